@@ -1,0 +1,169 @@
+/*
+ * csa.h -- C ABI of libcsa.so: the DeepSeek-V4 hybrid-attention hot path
+ * (CSA: Compressed Sparse Attention, HCA: Heavily Compressed Attention) as
+ * hand-written CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * The method (DeepSeek-V4 pages):
+ *   - blog.nickys.cn/?p=150, "1. CSA": every m tokens' key/value entries are
+ *     compressed into one entry (sequence length -> 1/m); a lightning indexer
+ *     selects the k compressed entries most relevant to each query; attention
+ *     runs over those plus a few sliding-window (uncompressed) entries.
+ *     "2. HCA": compression ratio m' >> m, no selection, dense attention over
+ *     every compressed entry.
+ *   - sz-guanghua.com.cn ifanr repost, attention section: the indexer scores
+ *     query/block relevance in FP4 and keeps the top-k blocks; both CSA and HCA
+ *     carry the sliding-window branch.
+ *   - m.youleyou.com/wenzhang/2906406.html, section 1: MXFP4 on the indexer's
+ *     query-key path.
+ * Where the pages leave a formula open, this library computes:
+ *   compression   a_i = exp(Z[i,c]+B[i mod m,c]) / sum_{block} exp(...),
+ *                 Kc[j,c] = sum_i a_i K[i,c], Vc[j,c] = sum_i a_i V[i,c]
+ *   indexer       I[t,j] = sum_h w[t,h] * ReLU(qI[t,h] . kI[j]) on MXFP4
+ *   visibility    block j (tokens j*m .. j*m+m-1) is visible to token t iff
+ *                 j*m+m-1 <= t, i.e. j < n_vis(t) = floor((t+1)/m)
+ *   top-k         k largest visible I[t,j]; ties -> smaller j
+ *   attention     one joint softmax over {selected (CSA) / all visible (HCA)
+ *                 compressed entries} U {raw tokens max(0,t-W+1) .. t}
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory, dense
+ *     row-major (last index fastest), 16-byte aligned.  bf16 tensors are passed
+ *     as `const void*` holding IEEE bfloat16 values.
+ *   - MXFP4 tensors: `*_codes` hold two E2M1 codes per byte (element 2i in the
+ *     low nibble of byte i); `*_scales` hold one E8M0 byte (2^(e-127)) per 32
+ *     consecutive elements.  Head weights w are one E2M1 code per byte (low
+ *     nibble).  Exactness precondition: every scale byte lies in [125, 128]
+ *     (2^-2 .. 2^1); a kernel that sees a byte outside it reports
+ *     CSA_ERR_RANGE through the status word and its scores are then unspecified.
+ *   - Work is enqueued on `stream` (0 = legacy default stream); no entry point
+ *     synchronises, allocates device memory or frees it.  Scratch memory is the
+ *     caller's `workspace`, sized by the matching *_workspace_bytes() query.
+ *   - Arguments are validated on the host before anything is enqueued; on any
+ *     error nothing is enqueued and a negative csa_status_t is returned.
+ *   - Device-side failures (a bounded wait that timed out, a scale byte outside
+ *     the exact range) are recorded in a 32-bit status word at the start of the
+ *     workspace; read it with csa_check_status() after the stream completes.
+ *   - Kernels are deterministic: no floating-point atomics, fixed reduction order.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* csa_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = -1,       /* null pointer, negative size, k/W out of range */
+  CSA_ERR_MISALIGNED = -2,        /* a pointer is not 16-byte aligned */
+  CSA_ERR_UNSUPPORTED_SHAPE = -3, /* d, H, HI, dI or m outside the supported set */
+  CSA_ERR_CUDA = -4,              /* a CUDA call failed; see csa_last_cuda_error() */
+  CSA_ERR_WORKSPACE = -5,         /* workspace null or smaller than required */
+  CSA_ERR_DEVICE_TIMEOUT = -6,    /* (status word) a bounded device wait gave up */
+  CSA_ERR_RANGE = -7              /* (status word) MXFP4 scale outside [125,128] */
+} csa_status_t;
+
+/* Human-readable text of a status code (static storage). */
+const char* csa_status_string(int status);
+/* The cudaError_t of the last CSA_ERR_CUDA on this host thread (0 if none). */
+int csa_last_cuda_error(void);
+/* Library version, major*10000 + minor*100 + patch. */
+int csa_version(void);
+
+/* Reads the device status word at the start of `workspace` (synchronously on
+ * `stream`) and clears it.  Returns CSA_OK or the first device-side error. */
+int csa_check_status(void* workspace, csa_stream_t stream);
+
+/* ---------------------------------------------------------------- compress
+ * Softmax-gated per-channel pooling of every complete block of m tokens
+ * (blog.nickys.cn/?p=150 "1. CSA"; gate weights exp(Z[i]+B[i mod m])).
+ *   K, V, Z : [T, d] bf16      B : [m, d] float32 (bias by position in block)
+ *   Kc, Vc  : [T/m, d] bf16 outputs (round-to-nearest-even of an fp32 result)
+ * The trailing T % m tokens are not compressed.  d in {64, 128}; 1 <= m <= 512
+ * with m <= 8 or m % 8 == 0.  For chunked prefill pass the chunk's rows (the
+ * chunk must start at a multiple of m) and the matching rows of Kc/Vc.
+ * No workspace. */
+int csa_compress(const void* K, const void* V, const void* Z, const float* B, int64_t T, int d, int m, void* Kc,
+                 void* Vc, csa_stream_t stream);
+
+/* ---------------------------------------------------------------- indexer + top-k
+ * Lightning indexer on MXFP4 fused with the causal top-k (ifanr repost,
+ * attention section; blog.nickys.cn/?p=150 "1. CSA").
+ * For query rows r in [0, T) at absolute positions t = t0 + r:
+ *   qI_codes [T, HI, dI/2] u8, qI_scales [T, HI, dI/32] u8, w_codes [T, HI] u8
+ *   kI_codes [Nc, dI/2] u8, kI_scales [Nc, dI/32] u8  (entries 0..Nc-1 of the
+ *            compressed cache; entry j covers tokens j*m .. j*m+m-1)
+ * Outputs, per row, in rank order (score descending, then j ascending):
+ *   idx    [T, k] int32  -- selected entries; -1 when fewer than k are visible
+ *   scores [T, k] float  -- I[t, idx] rounded to nearest float (-inf padding);
+ *                           may be NULL.
+ * HI in {4, 8, 16, 32, 64}, dI in {64, 128}, 1 <= k <= 2048, m >= 1.
+ * Scores are computed exactly (integer head sum), so idx is bit-exact. */
+size_t csa_indexer_topk_workspace_bytes(int64_t T, int64_t Nc, int HI, int dI, int k);
+int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                     const uint8_t* kI_codes, const uint8_t* kI_scales, int64_t T, int64_t t0, int64_t Nc, int HI,
+                     int dI, int m, int k, int32_t* idx, float* scores, void* workspace, size_t workspace_bytes,
+                     csa_stream_t stream);
+
+/* ---------------------------------------------------------------- CSA attention
+ * Sparse + sliding-window attention (blog.nickys.cn/?p=150 "1. CSA"; window
+ * branch: ifanr repost, attention section).  MQA: one shared K/V head.
+ *   Q      [T, H, d] bf16 (rows at absolute positions t = t0 + r)
+ *   Kc, Vc [Nc, d] bf16 compressed entries; idx [T, k] int32 (-1 = none)
+ *   Kraw, Vraw : raw K/V rows indexed by ABSOLUTE position (row s at
+ *          Kraw + s*d); rows max(0, t0-W+1) .. t0+T-1 must be readable.
+ *   O      [T, H, d] bf16 output; lse [T, H] float natural-log sum of exp of
+ *          the scaled logits (may be NULL).
+ * One joint softmax over the selected entries and the window; scale is the
+ * logit multiplier (1/sqrt(d) for the usual reading).  A row with an empty key
+ * set gets O = 0, lse = -inf.  H in {4, 8, 16, 32, 64, 128}, d in {64, 128},
+ * 1 <= k <= 2048, 0 <= W <= 1024. */
+size_t csa_sparse_attn_workspace_bytes(int64_t T, int H, int d, int k, int W);
+int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t* idx, const void* Kraw,
+                    const void* Vraw, int64_t T, int64_t t0, int64_t Nc, int H, int d, int k, int W, float scale,
+                    void* O, float* lse, void* workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------- HCA attention
+ * Dense attention over every visible compressed entry plus the window
+ * (blog.nickys.cn/?p=150 "2. HCA").  Same layouts as csa_sparse_attn without
+ * idx; entries j < min(Nc, floor((t+1)/m)) are visible to position t. */
+size_t hca_attn_workspace_bytes(int64_t T, int H, int d, int W);
+int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, const void* Vraw, int64_t T, int64_t t0,
+             int64_t Nc, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
+             size_t workspace_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------- decode
+ * One new token per sequence against a compressed KV cache (the decode case of
+ * the same method; ferris-liu.github.io ... deepseek-v4 section 3 gives the
+ * 1M-token cache sizes).  For sequence b in [0, B) the new token sits at
+ * absolute position pos[b] (host array), and:
+ *   q        [B, H, d] bf16           qI_codes [B, HI, dI/2], qI_scales [B, HI, dI/32]
+ *   w_codes  [B, HI]                  Kc, Vc [B, Ncap, d] bf16 compressed cache
+ *   kI_codes [B, Ncap, dI/2]          kI_scales [B, Ncap, dI/32]
+ *   Kwin, Vwin [B, W, d] bf16: raw K/V of positions pos[b]-W+1 .. pos[b]
+ *            (newest last; rows for negative positions are ignored)
+ *   O [B, H, d] bf16; lse [B, H] float (nullable); idx [B, k] int32 and
+ *   scores [B, k] float (both nullable) receive the selection.
+ * Entries j < min(Ncap, floor((pos[b]+1)/m)) are visible. */
+size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int HI, int dI, int k, int W);
+int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+               const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
+               const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
+               int W, float scale, void* O, float* lse, int32_t* idx, float* scores, void* workspace,
+               size_t workspace_bytes, csa_stream_t stream);
+
+/* HCA decode: dense over every visible cached entry plus the window. */
+size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W);
+int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
+               int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
+               size_t workspace_bytes, csa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

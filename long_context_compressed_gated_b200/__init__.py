@@ -1,0 +1,225 @@
+"""Python binding of libcsa.so -- the DeepSeek-V4 CSA/HCA hot path on B200.
+
+Argument marshalling only: every step runs in the CUDA kernels of libcsa.so
+(declared in include/csa.h).  Functions carry the C ABI names and take torch
+tensors that already live on the current CUDA device; outputs are allocated
+here when not supplied, scratch memory is a torch uint8 workspace sized by the
+library's *_workspace_bytes() query, and work is enqueued on torch's current
+stream.  A non-zero status from the library raises CsaError.  There is no CPU
+path: importing works without a GPU, but every call needs the CUDA library.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "CsaError", "lib", "csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode",
+    "hca_decode", "csa_check_status", "csa_status_string", "csa_version", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
+
+_lib = None
+
+
+class CsaError(RuntimeError):
+    def __init__(self, code, what):
+        super().__init__("%s failed: %s (status %d)" % (what, csa_status_string(code), code))
+        self.code = code
+
+
+def lib():
+    """The loaded libcsa.so. Raises if the CUDA library has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libcsa.so not found at %s; build it with "
+                               "`python -m long_context_compressed_gated_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I, SZ, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        sig = {
+            "csa_status_string": ([I], ctypes.c_char_p),
+            "csa_last_cuda_error": ([], I),
+            "csa_version": ([], I),
+            "csa_check_status": ([P, P], I),
+            "csa_compress": ([P, P, P, P, I64, I, I, P, P, P], I),
+            "csa_indexer_topk_workspace_bytes": ([I64, I64, I, I, I], SZ),
+            "csa_indexer_topk": ([P, P, P, P, P, I64, I64, I64, I, I, I, I, P, P, P, SZ, P], I),
+            "csa_sparse_attn_workspace_bytes": ([I64, I, I, I, I], SZ),
+            "csa_sparse_attn": ([P, P, P, P, P, P, I64, I64, I64, I, I, I, I, F, P, P, P, SZ, P], I),
+            "hca_attn_workspace_bytes": ([I64, I, I, I], SZ),
+            "hca_attn": ([P, P, P, P, P, I64, I64, I64, I, I, I, I, F, P, P, P, SZ, P], I),
+            "csa_decode_workspace_bytes": ([I, I64, I, I, I, I, I, I], SZ),
+            "csa_decode": ([P, P, P, P, P, P, P, P, P, P, P, I, I64, I, I, I, I, I, I, I, F, P, P, P, P, P, SZ, P],
+                           I),
+            "hca_decode_workspace_bytes": ([I, I64, I, I, I], SZ),
+            "hca_decode": ([P, P, P, P, P, P, I, I64, I, I, I, I, F, P, P, P, SZ, P], I),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def csa_status_string(code):
+    return lib().csa_status_string(int(code)).decode()
+
+
+def csa_version():
+    return lib().csa_version()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got %d" % (name, ndim, t.dim()))
+    return t
+
+
+def _check(code, what):
+    if code != 0:
+        raise CsaError(code, what)
+
+
+def _workspace(nbytes, device, workspace=None):
+    if workspace is not None:
+        if workspace.numel() < nbytes:
+            raise ValueError("workspace too small: %d < %d bytes" % (workspace.numel(), nbytes))
+        return workspace
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    ws[:4].zero_()  # status word
+    return ws
+
+
+def csa_check_status(workspace):
+    """Synchronise the current stream, return and clear the device status word."""
+    return lib().csa_check_status(_ptr(workspace), _stream())
+
+
+def csa_compress(K, V, Z, B, m, Kc=None, Vc=None):
+    """Gated pooling of every complete block of m tokens. K,V,Z [T,d] bf16, B [m,d] f32.
+    Returns (Kc, Vc) [T//m, d] bf16."""
+    _dev(K, torch.bfloat16, "K", 2), _dev(V, torch.bfloat16, "V", 2), _dev(Z, torch.bfloat16, "Z", 2)
+    _dev(B, torch.float32, "B", 2)
+    T, d = K.shape
+    nb = T // m
+    Kc = torch.empty(nb, d, dtype=torch.bfloat16, device=K.device) if Kc is None else _dev(Kc, torch.bfloat16, "Kc")
+    Vc = torch.empty(nb, d, dtype=torch.bfloat16, device=K.device) if Vc is None else _dev(Vc, torch.bfloat16, "Vc")
+    _check(lib().csa_compress(_ptr(K), _ptr(V), _ptr(Z), _ptr(B), T, d, m, _ptr(Kc), _ptr(Vc), _stream()),
+           "csa_compress")
+    return Kc, Vc
+
+
+def csa_indexer_topk(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, m, k, t0=0, idx=None, scores=None,
+                     want_scores=True, workspace=None):
+    """MXFP4 lightning indexer + causal top-k. Returns (idx [T,k] int32, scores [T,k] f32 or None, workspace)."""
+    _dev(qI_codes, torch.uint8, "qI_codes", 3), _dev(qI_scales, torch.uint8, "qI_scales", 3)
+    _dev(w_codes, torch.uint8, "w_codes", 2), _dev(kI_codes, torch.uint8, "kI_codes", 2)
+    _dev(kI_scales, torch.uint8, "kI_scales", 2)
+    T, HI, half = qI_codes.shape
+    dI = half * 2
+    Nc = kI_codes.shape[0]
+    dev = qI_codes.device
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev) if idx is None else _dev(idx, torch.int32, "idx")
+    if want_scores and scores is None:
+        scores = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ws = _workspace(lib().csa_indexer_topk_workspace_bytes(T, Nc, HI, dI, k), dev, workspace)
+    _check(lib().csa_indexer_topk(_ptr(qI_codes), _ptr(qI_scales), _ptr(w_codes), _ptr(kI_codes), _ptr(kI_scales),
+                                  T, t0, Nc, HI, dI, m, k, _ptr(idx), _ptr(scores), _ptr(ws), ws.numel(),
+                                  _stream()), "csa_indexer_topk")
+    return idx, scores, ws
+
+
+def csa_sparse_attn(Q, Kc, Vc, idx, Kraw, Vraw, W, scale, t0=0, O=None, lse=None, want_lse=True, workspace=None):
+    """CSA attention over the selected entries plus the raw window. Returns (O, lse, workspace)."""
+    _dev(Q, torch.bfloat16, "Q", 3), _dev(Kc, torch.bfloat16, "Kc", 2), _dev(Vc, torch.bfloat16, "Vc", 2)
+    _dev(idx, torch.int32, "idx", 2), _dev(Kraw, torch.bfloat16, "Kraw", 2), _dev(Vraw, torch.bfloat16, "Vraw", 2)
+    T, H, d = Q.shape
+    k = idx.shape[1]
+    dev = Q.device
+    O = torch.empty_like(Q) if O is None else _dev(O, torch.bfloat16, "O")
+    if want_lse and lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    ws = _workspace(lib().csa_sparse_attn_workspace_bytes(T, H, d, k, W), dev, workspace)
+    _check(lib().csa_sparse_attn(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(idx), _ptr(Kraw), _ptr(Vraw), T, t0,
+                                 Kc.shape[0], H, d, k, W, float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
+                                 _stream()), "csa_sparse_attn")
+    return O, lse, ws
+
+
+def hca_attn(Q, Kc, Vc, Kraw, Vraw, m, W, scale, t0=0, O=None, lse=None, want_lse=True, workspace=None):
+    """HCA attention over every visible compressed entry plus the raw window. Returns (O, lse, workspace)."""
+    _dev(Q, torch.bfloat16, "Q", 3), _dev(Kc, torch.bfloat16, "Kc", 2), _dev(Vc, torch.bfloat16, "Vc", 2)
+    _dev(Kraw, torch.bfloat16, "Kraw", 2), _dev(Vraw, torch.bfloat16, "Vraw", 2)
+    T, H, d = Q.shape
+    dev = Q.device
+    O = torch.empty_like(Q) if O is None else _dev(O, torch.bfloat16, "O")
+    if want_lse and lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    ws = _workspace(lib().hca_attn_workspace_bytes(T, H, d, W), dev, workspace)
+    _check(lib().hca_attn(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(Kraw), _ptr(Vraw), T, t0, Kc.shape[0], H, d, m, W,
+                          float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(), _stream()), "hca_attn")
+    return O, lse, ws
+
+
+def csa_decode(q, qI_codes, qI_scales, w_codes, Kc, Vc, kI_codes, kI_scales, Kwin, Vwin, pos, m, k, scale,
+               O=None, lse=None, idx=None, scores=None, want_lse=True, want_sel=True, workspace=None):
+    """One new token per sequence against its compressed cache (indexer, top-k,
+    sparse + window attention). pos: list of absolute positions (host).
+    Returns (O [B,H,d], lse, idx [B,k], scores [B,k], workspace)."""
+    _dev(q, torch.bfloat16, "q", 3), _dev(qI_codes, torch.uint8, "qI_codes", 3)
+    _dev(qI_scales, torch.uint8, "qI_scales", 3), _dev(w_codes, torch.uint8, "w_codes", 2)
+    _dev(Kc, torch.bfloat16, "Kc", 3), _dev(Vc, torch.bfloat16, "Vc", 3)
+    _dev(kI_codes, torch.uint8, "kI_codes", 3), _dev(kI_scales, torch.uint8, "kI_scales", 3)
+    _dev(Kwin, torch.bfloat16, "Kwin", 3), _dev(Vwin, torch.bfloat16, "Vwin", 3)
+    B, H, d = q.shape
+    HI, dI = qI_codes.shape[1], qI_codes.shape[2] * 2
+    Ncap = Kc.shape[1]
+    W = Kwin.shape[1]
+    dev = q.device
+    O = torch.empty_like(q) if O is None else _dev(O, torch.bfloat16, "O")
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    if want_sel:
+        idx = torch.empty(B, k, dtype=torch.int32, device=dev) if idx is None else idx
+        scores = torch.empty(B, k, dtype=torch.float32, device=dev) if scores is None else scores
+    posa = (ctypes.c_int64 * B)(*[int(p) for p in pos])
+    ws = _workspace(lib().csa_decode_workspace_bytes(B, Ncap, H, d, HI, dI, k, W), dev, workspace)
+    _check(lib().csa_decode(_ptr(q), _ptr(qI_codes), _ptr(qI_scales), _ptr(w_codes), _ptr(Kc), _ptr(Vc),
+                            _ptr(kI_codes), _ptr(kI_scales), _ptr(Kwin), _ptr(Vwin), posa, B, Ncap, H, d, HI, dI,
+                            m, k, W, float(scale), _ptr(O), _ptr(lse), _ptr(idx), _ptr(scores), _ptr(ws),
+                            ws.numel(), _stream()), "csa_decode")
+    return O, lse, idx, scores, ws
+
+
+def hca_decode(q, Kc, Vc, Kwin, Vwin, pos, m, scale, O=None, lse=None, want_lse=True, workspace=None):
+    """HCA decode: one token per sequence, dense over its visible cache + window."""
+    _dev(q, torch.bfloat16, "q", 3), _dev(Kc, torch.bfloat16, "Kc", 3), _dev(Vc, torch.bfloat16, "Vc", 3)
+    _dev(Kwin, torch.bfloat16, "Kwin", 3), _dev(Vwin, torch.bfloat16, "Vwin", 3)
+    B, H, d = q.shape
+    Ncap, W = Kc.shape[1], Kwin.shape[1]
+    dev = q.device
+    O = torch.empty_like(q) if O is None else _dev(O, torch.bfloat16, "O")
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    posa = (ctypes.c_int64 * B)(*[int(p) for p in pos])
+    ws = _workspace(lib().hca_decode_workspace_bytes(B, Ncap, H, d, W), dev, workspace)
+    _check(lib().hca_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Kwin), _ptr(Vwin), posa, B, Ncap, H, d, m, W,
+                            float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(), _stream()), "hca_decode")
+    return O, lse, ws

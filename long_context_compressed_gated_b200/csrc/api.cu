@@ -1,0 +1,402 @@
+// api.cu - the C ABI of libcsa.so (declared in include/csa.h): host-side
+// argument validation, workspace layout, status word, launch orchestration.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "attention.cuh"
+#include "common.cuh"
+
+namespace csa {
+
+// ---- kernels' host launchers (defined in the other translation units)
+cudaError_t launch_compress(const void* K, const void* V, const void* Z, const float* B, int64_t T, int d, int m,
+                            void* Kc, void* Vc, cudaStream_t stream);
+cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
+                                   const uint8_t* k_codes, const uint8_t* k_scales, int64_t T, int64_t t0, int64_t Nc,
+                                   int HI, int DI, int m, int k, int32_t* idx, float* scores, int* status,
+                                   cudaStream_t stream);
+cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
+                                  const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
+                                  int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
+                                  uint64_t* cand, int32_t* idx, float* scores, uint64_t* keys_out, int* status,
+                                  cudaStream_t stream);
+
+
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  if (e == cudaErrorInvalidConfiguration) return CSA_ERR_UNSUPPORTED_SHAPE;
+  return CSA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename... P>
+int check_ptrs(P... ps) {
+  const void* arr[] = {static_cast<const void*>(ps)...};
+  for (const void* p : arr) {
+    if (p == nullptr) return CSA_ERR_INVALID_ARG;
+    if (!aligned16(p)) return CSA_ERR_MISALIGNED;
+  }
+  return CSA_OK;
+}
+
+int check_opt(const void* p) { return (p != nullptr && !aligned16(p)) ? CSA_ERR_MISALIGNED : CSA_OK; }
+
+bool valid_H(int H) { return H == 4 || H == 8 || H == 16 || H == 32 || H == 64 || H == 128; }
+bool valid_HI(int HI) { return HI == 4 || HI == 8 || HI == 16 || HI == 32 || HI == 64; }
+
+int check_ws(void* ws, size_t bytes, size_t need) {
+  if (ws == nullptr || bytes < need) return CSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return CSA_ERR_MISALIGNED;
+  return CSA_OK;
+}
+
+int* status_word(void* ws) { return static_cast<int*>(ws); }
+
+// window tiles a CTA of gq consecutive tokens may need
+int64_t window_tiles(int W, int gq) { return W > 0 ? ceil_div((int64_t)W + gq - 1, 128) : 0; }
+
+struct PosBlock {
+  int64_t v[64];
+};
+
+__global__ void fill_i64_kernel(int64_t* dst, PosBlock blk, int n) {
+  if ((int)threadIdx.x < n) dst[threadIdx.x] = blk.v[threadIdx.x];
+}
+
+cudaError_t upload_positions(int64_t* dst, const int64_t* host, int B, cudaStream_t stream) {
+  for (int b0 = 0; b0 < B; b0 += 64) {
+    PosBlock blk{};
+    const int n = B - b0 < 64 ? B - b0 : 64;
+    for (int i = 0; i < n; ++i) blk.v[i] = host[b0 + i];
+    fill_i64_kernel<<<1, 64, 0, stream>>>(dst + b0, blk, n);
+  }
+  return cudaGetLastError();
+}
+
+// decode workspace: [header][pos B*8][idx B*k*4][cand B*nsplit*k*8]
+int decode_nsplit(int B, int64_t Ncap, int k) {
+  int sms = 148;
+  int ns = (int)((2 * sms + B - 1) / B);
+  const int64_t tiles = ceil_div(Ncap > 0 ? Ncap : 1, 128);
+  if (ns > tiles) ns = (int)tiles;
+  const int lim = 256 * 40 / k;  // merge capacity
+  if (ns > lim) ns = lim;
+  return ns < 1 ? 1 : ns;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+const char* csa_status_string(int status) {
+  switch (status) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case CSA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case CSA_ERR_CUDA: return "CUDA error (see csa_last_cuda_error)";
+    case CSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    case CSA_ERR_RANGE: return "MXFP4 scale byte outside [125, 128]";
+    default: return "unknown status";
+  }
+}
+
+int csa_last_cuda_error(void) { return g_last_cuda_error; }
+
+int csa_version(void) { return 100; }
+
+int csa_check_status(void* workspace, csa_stream_t stream) {
+  if (workspace == nullptr) return CSA_ERR_WORKSPACE;
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(int), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return v;
+}
+
+int csa_compress(const void* K, const void* V, const void* Z, const float* B, int64_t T, int d, int m, void* Kc,
+                 void* Vc, csa_stream_t stream) {
+  if (T < 0 || m < 1) return CSA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return CSA_ERR_UNSUPPORTED_SHAPE;
+  // rows per thread L and slices S = m / L with (d/8) * S <= 256 threads per block
+  const int CG = d / 8;
+  int L = m <= 8 ? m : 8;
+  while ((int64_t)CG * (m / L) > 256) L *= 2;
+  if (m % L != 0 || m > 4096) return CSA_ERR_UNSUPPORTED_SHAPE;
+  if (T / m == 0) return CSA_OK;
+  int rc = check_ptrs(K, V, Z, B, Kc, Vc);
+  if (rc) return rc;
+  cudaError_t e = launch_compress(K, V, Z, B, T, d, m, Kc, Vc, (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+size_t csa_indexer_topk_workspace_bytes(int64_t, int64_t, int, int, int) { return kWorkspaceHeader; }
+
+int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                     const uint8_t* kI_codes, const uint8_t* kI_scales, int64_t T, int64_t t0, int64_t Nc, int HI,
+                     int dI, int m, int k, int32_t* idx, float* scores, void* workspace, size_t workspace_bytes,
+                     csa_stream_t stream) {
+  if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || k < 1 || k > 2048) return CSA_ERR_INVALID_ARG;
+  if (!valid_HI(HI) || (dI != 64 && dI != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
+  if (rc) return rc;
+  if (T == 0) return CSA_OK;
+  rc = check_ptrs(qI_codes, qI_scales, w_codes, idx);
+  if (rc) return rc;
+  if (Nc > 0 && (rc = check_ptrs(kI_codes, kI_scales))) return rc;
+  if ((rc = check_opt(scores))) return rc;
+  cudaError_t e = launch_indexer_prefill(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, T, t0, Nc, HI, dI, m, k,
+                                         idx, scores, status_word(workspace), (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+size_t csa_sparse_attn_workspace_bytes(int64_t, int, int, int, int) { return kWorkspaceHeader; }
+
+int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t* idx, const void* Kraw,
+                    const void* Vraw, int64_t T, int64_t t0, int64_t Nc, int H, int d, int k, int W, float scale,
+                    void* O, float* lse, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  if (T < 0 || t0 < 0 || Nc < 0 || k < 1 || k > 2048 || W < 0 || W > 1024 || !std::isfinite(scale))
+    return CSA_ERR_INVALID_ARG;
+  if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  const int gq = 128 / H;
+  if (gq * ceil_div(k, 128) + window_tiles(W, gq) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
+  if (rc) return rc;
+  if (T == 0) return CSA_OK;
+  rc = check_ptrs(Q, idx, O);
+  if (rc) return rc;
+  if (Nc > 0 && (rc = check_ptrs(Kc, Vc))) return rc;
+  if (W > 0 && (rc = check_ptrs(Kraw, Vraw))) return rc;
+  if ((rc = check_opt(lse))) return rc;
+  AttnArgs a{};
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.Kc = static_cast<const __nv_bfloat16*>(Nc > 0 ? Kc : Q);
+  a.Vc = static_cast<const __nv_bfloat16*>(Nc > 0 ? Vc : Q);
+  a.idx = idx;
+  a.Kr = static_cast<const __nv_bfloat16*>(W > 0 ? Kraw : Q);
+  a.Vr = static_cast<const __nv_bfloat16*>(W > 0 ? Vraw : Q);
+  a.T = T;
+  a.t0 = t0;
+  a.Nc = Nc;
+  a.raw_lo = 0;
+  a.H = H;
+  a.k = k;
+  a.m = 1;
+  a.W = W;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.status = status_word(workspace);
+  cudaError_t e = launch_attention(a, d, (unsigned)ceil_div(T, gq), (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+size_t hca_attn_workspace_bytes(int64_t, int, int, int) { return kWorkspaceHeader; }
+
+int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, const void* Vraw, int64_t T, int64_t t0,
+             int64_t Nc, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
+             size_t workspace_bytes, csa_stream_t stream) {
+  if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || W < 0 || W > 1024 || !std::isfinite(scale)) return CSA_ERR_INVALID_ARG;
+  if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  const int gq = 128 / H;
+  int64_t nv = n_visible(t0 + T - 1, m);
+  if (nv > Nc) nv = Nc;
+  if (ceil_div(nv, 128) + window_tiles(W, gq) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
+  if (rc) return rc;
+  if (T == 0) return CSA_OK;
+  rc = check_ptrs(Q, O);
+  if (rc) return rc;
+  if (Nc > 0 && (rc = check_ptrs(Kc, Vc))) return rc;
+  if (W > 0 && (rc = check_ptrs(Kraw, Vraw))) return rc;
+  if ((rc = check_opt(lse))) return rc;
+  AttnArgs a{};
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.Kc = static_cast<const __nv_bfloat16*>(Nc > 0 ? Kc : Q);
+  a.Vc = static_cast<const __nv_bfloat16*>(Nc > 0 ? Vc : Q);
+  a.idx = nullptr;
+  a.Kr = static_cast<const __nv_bfloat16*>(W > 0 ? Kraw : Q);
+  a.Vr = static_cast<const __nv_bfloat16*>(W > 0 ? Vraw : Q);
+  a.T = T;
+  a.t0 = t0;
+  a.Nc = Nc;
+  a.raw_lo = 0;
+  a.H = H;
+  a.k = 0;
+  a.m = m;
+  a.W = W;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.status = status_word(workspace);
+  cudaError_t e = launch_attention(a, d, (unsigned)ceil_div(T, gq), (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int, int, int, int, int k, int) {
+  if (B <= 0 || k <= 0) return kWorkspaceHeader;
+  const int ns = decode_nsplit(B, Ncap, k);
+  return kWorkspaceHeader + align256((size_t)B * 8) + align256((size_t)B * k * 4) +
+         align256((size_t)B * ns * k * 8);
+}
+
+int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+               const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
+               const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
+               int W, float scale, void* O, float* lse, int32_t* idx, float* scores, void* workspace,
+               size_t workspace_bytes, csa_stream_t stream) {
+  if (B < 0 || Ncap < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 || !std::isfinite(scale))
+    return CSA_ERR_INVALID_ARG;
+  if (!valid_H(H) || (d != 64 && d != 128) || !valid_HI(HI) || (dI != 64 && dI != 128))
+    return CSA_ERR_UNSUPPORTED_SHAPE;
+  if (ceil_div(k, 128) + window_tiles(W, 1) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, csa_decode_workspace_bytes(B, Ncap, H, d, HI, dI, k, W));
+  if (rc) return rc;
+  if (B == 0) return CSA_OK;
+  if (pos == nullptr) return CSA_ERR_INVALID_ARG;
+  int64_t nvis_max = 0;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0) return CSA_ERR_INVALID_ARG;
+    int64_t nv = n_visible(pos[b], m);
+    if (nv > Ncap) nv = Ncap;
+    if (nv > nvis_max) nvis_max = nv;
+  }
+  rc = check_ptrs(q, qI_codes, qI_scales, w_codes, O);
+  if (rc) return rc;
+  if (Ncap > 0 && (rc = check_ptrs(Kc, Vc, kI_codes, kI_scales))) return rc;
+  if (W > 0 && (rc = check_ptrs(Kwin, Vwin))) return rc;
+  if ((rc = check_opt(lse)) || (rc = check_opt(idx)) || (rc = check_opt(scores))) return rc;
+  const int ns = decode_nsplit(B, Ncap, k);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int64_t* pos_dev = reinterpret_cast<int64_t*>(w + kWorkspaceHeader);
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(w + kWorkspaceHeader + align256((size_t)B * 8));
+  uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader + align256((size_t)B * 8) +
+                                               align256((size_t)B * k * 4));
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int32_t* sel = idx ? idx : idx_ws;
+  if (Ncap > 0) {
+    e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, nvis_max, Ncap, HI, dI,
+                              m, k, ns, cand, sel, scores, nullptr, status_word(workspace), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  } else {
+    e = cudaMemsetAsync(sel, 0xFF, (size_t)B * k * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  AttnArgs a{};
+  a.Q = static_cast<const __nv_bfloat16*>(q);
+  a.Kc = static_cast<const __nv_bfloat16*>(Ncap > 0 ? Kc : q);
+  a.Vc = static_cast<const __nv_bfloat16*>(Ncap > 0 ? Vc : q);
+  a.idx = sel;
+  a.Kr = static_cast<const __nv_bfloat16*>(W > 0 ? Kwin : q);
+  a.Vr = static_cast<const __nv_bfloat16*>(W > 0 ? Vwin : q);
+  a.T = 1;
+  a.t0 = 0;
+  a.Nc = Ncap;
+  a.H = H;
+  a.k = k;
+  a.m = m;
+  a.W = W;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.status = status_word(workspace);
+  a.q_batch_stride = (int64_t)H * d;
+  a.kc_batch_stride = Ncap * d;
+  a.raw_batch_stride = (int64_t)W * d;
+  a.o_batch_stride = (int64_t)H * d;
+  a.pos = pos_dev;
+  e = launch_attention(a, d, (unsigned)B, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+size_t hca_decode_workspace_bytes(int B, int64_t, int, int, int) {
+  return kWorkspaceHeader + align256((size_t)(B > 0 ? B : 0) * 8);
+}
+
+int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
+               int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
+               size_t workspace_bytes, csa_stream_t stream) {
+  if (B < 0 || Ncap < 0 || m < 1 || W < 0 || W > 1024 || !std::isfinite(scale)) return CSA_ERR_INVALID_ARG;
+  if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, hca_decode_workspace_bytes(B, Ncap, H, d, W));
+  if (rc) return rc;
+  if (B == 0) return CSA_OK;
+  if (pos == nullptr) return CSA_ERR_INVALID_ARG;
+  int64_t nvis_max = 0;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0) return CSA_ERR_INVALID_ARG;
+    int64_t nv = n_visible(pos[b], m);
+    if (nv > Ncap) nv = Ncap;
+    if (nv > nvis_max) nvis_max = nv;
+  }
+  if (ceil_div(nvis_max, 128) + window_tiles(W, 1) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
+  rc = check_ptrs(q, O);
+  if (rc) return rc;
+  if (Ncap > 0 && (rc = check_ptrs(Kc, Vc))) return rc;
+  if (W > 0 && (rc = check_ptrs(Kwin, Vwin))) return rc;
+  if ((rc = check_opt(lse))) return rc;
+  int64_t* pos_dev = reinterpret_cast<int64_t*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  AttnArgs a{};
+  a.Q = static_cast<const __nv_bfloat16*>(q);
+  a.Kc = static_cast<const __nv_bfloat16*>(Ncap > 0 ? Kc : q);
+  a.Vc = static_cast<const __nv_bfloat16*>(Ncap > 0 ? Vc : q);
+  a.idx = nullptr;
+  a.Kr = static_cast<const __nv_bfloat16*>(W > 0 ? Kwin : q);
+  a.Vr = static_cast<const __nv_bfloat16*>(W > 0 ? Vwin : q);
+  a.T = 1;
+  a.Nc = Ncap;
+  a.H = H;
+  a.m = m;
+  a.W = W;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.status = status_word(workspace);
+  a.q_batch_stride = (int64_t)H * d;
+  a.kc_batch_stride = Ncap * d;
+  a.raw_batch_stride = (int64_t)W * d;
+  a.o_batch_stride = (int64_t)H * d;
+  a.pos = pos_dev;
+  e = launch_attention(a, d, (unsigned)B, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

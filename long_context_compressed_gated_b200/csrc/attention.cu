@@ -1,0 +1,479 @@
+// attention.cu - CSA sparse + window attention and HCA dense + window attention.
+//
+// blog.nickys.cn/?p=150, "1. CSA": each query attends only to its k selected
+// compressed entries plus a few sliding-window (uncompressed) entries; "2. HCA":
+// dense attention over every compressed entry.  Window branch in both: ifanr
+// repost (sz-guanghua.com.cn), attention section.  One joint softmax over the
+// whole key set (the specification's reading); MQA: all heads share K/V.
+//
+// One CTA = 128 query rows = GQ = 128/H consecutive tokens x H heads.  The CTA
+// walks a list of key tiles (<= 128 keys each, width a multiple of 16):
+//   SEG(g)  : up to 128 of token g's selected compressed entries (CSA)
+//   HCA(j0) : compressed entries j0 .. j0+127 (HCA)
+//   WIN(w0) : raw tokens at positions w0 .. w0+127 (window union of the group)
+// and every row sees, per tile, one contiguous range of its columns (its own
+// segment / the visible prefix / its window), so masking needs no per-key data.
+//
+// Per tile: S = Q K^T (tcgen05 kind::f16, M=128, N=width, fp32 in TMEM),
+// online softmax in the softmax warps (one row per thread, exp2 with a lazily
+// raised running max), P (bf16) to shared memory, O += P V (tcgen05, V read as
+// an MN-major operand, O accumulated in TMEM).  K/V rows are gathered by four
+// producer warps with 16-byte cp.async into 128B-swizzled tiles (K and V in
+// separate double-buffered rings, so S of tile i+2 can start while PV of tile i
+// still reads V).
+#include "attention.cuh"
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kRows = 128;
+constexpr int kTileKeys = 128;
+constexpr int kMaxTiles = 80;
+constexpr int kSoftmaxWarps = 4, kProducerWarps = 3;
+constexpr int kThreads = (kSoftmaxWarps + kProducerWarps + 1) * 32;  // + 1 MMA warp
+constexpr float kRescaleSlack = 8.0f;  // raise the running max only when it grows by > 2^8
+
+enum TileType : int { kSeg = 0, kHca = 1, kWin = 2 };
+
+struct Tile {
+  int type, owner, width, valid;  // valid: SEG entries in this tile
+  int64_t base;                   // SEG: offset in the token's list; HCA: j0; WIN: w0
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Arrive on `bar` once all prior cp.async of this thread have landed (no extra pending count).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+}  // namespace
+
+
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kHalf = kRows * 128;                // one 64-column half of a 128-row tile
+  static constexpr int kTileBytes = (D / 64) * kHalf;      // 128 rows x D bf16
+  static constexpr size_t off_q = 0;
+  static constexpr size_t off_k = off_q + kTileBytes;      // 2 stages
+  static constexpr size_t off_v = off_k + 2 * kTileBytes;  // 2 stages
+  static constexpr size_t off_p = off_v + 2 * kTileBytes;  // 128 x 128 bf16
+  static constexpr size_t off_tiles = off_p + 2 * kHalf;
+  static constexpr size_t off_bar = off_tiles + kMaxTiles * sizeof(Tile);
+  static constexpr size_t off_misc = off_bar + 16 * 8;
+  static constexpr size_t off_idx = off_misc + 256;
+  static size_t bytes(int idx_entries) { return off_idx + (size_t)idx_entries * 4 + 1024; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a) {
+  using L = AttnSmem<D>;
+  constexpr int KSTEPS_QK = D / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_q = smem + L::off_q;
+  uint8_t* s_k = smem + L::off_k;
+  uint8_t* s_v = smem + L::off_v;
+  uint8_t* s_p = smem + L::off_p;
+  Tile* s_tiles = reinterpret_cast<Tile*>(smem + L::off_tiles);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+  uint64_t* q_full = bar + 0;
+  uint64_t* k_full = bar + 1;   // [2]
+  uint64_t* k_empty = bar + 3;  // [2]
+  uint64_t* v_full = bar + 5;   // [2]
+  uint64_t* v_empty = bar + 7;  // [2]
+  uint64_t* s_full = bar + 9;   // [2]
+  uint64_t* s_free = bar + 11;  // [2]
+  uint64_t* p_full = bar + 13;
+  uint64_t* pv_done = bar + 14;
+  int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [0] ntiles, [1] tmem, [2..] seg counts
+  int* s_idx = reinterpret_cast<int*>(smem + L::off_idx);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = a.H;
+  const int GQ = kRows / H;
+  const bool decode = a.pos != nullptr;
+  const int64_t b = decode ? blockIdx.x : 0;
+  const int64_t row_tok0 = decode ? 0 : (int64_t)blockIdx.x * GQ;  // first token row of this CTA
+  const __nv_bfloat16* Q = a.Q + b * a.q_batch_stride;
+  const __nv_bfloat16* Kc = a.Kc + b * a.kc_batch_stride;
+  const __nv_bfloat16* Vc = a.Vc + b * a.kc_batch_stride;
+  const __nv_bfloat16* Kr = a.Kr + b * a.raw_batch_stride;
+  const __nv_bfloat16* Vr = a.Vr + b * a.raw_batch_stride;
+  const int32_t* idx = a.idx ? a.idx + b * (decode ? (int64_t)a.k : 0) : nullptr;
+  const int64_t T = decode ? 1 : a.T;
+  const int64_t raw_lo = decode ? a.pos[b] - a.W + 1 : a.raw_lo;  // absolute position of raw row 0
+  auto token_pos = [&](int g) -> int64_t {
+    const int64_t r = row_tok0 + g;
+    if (r >= T) return -1;
+    return decode ? a.pos[b] : a.t0 + r;
+  };
+  const int ntok = (int)((T - row_tok0) < GQ ? (T - row_tok0) : GQ);
+  const int64_t t_first = token_pos(0), t_last = token_pos(ntok - 1);
+
+  // ---- setup: barriers, TMEM, selected-index lists, tile list
+  if (tid == 0) {
+    mbar_init(q_full, kProducerWarps * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], kProducerWarps * 32);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], kProducerWarps * 32);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kSoftmaxWarps);
+    }
+    mbar_init(p_full, kSoftmaxWarps);
+    mbar_init(pv_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == kSoftmaxWarps + kProducerWarps) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(&misc[1]), 512);
+    tmem_relinquish();
+  }
+  // compact each token's selected list (drop -1 / out-of-range), one warp per token
+  if (idx != nullptr) {
+    for (int g = warp; g < ntok; g += kThreads / 32) {
+      const int32_t* src = idx + (row_tok0 + g) * a.k;
+      int n = 0;
+      for (int base = 0; base < a.k; base += 32) {
+        const int q = base + lane;
+        int32_t j = q < a.k ? src[q] : -1;
+        const bool ok = j >= 0 && j < a.Nc;
+        const uint32_t bal = __ballot_sync(0xffffffffu, ok);
+        if (ok) s_idx[g * a.k + n + __popc(bal & ((1u << lane) - 1u))] = j;
+        n += __popc(bal);
+      }
+      if (lane == 0) misc[2 + g] = n;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nt = 0;
+    if (idx != nullptr) {
+      for (int g = 0; g < ntok; ++g) {
+        const int n = misc[2 + g];
+        for (int off = 0; off < n && nt < kMaxTiles; off += kTileKeys) {
+          const int v = n - off < kTileKeys ? n - off : kTileKeys;
+          s_tiles[nt++] = Tile{kSeg, g, (v + 15) & ~15, v, (int64_t)off};
+        }
+      }
+    } else {
+      int64_t nv = n_visible(t_last, a.m);
+      if (nv > a.Nc) nv = a.Nc;
+      for (int64_t j0 = 0; j0 < nv && nt < kMaxTiles; j0 += kTileKeys) {
+        const int v = (int)(nv - j0 < kTileKeys ? nv - j0 : kTileKeys);
+        s_tiles[nt++] = Tile{kHca, 0, (v + 15) & ~15, v, j0};
+      }
+    }
+    if (a.W > 0 && ntok > 0) {
+      int64_t w_lo = t_first - a.W + 1;
+      if (w_lo < raw_lo) w_lo = raw_lo;
+      if (w_lo < 0) w_lo = 0;
+      for (int64_t w0 = w_lo; w0 <= t_last && nt < kMaxTiles; w0 += kTileKeys) {
+        const int v = (int)(t_last - w0 + 1 < kTileKeys ? t_last - w0 + 1 : kTileKeys);
+        s_tiles[nt++] = Tile{kWin, 0, (v + 15) & ~15, v, w0};
+      }
+    }
+    misc[0] = nt;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int ntiles = misc[0];
+  const uint32_t tbase = (uint32_t)misc[1];
+  constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+
+  if (warp >= kSoftmaxWarps && warp < kSoftmaxWarps + kProducerWarps) {
+    // =========================== producers: Q once, then K/V tiles
+    constexpr int NP = kProducerWarps * 32;
+    const int pt = tid - kSoftmaxWarps * 32;  // 0..NP-1
+    constexpr int CH = D / 8;                  // 16-byte chunks per row
+    constexpr int ROWS_PER_PASS = NP / CH;
+    auto dst_off = [](int row, int c) -> uint32_t {
+      const int half = c >> 3, cc = c & 7;
+      return (uint32_t)(half * (kRows * 128) + row * 128 + ((cc ^ (row & 7)) << 4));
+    };
+    {
+      const uint32_t sq = smem_u32(s_q);
+      const int c = pt % CH;
+      for (int row = pt / CH; row < kRows; row += ROWS_PER_PASS) {
+        const int g = row / H, h = row % H;
+        const bool ok = g < ntok;
+        const __nv_bfloat16* src = ok ? Q + ((row_tok0 + g) * H + h) * (int64_t)D + c * 8 : a.Q;
+        cp_async16(sq + dst_off(row, c), src, ok ? 16u : 0u);
+      }
+      cp_async_arrive(q_full);
+    }
+    auto row_src = [&](const Tile& tl, int x, bool value) -> const __nv_bfloat16* {
+      if (x >= tl.valid) return nullptr;
+      if (tl.type == kSeg) {
+        const int j = s_idx[tl.owner * a.k + (int)tl.base + x];
+        return (value ? Vc : Kc) + (int64_t)j * D;
+      }
+      if (tl.type == kHca) return (value ? Vc : Kc) + (tl.base + x) * D;
+      return (value ? Vr : Kr) + (tl.base + x - raw_lo) * D;
+    };
+    for (int i = 0; i < ntiles; ++i) {
+      const Tile tl = s_tiles[i];
+      const int st = i & 1;
+      const uint32_t ph = (i >> 1) & 1;
+      for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
+        uint64_t* empty = which ? &v_empty[st] : &k_empty[st];
+        uint64_t* fullb = which ? &v_full[st] : &k_full[st];
+        if (!mbar_wait(empty, ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
+        const uint32_t base = smem_u32((which ? s_v : s_k) + (size_t)st * L::kTileBytes);
+        const int c = pt % CH;
+        for (int x = pt / CH; x < tl.width; x += ROWS_PER_PASS) {
+          const __nv_bfloat16* src = row_src(tl, x, which == 1);
+          cp_async16(base + dst_off(x, c), src ? src + c * 8 : a.Kc, src ? 16u : 0u);
+        }
+        cp_async_arrive(fullb);
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp == kSoftmaxWarps + kProducerWarps) {
+    // =========================== MMA issuer
+    if (ntiles > 0) mbar_wait(q_full, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
+    fence_proxy_async_smem();
+    tc_fence_after();
+    const uint32_t sq = smem_u32(s_q), sp = smem_u32(s_p);
+    auto issue_s = [&](int i) {
+      const int st = i & 1;
+      const uint32_t ph = (i >> 1) & 1;
+      mbar_wait(&k_full[st], ph, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      mbar_wait(&s_free[st], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tcgen05 (async proxy) reads
+      tc_fence_after();
+      if (lane == 0) {
+        const int width = s_tiles[i].width;
+        const uint32_t sk = smem_u32(s_k + (size_t)st * L::kTileBytes);
+        const uint32_t d = tbase + (st ? kTmemS1 : kTmemS0);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS_QK; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+          mma_bf16_ss(d, make_sdesc(sq + off, 16, 1024, kSwizzle128), make_sdesc(sk + off, 16, 1024, kSwizzle128),
+                      idesc_bf16(128, width, 0, 0), kk > 0);
+        }
+        mma_commit(&s_full[st]);
+        mma_commit(&k_empty[st]);
+      }
+      __syncwarp();
+    };
+    if (ntiles > 0) issue_s(0);
+    if (ntiles > 1) issue_s(1);
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i & 1;
+      mbar_wait(p_full, i & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      mbar_wait(&v_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      fence_proxy_async_smem();
+      tc_fence_after();
+      if (lane == 0) {
+        const int width = s_tiles[i].width;
+        const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
+        for (int ks = 0; ks < width / 16; ++ks) {
+          const uint32_t aoff = (uint32_t)((ks >> 2) * (kRows * 128) + (ks & 3) * 32);
+          mma_bf16_ss(tbase + kTmemO, make_sdesc(sp + aoff, 16, 1024, kSwizzle128),
+                      make_sdesc(sv + ks * 2048, kRows * 128, 1024, kSwizzle128), idesc_bf16(128, D, 0, 1),
+                      (i > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(pv_done);
+        mma_commit(&v_empty[st]);
+      }
+      __syncwarp();
+      if (i + 2 < ntiles) issue_s(i + 2);
+    }
+  } else {
+    // =========================== softmax (warps 0..3, one row per thread)
+    const int row = warp * 32 + lane;
+    const int g = row / H, h = row % H;
+    const int64_t t = g < ntok ? token_pos(g) : -1;
+    int64_t nvis = n_visible(t, a.m);
+    if (nvis > a.Nc) nvis = a.Nc;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t prow = smem_u32(s_p) + (uint32_t)row * 128;
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i & 1;
+      const Tile tl = s_tiles[i];
+      int lo = 0, hi = 0;
+      if (t >= 0) {
+        if (tl.type == kSeg) {
+          if (tl.owner == g) hi = tl.valid;
+        } else if (tl.type == kHca) {
+          const int64_t e = nvis - tl.base;
+          hi = (int)(e < 0 ? 0 : (e > tl.valid ? tl.valid : e));
+        } else {
+          int64_t l0 = t - a.W + 1 - tl.base, h0 = t - tl.base + 1;
+          if (l0 < 0) l0 = 0;
+          if (h0 > tl.valid) h0 = tl.valid;
+          lo = (int)l0;
+          hi = (int)(h0 > l0 ? h0 : l0);
+        }
+      }
+      mbar_wait(&s_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      tc_fence_after();
+      const uint32_t scol = tbase + lane_base + (st ? kTmemS1 : kTmemS0);
+      // pass 1: tile maximum over this row's visible range (log2 units of the scaled logits)
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c0 = 0; c0 < kTileKeys; c0 += 32) {
+        if (c0 < tl.width) {  // warp-uniform
+          uint32_t v[32];
+          tmem_ld32(scol + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e >= lo && c0 + e < hi) mt = fmaxf(mt, __uint_as_float(v[e]) * a.scale_log2);
+        }
+      }
+      const bool raise = mt > m_run + kRescaleSlack || (m_run == -INFINITY && mt > -INFINITY);
+      const float m_new = raise ? mt : m_run;
+      const float alpha = raise ? exp2f(m_run - m_new) : 1.0f;  // exp2(-inf) = 0 on the first raise
+      // pass 2: probabilities, packed to bf16 pairs
+      uint32_t pk[kTileKeys / 2];
+      float lsum = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < kTileKeys; c0 += 32) {
+        if (c0 < tl.width) {
+          uint32_t v[32];
+          tmem_ld32(scol + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int x = c0 + e;
+            float p0 = 0.f, p1 = 0.f;
+            if (x >= lo && x < hi) p0 = exp2f(__uint_as_float(v[e]) * a.scale_log2 - m_new);
+            if (x + 1 >= lo && x + 1 < hi) p1 = exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - m_new);
+            lsum += p0 + p1;
+            pk[x / 2] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) pk[(c0 + e) / 2] = 0u;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      // wait until PV of the previous tile finished: P buffer free, O stable
+      if (i > 0) {
+        mbar_wait(pv_done, (i - 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
+        const float sc = (raise && i > 0) ? alpha : 1.0f;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tbase + lane_base + kTmemO + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+              "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+                  tbase + lane_base + kTmemO + c0),
+              "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+              "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+              "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+              "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+              : "memory");
+        }
+        tmem_wait_st();
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+      // store the P row (K-major, 128B swizzle, two 64-key halves)
+#pragma unroll
+      for (int cc = 0; cc < kTileKeys / 8; ++cc) {
+        if (cc * 8 < tl.width) {
+          const uint32_t off = (uint32_t)((cc >> 3) * (kRows * 128) + (((cc & 7) ^ (row & 7)) << 4));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + off), "r"(pk[cc * 4]),
+                       "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // epilogue: O / l
+    if (ntiles > 0) {
+      mbar_wait(pv_done, (ntiles - 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      tc_fence_after();
+    }
+    const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
+    __nv_bfloat16* orow = nullptr;
+    if (t >= 0) orow = a.O + b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t v[32];
+      if (ntiles > 0) {
+        tmem_ld32(tbase + lane_base + kTmemO + c0, v);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (orow) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
+          o.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
+          o.z = pack_bf16x2(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
+          o.w = pack_bf16x2(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + c0 + e) = o;
+        }
+      }
+    }
+    if (t >= 0 && a.lse) {
+      const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kSoftmaxWarps + kProducerWarps) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+size_t attention_smem_bytes(int d, int idx_entries) {
+  return d == 128 ? AttnSmem<128>::bytes(idx_entries) : AttnSmem<64>::bytes(idx_entries);
+}
+
+int attention_max_tiles() { return kMaxTiles; }
+
+cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream) {
+  const int GQ = kRows / a.H;
+  const int idx_entries = a.idx ? GQ * a.k : 0;
+  const size_t smem = attention_smem_bytes(d, idx_entries);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attention_kernel<128><<<grid, kThreads, smem, stream>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attention_kernel<64><<<grid, kThreads, smem, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -1,0 +1,31 @@
+// attention.cuh - arguments of the attention kernel (CSA sparse / HCA dense,
+// prefill and decode) shared by its launcher and the C ABI.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace csa {
+
+struct AttnArgs {
+  const __nv_bfloat16* Q;   // [T, H, d] (decode: [B, H, d])
+  const __nv_bfloat16* Kc;  // [Nc, d] compressed keys (decode: per-sequence cache)
+  const __nv_bfloat16* Vc;
+  const int32_t* idx;       // [T, k] selected entries (CSA) or null (HCA)
+  const __nv_bfloat16* Kr;  // raw K rows, row 0 at absolute position raw_lo
+  const __nv_bfloat16* Vr;
+  int64_t T, t0, Nc, raw_lo;
+  int H, k, m, W;
+  float scale_log2;         // softmax scale * log2(e)
+  __nv_bfloat16* O;         // [T, H, d]
+  float* lse;               // [T, H] natural-log normaliser, nullable
+  int* status;              // device status word
+  // decode (pos != null): one sequence per CTA, batch strides in elements
+  int64_t q_batch_stride, kc_batch_stride, raw_batch_stride, o_batch_stride;
+  const int64_t* pos;       // device, absolute position of each sequence's new token
+};
+
+cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);
+int attention_max_tiles();
+
+}  // namespace csa

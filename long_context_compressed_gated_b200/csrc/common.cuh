@@ -1,0 +1,34 @@
+// common.cuh - shared definitions of the CUDA kernels of libcsa (device side).
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+// Device status word: first 4 bytes of every workspace. The first error wins.
+__device__ __forceinline__ void report(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Compressed entries visible to absolute position t: block j (tokens j*m..j*m+m-1)
+// is visible iff j*m + m - 1 <= t.
+__host__ __device__ __forceinline__ int64_t n_visible(int64_t t, int m) { return t < 0 ? 0 : (t + 1) / m; }
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Two floats -> packed bf16x2 (round to nearest even), low half = a.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Workspace header: status word + padding to 256 bytes.
+constexpr size_t kWorkspaceHeader = 256;
+
+}  // namespace csa

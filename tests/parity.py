@@ -1,0 +1,62 @@
+"""Comparison helpers shared by the GPU parity tests (no method arithmetic here)."""
+import numpy as np
+import torch
+
+import oracle
+
+# Attention tolerance of the specification: max-abs 1e-2, relative Frobenius 5e-3.
+ATTN_MAX_ABS = 1e-2
+ATTN_REL_FRO = 5e-3
+
+
+def bf16_to_f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def words(t):
+    """torch bf16 tensor -> numpy uint16 storage words."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def from_words(w, device):
+    return torch.from_numpy(np.ascontiguousarray(w).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def assert_within_bf16_ulp(got_bf16, exact_f64, what):
+    """|got - exact| <= 1 ulp of bf16 at |exact| (the GPU rounds an fp32 result to
+    nearest-even bf16; the exact value is the oracle's fp64 result)."""
+    got = bf16_to_f64(got_bf16)
+    ex = np.asarray(exact_f64, np.float64)
+    mag = np.maximum(np.abs(ex), 2.0 ** -126)
+    ulp = 2.0 ** (np.floor(np.log2(mag)) - 7)
+    err = np.abs(got - ex)
+    bad = err > ulp
+    assert not bad.any(), "%s: %d of %d elements off by more than 1 bf16 ulp (max err/ulp %.3f)" % (
+        what, int(bad.sum()), bad.size, float((err / ulp).max()))
+
+
+def assert_attention_close(got_bf16, want_f64, what):
+    got = bf16_to_f64(got_bf16)
+    want = np.asarray(want_f64, np.float64)
+    diff = got - want
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    fro = float(np.linalg.norm(diff) / max(np.linalg.norm(want), 1e-30)) if diff.size else 0.0
+    assert max_abs <= ATTN_MAX_ABS and fro <= ATTN_REL_FRO, "%s: max-abs %.3e (<= %.0e), rel-Frobenius %.3e (<= %.0e)" % (
+        what, max_abs, ATTN_MAX_ABS, fro, ATTN_REL_FRO)
+    return max_abs, fro
+
+
+def assert_topk_exact(idx_gpu, scores_gpu, idx_want, top_want, what):
+    ig = idx_gpu.cpu().numpy()
+    np.testing.assert_array_equal(ig, idx_want, err_msg=what + ": top-k indices differ")
+    if scores_gpu is not None:
+        sg = scores_gpu.cpu().numpy()
+        sw = np.asarray(top_want, np.float64).astype(np.float32)  # round-to-nearest of the exact score
+        np.testing.assert_array_equal(sg, sw, err_msg=what + ": top-k scores differ")
+
+
+def sample_rows(T, n, special, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(int(r) for r in special if 0 <= r < T)
+    rows.update(int(r) for r in rng.choice(T, size=min(n, T), replace=False))
+    return np.array(sorted(rows), dtype=np.int64)
