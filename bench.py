@@ -1,0 +1,447 @@
+"""Benchmark of the CSA/HCA hot path on B200 (one JSON line on rank 0).
+
+Step = one pass of the whole CSA prefill path (gated compression m=4, MXFP4
+indexer + causal top-k, sparse + window attention) over one sequence of the
+T=32768, 64x128 workload, inputs resident in HBM.  The HCA prefill
+(T=131072, m'=128) and the 1M-context CSA decode (B=16) are measured the same
+way and reported under "workloads".  With --gpus N each rank runs its own
+sequence (independent problems, no collective): weak scaling.
+
+--impl reference times the CPU oracle (the only reference this method has) on
+a bounded sample of the same workload.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_compressed_gated_b200 import inputs  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+METRIC = "CSA/HCA prefill tokens/s & TFLOP/s; 1M-ctx decode GB/s; % of B200 roofline"
+FP4_OVER_BF16 = 4.0  # nominal dense ratio (9 vs 2.25 PFLOP/s)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------- algorithmic work
+def csa_prefill_work(wl):
+    t = np.arange(wl.T, dtype=np.int64)
+    nv = (t + 1) // wl.m
+    pairs = int(nv.sum())
+    visits = int((np.minimum(nv, wl.k) + np.minimum(t + 1, wl.W)).sum())
+    return {
+        "indexer_flop": 2.0 * pairs * wl.HI * wl.dI,
+        "attn_flop": 4.0 * visits * wl.H * wl.d,
+        "compress_bytes": 3 * wl.T * wl.d * 2 + 2 * (wl.T // wl.m) * wl.d * 2 + wl.m * wl.d * 4,
+        "pairs": pairs, "visits": visits,
+    }
+
+
+def hca_prefill_work(wl):
+    t = np.arange(wl.T, dtype=np.int64)
+    nv = (t + 1) // wl.m_hca
+    visits = int((nv + np.minimum(t + 1, wl.W_hca)).sum())
+    return {"attn_flop": 4.0 * visits * wl.H * wl.d,
+            "compress_bytes": 3 * wl.T * wl.d * 2 + 2 * (wl.T // wl.m_hca) * wl.d * 2 + wl.m_hca * wl.d * 4,
+            "visits": visits}
+
+
+def decode_bytes(wl, B=None):
+    B = wl.batch if B is None else B
+    n = wl.context // wl.m
+    per = (n * (wl.dI // 2 + wl.dI // 32)            # every visible indexer key: codes + scales
+           + wl.k * wl.d * 2 * 2                      # gathered compressed K and V rows
+           + wl.W * wl.d * 2 * 2                      # raw window K and V
+           + wl.H * wl.d * 2 + wl.HI * (wl.dI // 2 + wl.dI // 32) + wl.HI  # q, qI, w
+           + wl.H * wl.d * 2 + wl.k * 4)              # O, idx
+    return per * B
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[5 + i].lower() == "active"})
+        under = [v for v in sm if v > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(under) if under else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- timing helpers
+class Timer:
+    """CUDA events on the current stream around each named phase of a step."""
+
+    def __init__(self, names):
+        self.names = names
+        self.events = []
+
+    def step(self):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.names) + 1)]
+        self.events.append(ev)
+        return ev
+
+    def per_phase_ms(self):
+        out = {n: 0.0 for n in self.names}
+        for ev in self.events:
+            for i, n in enumerate(self.names):
+                out[n] += ev[i].elapsed_time(ev[i + 1])
+        k = max(1, len(self.events))
+        return {n: v / k for n, v in out.items()}
+
+
+def barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, dist_on):
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- workloads (ours)
+def run_csa_prefill(csa, wl, steps, warmup, dist_on, rank):
+    d = inputs.prefill_layer(wl, device="cuda", seed=wl.seed + 1000 * rank)
+    scale = 1.0 / math.sqrt(wl.d)
+    T, H = wl.T, wl.H
+    Kc = torch.empty(T // wl.m, wl.d, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    idx = torch.empty(T, wl.k, dtype=torch.int32, device="cuda")
+    O = torch.empty_like(d["Q"])
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    timer = Timer(["compress", "indexer_topk", "sparse_attn"])
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        csa.csa_compress(d["K"], d["V"], d["Z"], d["B"], wl.m, Kc=Kc, Vc=Vc)
+        if ev: ev[1].record()
+        csa.csa_indexer_topk(d["qI_codes"], d["qI_scales"], d["w_codes"], d["kI_codes"], d["kI_scales"], wl.m,
+                             wl.k, idx=idx, want_scores=False, workspace=ws)
+        if ev: ev[2].record()
+        csa.csa_sparse_attn(d["Q"], Kc, Vc, idx, d["K"], d["V"], wl.W, scale, O=O, want_lse=False, workspace=ws)
+        if ev: ev[3].record()
+
+    for _ in range(warmup):
+        step()
+    barrier(dist_on)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step(timer.step())
+    t1.record()
+    barrier(dist_on)
+    ms = t0.elapsed_time(t1) / steps
+    status = csa.csa_check_status(ws)
+    phases = timer.per_phase_ms()
+    # e2e through the public API with host buffers: H2D of the step's inputs, D2H of O
+    host = {k: v.cpu().pin_memory() for k, v in d.items() if k != "B_hca"}
+    O_host = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = O.numel() * O.element_size()
+    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+
+    def e2e_step():
+        for k, v in host.items():
+            dev[k].copy_(v, non_blocking=True)
+        csa.csa_compress(dev["K"], dev["V"], dev["Z"], dev["B"], wl.m, Kc=Kc, Vc=Vc)
+        csa.csa_indexer_topk(dev["qI_codes"], dev["qI_scales"], dev["w_codes"], dev["kI_codes"], dev["kI_scales"],
+                             wl.m, wl.k, idx=idx, want_scores=False, workspace=ws)
+        csa.csa_sparse_attn(dev["Q"], Kc, Vc, idx, dev["K"], dev["V"], wl.W, scale, O=O, want_lse=False,
+                            workspace=ws)
+        O_host.copy_(O, non_blocking=True)
+
+    e2e_step()
+    barrier(dist_on)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(steps, 3))
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    barrier(dist_on)
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    del dev, host
+    return {"ms": ms, "phases": phases, "status": status, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+            "launches_per_step": 3}
+
+
+def run_hca_prefill(csa, wl, steps, warmup):
+    d = inputs.prefill_layer(wl, device="cuda", with_indexer=False)
+    scale = 1.0 / math.sqrt(wl.d)
+    Kc = torch.empty(wl.T // wl.m_hca, wl.d, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    O = torch.empty_like(d["Q"])
+    ws = torch.zeros(1 << 12, dtype=torch.uint8, device="cuda")
+    timer = Timer(["compress", "hca_attn"])
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        csa.csa_compress(d["K"], d["V"], d["Z"], d["B_hca"], wl.m_hca, Kc=Kc, Vc=Vc)
+        if ev: ev[1].record()
+        csa.hca_attn(d["Q"], Kc, Vc, d["K"], d["V"], wl.m_hca, wl.W_hca, scale, O=O, want_lse=False, workspace=ws)
+        if ev: ev[2].record()
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step(timer.step())
+    t1.record()
+    torch.cuda.synchronize()
+    return {"ms": t0.elapsed_time(t1) / steps, "phases": timer.per_phase_ms(), "status": csa.csa_check_status(ws)}
+
+
+def run_decode(csa, wl, steps, warmup):
+    d = inputs.decode_batch(wl, device="cuda")
+    scale = 1.0 / math.sqrt(wl.d)
+    pos = [wl.context - 1] * wl.batch
+    O = torch.empty_like(d["q"])
+    idx = torch.empty(wl.batch, wl.k, dtype=torch.int32, device="cuda")
+    ws = None
+
+    def step():
+        nonlocal ws
+        _, _, _, _, ws = csa.csa_decode(d["q"], d["qI_codes"], d["qI_scales"], d["w_codes"], d["Kc"], d["Vc"],
+                                        d["kI_codes"], d["kI_scales"], d["Kwin"], d["Vwin"], pos, wl.m, wl.k, scale,
+                                        O=O, idx=idx, want_lse=False, want_sel=True, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    # L2 is smaller than the streamed indexer keys (285 MB), so back-to-back steps read HBM.
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    return {"ms": t0.elapsed_time(t1) / steps, "status": csa.csa_check_status(ws)}
+
+
+# ----------------------------------------------------------------- CPU oracle (reference arm / baseline)
+def oracle_sample(wl, seconds=12.0, max_rows=4096):
+    """Time the CPU oracle on a bounded sample of the CSA prefill workload: the
+    compression of every block, then indexer + top-k + attention for sampled
+    query rows, until about `seconds` have passed. Returns tokens/s and details."""
+    import oracle
+    d = inputs.prefill_layer(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    nthreads = oracle.default_threads()
+    t_start = time.perf_counter()
+    Kc64, Vc64 = oracle.compress(d["K"], d["V"], d["Z"], d["B"], wl.m, nthreads)
+    Kcw, Vcw = oracle.to_bf16_words(Kc64), oracle.to_bf16_words(Vc64)
+    t_comp = time.perf_counter() - t_start
+    rng = np.random.default_rng(0)
+    order = rng.permutation(wl.T)
+    done, t_rows, batch = 0, 0.0, max(8, nthreads)
+    while t_rows < seconds and done < max_rows:
+        rows = np.sort(order[done:done + batch])
+        t1 = time.perf_counter()
+        I = oracle.indexer(d["qI_codes"], d["qI_scales"], d["w_codes"], d["kI_codes"], d["kI_scales"], 0, wl.m,
+                           rows, nthreads)
+        sel, _ = oracle.topk(I, oracle.n_vis(rows, wl.m), wl.k, nthreads)
+        oracle.attention(d["Q"], Kcw, Vcw, d["K"], d["V"], 0, wl.m, wl.W, scale, sel=sel, rows=rows,
+                         nthreads=nthreads)
+        t_rows += time.perf_counter() - t1
+        done += len(rows)
+    per_row = t_rows / done
+    total_s = t_comp + per_row * wl.T  # extrapolated full step
+    return {"tokens_per_s": wl.T / total_s, "rows": done, "seconds": t_comp + t_rows, "cores": nthreads,
+            "sample": "compression of all %d blocks + indexer/top-k/attention of %d uniformly sampled query rows "
+                      "of %d (%.1f s of CPU time); full step extrapolated as compress + T * per-row"
+                      % (wl.T // wl.m, done, wl.T, t_comp + t_rows)}
+
+
+# ----------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the HCA and decode workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = inputs.CSA_PREFILL
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        r = oracle_sample(wl, seconds=max(5.0, 4.0 * args.steps / max(1, args.steps)))
+        v = r["tokens_per_s"]
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.T / v,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "d": wl.d, "m": wl.m,
+                                                 "k": wl.k, "W": wl.W, "HI": wl.HI, "dI": wl.dI},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+                                 "sample": r["sample"]},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    import long_context_compressed_gated_b200 as csa
+    csa.lib()
+    peaks = load_peaks()
+    work = csa_prefill_work(wl)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    res = run_csa_prefill(csa, wl, args.steps, args.warmup, dist_on, rank)
+    sampler.stop()
+    ms = max_over_ranks(res["ms"], dist_on)
+    e2e_ms = max_over_ranks(res["e2e_ms"], dist_on)
+
+    extra = {}
+    if not args.no_extra and rank == 0:
+        w2 = inputs.HCA_PREFILL
+        r2 = run_hca_prefill(csa, w2, max(3, args.steps // 2), args.warmup)
+        hw = hca_prefill_work(w2)
+        extra["hca_prefill_T131072"] = {
+            "tokens_per_s": w2.T / (r2["ms"] * 1e-3), "ms_per_step": r2["ms"],
+            "attn_tflops": hw["attn_flop"] / (r2["phases"]["hca_attn"] * 1e-3) / 1e12,
+            "attn_frac_bf16": hw["attn_flop"] / (r2["phases"]["hca_attn"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "compress_gbs": hw["compress_bytes"] / (r2["phases"]["compress"] * 1e-3) / 1e9,
+            "phases_ms": r2["phases"], "status": r2["status"]}
+        torch.cuda.empty_cache()
+        w3 = inputs.CSA_DECODE
+        r3 = run_decode(csa, w3, max(5, args.steps), args.warmup)
+        by = decode_bytes(w3)
+        extra["csa_decode_B16_L1M"] = {
+            "us_per_step": r3["ms"] * 1e3, "algorithmic_bytes": by, "gbs": by / (r3["ms"] * 1e-3) / 1e9,
+            "frac_hbm": by / (r3["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], "status": r3["status"]}
+        torch.cuda.empty_cache()
+
+    ph = res["phases"]
+    dominant = max(ph, key=ph.get)
+    idx_tf = work["indexer_flop"] / (ph["indexer_topk"] * 1e-3) / 1e12
+    attn_tf = work["attn_flop"] / (ph["sparse_attn"] * 1e-3) / 1e12
+    comp_gbs = work["compress_bytes"] / (ph["compress"] * 1e-3) / 1e9
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    if dominant == "indexer_topk":
+        roof = {"kernel": "indexer_topk", "bound": "tensor", "achieved": idx_tf, "peak": fp4_peak,
+                "unit": "TFLOP/s", "frac": idx_tf / fp4_peak, "traffic": None,
+                "peak_note": "FP4 peak = measured bf16 burst x 4 (nominal dense ratio)"}
+    elif dominant == "sparse_attn":
+        roof = {"kernel": "sparse_attn", "bound": "tensor", "achieved": attn_tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_tflops"], "traffic": None,
+                "peak_note": "bf16 burst, %s" % peaks["source"]}
+    else:
+        roof = {"kernel": "compress", "bound": "hbm", "achieved": comp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": comp_gbs / peaks["hbm_gbs"], "traffic": None}
+    total_tokens = wl.T * world
+    value = total_tokens / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16+mxfp4", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "d": wl.d, "m": wl.m, "k": wl.k, "W": wl.W,
+                   "HI": wl.HI, "dI": wl.dI, "sequences_per_gpu": 1, "parallelism": "independent sequences per GPU",
+                   "l2": "inputs larger than L2 (Q alone 512 MiB), no flush"},
+        "roofline": roof,
+        "kernels": {"compress_ms": ph["compress"], "compress_gbs": comp_gbs,
+                    "indexer_topk_ms": ph["indexer_topk"], "indexer_tflops": idx_tf,
+                    "indexer_frac_fp4": idx_tf / fp4_peak,
+                    "sparse_attn_ms": ph["sparse_attn"], "sparse_attn_tflops": attn_tf,
+                    "sparse_attn_frac_bf16": attn_tf / peaks["bf16_tflops"]},
+        "e2e": {"value": total_tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches_per_step"] * args.steps,
+        "clocks": sampler.summary(),
+        "device_status": res["status"],
+        "peaks": peaks,
+        "workloads": extra,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_sample(wl, seconds=12.0)
+        line["cpu_baseline"] = {"value": r["tokens_per_s"], "unit": "tokens/s", "cores": r["cores"],
+                                "kind": "oracle", "sample": r["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     int64_t nvis = n_visible(t, a.m);
     if (nvis > a.Nc) nvis = a.Nc;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f, l_run32 = 0.f;
     const uint32_t prow = smem_u32(s_p) + (uint32_t)row * 128;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
@@ -324,13 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       // pass 1: tile maximum over this row's visible range (log2 units of the scaled logits)
       float mt = -INFINITY;
 #pragma unroll
-      for (int c0 = 0; c0 < kTileKeys; c0 += 32) {
+      for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
         if (c0 < tl.width) {  // warp-uniform
-          uint32_t v[32];
-          tmem_ld32(scol + c0, v);
+          uint32_t v[64];
+          tmem_ld32p(scol + c0, v);
+          if (c0 + 32 < tl.width) tmem_ld32p(scol + c0 + 32, v + 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
+          for (int e = 0; e < 64; ++e)
             if (c0 + e >= lo && c0 + e < hi) mt = fmaxf(mt, __uint_as_float(v[e]) * a.scale_log2);
         }
       }
@@ -339,25 +340,30 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const float alpha = raise ? exp2f(m_run - m_new) : 1.0f;  // exp2(-inf) = 0 on the first raise
       // pass 2: probabilities, packed to bf16 pairs
       uint32_t pk[kTileKeys / 2];
-      float lsum = 0.f;
+      float lsum = 0.f, lsum32 = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < kTileKeys; c0 += 32) {
+      for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
         if (c0 < tl.width) {
-          uint32_t v[32];
-          tmem_ld32(scol + c0, v);
+          uint32_t v[64];
+          tmem_ld32p(scol + c0, v);
+          if (c0 + 32 < tl.width) tmem_ld32p(scol + c0 + 32, v + 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = 0; e < 64; e += 2) {
             const int x = c0 + e;
             float p0 = 0.f, p1 = 0.f;
             if (x >= lo && x < hi) p0 = exp2f(__uint_as_float(v[e]) * a.scale_log2 - m_new);
             if (x + 1 >= lo && x + 1 < hi) p1 = exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - m_new);
-            lsum += p0 + p1;
-            pk[x / 2] = pack_bf16x2(p0, p1);
+            const uint32_t pp = pack_bf16x2(p0, p1);
+            // O is normalised by the same bf16-rounded weights the PV MMA consumes;
+            // the log-sum-exp output uses the fp32 weights
+            lsum += bf16_lo(pp) + bf16_hi(pp);
+            lsum32 += p0 + p1;
+            pk[x / 2] = pp;
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) pk[(c0 + e) / 2] = 0u;
+          for (int e = 0; e < 64; e += 2) pk[(c0 + e) / 2] = 0u;
         }
       }
       tc_fence_before();
@@ -371,25 +377,20 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
         const float sc = (raise && i > 0) ? alpha : 1.0f;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tbase + lane_base + kTmemO + c0, v);
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          uint32_t v[64];
+          tmem_ld32p(tbase + lane_base + kTmemO + c0, v);
+          tmem_ld32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
-          asm volatile(
-              "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-              "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
-                  tbase + lane_base + kTmemO + c0),
-              "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-              "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-              "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-              "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-              : "memory");
+          for (int e = 0; e < 64; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
+          tmem_st32p(tbase + lane_base + kTmemO + c0, v);
+          tmem_st32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
         }
         tmem_wait_st();
       }
       l_run = l_run * alpha + lsum;
+      l_run32 = l_run32 * alpha + lsum32;
       m_run = m_new;
       // store the P row (K-major, 128B swizzle, two 64-key halves)
 #pragma unroll
@@ -415,18 +416,19 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     __nv_bfloat16* orow = nullptr;
     if (t >= 0) orow = a.O + b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t v[32];
+    for (int c0 = 0; c0 < D; c0 += 64) {
+      uint32_t v[64];
       if (ntiles > 0) {
-        tmem_ld32(tbase + lane_base + kTmemO + c0, v);
+        tmem_ld32p(tbase + lane_base + kTmemO + c0, v);
+        tmem_ld32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0u;
+        for (int e = 0; e < 64; ++e) v[e] = 0u;
       }
       if (orow) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
+        for (int e = 0; e < 64; e += 8) {
           uint4 o;
           o.x = pack_bf16x2(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
           o.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
@@ -437,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       }
     }
     if (t >= 0 && a.lse) {
-      const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      const float lse = l_run32 > 0.f ? (m_run + log2f(l_run32)) * 0.69314718055994531f : -INFINITY;
       a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
     }
   }

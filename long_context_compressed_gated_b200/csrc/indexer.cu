@@ -68,6 +68,36 @@ __device__ __forceinline__ int e2m1_times2(uint32_t code) {
 
 }  // namespace
 
+// Head sums of this thread's key lane for the tokens of one half of the group:
+// acc[g] += w2[h] * max(bits(D[g*HI+h]), bits(196608)) over the half's columns,
+// loading up to 64 TMEM columns per wait.
+template <int HI, int G, int HALF>
+__device__ __forceinline__ void head_sums(uint32_t dcol, const int* s_w2, uint32_t (&acc)[G]) {
+  constexpr int G0 = (G + 1) / 2;
+  constexpr int c_lo = (HALF ? G0 : 0) * HI;
+  constexpr int c_hi = (HALF ? G : G0) * HI;
+#pragma unroll
+  for (int b0 = c_lo; b0 < c_hi; b0 += 64) {
+    uint32_t v[64];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (b0 + 16 * q < c_hi) tmem_ld16p(dcol + b0 + 16 * q, v + 16 * q);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 64; i += 4) {
+      if (b0 + i < c_hi) {
+        const int4 w = *reinterpret_cast<const int4*>(s_w2 + b0 + i);
+        const int ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int col = b0 + i + q;
+          acc[col / HI] += (uint32_t)ww[q] * (uint32_t)max((int)v[i + q], (int)kMagicBits);
+        }
+      }
+    }
+  }
+}
+
 struct IndexerArgs {
   const uint8_t* q_scales;  // [rows, HI, dI/32]
   const uint8_t* w_codes;   // [rows, HI]
@@ -97,7 +127,8 @@ struct IndexerSmem {
   static constexpr size_t off_q = 0;
   static constexpr size_t off_a = off_q + kQBytes;
   static constexpr size_t off_sf = off_a + (size_t)kStages * kABytes;
-  static constexpr size_t off_ma = off_sf + (size_t)kStages * 512;
+  static constexpr size_t off_sfraw = off_sf + (size_t)kStages * 512;  // scales as loaded, [128 rows][DI/32]
+  static constexpr size_t off_ma = off_sfraw + (size_t)kStages * 512;
   static constexpr size_t off_mb = off_ma + 4096;
   static constexpr size_t off_w2 = off_mb + (size_t)N * 32;
   static constexpr size_t off_sumw = off_w2 + (size_t)N * 4;
@@ -125,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* s_q = smem + L::off_q;
   uint8_t* s_a = smem + L::off_a;
   uint8_t* s_sf = smem + L::off_sf;
+  uint8_t* s_sfraw = smem + L::off_sfraw;
   uint8_t* s_ma = smem + L::off_ma;
   uint8_t* s_mb = smem + L::off_mb;
   int* s_w2 = reinterpret_cast<int*>(smem + L::off_w2);
@@ -225,36 +257,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (it / NST) & 1;
       if (!mbar_wait(&empty[s], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       const int64_t j0 = j_begin + (int64_t)it * 128;
+      const int64_t row0k = key_row_base + j0;
+      constexpr uint32_t kSfRow = DI / 32;  // scale bytes per key row
+      // whole tile inside the kI tensor: scales by one bulk copy; else plain loads
+      const bool bulk = row0k + 128 <= a.key_rows;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], L::kABytes);
-        tma_load_2d(s_a + (size_t)s * L::kABytes, &kmap, &full[s], 0, (int)(key_row_base + j0));
+        mbar_arrive_expect_tx(&full[s], L::kABytes + (bulk ? 128 * kSfRow : 0u));
+        tma_load_2d(s_a + (size_t)s * L::kABytes, &kmap, &full[s], 0, (int)row0k);
+        if (bulk) bulk_load(s_sfraw + (size_t)s * 512, a.k_scales + row0k * kSfRow, 128 * kSfRow, &full[s]);
       }
-      // scale factors: lane l stages rows l, l+32, l+64, l+96 (tcgen05.cp 32x128b layout)
-      uint32_t wv[4];
-      bool bad = false;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int64_t j = j0 + lane + 32 * c;
-        const int64_t row = key_row_base + j;
-        uint32_t w = 0x7F7F7F7Fu;
-        if (j < j_end && row < a.key_rows) {
+      if (!bulk) {
+        for (int r = lane; r < 128; r += 32) {
+          const int64_t row = row0k + r;
           if (DI == 128) {
-            w = *reinterpret_cast<const uint32_t*>(a.k_scales + row * 4);
+            const uint32_t w = row < a.key_rows ? *reinterpret_cast<const uint32_t*>(a.k_scales + row * 4)
+                                                 : 0x7F7F7F7Fu;
+            reinterpret_cast<uint32_t*>(s_sfraw + (size_t)s * 512)[r] = w;
           } else {
-            w = (uint32_t)*reinterpret_cast<const uint16_t*>(a.k_scales + row * 2) | 0x7F7F0000u;
-          }
-#pragma unroll
-          for (int b = 0; b < DI / 32; ++b) {
-            const uint32_t e = (w >> (8 * b)) & 255u;
-            bad |= (e < 125u) | (e > 128u);
+            const uint16_t w = row < a.key_rows ? *reinterpret_cast<const uint16_t*>(a.k_scales + row * 2)
+                                                : (uint16_t)0x7F7F;
+            reinterpret_cast<uint16_t*>(s_sfraw + (size_t)s * 512)[r] = w;
           }
         }
-        wv[c] = w;
+        __syncwarp();
       }
-      if (bad) report(a.status, CSA_ERR_RANGE);
-      *reinterpret_cast<uint4*>(s_sf + (size_t)s * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-      fence_proxy_async_smem();
-      __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
     }
   } else if (warp == 1) {
@@ -273,6 +299,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dph = (it >> 1) & 1;
       if (!mbar_wait(&dempty[b], dph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       if (!mbar_wait(&full[s], ph, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
+      {
+        // scales -> tcgen05.cp 32x128b layout: lane l holds rows l, l+32, l+64, l+96
+        const int64_t j0 = j_begin + (int64_t)it * 128;
+        uint32_t wv[4];
+        bool bad = false;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int r = lane + 32 * c;
+          uint32_t w;
+          if (DI == 128) w = reinterpret_cast<const uint32_t*>(s_sfraw + (size_t)s * 512)[r];
+          else w = (uint32_t)reinterpret_cast<const uint16_t*>(s_sfraw + (size_t)s * 512)[r] | 0x7F7F0000u;
+          if (j0 + r < j_end) {
+#pragma unroll
+            for (int q = 0; q < DI / 32; ++q) {
+              const uint32_t e = (w >> (8 * q)) & 255u;
+              bad |= (e < 125u) | (e > 128u);
+            }
+          }
+          wv[c] = w;
+        }
+        if (bad) report(a.status, CSA_ERR_RANGE);
+        *reinterpret_cast<uint4*>(s_sf + (size_t)s * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t d = tbase + (b ? kTmemD1 : 0u);
@@ -350,29 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc[G];  // arithmetic mod 2^32: the true head sum fits in int32
 #pragma unroll
       for (int g = 0; g < G; ++g) acc[g] = 0u;
-      // columns of this half: [g_lo*HI, g_hi*HI) in chunks of 16
-#pragma unroll
-      for (int c0 = 0; c0 < G * HI; c0 += 16) {
-        const int gc = c0 / HI;  // token of the chunk's first column
-        const bool mine = half == 0 ? (gc < G0) : (gc >= G0);
-        if (!mine) continue;
-        uint32_t v[16];
-        tmem_ld16(dcol + c0, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-          const int4 w = *reinterpret_cast<const int4*>(s_w2 + c0 + i);
-          const int ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = c0 + i + q;
-            if (col < G * HI) {
-              const int g = col / HI;
-              acc[g] += (uint32_t)ww[q] * (uint32_t)max((int)v[i + q], (int)kMagicBits);
-            }
-          }
-        }
-      }
+      if (half == 0) head_sums<HI, G, 0>(dcol, s_w2, acc);
+      else head_sums<HI, G, 1>(dcol, s_w2, acc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dempty[b]);
@@ -578,17 +608,6 @@ int indexer_tokens_per_cta(int HI) {
   }
 }
 
-size_t indexer_smem_bytes(int HI, int DI, int G, int cap) {
-  // mirrors IndexerSmem<>::bytes for the instantiated shapes
-  const int N = ((G * HI + 15) / 16) * 16;
-  const int stages = G == 1 ? 8 : 4;
-  const int rowb = DI / 2;
-  size_t off = (size_t)((N * rowb + 1023) / 1024) * 1024;
-  off += (size_t)stages * 128 * rowb + (size_t)stages * 512 + 4096 + (size_t)N * 32 + (size_t)N * 4 + 256 + 256 +
-         512 + 1024 + 64 + (2 * stages + 5) * 8;
-  off = ((off + 16 + 15) / 16) * 16;
-  return off + (size_t)G * cap * 8 + 1024;
-}
 
 // Prefill: rows = T, one range per group (direct output).
 cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,

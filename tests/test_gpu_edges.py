@@ -1,0 +1,212 @@
+"""GPU parity on edge cases: ragged sizes, chunk offsets (t0 > 0, a cache that
+holds only the entries visible so far), an empty cache, no window, fewer
+visible entries than k, decode at short contexts, the MXFP4 exact-range check,
+and the indexer shapes of the decode/stack workloads (16 heads x 128).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_compressed_gated_b200 import inputs
+from tests.parity import assert_attention_close, assert_topk_exact, from_words
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csa():
+    import long_context_compressed_gated_b200 as m
+    m.lib()
+    return m
+
+
+def _indexer_case(csa, T, Nc, HI, dI, m, k, t0, seed):
+    wl = inputs.Workload("edge", T=T, HI=HI, dI=dI, m=m, k=k, seed=seed)
+    qc, qs = inputs.mxfp4((T, HI), dI, seed, "qI")
+    w = inputs.uniform_u8((T, HI), seed, "w", 0, 15)
+    kc, ks = inputs.mxfp4((Nc,), dI, seed, "kI")
+    idx, sc, ws = csa.csa_indexer_topk(qc.cuda(), qs.cuda(), w.cuda(), kc.cuda(), ks.cuda(), m, k, t0=t0)
+    assert csa.csa_check_status(ws) == 0
+    I = oracle.indexer(qc, qs, w, kc, ks, t0, m)
+    rows = np.arange(T)
+    want_idx, want_top = oracle.topk(I, np.minimum(oracle.n_vis(t0 + rows, m), Nc), k)
+    assert_topk_exact(idx, sc, want_idx, want_top, "indexer T=%d Nc=%d HI=%d dI=%d k=%d t0=%d" % (T, Nc, HI, dI, k, t0))
+
+
+@pytest.mark.parametrize("T,Nc,HI,dI,m,k,t0", [
+    (1000, 250, 4, 64, 4, 16, 0),        # ragged T (not a multiple of the token group)
+    (777, 194, 16, 128, 4, 64, 0),       # decode/stack indexer shape, ragged
+    (300, 900, 64, 128, 4, 512, 3300),   # chunk at t0 > 0 against an accumulated cache
+    (256, 1000, 16, 128, 4, 1024, 2000), # k > visible entries for every row
+    (129, 40, 8, 64, 3, 7, 0),           # odd m and k
+    (64, 0, 16, 128, 4, 32, 0),          # empty cache: every idx is -1
+    (200, 3000, 32, 128, 4, 2048, 9000), # k = 2048 (largest), 32 heads
+])
+def test_indexer_edges(csa, T, Nc, HI, dI, m, k, t0):
+    _indexer_case(csa, T, Nc, HI, dI, m, k, t0, seed=T + Nc)
+
+
+def test_indexer_many_ties(csa):
+    """Exact integer scores make ties common (w = 0 and ReLU zeros): ties must go
+    to the smaller block index."""
+    T, Nc, HI, dI, m, k = 96, 400, 16, 128, 4, 64
+    qc, qs = inputs.mxfp4((T, HI), dI, 5, "qI")
+    w = inputs.uniform_u8((T, HI), 5, "w", 0, 15)
+    w[:, 4:] = 0                               # only 4 heads count
+    qs[:] = 127
+    kc, ks = inputs.mxfp4((Nc,), dI, 5, "kI")
+    kc[::3] = 0                                # every third key scores exactly 0
+    ks[:] = 127
+    kc[1::7] = kc[0]                           # duplicated keys -> equal scores
+    idx, sc, ws = csa.csa_indexer_topk(qc.cuda(), qs.cuda(), w.cuda(), kc.cuda(), ks.cuda(), m, k)
+    assert csa.csa_check_status(ws) == 0
+    I = oracle.indexer(qc, qs, w, kc, ks, 0, m)
+    want_idx, want_top = oracle.topk(I, np.minimum(oracle.n_vis(np.arange(T), m), Nc), k)
+    assert_topk_exact(idx, sc, want_idx, want_top, "indexer ties")
+
+
+def test_indexer_extreme_magnitudes(csa):
+    """All |codes| = 6 with scale 2^1 against mixed 2^-2 / 2^1 blocks: the largest
+    head sums the exact range allows."""
+    T, Nc, HI, dI, m, k = 32, 64, 64, 128, 1, 16
+    qc = torch.full((T, HI, dI // 2), 0x77, dtype=torch.uint8)
+    qc[::2] = 0xFF                                 # -6 on every other token
+    qs = torch.full((T, HI, dI // 32), 128, dtype=torch.uint8)
+    w = torch.full((T, HI), 7, dtype=torch.uint8)  # w = 6
+    kc = torch.full((Nc, dI // 2), 0x77, dtype=torch.uint8)
+    ks = inputs.uniform_u8((Nc, dI // 32), 9, "ks", 125, 128)
+    kc[5::4] = 0x7F                                # mixed signs inside a row
+    idx, sc, ws = csa.csa_indexer_topk(qc.cuda(), qs.cuda(), w.cuda(), kc.cuda(), ks.cuda(), m, k)
+    assert csa.csa_check_status(ws) == 0
+    I = oracle.indexer(qc, qs, w, kc, ks, 0, m)
+    want_idx, want_top = oracle.topk(I, np.minimum(oracle.n_vis(np.arange(T), m), Nc), k)
+    assert_topk_exact(idx, sc, want_idx, want_top, "indexer extreme magnitudes")
+
+
+def test_indexer_reports_scale_out_of_range(csa):
+    T, Nc, HI, dI = 8, 64, 16, 128
+    qc, qs = inputs.mxfp4((T, HI), dI, 1, "qI")
+    w = inputs.uniform_u8((T, HI), 1, "w", 0, 15)
+    kc, ks = inputs.mxfp4((Nc,), dI, 1, "kI")
+    ks[3, 1] = 124                                  # 2^-3: outside the exact range
+    _, _, ws = csa.csa_indexer_topk(qc.cuda(), qs.cuda(), w.cuda(), kc.cuda(), ks.cuda(), 1, 8)
+    assert csa.csa_check_status(ws) == -7           # CSA_ERR_RANGE
+    assert csa.csa_check_status(ws) == 0            # cleared by the read
+
+
+def _attn_inputs(T, H, d, Nc, seed):
+    g = torch.Generator().manual_seed(seed)
+    f = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    return f(T, H, d), f(Nc, d), f(Nc, d)
+
+
+def _raw_kv(n, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(n, d, generator=g).to(torch.bfloat16), torch.randn(n, d, generator=g).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("T,t0,H,d,m,k,W", [
+    (300, 0, 64, 128, 4, 512, 128),     # ragged T, early rows see < k entries
+    (200, 5000, 16, 64, 4, 64, 100),    # chunk offset, odd window
+    (130, 40, 128, 128, 4, 16, 0),      # no window, one token per CTA (H=128)
+    (97, 0, 8, 64, 5, 9, 33),
+])
+def test_sparse_attention_edges(csa, T, t0, H, d, m, k, W):
+    Nc = (t0 + T) // m
+    Q, Kc, Vc = _attn_inputs(T, H, d, Nc, seed=T + t0)
+    Kraw, Vraw = _raw_kv(t0 + T, d, seed=7 + T)
+    rng = np.random.default_rng(T)
+    sel = np.full((T, k), -1, np.int32)
+    for r in range(T):
+        nv = min((t0 + r + 1) // m, Nc)
+        c = rng.choice(nv, size=min(k, nv), replace=False) if nv else []
+        sel[r, : len(c)] = c
+    scale = 1.0 / math.sqrt(d)
+    O, lse, ws = csa.csa_sparse_attn(Q.cuda(), Kc.cuda(), Vc.cuda(), torch.from_numpy(sel).cuda(), Kraw.cuda(),
+                                     Vraw.cuda(), W, scale, t0=t0)
+    assert csa.csa_check_status(ws) == 0
+    O_want, lse_want = oracle.attention(Q, Kc, Vc, Kraw, Vraw, t0, m, W, scale, sel=sel)
+    assert_attention_close(O, O_want, "sparse attention edge %s" % ((T, t0, H, d, m, k, W),))
+    got = lse.cpu().numpy()
+    empty = np.isneginf(lse_want)
+    assert np.all(np.isneginf(got[empty])), "rows with no keys must give lse = -inf"
+    np.testing.assert_allclose(got[~empty], lse_want[~empty], atol=2e-3)
+
+
+@pytest.mark.parametrize("T,t0,H,d,m,W", [
+    (500, 0, 64, 128, 16, 128),
+    (260, 3000, 32, 64, 128, 64),
+    (64, 10, 64, 128, 8, 0),            # no window: the first rows see nothing
+])
+def test_hca_attention_edges(csa, T, t0, H, d, m, W):
+    Nc = (t0 + T) // m
+    Q, Kc, Vc = _attn_inputs(T, H, d, max(Nc, 1), seed=3 * T + t0)
+    Kc, Vc = Kc[:Nc], Vc[:Nc]
+    Kraw, Vraw = _raw_kv(t0 + T, d, seed=11 + T)
+    scale = 1.0 / math.sqrt(d)
+    if Nc == 0:
+        pytest.skip("empty cache")
+    O, lse, ws = csa.hca_attn(Q.cuda(), Kc.cuda(), Vc.cuda(), Kraw.cuda(), Vraw.cuda(), m, W, scale, t0=t0)
+    assert csa.csa_check_status(ws) == 0
+    O_want, lse_want = oracle.attention(Q, Kc, Vc, Kraw, Vraw, t0, m, W, scale)
+    assert_attention_close(O, O_want, "HCA edge %s" % ((T, t0, H, d, m, W),))
+    got = lse.cpu().numpy()
+    empty = np.isneginf(lse_want)
+    assert np.all(np.isneginf(got[empty]))
+    np.testing.assert_allclose(got[~empty], lse_want[~empty], atol=2e-3)
+
+
+def test_decode_short_contexts_all_sequences(csa):
+    """Decode with different positions per sequence, including one whose window
+    reaches before position 0 and one with fewer visible entries than k."""
+    wl = inputs.Workload("dec_small", H=64, d=128, m=4, k=64, W=32, HI=16, dI=128, batch=5, context=4096, seed=21)
+    g = inputs.decode_batch(wl)
+    pos = [4095, 20, 1000, 255, 3]
+    scale = 1.0 / math.sqrt(wl.d)
+    gc = {k: v.cuda() for k, v in g.items()}
+    O, lse, idx, scores, ws = csa.csa_decode(gc["q"], gc["qI_codes"], gc["qI_scales"], gc["w_codes"], gc["Kc"],
+                                             gc["Vc"], gc["kI_codes"], gc["kI_scales"], gc["Kwin"], gc["Vwin"], pos,
+                                             wl.m, wl.k, scale)
+    assert csa.csa_check_status(ws) == 0
+    for b, t in enumerate(pos):
+        I = oracle.indexer(g["qI_codes"][b:b + 1], g["qI_scales"][b:b + 1], g["w_codes"][b:b + 1], g["kI_codes"][b],
+                           g["kI_scales"][b], t, wl.m)
+        want_idx, want_top = oracle.topk(I, oracle.n_vis([t], wl.m), wl.k)
+        assert_topk_exact(idx[b:b + 1], scores[b:b + 1], want_idx, want_top, "decode seq %d" % b)
+        o, l = oracle.attention(g["q"][b:b + 1], g["Kc"][b], g["Vc"][b], g["Kwin"][b], g["Vwin"][b], t, wl.m, wl.W,
+                                scale, sel=want_idx, rows=[0], raw_pos0=t - wl.W + 1)
+        assert_attention_close(O[b:b + 1], o, "decode attention seq %d" % b)
+
+
+def test_hca_decode(csa):
+    wl = inputs.Workload("hdec", H=64, d=128, m=128, W=128, batch=3, context=1 << 20, seed=22)
+    n = wl.context // wl.m
+    gen = torch.Generator().manual_seed(22)
+    f = lambda *s: torch.randn(*s, generator=gen).to(torch.bfloat16)
+    q, Kc, Vc = f(wl.batch, wl.H, wl.d), f(wl.batch, n, wl.d), f(wl.batch, n, wl.d)
+    Kw, Vw = f(wl.batch, wl.W, wl.d), f(wl.batch, wl.W, wl.d)
+    pos = [wl.context - 1, 5000, 127]
+    scale = 1.0 / math.sqrt(wl.d)
+    O, lse, ws = csa.hca_decode(q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), pos, wl.m, scale)
+    assert csa.csa_check_status(ws) == 0
+    for b, t in enumerate(pos):
+        o, l = oracle.attention(q[b:b + 1], Kc[b], Vc[b], Kw[b], Vw[b], t, wl.m, wl.W, scale, rows=[0],
+                                raw_pos0=t - wl.W + 1)
+        assert_attention_close(O[b:b + 1], o, "HCA decode seq %d" % b)
+        np.testing.assert_allclose(lse[b:b + 1].cpu().numpy(), l, atol=2e-3)
+
+
+@pytest.mark.parametrize("T,d,m", [(1000, 128, 4), (1000, 64, 64), (4096, 128, 128), (333, 128, 8), (640, 64, 1)])
+def test_compress_edges(csa, T, d, m):
+    from tests.parity import assert_within_bf16_ulp, fp32_pool_slack
+    g = torch.Generator().manual_seed(T + m)
+    K, V, Z = (torch.randn(T, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    B = torch.randn(m, d, generator=g) * 0.5
+    Kc, Vc = csa.csa_compress(K.cuda(), V.cuda(), Z.cuda(), B.cuda(), m)
+    Kx, Vx = oracle.compress(K, V, Z, B, m)
+    assert Kc.shape[0] == T // m
+    assert_within_bf16_ulp(Kc, Kx, "Kc", fp32_pool_slack(K, m))
+    assert_within_bf16_ulp(Vc, Vx, "Vc", fp32_pool_slack(V, m))

@@ -12,7 +12,8 @@ import torch
 
 import oracle
 from long_context_compressed_gated_b200 import inputs
-from tests.parity import (assert_attention_close, assert_topk_exact, assert_within_bf16_ulp, from_words, words)
+from tests.parity import (assert_attention_close, assert_topk_exact, assert_within_bf16_ulp, fp32_pool_slack,
+                          from_words, words)
 
 pytestmark = pytest.mark.gpu
 
@@ -41,8 +42,8 @@ def test_compress_csa_and_hca(lib, data):
         Kc, Vc = lib.csa_compress(g["K"], g["V"], g["Z"], g[B], m)
         torch.cuda.synchronize()
         Kx, Vx = oracle.compress(data["K"], data["V"], data["Z"], data[B], m)
-        assert_within_bf16_ulp(Kc, Kx, "Kc m=%d" % m)
-        assert_within_bf16_ulp(Vc, Vx, "Vc m=%d" % m)
+        assert_within_bf16_ulp(Kc, Kx, "Kc m=%d" % m, fp32_pool_slack(data["K"], m))
+        assert_within_bf16_ulp(Vc, Vx, "Vc m=%d" % m, fp32_pool_slack(data["V"], m))
 
 
 def test_indexer_topk_exact(lib, data):
