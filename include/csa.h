@@ -120,7 +120,7 @@ int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const ui
  *   O      [T, H, d] bf16 output; lse [T, H] float natural-log sum of exp of
  *          the scaled logits (may be NULL).
  * One joint softmax over the selected entries and the window; scale is the
- * logit multiplier (1/sqrt(d) for the usual reading).  A row with an empty key
+ * logit multiplier (> 0; 1/sqrt(d) for the usual reading).  A row with an empty key
  * set gets O = 0, lse = -inf.  H in {4, 8, 16, 32, 64, 128}, d in {64, 128},
  * 1 <= k <= 2048, 0 <= W <= 1024. */
 size_t csa_sparse_attn_workspace_bytes(int64_t T, int H, int d, int k, int W);

@@ -188,7 +188,7 @@ size_t csa_sparse_attn_workspace_bytes(int64_t, int, int, int, int) { return kWo
 int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t* idx, const void* Kraw,
                     const void* Vraw, int64_t T, int64_t t0, int64_t Nc, int H, int d, int k, int W, float scale,
                     void* O, float* lse, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
-  if (T < 0 || t0 < 0 || Nc < 0 || k < 1 || k > 2048 || W < 0 || W > 1024 || !std::isfinite(scale))
+  if (T < 0 || t0 < 0 || Nc < 0 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f))
     return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   const int gq = 128 / H;
@@ -220,6 +220,9 @@ int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t
   a.O = static_cast<__nv_bfloat16*>(O);
   a.lse = lse;
   a.status = status_word(workspace);
+  a.q_rows = T * H;
+  a.kc_rows = Nc > 0 ? Nc : 1;
+  a.raw_rows = W > 0 ? t0 + T : 1;
   cudaError_t e = launch_attention(a, d, (unsigned)ceil_div(T, gq), (cudaStream_t)stream);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
@@ -229,7 +232,7 @@ size_t hca_attn_workspace_bytes(int64_t, int, int, int) { return kWorkspaceHeade
 int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, const void* Vraw, int64_t T, int64_t t0,
              int64_t Nc, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
              size_t workspace_bytes, csa_stream_t stream) {
-  if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || W < 0 || W > 1024 || !std::isfinite(scale)) return CSA_ERR_INVALID_ARG;
+  if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f)) return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   const int gq = 128 / H;
   int64_t nv = n_visible(t0 + T - 1, m);
@@ -262,6 +265,9 @@ int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, co
   a.O = static_cast<__nv_bfloat16*>(O);
   a.lse = lse;
   a.status = status_word(workspace);
+  a.q_rows = T * H;
+  a.kc_rows = Nc > 0 ? Nc : 1;
+  a.raw_rows = W > 0 ? t0 + T : 1;
   cudaError_t e = launch_attention(a, d, (unsigned)ceil_div(T, gq), (cudaStream_t)stream);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
@@ -278,7 +284,7 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
                const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
                int W, float scale, void* O, float* lse, int32_t* idx, float* scores, void* workspace,
                size_t workspace_bytes, csa_stream_t stream) {
-  if (B < 0 || Ncap < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 || !std::isfinite(scale))
+  if (B < 0 || Ncap < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f))
     return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128) || !valid_HI(HI) || (dI != 64 && dI != 128))
     return CSA_ERR_UNSUPPORTED_SHAPE;
@@ -340,6 +346,9 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
+  a.q_rows = (int64_t)B * H;
+  a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
+  a.raw_rows = W > 0 ? (int64_t)B * W : 1;
   e = launch_attention(a, d, (unsigned)B, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
@@ -351,7 +360,7 @@ size_t hca_decode_workspace_bytes(int B, int64_t, int, int, int) {
 int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
                int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
                size_t workspace_bytes, csa_stream_t stream) {
-  if (B < 0 || Ncap < 0 || m < 1 || W < 0 || W > 1024 || !std::isfinite(scale)) return CSA_ERR_INVALID_ARG;
+  if (B < 0 || Ncap < 0 || m < 1 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f)) return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   int rc = check_ws(workspace, workspace_bytes, hca_decode_workspace_bytes(B, Ncap, H, d, W));
   if (rc) return rc;
@@ -395,6 +404,9 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
+  a.q_rows = (int64_t)B * H;
+  a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
+  a.raw_rows = W > 0 ? (int64_t)B * W : 1;
   e = launch_attention(a, d, (unsigned)B, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }

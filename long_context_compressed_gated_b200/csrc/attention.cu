@@ -21,6 +21,8 @@
 // producer warps with 16-byte cp.async into 128B-swizzled tiles (K and V in
 // separate double-buffered rings, so S of tile i+2 can start while PV of tile i
 // still reads V).
+#include <cuda.h>
+
 #include "attention.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
@@ -34,7 +36,7 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kTileKeys = 128;
 constexpr int kMaxTiles = 80;
-constexpr int kSoftmaxWarps = 4, kProducerWarps = 3;
+constexpr int kSoftmaxWarps = 4, kProducerWarps = 1;
 constexpr int kThreads = (kSoftmaxWarps + kProducerWarps + 1) * 32;  // + 1 MMA warp
 constexpr float kRescaleSlack = 8.0f;  // raise the running max only when it grows by > 2^8
 
@@ -45,18 +47,30 @@ struct Tile {
   int64_t base;                   // SEG: offset in the token's list; HCA: j0; WIN: w0
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// 2^x with the SFU (ex2.approx, ~2 ulp; -inf -> +0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-// Arrive on `bar` once all prior cp.async of this thread have landed (no extra pending count).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+
+
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
 }
 
 }  // namespace
 
-
+// TMA descriptors of one launch: 128-row boxes (two 64-column halves, 128B
+// swizzle) for contiguous rows, and 1-row boxes for 4-row gathers.
+struct alignas(64) AttnMaps {
+  CUtensorMap q, kc, vc, kc_g4, vc_g4, kr, vr;
+};
 
 template <int D>
 struct AttnSmem {
@@ -69,12 +83,14 @@ struct AttnSmem {
   static constexpr size_t off_tiles = off_p + 2 * kHalf;
   static constexpr size_t off_bar = off_tiles + kMaxTiles * sizeof(Tile);
   static constexpr size_t off_misc = off_bar + 16 * 8;
-  static constexpr size_t off_idx = off_misc + 256;
+  static constexpr size_t off_ones = off_misc + 256;        // 16 x 16 bf16 ones (row-sum MMA operand)
+  static constexpr size_t off_idx = off_ones + 512;
   static size_t bytes(int idx_entries) { return off_idx + (size_t)idx_entries * 4 + 1024; }
 };
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a) {
+template <int D, bool WANT_LSE>
+__global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a,
+                                                                const __grid_constant__ AttnMaps maps) {
   using L = AttnSmem<D>;
   constexpr int KSTEPS_QK = D / 16;
   extern __shared__ uint8_t smem_raw[];
@@ -96,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   uint64_t* pv_done = bar + 14;
   int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [0] ntiles, [1] tmem, [2..] seg counts
   int* s_idx = reinterpret_cast<int*>(smem + L::off_idx);
+  uint8_t* s_ones = smem + L::off_ones;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
@@ -121,11 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
 
   // ---- setup: barriers, TMEM, selected-index lists, tile list
   if (tid == 0) {
-    mbar_init(q_full, kProducerWarps * 32);
+    mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], kProducerWarps * 32);
+      mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], kProducerWarps * 32);
+      mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftmaxWarps);
@@ -138,6 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     tmem_alloc(reinterpret_cast<uint32_t*>(&misc[1]), 512);
     tmem_relinquish();
   }
+  if (tid < 32) reinterpret_cast<uint4*>(s_ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async_smem();
   // compact each token's selected list (drop -1 / out-of-range), one warp per token
   if (idx != nullptr) {
     for (int g = warp; g < ntok; g += kThreads / 32) {
@@ -192,35 +211,17 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
 
   if (warp >= kSoftmaxWarps && warp < kSoftmaxWarps + kProducerWarps) {
-    // =========================== producers: Q once, then K/V tiles
-    constexpr int NP = kProducerWarps * 32;
-    const int pt = tid - kSoftmaxWarps * 32;  // 0..NP-1
-    constexpr int CH = D / 8;                  // 16-byte chunks per row
-    constexpr int ROWS_PER_PASS = NP / CH;
-    auto dst_off = [](int row, int c) -> uint32_t {
-      const int half = c >> 3, cc = c & 7;
-      return (uint32_t)(half * (kRows * 128) + row * 128 + ((cc ^ (row & 7)) << 4));
-    };
-    {
-      const uint32_t sq = smem_u32(s_q);
-      const int c = pt % CH;
-      for (int row = pt / CH; row < kRows; row += ROWS_PER_PASS) {
-        const int g = row / H, h = row % H;
-        const bool ok = g < ntok;
-        const __nv_bfloat16* src = ok ? Q + ((row_tok0 + g) * H + h) * (int64_t)D + c * 8 : a.Q;
-        cp_async16(sq + dst_off(row, c), src, ok ? 16u : 0u);
-      }
-      cp_async_arrive(q_full);
+    // =========================== producer (one warp): Q once, then K/V tiles by TMA
+    constexpr int HALVES = D / 64;
+    constexpr uint32_t kHalfBytes = kRows * 128;
+    const int64_t kc_base = decode ? b * a.Nc : 0;           // first compressed row of this sequence
+    const int64_t raw_base = decode ? b * (int64_t)a.W : 0;  // first raw row of this sequence
+    if (lane == 0) {
+      prefetch_tmap(&maps.q);
+      mbar_arrive_expect_tx(q_full, HALVES * kHalfBytes);
+      const int qrow = (int)(decode ? b * H : row_tok0 * H);
+      for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(s_q + hf * kHalfBytes, &maps.q, q_full, hf * 64, qrow);
     }
-    auto row_src = [&](const Tile& tl, int x, bool value) -> const __nv_bfloat16* {
-      if (x >= tl.valid) return nullptr;
-      if (tl.type == kSeg) {
-        const int j = s_idx[tl.owner * a.k + (int)tl.base + x];
-        return (value ? Vc : Kc) + (int64_t)j * D;
-      }
-      if (tl.type == kHca) return (value ? Vc : Kc) + (tl.base + x) * D;
-      return (value ? Vr : Kr) + (tl.base + x - raw_lo) * D;
-    };
     for (int i = 0; i < ntiles; ++i) {
       const Tile tl = s_tiles[i];
       const int st = i & 1;
@@ -228,21 +229,37 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
         uint64_t* empty = which ? &v_empty[st] : &k_empty[st];
         uint64_t* fullb = which ? &v_full[st] : &k_full[st];
+        uint8_t* dst = (which ? s_v : s_k) + (size_t)st * L::kTileBytes;
         if (!mbar_wait(empty, ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
-        const uint32_t base = smem_u32((which ? s_v : s_k) + (size_t)st * L::kTileBytes);
-        const int c = pt % CH;
-        for (int x = pt / CH; x < tl.width; x += ROWS_PER_PASS) {
-          const __nv_bfloat16* src = row_src(tl, x, which == 1);
-          cp_async16(base + dst_off(x, c), src ? src + c * 8 : a.Kc, src ? 16u : 0u);
+        if (tl.type == kSeg) {
+          // selected entries: 4-row gathers, lane l loads rows 4l..4l+3 of every half
+          if (lane == 0) mbar_arrive_expect_tx(fullb, (uint32_t)(HALVES * tl.width * 128));
+          __syncwarp();
+          const int* sel = s_idx + tl.owner * a.k + (int)tl.base;
+          const CUtensorMap* m = which ? &maps.vc_g4 : &maps.kc_g4;
+          for (int grp = lane; grp * 4 < tl.width; grp += 32) {
+            int y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int x = grp * 4 + e;
+              y[e] = (int)(kc_base + (x < tl.valid ? sel[x] : sel[0]));
+            }
+            for (int hf = 0; hf < HALVES; ++hf)
+              tma_gather4(dst + hf * kHalfBytes + grp * 512, m, fullb, hf * 64, y[0], y[1], y[2], y[3]);
+          }
+        } else if (lane == 0) {
+          // contiguous rows: one 128-row box per half
+          const CUtensorMap* m = tl.type == kHca ? (which ? &maps.vc : &maps.kc) : (which ? &maps.vr : &maps.kr);
+          const int row = (int)(tl.type == kHca ? kc_base + tl.base : raw_base + (tl.base - raw_lo));
+          mbar_arrive_expect_tx(fullb, HALVES * kHalfBytes);
+          for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(dst + hf * kHalfBytes, m, fullb, hf * 64, row);
         }
-        cp_async_arrive(fullb);
+        __syncwarp();
       }
     }
-    cp_async_wait_all();
   } else if (warp == kSoftmaxWarps + kProducerWarps) {
     // =========================== MMA issuer
     if (ntiles > 0) mbar_wait(q_full, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
-    fence_proxy_async_smem();
     tc_fence_after();
     const uint32_t sq = smem_u32(s_q), sp = smem_u32(s_p);
     auto issue_s = [&](int i) {
@@ -250,7 +267,6 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const uint32_t ph = (i >> 1) & 1;
       mbar_wait(&k_full[st], ph, a.status, CSA_ERR_DEVICE_TIMEOUT);
       mbar_wait(&s_free[st], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
-      fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tcgen05 (async proxy) reads
       tc_fence_after();
       if (lane == 0) {
         const int width = s_tiles[i].width;
@@ -273,16 +289,19 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const int st = i & 1;
       mbar_wait(p_full, i & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       mbar_wait(&v_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
-      fence_proxy_async_smem();
       tc_fence_after();
       if (lane == 0) {
         const int width = s_tiles[i].width;
         const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
+        const uint64_t ones = make_sdesc(smem_u32(s_ones), 128, 256, kSwizzleNone);
         for (int ks = 0; ks < width / 16; ++ks) {
           const uint32_t aoff = (uint32_t)((ks >> 2) * (kRows * 128) + (ks & 3) * 32);
-          mma_bf16_ss(tbase + kTmemO, make_sdesc(sp + aoff, 16, 1024, kSwizzle128),
-                      make_sdesc(sv + ks * 2048, kRows * 128, 1024, kSwizzle128), idesc_bf16(128, D, 0, 1),
-                      (i > 0 || ks > 0) ? 1u : 0u);
+          const uint64_t pdesc = make_sdesc(sp + aoff, 16, 1024, kSwizzle128);
+          const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
+          mma_bf16_ss(tbase + kTmemO, pdesc, make_sdesc(sv + ks * 2048, kRows * 128, 1024, kSwizzle128),
+                      idesc_bf16(128, D, 0, 1), acc);
+          // row sums of the same bf16 weights: P x ones -> 16 columns after O
+          mma_bf16_ss(tbase + kTmemO + D, pdesc, ones, idesc_bf16(128, 16, 0, 0), acc);
         }
         mma_commit(pv_done);
         mma_commit(&v_empty[st]);
@@ -298,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     int64_t nvis = n_visible(t, a.m);
     if (nvis > a.Nc) nvis = a.Nc;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.f, l_run32 = 0.f;
+    const float c = a.scale_log2;  // > 0: max of raw logits * c = max of scaled logits
+    float m_run = -INFINITY, l_run32 = 0.f;
     const uint32_t prow = smem_u32(s_p) + (uint32_t)row * 128;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
@@ -318,52 +338,72 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
           hi = (int)(h0 > l0 ? h0 : l0);
         }
       }
+      const int width = tl.width;
+      const bool mine = hi > lo;
+      const bool full = lo == 0 && hi == width;
+      const bool warp_any = __any_sync(0xffffffffu, mine);
+      const bool warp_full = __all_sync(0xffffffffu, full);
       mbar_wait(&s_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       tc_fence_after();
       const uint32_t scol = tbase + lane_base + (st ? kTmemS1 : kTmemS0);
-      // pass 1: tile maximum over this row's visible range (log2 units of the scaled logits)
-      float mt = -INFINITY;
+      // pass 1: row maximum of the raw logits over the visible range
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (warp_any) {
 #pragma unroll
-      for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
-        if (c0 < tl.width) {  // warp-uniform
-          uint32_t v[64];
-          tmem_ld32p(scol + c0, v);
-          if (c0 + 32 < tl.width) tmem_ld32p(scol + c0 + 32, v + 32);
-          tmem_wait_ld();
+        for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
+          if (c0 < width) {
+            uint32_t v[64];
+            tmem_ld32p(scol + c0, v);
+            if (c0 + 32 < width) tmem_ld32p(scol + c0 + 32, v + 32);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (c0 + e >= lo && c0 + e < hi) mt = fmaxf(mt, __uint_as_float(v[e]) * a.scale_log2);
+            for (int q = 0; q < 4; ++q) {
+              if (c0 + 16 * q < width) {
+#pragma unroll
+                for (int e = 16 * q; e < 16 * q + 16; ++e) {
+                  const float x = __uint_as_float(v[e]);
+                  if (warp_full || (c0 + e >= lo && c0 + e < hi)) mx[e & 3] = fmaxf(mx[e & 3], x);
+                }
+              }
+            }
+          }
         }
       }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
       const bool raise = mt > m_run + kRescaleSlack || (m_run == -INFINITY && mt > -INFINITY);
       const float m_new = raise ? mt : m_run;
       const float alpha = raise ? exp2f(m_run - m_new) : 1.0f;  // exp2(-inf) = 0 on the first raise
-      // pass 2: probabilities, packed to bf16 pairs
+      // pass 2: p = 2^(s*c - m), packed to bf16 pairs (zero outside the visible range)
       uint32_t pk[kTileKeys / 2];
-      float lsum = 0.f, lsum32 = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
-        if (c0 < tl.width) {
-          uint32_t v[64];
-          tmem_ld32p(scol + c0, v);
-          if (c0 + 32 < tl.width) tmem_ld32p(scol + c0 + 32, v + 32);
-          tmem_wait_ld();
+      for (int q = 0; q < kTileKeys / 2; ++q) pk[q] = 0u;
+      if (warp_any) {
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const int x = c0 + e;
-            float p0 = 0.f, p1 = 0.f;
-            if (x >= lo && x < hi) p0 = exp2f(__uint_as_float(v[e]) * a.scale_log2 - m_new);
-            if (x + 1 >= lo && x + 1 < hi) p1 = exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - m_new);
-            const uint32_t pp = pack_bf16x2(p0, p1);
-            // O is normalised by the same bf16-rounded weights the PV MMA consumes;
-            // the log-sum-exp output uses the fp32 weights
-            lsum += bf16_lo(pp) + bf16_hi(pp);
-            lsum32 += p0 + p1;
-            pk[x / 2] = pp;
+        for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
+          if (c0 < width) {
+            uint32_t v[64];
+            tmem_ld32p(scol + c0, v);
+            if (c0 + 32 < width) tmem_ld32p(scol + c0 + 32, v + 32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (c0 + 16 * q < width) {
+#pragma unroll
+                for (int e = 16 * q; e < 16 * q + 16; e += 2) {
+                  const int x = c0 + e;
+                  float p0 = fast_exp2(fmaf(__uint_as_float(v[e]), c, -m_new));
+                  float p1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), c, -m_new));
+                  if (!warp_full) {
+                    p0 = (x >= lo && x < hi) ? p0 : 0.f;
+                    p1 = (x + 1 >= lo && x + 1 < hi) ? p1 : 0.f;
+                  }
+                  if (WANT_LSE) ls[(e >> 1) & 3] += p0 + p1;
+                  pk[x / 2] = pack_bf16x2(p0, p1);
+                }
+              }
+            }
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 64; e += 2) pk[(c0 + e) / 2] = 0u;
         }
       }
       tc_fence_before();
@@ -375,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
+        // rescale O and its row-sum columns (the PV accumulation continues on top)
         const float sc = (raise && i > 0) ? alpha : 1.0f;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 64) {
@@ -387,15 +428,22 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
           tmem_st32p(tbase + lane_base + kTmemO + c0, v);
           tmem_st32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
         }
+        {
+          uint32_t v[16];
+          tmem_ld16p(tbase + lane_base + kTmemO + D, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
+          tmem_st16p(tbase + lane_base + kTmemO + D, v);
+        }
         tmem_wait_st();
       }
-      l_run = l_run * alpha + lsum;
-      l_run32 = l_run32 * alpha + lsum32;
+      if (WANT_LSE) l_run32 = l_run32 * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
       m_run = m_new;
       // store the P row (K-major, 128B swizzle, two 64-key halves)
 #pragma unroll
       for (int cc = 0; cc < kTileKeys / 8; ++cc) {
-        if (cc * 8 < tl.width) {
+        if (cc * 8 < width) {
           const uint32_t off = (uint32_t)((cc >> 3) * (kRows * 128) + (((cc & 7) ^ (row & 7)) << 4));
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + off), "r"(pk[cc * 4]),
                        "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
@@ -407,10 +455,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // epilogue: O / l
+    // epilogue: O / l, with l the row sum of the bf16 weights (tensor-core P x ones)
+    float l_run = 0.f;
     if (ntiles > 0) {
       mbar_wait(pv_done, (ntiles - 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       tc_fence_after();
+      uint32_t v[16];
+      tmem_ld16p(tbase + lane_base + kTmemO + D, v);
+      tmem_wait_ld();
+      l_run = __uint_as_float(v[0]);
     }
     const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
     __nv_bfloat16* orow = nullptr;
@@ -438,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         }
       }
     }
-    if (t >= 0 && a.lse) {
+    if (WANT_LSE && t >= 0 && a.lse) {
       const float lse = l_run32 > 0.f ? (m_run + log2f(l_run32)) * 0.69314718055994531f : -INFINITY;
       a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
     }
@@ -460,22 +513,48 @@ size_t attention_smem_bytes(int d, int idx_entries) {
 
 int attention_max_tiles() { return kMaxTiles; }
 
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeFn get_encode_fn();
+
+// bf16 matrix [rows, d] with 128B-swizzled boxes of 64 columns x box_rows rows
+static bool bf16_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+  EncodeFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool L>
+static cudaError_t launch_t(const AttnArgs& a, const AttnMaps& maps, unsigned grid, size_t smem,
+                            cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  attention_kernel<D, L><<<grid, kThreads, smem, stream>>>(a, maps);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream) {
   const int GQ = kRows / a.H;
   const int idx_entries = a.idx ? GQ * a.k : 0;
   const size_t smem = attention_smem_bytes(d, idx_entries);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attention_kernel<128><<<grid, kThreads, smem, stream>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attention_kernel<64><<<grid, kThreads, smem, stream>>>(a);
-  }
-  return cudaGetLastError();
+  AttnMaps maps;
+  if (!bf16_map(&maps.q, a.Q, a.q_rows, d, 128) || !bf16_map(&maps.kc, a.Kc, a.kc_rows, d, 128) ||
+      !bf16_map(&maps.vc, a.Vc, a.kc_rows, d, 128) || !bf16_map(&maps.kc_g4, a.Kc, a.kc_rows, d, 1) ||
+      !bf16_map(&maps.vc_g4, a.Vc, a.kc_rows, d, 1) || !bf16_map(&maps.kr, a.Kr, a.raw_rows, d, 128) ||
+      !bf16_map(&maps.vr, a.Vr, a.raw_rows, d, 128))
+    return cudaErrorInvalidValue;
+  const bool lse = a.lse != nullptr;
+  if (d == 128)
+    return lse ? launch_t<128, true>(a, maps, grid, smem, stream) : launch_t<128, false>(a, maps, grid, smem, stream);
+  return lse ? launch_t<64, true>(a, maps, grid, smem, stream) : launch_t<64, false>(a, maps, grid, smem, stream);
 }
 
 }  // namespace csa

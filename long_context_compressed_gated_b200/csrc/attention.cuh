@@ -23,6 +23,8 @@ struct AttnArgs {
   // decode (pos != null): one sequence per CTA, batch strides in elements
   int64_t q_batch_stride, kc_batch_stride, raw_batch_stride, o_batch_stride;
   const int64_t* pos;       // device, absolute position of each sequence's new token
+  // extents (rows) of the tensors, for the TMA descriptors
+  int64_t q_rows, kc_rows, raw_rows;
 };
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);

@@ -70,12 +70,19 @@ __device__ __forceinline__ int e2m1_times2(uint32_t code) {
 
 // Head sums of this thread's key lane for the tokens of one half of the group:
 // acc[g] += w2[h] * max(bits(D[g*HI+h]), bits(196608)) over the half's columns,
-// loading up to 64 TMEM columns per wait.
+// loading up to 64 TMEM columns per wait.  NP partial sums per token break the
+// dependent multiply-add chain when a token has many heads.
 template <int HI, int G, int HALF>
 __device__ __forceinline__ void head_sums(uint32_t dcol, const int* s_w2, uint32_t (&acc)[G]) {
   constexpr int G0 = (G + 1) / 2;
   constexpr int c_lo = (HALF ? G0 : 0) * HI;
   constexpr int c_hi = (HALF ? G : G0) * HI;
+  constexpr int NP = HI >= 32 ? 4 : 1;
+  uint32_t part[G][NP];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int p = 0; p < NP; ++p) part[g][p] = 0u;
 #pragma unroll
   for (int b0 = c_lo; b0 < c_hi; b0 += 64) {
     uint32_t v[64];
@@ -91,11 +98,15 @@ __device__ __forceinline__ void head_sums(uint32_t dcol, const int* s_w2, uint32
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int col = b0 + i + q;
-          acc[col / HI] += (uint32_t)ww[q] * (uint32_t)max((int)v[i + q], (int)kMagicBits);
+          part[col / HI][col % NP] += (uint32_t)ww[q] * (uint32_t)max((int)v[i + q], (int)kMagicBits);
         }
       }
     }
   }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int p = 0; p < NP; ++p) acc[g] += part[g][p];
 }
 
 struct IndexerArgs {
@@ -109,6 +120,7 @@ struct IndexerArgs {
   int64_t key_rows;         // rows of the kI tensor (bounds for scale loads)
   int m, k;
   int cap;                  // candidate buffer capacity per token
+  int check;                // tiles between buffer cut-backs (cap >= k + 128 * check)
   int nsplit;               // key ranges per query group
   int64_t split_tiles;      // 128-key tiles per range
   int32_t* idx;             // [rows, k]      (nsplit == 1)
@@ -182,16 +194,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t grp = decode ? blockIdx.x : (int64_t)(gridDim.x - 1 - blockIdx.x);  // heavy groups first
   const int64_t row0 = grp * G;
   const int split = blockIdx.y;
-  int64_t tpos[G];
+  int64_t tnvis[G];  // entries visible to each token of the group (0 for rows past the end)
   int64_t nvis_max = 0;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const int64_t r = row0 + g;
     int64_t t = -1;
     if (r < a.rows) t = decode ? a.pos[r] : a.t0 + r;
-    tpos[g] = t;
     int64_t nv = n_visible(t, a.m);
     if (nv > a.Nc) nv = a.Nc;
+    tnvis[g] = nv;
     if (nv > nvis_max) nvis_max = nv;
   }
   const int64_t key_row_base = decode ? row0 * a.Nc : 0;  // per-sequence cache (decode)
@@ -412,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         if (g < g_lo || g >= g_hi) continue;
-        const int64_t nv = tpos[g] < 0 ? 0 : (n_visible(tpos[g], a.m) < a.Nc ? n_visible(tpos[g], a.m) : a.Nc);
+        const int64_t nv = tnvis[g];
         const int32_t units = (int32_t)(acc[g] - kMagicBits * (uint32_t)s_sumw[g]);
         const uint64_t key = topk::make_key(units, (uint32_t)j);
         const bool take = (j < nv) && (j < j_end) && (key >= s_thr[g]);
@@ -424,12 +436,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (take) s_cand[(size_t)g * cap + base + __popc(bal & ((1u << lane) - 1u))] = key;
         }
       }
+      // every `check` tiles (and before the last one) cut back each buffer that
+      // could overflow within the next `check` tiles
+      if ((it + 1) % a.check != 0 && it + 1 != ntiles) continue;
       topk::named_sync(kEpiBar, kEpiThreads);
-      // cut back every buffer that could overflow on the next tile
 #pragma unroll 1
       for (int g = 0; g < G; ++g) {
         const int cnt = s_cnt[g];
-        if (cnt > cap - 128) {
+        if (cnt > cap - 128 * a.check) {
           uint64_t* buf = s_cand + (size_t)g * cap;
           const uint64_t thr = topk::radix_threshold<kEpiThreads>(buf, cnt, a.k, s_hist, s_sh, et, kEpiBar);
           const int n = topk::compact_ge<kEpiThreads, kCompactPer>(buf, cnt, thr, s_sh + 4, et, kEpiBar);
@@ -552,11 +566,16 @@ static bool make_u8_map(CUtensorMap* m, const void* base, int64_t rows, int row_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tiles between candidate cut-backs: fewer barriers when the buffers have room.
+int indexer_check(int k, int G) {
+  int c = G == 1 ? 8 : (G <= 4 ? 4 : 1);
+  while (c > 1 && k + 128 * c > kEpiThreads * kCompactPer) c >>= 1;
+  return c;
+}
+
 int indexer_cap(int k, int G) {
-  // room for k survivors plus at least one full tile (more when few tokens share
-  // the CTA, so that cut-backs are rarer), at least a power of two >= k
-  int cap = k + 128 * (G == 1 ? 8 : (G <= 4 ? 4 : 1));
-  if (cap > kEpiThreads * kCompactPer) cap = kEpiThreads * kCompactPer;
+  // room for k survivors plus `check` full tiles, at least a power of two >= k
+  int cap = k + 128 * indexer_check(k, G);
   const int p = topk::next_pow2(k);
   if (cap < p) cap = p;
   return ((cap + 127) / 128) * 128;
@@ -627,6 +646,7 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
   a.m = m;
   a.k = k;
   a.cap = indexer_cap(k, G);
+  a.check = indexer_check(k, G);
   a.nsplit = 1;
   a.split_tiles = ceil_div(Nc > 0 ? Nc : 1, 128);
   a.idx = idx;
@@ -658,6 +678,7 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
   a.m = m;
   a.k = k;
   a.cap = indexer_cap(k, 1);
+  a.check = indexer_check(k, 1);
   a.nsplit = nsplit;
   a.split_tiles = ceil_div(ceil_div(nvis_max > 0 ? nvis_max : 1, nsplit), 128);
   a.idx = nullptr;
