@@ -163,6 +163,32 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
                int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
                size_t workspace_bytes, csa_stream_t stream);
 
+/* ---------------------------------------------------------------- decode without allocation
+ * csa_decode for callers that cannot allocate device memory: code recording a
+ * CUDA graph (an allocation would break the capture), serving loops that ban
+ * allocator calls on the hot path, and embedders that own every buffer and hand
+ * the library nothing else.  The pages describe no such interface; it exists
+ * only for these callers.
+ * Same arguments and results as csa_decode, minus the workspace: the scratch
+ * lives in one static 8 MiB device array inside libcsa.so that every GPU loading
+ * the library keeps until the process exits.  Calls whose
+ * csa_decode_workspace_bytes() exceeds 8 MiB are rejected with
+ * CSA_ERR_WORKSPACE (B = 16, k = 1024 fits for any cache length).
+ * The first call on a device looks up the array's device address (a runtime
+ * call, once per device, with that device current); make that first call
+ * before capturing a stream into a graph.  All calls on a device share the
+ * array, so calls that can overlap on the GPU (different streams, no ordering
+ * between them) race with each other; issue them on one stream or order them.
+ * The call clears the array's status word itself.  status_out (device int,
+ * nullable) receives the device status word of the call (CSA_OK, or
+ * CSA_ERR_DEVICE_TIMEOUT / CSA_ERR_RANGE) in stream order.
+ * Allocates nothing: no cudaMalloc/cudaFree, no allocating library routine. */
+int csa_decode_noalloc(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                       const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales,
+                       const void* Kwin, const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d,
+                       int HI, int dI, int m, int k, int W, float scale, void* O, float* lse, int32_t* idx,
+                       float* scores, int* status_out, csa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
