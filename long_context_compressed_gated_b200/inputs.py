@@ -92,17 +92,17 @@ def mxfp4(rows_shape, dI, seed, name, device="cpu"):
     return codes, scales
 
 
-def prefill_layer(wl: Workload, T=None, seed=None, device="cpu", prefix="", with_indexer=True):
+def prefill_layer(wl: Workload, T=None, seed=None, device="cpu", prefix="", with_indexer=True, with_q=True):
     """Inputs of one CSA/HCA prefill layer: Q,K,V,Z,B (+ indexer tensors)."""
     T = wl.T if T is None else T
     s = wl.seed if seed is None else seed
     p = prefix
-    out = {
-        "Q": normal_bf16((T, wl.H, wl.d), s, p + "Q", device=device),
-        "K": normal_bf16((T, wl.d), s, p + "K", device=device),
-        "V": normal_bf16((T, wl.d), s, p + "V", device=device),
-        "Z": normal_bf16((T, wl.d), s, p + "Z", device=device),
-    }
+    out = {}
+    if with_q:
+        out["Q"] = normal_bf16((T, wl.H, wl.d), s, p + "Q", device=device)
+    out["K"] = normal_bf16((T, wl.d), s, p + "K", device=device)
+    out["V"] = normal_bf16((T, wl.d), s, p + "V", device=device)
+    out["Z"] = normal_bf16((T, wl.d), s, p + "Z", device=device)
     out["B"] = normal_f32((wl.m, wl.d), s, p + "B", std=0.5, device=device)
     out["B_hca"] = normal_f32((wl.m_hca, wl.d), s, p + "B_hca", std=0.5, device=device)
     if with_indexer:
