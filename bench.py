@@ -288,6 +288,43 @@ def run_decode(csa, wl, steps, warmup):
     return {"ms": t0.elapsed_time(t1) / steps, "status": csa.csa_check_status(ws)}
 
 
+def stack_work(wl):
+    t = np.arange(wl.T, dtype=np.int64)
+    nv1 = (t + 1) // wl.m
+    nv2 = (t + 1) // wl.m_hca
+    win = np.minimum(t + 1, wl.W)
+    return {"indexer_flop": 2.0 * float(nv1.sum()) * wl.HI * wl.dI,
+            "csa_attn_flop": 4.0 * float((np.minimum(nv1, wl.k) + win).sum()) * wl.H * wl.d,
+            "hca_attn_flop": 4.0 * float((nv2 + np.minimum(t + 1, wl.W_hca)).sum()) * wl.H * wl.d,
+            "projection_flop": 2.0 * wl.T * wl.H * wl.d * wl.d}
+
+
+def run_stack(csa, wl, steps, warmup):
+    from long_context_compressed_gated_b200.stack import stack_inputs, stack_prefill_chunked
+    l1, l2, P = stack_inputs(wl, device="cuda")
+    O2 = torch.empty_like(l1["Q"])
+
+    def step(events=None):
+        stack_prefill_chunked(l1, l2, P, wl.chunk, wl.m, wl.k, wl.W, wl.m_hca, wl.W_hca, out=O2,
+                              phase_events=events)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    events = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step(events)
+    t1.record()
+    torch.cuda.synchronize()
+    phases = {}
+    for name, e0, e1 in events:
+        phases[name] = phases.get(name, 0.0) + e0.elapsed_time(e1) / steps
+    return {"ms": t0.elapsed_time(t1) / steps, "phases": phases}
+
+
 # ----------------------------------------------------------------- CPU oracle (reference arm / baseline)
 def oracle_sample(wl, seconds=12.0, max_rows=4096):
     """Time the CPU oracle on a bounded sample of the CSA prefill workload: the
@@ -390,6 +427,19 @@ def main():
         extra["csa_decode_B16_L1M"] = {
             "us_per_step": r3["ms"] * 1e3, "algorithmic_bytes": by, "gbs": by / (r3["ms"] * 1e-3) / 1e9,
             "frac_hbm": by / (r3["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], "status": r3["status"]}
+        torch.cuda.empty_cache()
+        w4 = inputs.STACK
+        r4 = run_stack(csa, w4, 2, 1)
+        sw = stack_work(w4)
+        ph4 = r4["phases"]
+        method_ms = r4["ms"] - ph4.get("projection", 0.0)
+        extra["csa_hca_stack_T262144_chunk16384"] = {
+            "tokens_per_s": w4.T / (r4["ms"] * 1e-3), "ms_per_step": r4["ms"],
+            "tokens_per_s_without_projection": w4.T / (method_ms * 1e-3),
+            "indexer_tflops": sw["indexer_flop"] / (ph4["indexer_topk"] * 1e-3) / 1e12,
+            "csa_attn_tflops": sw["csa_attn_flop"] / (ph4["sparse_attn"] * 1e-3) / 1e12,
+            "hca_attn_tflops": sw["hca_attn_flop"] / (ph4["hca_attn"] * 1e-3) / 1e12,
+            "phases_ms": ph4, "projection_excluded_from_method": True}
         torch.cuda.empty_cache()
 
     ph = res["phases"]

@@ -14,13 +14,19 @@
 // and every row sees, per tile, one contiguous range of its columns (its own
 // segment / the visible prefix / its window), so masking needs no per-key data.
 //
-// Per tile: S = Q K^T (tcgen05 kind::f16, M=128, N=width, fp32 in TMEM),
-// online softmax in the softmax warps (one row per thread, exp2 with a lazily
-// raised running max), P (bf16) to shared memory, O += P V (tcgen05, V read as
-// an MN-major operand, O accumulated in TMEM).  K/V rows are gathered by four
-// producer warps with 16-byte cp.async into 128B-swizzled tiles (K and V in
-// separate double-buffered rings, so S of tile i+2 can start while PV of tile i
-// still reads V).
+// Per tile: S = Q K^T (tcgen05 kind::f16, M=128, N=width, fp32 in TMEM), online
+// softmax, P (bf16) to shared memory, O += P V (tcgen05, V as an MN-major
+// operand) and l += P 1 (row sums of the same bf16 weights, tensor core), with
+// O and l accumulated in TMEM.  Warp roles:
+//   warps 0..7   softmax: two warps per TMEM lane quarter, each owning 64 of the
+//                128 columns of a tile (the row maximum is taken over all columns
+//                by both warps, so they agree without exchanging data);
+//   warps 8..11  loaders: 16-byte cp.async gathers of selected rows into
+//                128B-swizzled tiles; contiguous tiles (HCA, window) and Q come
+//                in whole 128-row boxes by TMA;
+//   warp 12      TMEM allocation and MMA issue.
+// K and V have separate double-buffered rings, so S of tile i+2 can start while
+// PV of tile i still reads V.
 #include <cuda.h>
 
 #include "attention.cuh"
@@ -36,14 +42,17 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kTileKeys = 128;
 constexpr int kMaxTiles = 80;
-constexpr int kSoftmaxWarps = 4, kProducerWarps = 1;
-constexpr int kThreads = (kSoftmaxWarps + kProducerWarps + 1) * 32;  // + 1 MMA warp
+constexpr int kSoftmaxWarps = 8, kLoaderWarps = 4;
+constexpr int kLoaderThreads = kLoaderWarps * 32;
+constexpr int kMmaWarp = kSoftmaxWarps + kLoaderWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr float kRescaleSlack = 8.0f;  // raise the running max only when it grows by > 2^8
+constexpr int kSoftmaxBar = 1;         // named barrier of the softmax warps (end of kernel)
 
 enum TileType : int { kSeg = 0, kHca = 1, kWin = 2 };
 
 struct Tile {
-  int type, owner, width, valid;  // valid: SEG entries in this tile
+  int type, owner, width, valid;  // valid: keys of the tile that exist (<= width)
   int64_t base;                   // SEG: offset in the token's list; HCA: j0; WIN: w0
 };
 
@@ -54,22 +63,35 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-
-__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-      : "memory");
+// (a*c - m, b*c - m) with one packed fp32x2 fma.
+__device__ __forceinline__ float2 scale_sub2(float a, float b, float c, float m) {
+  unsigned long long x, y;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
+  asm("{\n\t.reg .b64 cc, mm;\n\t"
+      "mov.b64 cc, {%2, %2};\n\t"
+      "mov.b64 mm, {%3, %3};\n\t"
+      "fma.rn.f32x2 %0, %1, cc, mm;\n\t}"
+      : "=l"(y)
+      : "l"(x), "f"(c), "f"(-m));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(y));
+  return r;
 }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on `bar` once all prior cp.async of this thread have landed (counts as one arrival).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 }  // namespace
 
-// TMA descriptors of one launch: 128-row boxes (two 64-column halves, 128B
-// swizzle) for contiguous rows, and 1-row boxes for 4-row gathers.
+// TMA descriptors of one launch: 128-row boxes (64-column halves, 128B swizzle).
 struct alignas(64) AttnMaps {
-  CUtensorMap q, kc, vc, kc_g4, vc_g4, kr, vr;
+  CUtensorMap q, kc, vc, kr, vr;
 };
 
 template <int D>
@@ -83,8 +105,9 @@ struct AttnSmem {
   static constexpr size_t off_tiles = off_p + 2 * kHalf;
   static constexpr size_t off_bar = off_tiles + kMaxTiles * sizeof(Tile);
   static constexpr size_t off_misc = off_bar + 16 * 8;
-  static constexpr size_t off_ones = off_misc + 256;        // 16 x 16 bf16 ones (row-sum MMA operand)
-  static constexpr size_t off_idx = off_ones + 512;
+  static constexpr size_t off_ones = off_misc + 256;       // 16 x 16 bf16 ones (row-sum MMA operand)
+  static constexpr size_t off_red = off_ones + 512;        // [2][128] floats: partial fp32 row sums
+  static constexpr size_t off_idx = off_red + 1024;
   static size_t bytes(int idx_entries) { return off_idx + (size_t)idx_entries * 4 + 1024; }
 };
 
@@ -93,6 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
                                                                 const __grid_constant__ AttnMaps maps) {
   using L = AttnSmem<D>;
   constexpr int KSTEPS_QK = D / 16;
+  constexpr int HALVES = D / 64;
+  constexpr uint32_t kHalfBytes = kRows * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_q = smem + L::off_q;
@@ -111,8 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   uint64_t* p_full = bar + 13;
   uint64_t* pv_done = bar + 14;
   int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [0] ntiles, [1] tmem, [2..] seg counts
-  int* s_idx = reinterpret_cast<int*>(smem + L::off_idx);
   uint8_t* s_ones = smem + L::off_ones;
+  float* s_red = reinterpret_cast<float*>(smem + L::off_red);
+  int* s_idx = reinterpret_cast<int*>(smem + L::off_idx);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
@@ -120,11 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   const bool decode = a.pos != nullptr;
   const int64_t b = decode ? blockIdx.x : 0;
   const int64_t row_tok0 = decode ? 0 : (int64_t)blockIdx.x * GQ;  // first token row of this CTA
-  const __nv_bfloat16* Q = a.Q + b * a.q_batch_stride;
   const __nv_bfloat16* Kc = a.Kc + b * a.kc_batch_stride;
   const __nv_bfloat16* Vc = a.Vc + b * a.kc_batch_stride;
-  const __nv_bfloat16* Kr = a.Kr + b * a.raw_batch_stride;
-  const __nv_bfloat16* Vr = a.Vr + b * a.raw_batch_stride;
   const int32_t* idx = a.idx ? a.idx + b * (decode ? (int64_t)a.k : 0) : nullptr;
   const int64_t T = decode ? 1 : a.T;
   const int64_t raw_lo = decode ? a.pos[b] - a.W + 1 : a.raw_lo;  // absolute position of raw row 0
@@ -140,9 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   if (tid == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
+      mbar_init(&k_full[i], kLoaderThreads + 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
+      mbar_init(&v_full[i], kLoaderThreads + 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftmaxWarps);
@@ -151,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     mbar_init(pv_done, 1);
     fence_mbar_init();
   }
-  if (warp == kSoftmaxWarps + kProducerWarps) {
+  if (warp == kMmaWarp) {
     tmem_alloc(reinterpret_cast<uint32_t*>(&misc[1]), 512);
     tmem_relinquish();
   }
@@ -210,18 +233,23 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   const uint32_t tbase = (uint32_t)misc[1];
   constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
 
-  if (warp >= kSoftmaxWarps && warp < kSoftmaxWarps + kProducerWarps) {
-    // =========================== producer (one warp): Q once, then K/V tiles by TMA
-    constexpr int HALVES = D / 64;
-    constexpr uint32_t kHalfBytes = kRows * 128;
+  if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
+    // =========================== loaders: Q and contiguous tiles by TMA, selected rows by cp.async
+    const int lt = tid - kSoftmaxWarps * 32;                 // 0..127
     const int64_t kc_base = decode ? b * a.Nc : 0;           // first compressed row of this sequence
     const int64_t raw_base = decode ? b * (int64_t)a.W : 0;  // first raw row of this sequence
-    if (lane == 0) {
+    if (lt == 0) {
       prefetch_tmap(&maps.q);
       mbar_arrive_expect_tx(q_full, HALVES * kHalfBytes);
       const int qrow = (int)(decode ? b * H : row_tok0 * H);
       for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(s_q + hf * kHalfBytes, &maps.q, q_full, hf * 64, qrow);
     }
+    // cp.async mapping: thread lt copies 16-byte chunk c of rows r0, r0 + RSTEP, ...; the
+    // 128B swizzle term (chunk ^ row%8) is the same for all of them.
+    constexpr int CH = D / 8;
+    constexpr int RSTEP = kLoaderThreads / CH;
+    const int c = lt % CH, r0 = lt / CH;
+    const uint32_t dst_lane = (uint32_t)((c >> 3) * kHalfBytes + r0 * 128 + (((c & 7) ^ (r0 & 7)) << 4));
     for (int i = 0; i < ntiles; ++i) {
       const Tile tl = s_tiles[i];
       const int st = i & 1;
@@ -232,32 +260,29 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         uint8_t* dst = (which ? s_v : s_k) + (size_t)st * L::kTileBytes;
         if (!mbar_wait(empty, ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
         if (tl.type == kSeg) {
-          // selected entries: 4-row gathers, lane l loads rows 4l..4l+3 of every half
-          if (lane == 0) mbar_arrive_expect_tx(fullb, (uint32_t)(HALVES * tl.width * 128));
-          __syncwarp();
           const int* sel = s_idx + tl.owner * a.k + (int)tl.base;
-          const CUtensorMap* m = which ? &maps.vc_g4 : &maps.kc_g4;
-          for (int grp = lane; grp * 4 < tl.width; grp += 32) {
-            int y[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int x = grp * 4 + e;
-              y[e] = (int)(kc_base + (x < tl.valid ? sel[x] : sel[0]));
-            }
-            for (int hf = 0; hf < HALVES; ++hf)
-              tma_gather4(dst + hf * kHalfBytes + grp * 512, m, fullb, hf * 64, y[0], y[1], y[2], y[3]);
+          const __nv_bfloat16* src0 = (which ? Vc : Kc) + c * 8;
+          const uint32_t d0 = smem_u32(dst) + dst_lane;
+          for (int x = r0; x < tl.width; x += RSTEP) {
+            const bool ok = x < tl.valid;
+            const int j = ok ? sel[x] : 0;
+            cp_async16(d0 + (uint32_t)(x - r0) * 128, src0 + (int64_t)j * D, ok ? 16u : 0u);
           }
-        } else if (lane == 0) {
-          // contiguous rows: one 128-row box per half
-          const CUtensorMap* m = tl.type == kHca ? (which ? &maps.vc : &maps.kc) : (which ? &maps.vr : &maps.kr);
-          const int row = (int)(tl.type == kHca ? kc_base + tl.base : raw_base + (tl.base - raw_lo));
-          mbar_arrive_expect_tx(fullb, HALVES * kHalfBytes);
-          for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(dst + hf * kHalfBytes, m, fullb, hf * 64, row);
+          cp_async_arrive(fullb);
+          if (lt == 0) mbar_arrive(fullb);
+        } else {
+          if (lt == 0) {
+            const CUtensorMap* m = tl.type == kHca ? (which ? &maps.vc : &maps.kc) : (which ? &maps.vr : &maps.kr);
+            const int row = (int)(tl.type == kHca ? kc_base + tl.base : raw_base + (tl.base - raw_lo));
+            mbar_arrive_expect_tx(fullb, HALVES * kHalfBytes);
+            for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(dst + hf * kHalfBytes, m, fullb, hf * 64, row);
+          }
+          mbar_arrive(fullb);
         }
-        __syncwarp();
       }
     }
-  } else if (warp == kSoftmaxWarps + kProducerWarps) {
+    cp_async_wait_all();
+  } else if (warp == kMmaWarp) {
     // =========================== MMA issuer
     if (ntiles > 0) mbar_wait(q_full, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
     tc_fence_after();
@@ -267,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const uint32_t ph = (i >> 1) & 1;
       mbar_wait(&k_full[st], ph, a.status, CSA_ERR_DEVICE_TIMEOUT);
       mbar_wait(&s_free[st], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tcgen05 (async proxy) reads
       tc_fence_after();
       if (lane == 0) {
         const int width = s_tiles[i].width;
@@ -274,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         const uint32_t d = tbase + (st ? kTmemS1 : kTmemS0);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS_QK; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+          const uint32_t off = (uint32_t)((kk >> 2) * kHalfBytes + (kk & 3) * 32);
           mma_bf16_ss(d, make_sdesc(sq + off, 16, 1024, kSwizzle128), make_sdesc(sk + off, 16, 1024, kSwizzle128),
                       idesc_bf16(128, width, 0, 0), kk > 0);
         }
@@ -285,20 +311,21 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     };
     if (ntiles > 0) issue_s(0);
     if (ntiles > 1) issue_s(1);
+    const uint64_t ones = make_sdesc(smem_u32(s_ones), 128, 256, kSwizzleNone);
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
       mbar_wait(p_full, i & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       mbar_wait(&v_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      fence_proxy_async_smem();
       tc_fence_after();
       if (lane == 0) {
         const int width = s_tiles[i].width;
         const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
-        const uint64_t ones = make_sdesc(smem_u32(s_ones), 128, 256, kSwizzleNone);
         for (int ks = 0; ks < width / 16; ++ks) {
-          const uint32_t aoff = (uint32_t)((ks >> 2) * (kRows * 128) + (ks & 3) * 32);
+          const uint32_t aoff = (uint32_t)((ks >> 2) * kHalfBytes + (ks & 3) * 32);
           const uint64_t pdesc = make_sdesc(sp + aoff, 16, 1024, kSwizzle128);
           const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
-          mma_bf16_ss(tbase + kTmemO, pdesc, make_sdesc(sv + ks * 2048, kRows * 128, 1024, kSwizzle128),
+          mma_bf16_ss(tbase + kTmemO, pdesc, make_sdesc(sv + ks * 2048, kHalfBytes, 1024, kSwizzle128),
                       idesc_bf16(128, D, 0, 1), acc);
           // row sums of the same bf16 weights: P x ones -> 16 columns after O
           mma_bf16_ss(tbase + kTmemO + D, pdesc, ones, idesc_bf16(128, 16, 0, 0), acc);
@@ -310,16 +337,18 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       if (i + 2 < ntiles) issue_s(i + 2);
     }
   } else {
-    // =========================== softmax (warps 0..3, one row per thread)
-    const int row = warp * 32 + lane;
+    // =========================== softmax (warps 0..7): row = TMEM lane, columns [64*half, +64)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
     const int g = row / H, h = row % H;
     const int64_t t = g < ntok ? token_pos(g) : -1;
     int64_t nvis = n_visible(t, a.m);
     if (nvis > a.Nc) nvis = a.Nc;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float c = a.scale_log2;  // > 0: max of raw logits * c = max of scaled logits
+    const int my0 = half * 64;     // first column this warp turns into probabilities
     float m_run = -INFINITY, l_run32 = 0.f;
-    const uint32_t prow = smem_u32(s_p) + (uint32_t)row * 128;
+    const uint32_t prow = smem_u32(s_p) + (uint32_t)(half * kHalfBytes + row * 128);
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
       const Tile tl = s_tiles[i];
@@ -339,30 +368,30 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         }
       }
       const int width = tl.width;
-      const bool mine = hi > lo;
-      const bool full = lo == 0 && hi == width;
-      const bool warp_any = __any_sync(0xffffffffu, mine);
-      const bool warp_full = __all_sync(0xffffffffu, full);
+      const bool warp_any = __any_sync(0xffffffffu, hi > lo);
+      const bool warp_full = __all_sync(0xffffffffu, lo == 0 && hi == width);
       mbar_wait(&s_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       tc_fence_after();
       const uint32_t scol = tbase + lane_base + (st ? kTmemS1 : kTmemS0);
-      // pass 1: row maximum of the raw logits over the visible range
+      // pass 1: row maximum of the raw logits over the visible range (all columns)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (warp_any) {
 #pragma unroll
-        for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
+        for (int c0 = 0; c0 < kTileKeys; c0 += 32) {
           if (c0 < width) {
-            uint32_t v[64];
+            uint32_t v[32];
             tmem_ld32p(scol + c0, v);
-            if (c0 + 32 < width) tmem_ld32p(scol + c0 + 32, v + 32);
             tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
               if (c0 + 16 * q < width) {
+                if (warp_full) {
 #pragma unroll
-                for (int e = 16 * q; e < 16 * q + 16; ++e) {
-                  const float x = __uint_as_float(v[e]);
-                  if (warp_full || (c0 + e >= lo && c0 + e < hi)) mx[e & 3] = fmaxf(mx[e & 3], x);
+                  for (int e = 16 * q; e < 16 * q + 16; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
+                } else {
+#pragma unroll
+                  for (int e = 16 * q; e < 16 * q + 16; ++e)
+                    if (c0 + e >= lo && c0 + e < hi) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
                 }
               }
             }
@@ -373,33 +402,32 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const bool raise = mt > m_run + kRescaleSlack || (m_run == -INFINITY && mt > -INFINITY);
       const float m_new = raise ? mt : m_run;
       const float alpha = raise ? exp2f(m_run - m_new) : 1.0f;  // exp2(-inf) = 0 on the first raise
-      // pass 2: p = 2^(s*c - m), packed to bf16 pairs (zero outside the visible range)
-      uint32_t pk[kTileKeys / 2];
+      // pass 2: p = 2^(s*c - m) over this warp's 64 columns, packed to bf16 pairs
+      uint32_t pk[32];
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < kTileKeys / 2; ++q) pk[q] = 0u;
-      if (warp_any) {
+      for (int q = 0; q < 32; ++q) pk[q] = 0u;
+      if (warp_any && my0 < width) {
 #pragma unroll
-        for (int c0 = 0; c0 < kTileKeys; c0 += 64) {
-          if (c0 < width) {
-            uint32_t v[64];
-            tmem_ld32p(scol + c0, v);
-            if (c0 + 32 < width) tmem_ld32p(scol + c0 + 32, v + 32);
+        for (int b0 = 0; b0 < 64; b0 += 32) {
+          if (my0 + b0 < width) {
+            uint32_t v[32];
+            tmem_ld32p(scol + my0 + b0, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (c0 + 16 * q < width) {
+            for (int q = 0; q < 2; ++q) {
+              if (my0 + b0 + 16 * q < width) {
 #pragma unroll
                 for (int e = 16 * q; e < 16 * q + 16; e += 2) {
-                  const int x = c0 + e;
-                  float p0 = fast_exp2(fmaf(__uint_as_float(v[e]), c, -m_new));
-                  float p1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), c, -m_new));
+                  const float2 z = scale_sub2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), c, m_new);
+                  float p0 = fast_exp2(z.x), p1 = fast_exp2(z.y);
                   if (!warp_full) {
+                    const int x = my0 + b0 + e;
                     p0 = (x >= lo && x < hi) ? p0 : 0.f;
                     p1 = (x + 1 >= lo && x + 1 < hi) ? p1 : 0.f;
                   }
                   if (WANT_LSE) ls[(e >> 1) & 3] += p0 + p1;
-                  pk[x / 2] = pack_bf16x2(p0, p1);
+                  pk[(b0 + e) / 2] = pack_bf16x2(p0, p1);
                 }
               }
             }
@@ -415,20 +443,20 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
-        // rescale O and its row-sum columns (the PV accumulation continues on top)
+        // rescale this warp's half of O (and, for half 0, the row-sum columns)
         const float sc = (raise && i > 0) ? alpha : 1.0f;
+        if (my0 < D) {
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 64) {
-          uint32_t v[64];
-          tmem_ld32p(tbase + lane_base + kTmemO + c0, v);
-          tmem_ld32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
-          tmem_wait_ld();
+          for (int b0 = 0; b0 < 64; b0 += 32) {
+            uint32_t v[32];
+            tmem_ld32p(tbase + lane_base + kTmemO + my0 + b0, v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 64; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
-          tmem_st32p(tbase + lane_base + kTmemO + c0, v);
-          tmem_st32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
+            tmem_st32p(tbase + lane_base + kTmemO + my0 + b0, v);
+          }
         }
-        {
+        if (half == 0) {
           uint32_t v[16];
           tmem_ld16p(tbase + lane_base + kTmemO + D, v);
           tmem_wait_ld();
@@ -440,14 +468,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       }
       if (WANT_LSE) l_run32 = l_run32 * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
       m_run = m_new;
-      // store the P row (K-major, 128B swizzle, two 64-key halves)
+      // store this warp's half of the P row (K-major, 128B swizzle)
+      if (my0 < width) {
 #pragma unroll
-      for (int cc = 0; cc < kTileKeys / 8; ++cc) {
-        if (cc * 8 < width) {
-          const uint32_t off = (uint32_t)((cc >> 3) * (kRows * 128) + (((cc & 7) ^ (row & 7)) << 4));
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + off), "r"(pk[cc * 4]),
-                       "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
-                       : "memory");
+        for (int cc = 0; cc < 8; ++cc) {
+          if (my0 + cc * 8 < width) {
+            const uint32_t off = (uint32_t)(((cc ^ (row & 7)) << 4));
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + off), "r"(pk[cc * 4]),
+                         "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
+                         : "memory");
+          }
         }
       }
       fence_proxy_async_smem();
@@ -469,37 +499,43 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     __nv_bfloat16* orow = nullptr;
     if (t >= 0) orow = a.O + b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 64) {
-      uint32_t v[64];
+    for (int b0 = 0; b0 < 64; b0 += 32) {
+      if (my0 >= D) break;
+      uint32_t v[32];
       if (ntiles > 0) {
-        tmem_ld32p(tbase + lane_base + kTmemO + c0, v);
-        tmem_ld32p(tbase + lane_base + kTmemO + c0 + 32, v + 32);
+        tmem_ld32p(tbase + lane_base + kTmemO + my0 + b0, v);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) v[e] = 0u;
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
       if (orow) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 8) {
+        for (int e = 0; e < 32; e += 8) {
           uint4 o;
           o.x = pack_bf16x2(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
           o.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
           o.z = pack_bf16x2(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
           o.w = pack_bf16x2(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + c0 + e) = o;
+          *reinterpret_cast<uint4*>(orow + my0 + b0 + e) = o;
         }
       }
     }
-    if (WANT_LSE && t >= 0 && a.lse) {
-      const float lse = l_run32 > 0.f ? (m_run + log2f(l_run32)) * 0.69314718055994531f : -INFINITY;
-      a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
+    if (WANT_LSE) {
+      // combine the two halves' fp32 row sums
+      s_red[half * kRows + row] = l_run32;
+      asm volatile("bar.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(kSoftmaxWarps * 32) : "memory");
+      if (half == 0 && t >= 0 && a.lse) {
+        const float l32 = l_run32 + s_red[kRows + row];
+        const float lse = l32 > 0.f ? (m_run + log2f(l32)) * 0.69314718055994531f : -INFINITY;
+        a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kSoftmaxWarps + kProducerWarps) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -547,8 +583,7 @@ cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   AttnMaps maps;
   if (!bf16_map(&maps.q, a.Q, a.q_rows, d, 128) || !bf16_map(&maps.kc, a.Kc, a.kc_rows, d, 128) ||
-      !bf16_map(&maps.vc, a.Vc, a.kc_rows, d, 128) || !bf16_map(&maps.kc_g4, a.Kc, a.kc_rows, d, 1) ||
-      !bf16_map(&maps.vc_g4, a.Vc, a.kc_rows, d, 1) || !bf16_map(&maps.kr, a.Kr, a.raw_rows, d, 128) ||
+      !bf16_map(&maps.vc, a.Vc, a.kc_rows, d, 128) || !bf16_map(&maps.kr, a.Kr, a.raw_rows, d, 128) ||
       !bf16_map(&maps.vr, a.Vr, a.raw_rows, d, 128))
     return cudaErrorInvalidValue;
   const bool lse = a.lse != nullptr;
