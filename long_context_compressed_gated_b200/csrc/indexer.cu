@@ -44,8 +44,8 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kMagicBits = 0x48400000u;  // bit pattern of 196608.0f
-constexpr int kEpiBar = 1;                    // named barrier of the epilogue warps
-constexpr int kCompactPer = 12;               // candidate capacity <= kEpiThreads * kCompactPer
+constexpr int kHalfBar0 = 1;                  // named barriers 1, 2: the four warps of each half
+constexpr size_t kSmemLimit = 227 * 1024;
 
 // TMEM column map (512 allocated): D[0] at 0, D[1] at 256; scale factors at 224..
 constexpr uint32_t kTmemD1 = 256;
@@ -56,7 +56,7 @@ constexpr uint32_t kTmemMagicSFB = 244;  // 8 columns
 
 template <int HI>
 struct Geometry {
-  static constexpr int G = kMaxCols / HI < 16 ? kMaxCols / HI : 16;  // tokens per CTA (prefill)
+  static constexpr int G = kMaxCols / HI < 8 ? kMaxCols / HI : 8;  // tokens per CTA (prefill)
 };
 
 __device__ __forceinline__ int e2m1_times2(uint32_t code) {
@@ -146,8 +146,8 @@ struct IndexerSmem {
   static constexpr size_t off_sumw = off_w2 + (size_t)N * 4;
   static constexpr size_t off_cnt = off_sumw + 64 * 4;
   static constexpr size_t off_thr = off_cnt + 64 * 4;
-  static constexpr size_t off_hist = off_thr + 64 * 8;
-  static constexpr size_t off_sh = off_hist + 256 * 4;
+  static constexpr size_t off_hist = off_thr + 64 * 8;               // per epilogue warp, kWarpBins ints
+  static constexpr size_t off_sh = off_hist + (size_t)kEpiWarps * topk::kWarpBins * 4;
   static constexpr size_t off_bar = off_sh + 64;
   static constexpr size_t off_tslot = off_bar + (2 * kStages + 5) * 8;
   static constexpr size_t off_cand = ((off_tslot + 16 + 15) / 16) * 16;
@@ -403,6 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(G == 1 || (G0 * HI) % 16 == 0, "halves must split on a 16-column chunk");
     const int g_lo = half == 0 ? 0 : G0;
     const int g_hi = half == 0 ? G0 : G;
+    static_assert(G0 <= 4, "one token per warp of a half");
+    const int my_g = g_lo + quarter;  // token whose buffer this warp maintains
+    int* my_hist = s_hist + (warp - 2) * topk::kWarpBins;
 
     for (int it = 0; it < ntiles; ++it) {
       const int b = it & 1;
@@ -436,43 +439,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (take) s_cand[(size_t)g * cap + base + __popc(bal & ((1u << lane) - 1u))] = key;
         }
       }
-      // every `check` tiles (and before the last one) cut back each buffer that
-      // could overflow within the next `check` tiles
+      // every `check` tiles (and after the last one) the half's warps meet; warp
+      // `quarter` then cuts back token g_lo + quarter's buffer if the next `check`
+      // tiles could overflow it (one-pass histogram threshold that keeps >= k)
       if ((it + 1) % a.check != 0 && it + 1 != ntiles) continue;
-      topk::named_sync(kEpiBar, kEpiThreads);
-#pragma unroll 1
-      for (int g = 0; g < G; ++g) {
-        const int cnt = s_cnt[g];
+      topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
+      if (my_g < g_hi) {
+        uint64_t* buf = s_cand + (size_t)my_g * cap;
+        const int cnt = s_cnt[my_g];
         if (cnt > cap - 128 * a.check) {
-          uint64_t* buf = s_cand + (size_t)g * cap;
-          const uint64_t thr = topk::radix_threshold<kEpiThreads>(buf, cnt, a.k, s_hist, s_sh, et, kEpiBar);
-          const int n = topk::compact_ge<kEpiThreads, kCompactPer>(buf, cnt, thr, s_sh + 4, et, kEpiBar);
-          if (et == 0) {
-            s_cnt[g] = n;
-            s_thr[g] = thr;
+          int kept;
+          const uint64_t thr = topk::warp_approx_threshold(buf, cnt, a.k, cap - 128 * a.check, my_hist, lane, &kept);
+          const int n = topk::warp_compact_ge(buf, cnt, thr, lane);
+          if (lane == 0) {
+            s_cnt[my_g] = n;
+            s_thr[my_g] = thr;
           }
-          topk::named_sync(kEpiBar, kEpiThreads);
         }
       }
+      topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
     }
 
-    // final selection and output, token by token
-#pragma unroll 1
-    for (int g = 0; g < G; ++g) {
-      const int64_t r = row0 + g;
-      if (r >= a.rows) break;
-      uint64_t* buf = s_cand + (size_t)g * cap;
-      int cnt = s_cnt[g];
+    // final exact selection and sort: one warp per token, all tokens in parallel
+    if (my_g < g_hi && row0 + my_g < a.rows) {
+      const int64_t r = row0 + my_g;
+      uint64_t* buf = s_cand + (size_t)my_g * cap;
+      int cnt = s_cnt[my_g];
       if (cnt > a.k) {
-        const uint64_t thr = topk::radix_threshold<kEpiThreads>(buf, cnt, a.k, s_hist, s_sh, et, kEpiBar);
-        cnt = topk::compact_ge<kEpiThreads, kCompactPer>(buf, cnt, thr, s_sh + 4, et, kEpiBar);
+        const uint64_t thr = topk::warp_exact_threshold(buf, cnt, a.k, my_hist, lane);
+        cnt = topk::warp_compact_ge(buf, cnt, thr, lane);
       }
       const int P = topk::next_pow2(cnt > 1 ? cnt : 1);
-      for (int i = cnt + et; i < P; i += kEpiThreads) buf[i] = 0;
-      topk::named_sync(kEpiBar, kEpiThreads);
-      topk::bitonic_desc<kEpiThreads>(buf, P, et, kEpiBar);
+      for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
+      __syncwarp();
+      topk::warp_bitonic_desc(buf, P, lane);
       if (a.nsplit == 1) {
-        for (int q = et; q < a.k; q += kEpiThreads) {
+        for (int q = lane; q < a.k; q += 32) {
           int32_t id = -1;
           float sc = -INFINITY;
           if (q < cnt) {
@@ -485,9 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
-        for (int q = et; q < a.k; q += kEpiThreads) out[q] = q < cnt ? buf[q] : 0;
+        for (int q = lane; q < a.k; q += 32) out[q] = q < cnt ? buf[q] : 0;
       }
-      topk::named_sync(kEpiBar, kEpiThreads);
     }
   }
 
@@ -566,19 +567,26 @@ static bool make_u8_map(CUtensorMap* m, const void* base, int64_t rows, int row_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tiles between candidate cut-backs: fewer barriers when the buffers have room.
-int indexer_check(int k, int G) {
-  int c = G == 1 ? 8 : (G <= 4 ? 4 : 1);
-  while (c > 1 && k + 128 * c > kEpiThreads * kCompactPer) c >>= 1;
-  return c;
-}
-
-int indexer_cap(int k, int G) {
-  // room for k survivors plus `check` full tiles, at least a power of two >= k
-  int cap = k + 128 * indexer_check(k, G);
+// Candidate capacity per token: whatever shared memory is left (cut-backs are
+// rarer the larger it is), at least k + 128*check and a power of two >= k.
+template <int HI, int DI, int G>
+static bool choose_cap(int k, int* cap, int* check) {
+  using L = IndexerSmem<HI, DI, G>;
+  const size_t base = L::bytes(0);
+  const int budget = base < kSmemLimit ? (int)((kSmemLimit - base) / (8 * (size_t)G)) & ~127 : 0;
   const int p = topk::next_pow2(k);
-  if (cap < p) cap = p;
-  return ((cap + 127) / 128) * 128;
+  for (int c = 4; c >= 1; c >>= 1) {
+    const int need = k + 128 * c > p ? k + 128 * c : p;
+    if (budget >= need) {
+      int want = k + (k > 128 * c ? k : 128 * c) + 128 * c;  // room for ~k more before a cut-back
+      if (want < need) want = need;
+      *cap = (want < budget ? want : budget) & ~127;
+      if (*cap < need) *cap = ((need + 127) / 128) * 128;
+      *check = c;
+      return true;
+    }
+  }
+  return false;
 }
 
 template <int HI, int DI, int G>
@@ -588,8 +596,9 @@ static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, In
   CUtensorMap qmap, kmap;
   if (!make_u8_map(&qmap, q_codes, a.rows * HI, DI / 2, L::N)) return cudaErrorInvalidValue;
   if (!make_u8_map(&kmap, k_codes, a.key_rows, DI / 2, 128)) return cudaErrorInvalidValue;
+  if (!choose_cap<HI, DI, G>(a.k, &a.cap, &a.check)) return cudaErrorInvalidConfiguration;
   const size_t smem = L::bytes(a.cap);
-  if (smem > 227 * 1024 || a.cap > kEpiThreads * kCompactPer) return cudaErrorInvalidConfiguration;
+  if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
   auto kern = indexer_topk_kernel<HI, DI, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -645,8 +654,6 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
   a.key_rows = Nc > 0 ? Nc : 1;
   a.m = m;
   a.k = k;
-  a.cap = indexer_cap(k, G);
-  a.check = indexer_check(k, G);
   a.nsplit = 1;
   a.split_tiles = ceil_div(Nc > 0 ? Nc : 1, 128);
   a.idx = idx;
@@ -677,8 +684,6 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
   a.key_rows = (int64_t)B * Ncap;
   a.m = m;
   a.k = k;
-  a.cap = indexer_cap(k, 1);
-  a.check = indexer_check(k, 1);
   a.nsplit = nsplit;
   a.split_tiles = ceil_div(ceil_div(nvis_max > 0 ? nvis_max : 1, nsplit), 128);
   a.idx = nullptr;

@@ -129,6 +129,177 @@ __device__ void bitonic_desc(uint64_t* buf, int P, int tid, int bar_id) {
   }
 }
 
+// ------------------------------------------------------------------ warp-level selection
+// One warp owns one token's candidate buffer in shared memory; only __syncwarp
+// is needed.  `hist` is a per-warp shared-memory array of kWarpBins ints.
+constexpr int kWarpBins = 1024;
+
+__device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w < v ? w : v;
+  }
+  return v;
+}
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+// Order-preserving in-place compaction of buf[0..cnt) to the keys >= thr.
+__device__ __forceinline__ int warp_compact_ge(uint64_t* buf, int cnt, uint64_t thr, int lane) {
+  int out = 0;
+  for (int base = 0; base < cnt; base += 32) {
+    const int i = base + lane;
+    const uint64_t v = i < cnt ? buf[i] : 0;
+    const bool keep = i < cnt && v >= thr;
+    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    __syncwarp();
+    if (keep) buf[out + __popc(bal & ((1u << lane) - 1u))] = v;
+    out += __popc(bal);
+    __syncwarp();
+  }
+  return out;
+}
+
+// Given a histogram of kWarpBins counts (bin index increasing with the key),
+// the highest bin b such that count(bins >= b) >= need, and that count.
+__device__ __forceinline__ void warp_hist_cut(const int* hist, int need, int lane, int* bin_out, int* kept_out) {
+  // lane l sums bins [kWarpBins - 32(l+1), kWarpBins - 32l): descending order across lanes
+  constexpr int PER = kWarpBins / 32;
+  const int hi_bin = kWarpBins - PER * lane;  // exclusive
+  int tot = 0;
+#pragma unroll 8
+  for (int e = 1; e <= PER; ++e) tot += hist[hi_bin - e];
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int excl = incl - tot;
+  int bin = -1, kept = 0;
+  if (excl < need && need <= incl) {
+    int cum = excl;
+    for (int e = 1; e <= PER; ++e) {
+      cum += hist[hi_bin - e];
+      if (cum >= need) {
+        bin = hi_bin - e;
+        kept = cum;
+        break;
+      }
+    }
+  }
+  const uint32_t who = __ballot_sync(0xffffffffu, bin >= 0);
+  const int src = who ? __ffs(who) - 1 : 0;
+  *bin_out = __shfl_sync(0xffffffffu, bin, src);
+  *kept_out = __shfl_sync(0xffffffffu, kept, src);
+}
+
+// Threshold t such that exactly min(keep, cnt) keys of buf[0..cnt) are >= t:
+// radix select over the bits where the keys differ, kWarpBins-ary digits.
+__device__ uint64_t warp_exact_threshold(const uint64_t* buf, int cnt, int keep, int* hist, int lane) {
+  if (cnt <= keep) return 0;
+  uint64_t lo = ~0ull, hi = 0;
+  for (int i = lane; i < cnt; i += 32) {
+    const uint64_t v = buf[i];
+    lo = v < lo ? v : lo;
+    hi = v > hi ? v : hi;
+  }
+  lo = warp_min_u64(lo);
+  hi = warp_max_u64(hi);
+  // bits below `top` are undetermined; the prefix above is common to all keys
+  int top = 64 - __clzll(lo ^ hi);  // number of differing low bits (keys unique => top >= 1)
+  uint64_t prefix = lo & ~((top >= 64) ? ~0ull : ((1ull << top) - 1));
+  int need = keep;
+  while (top > 0) {
+    const int w = top >= 10 ? 10 : top;  // digit width (kWarpBins = 1024 bins)
+    const int shift = top - w;
+    const uint64_t pmask = (top >= 64) ? 0ull : ~((1ull << top) - 1);
+    for (int b = lane; b < kWarpBins; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int i = lane; i < cnt; i += 32) {
+      const uint64_t v = buf[i];
+      if ((v & pmask) == prefix) atomicAdd(&hist[(int)((v >> shift) & ((1ull << w) - 1))], 1);
+    }
+    __syncwarp();
+    int bin, kept;
+    warp_hist_cut(hist, need, lane, &bin, &kept);
+    __syncwarp();
+    const int in_bin = hist[bin];
+    need -= kept - in_bin;  // keys in higher bins are all kept
+    prefix |= (uint64_t)bin << shift;
+    top = shift;
+    __syncwarp();
+    if (in_bin == need) break;  // the whole bin is kept
+  }
+  return prefix;
+}
+
+// One-pass approximate cut: a score threshold keeping at least `keep` keys (all
+// keys of the threshold bin are kept).  Returns the number kept through *kept.
+// Falls back to the exact threshold when ties would keep more than `room`.
+__device__ uint64_t warp_approx_threshold(const uint64_t* buf, int cnt, int keep, int room, int* hist, int lane,
+                                          int* kept_out) {
+  if (cnt <= keep) {
+    *kept_out = cnt;
+    return 0;
+  }
+  uint32_t lo = 0xFFFFFFFFu, hi = 0;
+  for (int i = lane; i < cnt; i += 32) {
+    const uint32_t sc = (uint32_t)(buf[i] >> 32);
+    lo = sc < lo ? sc : lo;
+    hi = sc > hi ? sc : hi;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const uint32_t range = hi - lo;
+  if (range > 0) {
+    const int bits = 32 - __clz(range);
+    const int shift = bits > 10 ? bits - 10 : 0;
+    for (int b = lane; b < kWarpBins; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int i = lane; i < cnt; i += 32) atomicAdd(&hist[((uint32_t)(buf[i] >> 32) - lo) >> shift], 1);
+    __syncwarp();
+    int bin, kept;
+    warp_hist_cut(hist, keep, lane, &bin, &kept);
+    __syncwarp();
+    if (kept <= room) {
+      *kept_out = kept;
+      return (uint64_t)(lo + ((uint32_t)bin << shift)) << 32;
+    }
+  }
+  *kept_out = keep;
+  return warp_exact_threshold(buf, cnt, keep, hist, lane);
+}
+
+// Sort buf[0..P) descending (P a power of two, padding zeros), one warp.
+__device__ void warp_bitonic_desc(uint64_t* buf, int P, int lane) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = lane; i < (P >> 1); i += 32) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = (lo & size) == 0;
+        const uint64_t x = buf[lo], y = buf[hi];
+        if ((x < y) == desc) {
+          buf[lo] = y;
+          buf[hi] = x;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
 __host__ __device__ constexpr int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;
