@@ -359,6 +359,45 @@ def oracle_sample(wl, seconds=12.0, max_rows=4096):
                       % (wl.T // wl.m, done, wl.T, t_comp + t_rows)}
 
 
+EXTRA_CASES = ("hca_prefill", "csa_decode", "stack")
+
+
+def run_extra(name, csa, peaks, steps, warmup, T=None):
+    """One of the workloads reported under "workloads" (T overrides its length)."""
+    import dataclasses
+    if name == "hca_prefill":
+        w2 = inputs.HCA_PREFILL if T is None else dataclasses.replace(inputs.HCA_PREFILL, T=T)
+        r2 = run_hca_prefill(csa, w2, max(3, steps // 2), warmup)
+        hw = hca_prefill_work(w2)
+        return {"hca_prefill_T%d" % w2.T: {
+            "tokens_per_s": w2.T / (r2["ms"] * 1e-3), "ms_per_step": r2["ms"],
+            "attn_tflops": hw["attn_flop"] / (r2["phases"]["hca_attn"] * 1e-3) / 1e12,
+            "attn_frac_bf16": hw["attn_flop"] / (r2["phases"]["hca_attn"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "compress_gbs": hw["compress_bytes"] / (r2["phases"]["compress"] * 1e-3) / 1e9,
+            "phases_ms": r2["phases"], "status": r2["status"]}}
+    if name == "csa_decode":
+        w3 = inputs.CSA_DECODE if T is None else dataclasses.replace(inputs.CSA_DECODE, context=T)
+        r3 = run_decode(csa, w3, max(5, steps), warmup)
+        by = decode_bytes(w3)
+        return {"csa_decode_B%d_L%s" % (w3.batch, "1M" if w3.context == 1 << 20 else str(w3.context)): {
+            "us_per_step": r3["ms"] * 1e3, "algorithmic_bytes": by, "gbs": by / (r3["ms"] * 1e-3) / 1e9,
+            "frac_hbm": by / (r3["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], "status": r3["status"]}}
+    if name == "stack":
+        w4 = inputs.STACK if T is None else dataclasses.replace(inputs.STACK, T=T)
+        r4 = run_stack(csa, w4, 2, 1)
+        sw = stack_work(w4)
+        ph4 = r4["phases"]
+        method_ms = r4["ms"] - ph4.get("projection", 0.0)
+        return {"csa_hca_stack_T%d_chunk%d" % (w4.T, w4.chunk): {
+            "tokens_per_s": w4.T / (r4["ms"] * 1e-3), "ms_per_step": r4["ms"],
+            "tokens_per_s_without_projection": w4.T / (method_ms * 1e-3),
+            "indexer_tflops": sw["indexer_flop"] / (ph4["indexer_topk"] * 1e-3) / 1e12,
+            "csa_attn_tflops": sw["csa_attn_flop"] / (ph4["sparse_attn"] * 1e-3) / 1e12,
+            "hca_attn_tflops": sw["hca_attn_flop"] / (ph4["hca_attn"] * 1e-3) / 1e12,
+            "phases_ms": ph4, "projection_excluded_from_method": True}}
+    raise ValueError(name)
+
+
 # ----------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -368,12 +407,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the HCA and decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default="all", choices=("all", "csa_prefill") + EXTRA_CASES,
+                    help="all: the CSA prefill line plus the other workloads; csa_prefill: that line alone; "
+                         "otherwise one other workload alone, on one GPU (for profiling)")
+    ap.add_argument("--T", type=int, default=None,
+                    help="with --case: override the sequence length (the context length for csa_decode)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     wl = inputs.CSA_PREFILL
+    if args.case == "csa_prefill" and args.T is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, T=args.T)
 
     if args.impl == "reference":
         if rank != 0:
@@ -400,6 +447,13 @@ def main():
     import long_context_compressed_gated_b200 as csa
     csa.lib()
     peaks = load_peaks()
+    if args.case in EXTRA_CASES:
+        if rank == 0:
+            print(json.dumps({"case": args.case, "workloads": run_extra(args.case, csa, peaks, args.steps,
+                                                                         args.warmup, args.T)}), flush=True)
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return
     work = csa_prefill_work(wl)
 
     sampler = ClockSampler(local)
@@ -410,37 +464,10 @@ def main():
     e2e_ms = max_over_ranks(res["e2e_ms"], dist_on)
 
     extra = {}
-    if not args.no_extra and rank == 0:
-        w2 = inputs.HCA_PREFILL
-        r2 = run_hca_prefill(csa, w2, max(3, args.steps // 2), args.warmup)
-        hw = hca_prefill_work(w2)
-        extra["hca_prefill_T131072"] = {
-            "tokens_per_s": w2.T / (r2["ms"] * 1e-3), "ms_per_step": r2["ms"],
-            "attn_tflops": hw["attn_flop"] / (r2["phases"]["hca_attn"] * 1e-3) / 1e12,
-            "attn_frac_bf16": hw["attn_flop"] / (r2["phases"]["hca_attn"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            "compress_gbs": hw["compress_bytes"] / (r2["phases"]["compress"] * 1e-3) / 1e9,
-            "phases_ms": r2["phases"], "status": r2["status"]}
-        torch.cuda.empty_cache()
-        w3 = inputs.CSA_DECODE
-        r3 = run_decode(csa, w3, max(5, args.steps), args.warmup)
-        by = decode_bytes(w3)
-        extra["csa_decode_B16_L1M"] = {
-            "us_per_step": r3["ms"] * 1e3, "algorithmic_bytes": by, "gbs": by / (r3["ms"] * 1e-3) / 1e9,
-            "frac_hbm": by / (r3["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], "status": r3["status"]}
-        torch.cuda.empty_cache()
-        w4 = inputs.STACK
-        r4 = run_stack(csa, w4, 2, 1)
-        sw = stack_work(w4)
-        ph4 = r4["phases"]
-        method_ms = r4["ms"] - ph4.get("projection", 0.0)
-        extra["csa_hca_stack_T262144_chunk16384"] = {
-            "tokens_per_s": w4.T / (r4["ms"] * 1e-3), "ms_per_step": r4["ms"],
-            "tokens_per_s_without_projection": w4.T / (method_ms * 1e-3),
-            "indexer_tflops": sw["indexer_flop"] / (ph4["indexer_topk"] * 1e-3) / 1e12,
-            "csa_attn_tflops": sw["csa_attn_flop"] / (ph4["sparse_attn"] * 1e-3) / 1e12,
-            "hca_attn_tflops": sw["hca_attn_flop"] / (ph4["hca_attn"] * 1e-3) / 1e12,
-            "phases_ms": ph4, "projection_excluded_from_method": True}
-        torch.cuda.empty_cache()
+    if not args.no_extra and args.case == "all" and rank == 0:
+        for name in EXTRA_CASES:
+            extra.update(run_extra(name, csa, peaks, args.steps, args.warmup))
+            torch.cuda.empty_cache()
 
     ph = res["phases"]
     dominant = max(ph, key=ph.get)
@@ -467,7 +494,7 @@ def main():
         "dtype": "bf16+mxfp4", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "d": wl.d, "m": wl.m, "k": wl.k, "W": wl.W,
                    "HI": wl.HI, "dI": wl.dI, "sequences_per_gpu": 1, "parallelism": "independent sequences per GPU",
-                   "l2": "inputs larger than L2 (Q alone 512 MiB), no flush"},
+                   "l2": "inputs larger than L2 (Q alone %d MiB), no flush" % (wl.T * wl.H * wl.d * 2 >> 20)},
         "roofline": roof,
         "kernels": {"compress_ms": ph["compress"], "compress_gbs": comp_gbs,
                     "indexer_topk_ms": ph["indexer_topk"], "indexer_tflops": idx_tf,

@@ -100,9 +100,11 @@ cudaError_t upload_positions(int64_t* dst, const int64_t* host, int B, cudaStrea
 }
 
 // decode workspace: [header][pos B*8][idx B*k*4][cand B*nsplit*k*8]
+// Key ranges per decode row: as many as fill the GPU in one wave of
+// one-CTA-per-SM indexer blocks (a second partial wave would double the time).
 int decode_nsplit(int B, int64_t Ncap, int k) {
   int sms = 148;
-  int ns = (int)((2 * sms + B - 1) / B);
+  int ns = B > 0 ? sms / B : 1;
   const int64_t tiles = ceil_div(Ncap > 0 ? Ncap : 1, 128);
   if (ns > tiles) ns = (int)tiles;
   const int lim = 256 * 40 / k;  // merge capacity

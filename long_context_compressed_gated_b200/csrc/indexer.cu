@@ -176,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_cnt = reinterpret_cast<int*>(smem + L::off_cnt);
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L::off_thr);
   int* s_hist = reinterpret_cast<int*>(smem + L::off_hist);
-  int* s_sh = reinterpret_cast<int*>(smem + L::off_sh);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* full = bar;                 // [NST] producer -> MMA
   uint64_t* empty = bar + NST;          // [NST] MMA -> producer
@@ -337,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {  // issue from a converged warp (much cheaper than a lane-0 branch)
         const uint32_t d = tbase + (b ? kTmemD1 : 0u);
         const uint32_t sfa = tbase + kTmemSFA0 + 4 * b;
         asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sfa),
@@ -360,7 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // =========================== epilogue + selection (warps 2..9)
-    const int et = tid - 64;            // 0..255
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;   // which half of the token group
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -466,14 +464,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* buf = s_cand + (size_t)my_g * cap;
       int cnt = s_cnt[my_g];
       if (cnt > a.k) {
-        const uint64_t thr = topk::warp_exact_threshold(buf, cnt, a.k, my_hist, lane);
+        const uint64_t thr = topk::warp_select_threshold(buf, cnt, a.k, my_hist, lane);
         cnt = topk::warp_compact_ge(buf, cnt, thr, lane);
       }
-      const int P = topk::next_pow2(cnt > 1 ? cnt : 1);
-      for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
-      __syncwarp();
-      topk::warp_bitonic_desc(buf, P, lane);
       if (a.nsplit == 1) {
+        // final order: descending key (the per-range lists of a split search are
+        // merged and sorted by topk_merge_kernel instead)
+        const int P = topk::next_pow2(cnt > 1 ? cnt : 1);
+        for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
+        __syncwarp();
+        topk::warp_bitonic_desc(buf, P, lane);
         for (int q = lane; q < a.k; q += 32) {
           int32_t id = -1;
           float sc = -INFINITY;

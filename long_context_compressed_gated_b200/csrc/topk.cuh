@@ -131,8 +131,11 @@ __device__ void bitonic_desc(uint64_t* buf, int P, int tid, int bar_id) {
 
 // ------------------------------------------------------------------ warp-level selection
 // One warp owns one token's candidate buffer in shared memory; only __syncwarp
-// is needed.  `hist` is a per-warp shared-memory array of kWarpBins ints.
+// is needed.  `hist` is a per-warp shared-memory array of kWarpBins ints (16-byte
+// aligned).  Every pass over a buffer loads kBatch keys per lane before using
+// any of them, so a pass costs about one shared-memory latency per 32*kBatch keys.
 constexpr int kWarpBins = 1024;
+constexpr int kBatch = 8;
 
 __device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
 #pragma unroll
@@ -151,17 +154,90 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
   return v;
 }
 
+// Bitonic sort of one key per lane across the warp, descending by lane.
+__device__ __forceinline__ uint64_t warp_sort32_desc(uint64_t x, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t y = __shfl_xor_sync(0xffffffffu, x, stride);
+      const bool lower = (lane & stride) == 0;
+      const bool desc = (lane & size) == 0;
+      x = (lower == desc) ? (x > y ? x : y) : (x < y ? x : y);
+    }
+  }
+  return x;
+}
+
+__device__ __forceinline__ void warp_clear_hist(int* hist, int lane) {
+#pragma unroll
+  for (int b = 4 * lane; b < kWarpBins; b += 128) *reinterpret_cast<int4*>(hist + b) = make_int4(0, 0, 0, 0);
+}
+
+// Range of the score field (upper 32 bits) over buf[0..cnt), cnt > 0.
+__device__ __forceinline__ void warp_score_range(const uint64_t* buf, int cnt, int lane, uint32_t* lo_out,
+                                                 uint32_t* hi_out) {
+  uint32_t lo = 0xFFFFFFFFu, hi = 0;
+  for (int base = 0; base < cnt; base += 32 * kBatch) {
+    uint32_t v[kBatch];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int i = base + 32 * t + lane;
+      v[t] = (uint32_t)(buf[i < cnt ? i : 0] >> 32);  // buf[0] is a member: neutral for min and max
+    }
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      lo = v[t] < lo ? v[t] : lo;
+      hi = v[t] > hi ? v[t] : hi;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  *lo_out = lo;
+  *hi_out = hi;
+}
+
+// Histogram of bin(key) = ((score - lo) >> shift) over buf[0..cnt) (bins < kWarpBins).
+__device__ __forceinline__ void warp_score_hist(const uint64_t* buf, int cnt, uint32_t lo, int shift, int* hist,
+                                                int lane) {
+  warp_clear_hist(hist, lane);
+  __syncwarp();
+  for (int base = 0; base < cnt; base += 32 * kBatch) {
+    uint32_t v[kBatch];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int i = base + 32 * t + lane;
+      v[t] = (uint32_t)(buf[i < cnt ? i : 0] >> 32);
+    }
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t)
+      if (base + 32 * t + lane < cnt) atomicAdd(&hist[(v[t] - lo) >> shift], 1);
+  }
+  __syncwarp();
+}
+
 // Order-preserving in-place compaction of buf[0..cnt) to the keys >= thr.
 __device__ __forceinline__ int warp_compact_ge(uint64_t* buf, int cnt, uint64_t thr, int lane) {
   int out = 0;
-  for (int base = 0; base < cnt; base += 32) {
-    const int i = base + lane;
-    const uint64_t v = i < cnt ? buf[i] : 0;
-    const bool keep = i < cnt && v >= thr;
-    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-    __syncwarp();
-    if (keep) buf[out + __popc(bal & ((1u << lane) - 1u))] = v;
-    out += __popc(bal);
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = 0; base < cnt; base += 32 * kBatch) {
+    uint64_t v[kBatch];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int i = base + 32 * t + lane;
+      v[t] = i < cnt ? buf[i] : 0;  // 0 is below every threshold of a real key set
+    }
+    __syncwarp();  // stores below only reach positions already loaded
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const bool keep = v[t] >= thr && v[t] != 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (keep) buf[out + __popc(bal & lt)] = v[t];
+      out += __popc(bal);
+    }
     __syncwarp();
   }
   return out;
@@ -170,12 +246,20 @@ __device__ __forceinline__ int warp_compact_ge(uint64_t* buf, int cnt, uint64_t 
 // Given a histogram of kWarpBins counts (bin index increasing with the key),
 // the highest bin b such that count(bins >= b) >= need, and that count.
 __device__ __forceinline__ void warp_hist_cut(const int* hist, int need, int lane, int* bin_out, int* kept_out) {
-  // lane l sums bins [kWarpBins - 32(l+1), kWarpBins - 32l): descending order across lanes
-  constexpr int PER = kWarpBins / 32;
-  const int hi_bin = kWarpBins - PER * lane;  // exclusive
+  constexpr int PER = kWarpBins / 32;  // lane l holds bins [kWarpBins - PER(l+1), kWarpBins - PER l)
+  const int lo_bin = kWarpBins - PER * (lane + 1);
+  int c[PER];
+#pragma unroll
+  for (int q = 0; q < PER / 4; ++q) {
+    const int4 x = *reinterpret_cast<const int4*>(hist + lo_bin + 4 * q);
+    c[4 * q] = x.x;
+    c[4 * q + 1] = x.y;
+    c[4 * q + 2] = x.z;
+    c[4 * q + 3] = x.w;
+  }
   int tot = 0;
-#pragma unroll 8
-  for (int e = 1; e <= PER; ++e) tot += hist[hi_bin - e];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) tot += c[e];
   int incl = tot;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -186,12 +270,12 @@ __device__ __forceinline__ void warp_hist_cut(const int* hist, int need, int lan
   int bin = -1, kept = 0;
   if (excl < need && need <= incl) {
     int cum = excl;
-    for (int e = 1; e <= PER; ++e) {
-      cum += hist[hi_bin - e];
-      if (cum >= need) {
-        bin = hi_bin - e;
+#pragma unroll
+    for (int e = PER - 1; e >= 0; --e) {
+      cum += c[e];
+      if (bin < 0 && cum >= need) {
+        bin = lo_bin + e;
         kept = cum;
-        break;
       }
     }
   }
@@ -203,42 +287,100 @@ __device__ __forceinline__ void warp_hist_cut(const int* hist, int need, int lan
 
 // Threshold t such that exactly min(keep, cnt) keys of buf[0..cnt) are >= t:
 // radix select over the bits where the keys differ, kWarpBins-ary digits.
+// General fallback of warp_select_threshold (heavy score ties).
 __device__ uint64_t warp_exact_threshold(const uint64_t* buf, int cnt, int keep, int* hist, int lane) {
   if (cnt <= keep) return 0;
   uint64_t lo = ~0ull, hi = 0;
-  for (int i = lane; i < cnt; i += 32) {
-    const uint64_t v = buf[i];
-    lo = v < lo ? v : lo;
-    hi = v > hi ? v : hi;
+  for (int base = 0; base < cnt; base += 32 * kBatch) {
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int i = base + 32 * t + lane;
+      const uint64_t v = buf[i < cnt ? i : 0];
+      lo = v < lo ? v : lo;
+      hi = v > hi ? v : hi;
+    }
   }
   lo = warp_min_u64(lo);
   hi = warp_max_u64(hi);
   // bits below `top` are undetermined; the prefix above is common to all keys
-  int top = 64 - __clzll(lo ^ hi);  // number of differing low bits (keys unique => top >= 1)
+  int top = 64 - __clzll(lo ^ hi);  // keys unique and cnt >= 2 => top >= 1
   uint64_t prefix = lo & ~((top >= 64) ? ~0ull : ((1ull << top) - 1));
   int need = keep;
   while (top > 0) {
     const int w = top >= 10 ? 10 : top;  // digit width (kWarpBins = 1024 bins)
     const int shift = top - w;
     const uint64_t pmask = (top >= 64) ? 0ull : ~((1ull << top) - 1);
-    for (int b = lane; b < kWarpBins; b += 32) hist[b] = 0;
+    warp_clear_hist(hist, lane);
     __syncwarp();
-    for (int i = lane; i < cnt; i += 32) {
-      const uint64_t v = buf[i];
-      if ((v & pmask) == prefix) atomicAdd(&hist[(int)((v >> shift) & ((1ull << w) - 1))], 1);
+    for (int base = 0; base < cnt; base += 32 * kBatch) {
+      uint64_t v[kBatch];
+#pragma unroll
+      for (int t = 0; t < kBatch; ++t) {
+        const int i = base + 32 * t + lane;
+        v[t] = buf[i < cnt ? i : 0];
+      }
+#pragma unroll
+      for (int t = 0; t < kBatch; ++t)
+        if (base + 32 * t + lane < cnt && (v[t] & pmask) == prefix)
+          atomicAdd(&hist[(int)((v[t] >> shift) & ((1ull << w) - 1))], 1);
     }
     __syncwarp();
     int bin, kept;
     warp_hist_cut(hist, need, lane, &bin, &kept);
-    __syncwarp();
     const int in_bin = hist[bin];
+    __syncwarp();
     need -= kept - in_bin;  // keys in higher bins are all kept
     prefix |= (uint64_t)bin << shift;
     top = shift;
-    __syncwarp();
     if (in_bin == need) break;  // the whole bin is kept
   }
   return prefix;
+}
+
+// Exact threshold (as warp_exact_threshold) in one histogram pass over the
+// score range plus, when the boundary bin must be split, one gather of that
+// bin's keys (at most 32) and an in-register sort.
+__device__ uint64_t warp_select_threshold(const uint64_t* buf, int cnt, int keep, int* hist, int lane) {
+  if (cnt <= keep) return 0;
+  uint32_t lo, hi;
+  warp_score_range(buf, cnt, lane, &lo, &hi);
+  if (hi > lo) {
+    const int bits = 32 - __clz(hi - lo);
+    const int shift = bits > 10 ? bits - 10 : 0;
+    warp_score_hist(buf, cnt, lo, shift, hist, lane);
+    int bin, kept;
+    warp_hist_cut(hist, keep, lane, &bin, &kept);
+    const int in_bin = hist[bin];
+    const int need = keep - (kept - in_bin);  // 1 <= need <= in_bin
+    if (need == in_bin) return (uint64_t)(lo + ((uint32_t)bin << shift)) << 32;
+    if (in_bin <= 32) {
+      __syncwarp();
+      uint64_t* sc = reinterpret_cast<uint64_t*>(hist);  // 32 keys of scratch
+      int n = 0;
+      for (int base = 0; base < cnt; base += 32 * kBatch) {
+        uint64_t v[kBatch];
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) {
+          const int i = base + 32 * t + lane;
+          v[t] = buf[i < cnt ? i : 0];
+        }
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) {
+          const bool in = base + 32 * t + lane < cnt && (int)(((uint32_t)(v[t] >> 32) - lo) >> shift) == bin;
+          const uint32_t bal = __ballot_sync(0xffffffffu, in);
+          if (in) sc[n + __popc(bal & ((1u << lane) - 1u))] = v[t];
+          n += __popc(bal);
+        }
+      }
+      __syncwarp();
+      uint64_t x = lane < in_bin ? sc[lane] : 0;
+      __syncwarp();
+      x = warp_sort32_desc(x, lane);
+      return __shfl_sync(0xffffffffu, x, need - 1);
+    }
+    __syncwarp();
+  }
+  return warp_exact_threshold(buf, cnt, keep, hist, lane);
 }
 
 // One-pass approximate cut: a score threshold keeping at least `keep` keys (all
@@ -250,25 +392,12 @@ __device__ uint64_t warp_approx_threshold(const uint64_t* buf, int cnt, int keep
     *kept_out = cnt;
     return 0;
   }
-  uint32_t lo = 0xFFFFFFFFu, hi = 0;
-  for (int i = lane; i < cnt; i += 32) {
-    const uint32_t sc = (uint32_t)(buf[i] >> 32);
-    lo = sc < lo ? sc : lo;
-    hi = sc > hi ? sc : hi;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  const uint32_t range = hi - lo;
-  if (range > 0) {
-    const int bits = 32 - __clz(range);
+  uint32_t lo, hi;
+  warp_score_range(buf, cnt, lane, &lo, &hi);
+  if (hi > lo) {
+    const int bits = 32 - __clz(hi - lo);
     const int shift = bits > 10 ? bits - 10 : 0;
-    for (int b = lane; b < kWarpBins; b += 32) hist[b] = 0;
-    __syncwarp();
-    for (int i = lane; i < cnt; i += 32) atomicAdd(&hist[((uint32_t)(buf[i] >> 32) - lo) >> shift], 1);
-    __syncwarp();
+    warp_score_hist(buf, cnt, lo, shift, hist, lane);
     int bin, kept;
     warp_hist_cut(hist, keep, lane, &bin, &kept);
     __syncwarp();
@@ -278,21 +407,41 @@ __device__ uint64_t warp_approx_threshold(const uint64_t* buf, int cnt, int keep
     }
   }
   *kept_out = keep;
-  return warp_exact_threshold(buf, cnt, keep, hist, lane);
+  return warp_select_threshold(buf, cnt, keep, hist, lane);
 }
 
-// Sort buf[0..P) descending (P a power of two, padding zeros), one warp.
+// Sort buf[0..P) descending (P a power of two, padding zeros), one warp.  Each
+// compare-exchange stage loads a batch of pairs per lane before swapping them.
 __device__ void warp_bitonic_desc(uint64_t* buf, int P, int lane) {
+  if (P <= 32) {
+    uint64_t x = lane < P ? buf[lane] : 0;
+    __syncwarp();
+    x = warp_sort32_desc(x, lane);
+    if (lane < P) buf[lane] = x;
+    __syncwarp();
+    return;
+  }
+  const int half = P >> 1;
   for (int size = 2; size <= P; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < (P >> 1); i += 32) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint64_t x = buf[lo], y = buf[hi];
-        if ((x < y) == desc) {
-          buf[lo] = y;
-          buf[hi] = x;
+      for (int base = 0; base < half; base += 32 * kBatch) {
+        uint64_t x[kBatch], y[kBatch];
+        int lo[kBatch];
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) {
+          const int i = base + 32 * t + lane;
+          const int ii = i < half ? i : 0;
+          lo[t] = 2 * ii - (ii & (stride - 1));
+          x[t] = buf[lo[t]];
+          y[t] = buf[lo[t] + stride];
+        }
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) {
+          const bool desc = (lo[t] & size) == 0;
+          if (base + 32 * t + lane < half && (x[t] < y[t]) == desc) {
+            buf[lo[t]] = y[t];
+            buf[lo[t] + stride] = x[t];
+          }
         }
       }
       __syncwarp();

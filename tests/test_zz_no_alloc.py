@@ -67,8 +67,8 @@ def test_noalloc_matches_workspace_decode_twice():
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
     csa, L = _lib()
-    # B = 256 sequences with k = 2048 needs more than the 8 MiB static scratch
-    B = 256
+    # B = 1024 sequences with k = 2048 need more than the 8 MiB static scratch
+    B = 1024
     need = csa.lib().csa_decode_workspace_bytes(B, 1 << 20, 64, 128, 16, 128, 2048, 128)
     assert need > (8 << 20)
     fake = ctypes.c_void_p(0x1000)
