@@ -78,15 +78,6 @@ __device__ __forceinline__ float2 scale_sub2(float a, float b, float c, float m)
   return r;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-// Arrive on `bar` once all prior cp.async of this thread have landed (counts as one arrival).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 }  // namespace
 
 // TMA descriptors of one launch: 128-row boxes (64-column halves, 128B swizzle).
@@ -294,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       mbar_wait(&s_free[st], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tcgen05 (async proxy) reads
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {  // converged-warp issue
         const int width = s_tiles[i].width;
         const uint32_t sk = smem_u32(s_k + (size_t)st * L::kTileBytes);
         const uint32_t d = tbase + (st ? kTmemS1 : kTmemS0);
@@ -318,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       mbar_wait(&v_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       fence_proxy_async_smem();
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {
         const int width = s_tiles[i].width;
         const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
         for (int ks = 0; ks < width / 16; ++ks) {

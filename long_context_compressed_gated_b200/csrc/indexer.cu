@@ -44,6 +44,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kMagicBits = 0x48400000u;  // bit pattern of 196608.0f
+constexpr int kCheckWarp = 6;                // epilogue warp that range-checks the key scales
 constexpr int kHalfBar0 = 1;                  // named barriers 1, 2: the four warps of each half
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -138,9 +139,8 @@ struct IndexerSmem {
   static constexpr int kABytes = 128 * kRowBytes;  // multiple of 1024
   static constexpr size_t off_q = 0;
   static constexpr size_t off_a = off_q + kQBytes;
-  static constexpr size_t off_sf = off_a + (size_t)kStages * kABytes;
-  static constexpr size_t off_sfraw = off_sf + (size_t)kStages * 512;  // scales as loaded, [128 rows][DI/32]
-  static constexpr size_t off_ma = off_sfraw + (size_t)kStages * 512;
+  static constexpr size_t off_sf = off_a + (size_t)kStages * kABytes;  // key scales, tcgen05.cp layout
+  static constexpr size_t off_ma = off_sf + (size_t)kStages * 512;
   static constexpr size_t off_mb = off_ma + 4096;
   static constexpr size_t off_w2 = off_mb + (size_t)N * 32;
   static constexpr size_t off_sumw = off_w2 + (size_t)N * 4;
@@ -153,6 +153,38 @@ struct IndexerSmem {
   static constexpr size_t off_cand = ((off_tslot + 16 + 15) / 16) * 16;
   static size_t bytes(int cap) { return off_cand + (size_t)G * cap * 8 + 1024; }
 };
+
+// Sort a token's final candidates (cnt <= 32*R) in registers and write idx /
+// scores in rank order, padding with -1 / -inf up to k.
+template <int R>
+__device__ __forceinline__ void write_sorted(const uint64_t* buf, int cnt, const IndexerArgs& a, int64_t r, int lane) {
+  uint64_t v[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int e = i * 32 + lane;
+    v[i] = e < cnt ? buf[e] : 0;
+  }
+  topk::warp_sort_regs_desc<R>(v, lane);
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int q = i * 32 + lane;
+    if (q < a.k) {
+      int32_t id = -1;
+      float sc = -INFINITY;
+      if (q < cnt) {
+        id = (int32_t)topk::key_index(v[i]);
+        sc = (float)topk::key_score(v[i]) * (1.0f / 128.0f);
+      }
+      a.idx[r * a.k + q] = id;
+      if (a.scores) a.scores[r * a.k + q] = sc;
+    }
+  }
+  // rows beyond 32*R (k > 32*R with cnt <= 32*R) are padding
+  for (int q = 32 * R + lane; q < a.k; q += 32) {
+    a.idx[r * a.k + q] = -1;
+    if (a.scores) a.scores[r * a.k + q] = -INFINITY;
+  }
+}
 
 template <int HI, int DI, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -168,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* s_q = smem + L::off_q;
   uint8_t* s_a = smem + L::off_a;
   uint8_t* s_sf = smem + L::off_sf;
-  uint8_t* s_sfraw = smem + L::off_sfraw;
   uint8_t* s_ma = smem + L::off_ma;
   uint8_t* s_mb = smem + L::off_mb;
   int* s_w2 = reinterpret_cast<int*>(smem + L::off_w2);
@@ -214,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- setup
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 2);
+      mbar_init(&full[s], 1 + 32);  // TMA transaction arrival + one per producer lane (scales)
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -269,31 +300,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&empty[s], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       const int64_t j0 = j_begin + (int64_t)it * 128;
       const int64_t row0k = key_row_base + j0;
-      constexpr uint32_t kSfRow = DI / 32;  // scale bytes per key row
-      // whole tile inside the kI tensor: scales by one bulk copy; else plain loads
-      const bool bulk = row0k + 128 <= a.key_rows;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], L::kABytes + (bulk ? 128 * kSfRow : 0u));
+        mbar_arrive_expect_tx(&full[s], L::kABytes);
         tma_load_2d(s_a + (size_t)s * L::kABytes, &kmap, &full[s], 0, (int)row0k);
-        if (bulk) bulk_load(s_sfraw + (size_t)s * 512, a.k_scales + row0k * kSfRow, 128 * kSfRow, &full[s]);
       }
-      if (!bulk) {
-        for (int r = lane; r < 128; r += 32) {
-          const int64_t row = row0k + r;
-          if (DI == 128) {
-            const uint32_t w = row < a.key_rows ? *reinterpret_cast<const uint32_t*>(a.k_scales + row * 4)
-                                                 : 0x7F7F7F7Fu;
-            reinterpret_cast<uint32_t*>(s_sfraw + (size_t)s * 512)[r] = w;
-          } else {
-            const uint16_t w = row < a.key_rows ? *reinterpret_cast<const uint16_t*>(a.k_scales + row * 2)
-                                                : (uint16_t)0x7F7F;
-            reinterpret_cast<uint16_t*>(s_sfraw + (size_t)s * 512)[r] = w;
-          }
+      // key scales straight into the tcgen05.cp 32x128b layout: lane l holds the
+      // scale words of rows l, l+32, l+64, l+96 (rows past the tensor read as 0)
+      const uint32_t sdst = smem_u32(s_sf + (size_t)s * 512) + lane * 16;
+      if (DI == 128) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int64_t row = row0k + lane + 32 * c;
+          const bool in = row < a.key_rows;
+          cp_async4(sdst + 4 * c, a.k_scales + (in ? row : 0) * 4, in ? 4u : 0u);
         }
-        __syncwarp();
+        cp_async_arrive(&full[s]);
+      } else {
+        // two scale bytes per row: plain loads, padded to the 4-byte word
+        uint32_t wv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int64_t row = row0k + lane + 32 * c;
+          wv[c] = row < a.key_rows ? (uint32_t)*reinterpret_cast<const uint16_t*>(a.k_scales + row * 2) | 0x7F7F0000u
+                                   : 0x7F7F7F7Fu;
+        }
+        *reinterpret_cast<uint4*>(s_sf + (size_t)s * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        fence_proxy_async_smem();  // generic-proxy writes -> tcgen05.cp
+        mbar_arrive(&full[s]);
       }
-      if (lane == 0) mbar_arrive(&full[s]);
     }
+    cp_async_wait_all();
   } else if (warp == 1) {
     // =========================== MMA issuer
     if (ntiles > 0) {
@@ -310,31 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dph = (it >> 1) & 1;
       if (!mbar_wait(&dempty[b], dph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       if (!mbar_wait(&full[s], ph, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
-      {
-        // scales -> tcgen05.cp 32x128b layout: lane l holds rows l, l+32, l+64, l+96
-        const int64_t j0 = j_begin + (int64_t)it * 128;
-        uint32_t wv[4];
-        bool bad = false;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int r = lane + 32 * c;
-          uint32_t w;
-          if (DI == 128) w = reinterpret_cast<const uint32_t*>(s_sfraw + (size_t)s * 512)[r];
-          else w = (uint32_t)reinterpret_cast<const uint16_t*>(s_sfraw + (size_t)s * 512)[r] | 0x7F7F0000u;
-          if (j0 + r < j_end) {
-#pragma unroll
-            for (int q = 0; q < DI / 32; ++q) {
-              const uint32_t e = (w >> (8 * q)) & 255u;
-              bad |= (e < 125u) | (e > 128u);
-            }
-          }
-          wv[c] = w;
-        }
-        if (bad) report(a.status, CSA_ERR_RANGE);
-        *reinterpret_cast<uint4*>(s_sf + (size_t)s * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
+      fence_proxy_async_smem();  // cp.async-written scales -> tcgen05.cp (async proxy)
       tc_fence_after();
       if (elect_one()) {  // issue from a converged warp (much cheaper than a lane-0 branch)
         const uint32_t d = tbase + (b ? kTmemD1 : 0u);
@@ -410,6 +422,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dph = (it >> 1) & 1;
       if (!mbar_wait(&dfull[b], dph, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       tc_fence_after();
+      if (warp == kCheckWarp) {
+        // exactness precondition on this tile's key scales (rows below j_end), read
+        // back from the replicated TMEM copy the MMA used
+        uint32_t sw[4];
+        tmem_ld4(tbase + lane_base + kTmemSFA0 + 4 * b, sw);
+        tmem_wait_ld();
+        const int64_t j0 = j_begin + (int64_t)it * 128;
+        bool bad = false;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (j0 + lane + 32 * c < j_end) {
+#pragma unroll
+            for (int q = 0; q < DI / 32; ++q) bad |= ((sw[c] >> (8 * q)) & 255u) - 125u > 3u;
+          }
+        if (bad) report(a.status, CSA_ERR_RANGE);
+      }
       const uint32_t dcol = tbase + lane_base + (b ? kTmemD1 : 0u);
       uint32_t acc[G];  // arithmetic mod 2^32: the true head sum fits in int32
 #pragma unroll
@@ -470,20 +498,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (a.nsplit == 1) {
         // final order: descending key (the per-range lists of a split search are
         // merged and sorted by topk_merge_kernel instead)
-        const int P = topk::next_pow2(cnt > 1 ? cnt : 1);
-        for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
-        __syncwarp();
-        topk::warp_bitonic_desc(buf, P, lane);
-        for (int q = lane; q < a.k; q += 32) {
-          int32_t id = -1;
-          float sc = -INFINITY;
-          if (q < cnt) {
-            const uint64_t key = buf[q];
-            id = (int32_t)topk::key_index(key);
-            sc = (float)topk::key_score(key) * (1.0f / 128.0f);
+        if (cnt <= 512) write_sorted<16>(buf, cnt, a, r, lane);
+        else if (cnt <= 1024) write_sorted<32>(buf, cnt, a, r, lane);
+        else {
+          const int P = topk::next_pow2(cnt);
+          for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
+          __syncwarp();
+          topk::warp_bitonic_desc(buf, P, lane);
+          for (int q = lane; q < a.k; q += 32) {
+            int32_t id = -1;
+            float sc = -INFINITY;
+            if (q < cnt) {
+              const uint64_t key = buf[q];
+              id = (int32_t)topk::key_index(key);
+              sc = (float)topk::key_score(key) * (1.0f / 128.0f);
+            }
+            a.idx[r * a.k + q] = id;
+            if (a.scores) a.scores[r * a.k + q] = sc;
           }
-          a.idx[r * a.k + q] = id;
-          if (a.scores) a.scores[r * a.k + q] = sc;
         }
       } else {
         uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
@@ -578,7 +610,8 @@ static bool choose_cap(int k, int* cap, int* check) {
   for (int c = 4; c >= 1; c >>= 1) {
     const int need = k + 128 * c > p ? k + 128 * c : p;
     if (budget >= need) {
-      int want = k + (k > 128 * c ? k : 128 * c) + 128 * c;  // room for ~k more before a cut-back
+      int want = 4 * k + 128 * c;  // cut-backs rare: room for several k between them
+      if (want < 4096) want = 4096;
       if (want < need) want = need;
       *cap = (want < budget ? want : budget) & ~127;
       if (*cap < need) *cap = ((need + 127) / 128) * 128;

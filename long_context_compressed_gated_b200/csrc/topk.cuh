@@ -449,6 +449,61 @@ __device__ void warp_bitonic_desc(uint64_t* buf, int P, int lane) {
   }
 }
 
+// Register-resident bitonic sort of 32*R keys, descending; element e = r*32 + lane
+// lives in v[r] of lane `lane`.  Strides below 32 exchange across lanes by
+// shuffles, strides of 32 and more swap registers within a lane (the register
+// pair is a compile-time choice per case).  Pad with zeros to fill 32*R.
+template <int R>
+__device__ __forceinline__ void sort_within_lane(uint64_t (&v)[R], int j, int size) {
+  // partner of register r is r ^ j (j = stride / 32, a power of two below R)
+#define CSA_WITHIN_CASE(J)                                                \
+  case J:                                                                 \
+    _Pragma("unroll") for (int r = 0; r < R; ++r) {                       \
+      if ((r & J) == 0 && (r ^ J) < R) {                                  \
+        const bool desc = ((r * 32) & size) == 0;                         \
+        const uint64_t x = v[r], y = v[r ^ J];                            \
+        const bool sw = (x < y) == desc;                                  \
+        v[r] = sw ? y : x;                                                \
+        v[r ^ J] = sw ? x : y;                                            \
+      }                                                                   \
+    }                                                                     \
+    break;
+  switch (j) {
+    CSA_WITHIN_CASE(1)
+    CSA_WITHIN_CASE(2)
+    CSA_WITHIN_CASE(4)
+    CSA_WITHIN_CASE(8)
+    CSA_WITHIN_CASE(16)
+    CSA_WITHIN_CASE(32)
+    default: break;
+  }
+#undef CSA_WITHIN_CASE
+}
+
+template <int R>
+__device__ __forceinline__ void warp_sort_regs_desc(uint64_t (&v)[R], int lane) {
+  constexpr int P = 32 * R;
+#pragma unroll 1
+  for (int size = 2; size <= P; size <<= 1) {
+#pragma unroll 1
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {
+        sort_within_lane<R>(v, stride >> 5, size);
+      } else {
+        const bool lower = (lane & stride) == 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint64_t y = __shfl_xor_sync(0xffffffffu, v[r], stride);
+          const bool desc = (((r << 5) | lane) & size) == 0;
+          const bool keep_max = lower == desc;
+          const bool gt = v[r] > y;
+          v[r] = (gt == keep_max) ? v[r] : y;
+        }
+      }
+    }
+  }
+}
+
 __host__ __device__ constexpr int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;
