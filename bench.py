@@ -172,7 +172,9 @@ def run_csa_prefill(csa, wl, steps, warmup, dist_on, rank):
     Vc = torch.empty_like(Kc)
     idx = torch.empty(T, wl.k, dtype=torch.int32, device="cuda")
     O = torch.empty_like(d["Q"])
-    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    ws_bytes = max(csa.lib().csa_indexer_topk_workspace_bytes(T, T // wl.m, wl.HI, wl.dI, wl.k),
+                   csa.lib().csa_sparse_attn_workspace_bytes(T, H, wl.d, wl.k, wl.W))
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
     timer = Timer(["compress", "indexer_topk", "sparse_attn"])
 
     def step(ev=None):

@@ -16,13 +16,13 @@ cudaError_t launch_compress(const void* K, const void* V, const void* Z, const f
                             void* Kc, void* Vc, cudaStream_t stream);
 cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
                                    const uint8_t* k_codes, const uint8_t* k_scales, int64_t T, int64_t t0, int64_t Nc,
-                                   int HI, int DI, int m, int k, int32_t* idx, float* scores, int* status,
-                                   cudaStream_t stream);
+                                   int HI, int DI, int m, int k, int32_t* idx, float* scores, uint64_t* cand,
+                                   int* cand_cnt, int* status, cudaStream_t stream);
 cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
                                   const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
                                   int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
-                                  uint64_t* cand, int32_t* idx, float* scores, uint64_t* keys_out, int* status,
-                                  cudaStream_t stream);
+                                  uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
+                                  int* status, cudaStream_t stream);
 
 
 
@@ -165,7 +165,12 @@ int csa_compress(const void* K, const void* V, const void* Z, const float* B, in
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
-size_t csa_indexer_topk_workspace_bytes(int64_t, int64_t, int, int, int) { return kWorkspaceHeader; }
+// Indexer workspace: status header, then per query row the k selected keys
+// (uint64) and their count, which the finalize pass sorts into idx / scores.
+size_t csa_indexer_topk_workspace_bytes(int64_t T, int64_t, int, int, int k) {
+  if (T <= 0 || k <= 0) return kWorkspaceHeader;
+  return kWorkspaceHeader + align256((size_t)T * k * 8) + align256((size_t)T * 4);
+}
 
 int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
                      const uint8_t* kI_codes, const uint8_t* kI_scales, int64_t T, int64_t t0, int64_t Nc, int HI,
@@ -173,15 +178,18 @@ int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const ui
                      csa_stream_t stream) {
   if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || k < 1 || k > 2048) return CSA_ERR_INVALID_ARG;
   if (!valid_HI(HI) || (dI != 64 && dI != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
-  int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
+  int rc = check_ws(workspace, workspace_bytes, csa_indexer_topk_workspace_bytes(T, Nc, HI, dI, k));
   if (rc) return rc;
   if (T == 0) return CSA_OK;
   rc = check_ptrs(qI_codes, qI_scales, w_codes, idx);
   if (rc) return rc;
   if (Nc > 0 && (rc = check_ptrs(kI_codes, kI_scales))) return rc;
   if ((rc = check_opt(scores))) return rc;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader);
+  int* cand_cnt = reinterpret_cast<int*>(w + kWorkspaceHeader + align256((size_t)T * k * 8));
   cudaError_t e = launch_indexer_prefill(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, T, t0, Nc, HI, dI, m, k,
-                                         idx, scores, status_word(workspace), (cudaStream_t)stream);
+                                         idx, scores, cand, cand_cnt, status_word(workspace), (cudaStream_t)stream);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
@@ -278,7 +286,7 @@ size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int, int, int, int, int k
   if (B <= 0 || k <= 0) return kWorkspaceHeader;
   const int ns = decode_nsplit(B, Ncap, k);
   return kWorkspaceHeader + align256((size_t)B * 8) + align256((size_t)B * k * 4) +
-         align256((size_t)B * ns * k * 8);
+         align256((size_t)B * ns * k * 8) + align256((size_t)B * ns * 4);
 }
 
 int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
@@ -313,13 +321,14 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   int32_t* idx_ws = reinterpret_cast<int32_t*>(w + kWorkspaceHeader + align256((size_t)B * 8));
   uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader + align256((size_t)B * 8) +
                                                align256((size_t)B * k * 4));
+  int* cand_cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cand) + align256((size_t)B * ns * k * 8));
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = upload_positions(pos_dev, pos, B, s);
   if (e != cudaSuccess) return cuda_fail(e);
   int32_t* sel = idx ? idx : idx_ws;
   if (Ncap > 0) {
     e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, nvis_max, Ncap, HI, dI,
-                              m, k, ns, cand, sel, scores, nullptr, status_word(workspace), s);
+                              m, k, ns, cand, cand_cnt, sel, scores, nullptr, status_word(workspace), s);
     if (e != cudaSuccess) return cuda_fail(e);
   } else {
     e = cudaMemsetAsync(sel, 0xFF, (size_t)B * k * 4, s);

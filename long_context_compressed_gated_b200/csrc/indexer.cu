@@ -9,24 +9,29 @@
 // Design (one CTA = G query tokens x one range of compressed entries):
 //  * tcgen05.mma kind::mxf4 (packed E2M1 x E2M1, UE8M0 scale per 32 elements):
 //    A = 128 compressed keys (TMEM lanes), B = the G*HI (token, head) rows of
-//    the query group (TMEM columns), K = dI.  A third MMA with constant
+//    the query group (TMEM columns), K = dI.  One more MMA with constant
 //    operands (all 1.0 x all 6.0 * 2^9) adds 196608 = 1.5*2^17 to every
 //    accumulator, which pins the fp32 exponent so the raw bit pattern of the
 //    accumulator minus that of 196608 is the exact dot product in units of
 //    2^-6 (valid while every scale exponent lies in [-2, 1]).
 //  * Epilogue (8 warps, two per TMEM lane quarter): per key lane, per token,
-//        acc += w2[h] * max(bits, bits(196608))          (int32, exact)
+//        acc += w2[h] * max(bits, bits(196608))          (uint32, exact)
 //    then I*2^7 = acc - bits(196608)*sum_h w2[h] (mod 2^32), with w2 = 2*w.
-//    Ranking uses the exact integer; no floating-point head sum.
+//    Ranking uses the exact integer; no floating-point head sum.  With G >= 2
+//    the two halves of the epilogue own G/2 tokens each and read every tile;
+//    with G = 1 (decode) they take alternate tiles.
 //  * Streaming top-k per token: candidates whose 64-bit key (score, -j) clears
 //    the token's running threshold are appended to a shared-memory buffer; when
-//    the buffer could overflow on the next tile it is cut back to the k best by
-//    radix select, which also raises the threshold.  At the end the k best are
-//    bitonic-sorted (score desc, j asc) and written out.
-//  * Warp roles: warp 0 TMA producer (key codes) + scale-factor staging, warp 1
-//    TMEM allocation and MMA issue (scales copied to TMEM with tcgen05.cp),
-//    warps 2..9 epilogue + selection.  Key tiles are 4-stage pipelined;
-//    accumulators double-buffered in TMEM.
+//    the buffer could overflow before the next meeting it is cut back (one-pass
+//    histogram threshold keeping >= k), which also raises the threshold.  At the
+//    end the exact k best of the CTA's key range are selected and written out
+//    unsorted; topk_finalize_kernel (one warp per row) merges the ranges of a
+//    row, selects its k best and sorts them (score desc, j asc).
+//  * Warp roles: warp 0 TMA producer (key codes; scales by cp.async straight
+//    into the tcgen05.cp layout), warp 1 TMEM allocation and MMA issue, warps
+//    2..9 epilogue + selection.  Key tiles are 4- or 8-stage pipelined; NB
+//    accumulator buffers in TMEM (3 for 128-column groups, 8 for decode) keep
+//    the MMAs ahead of the epilogue.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -39,25 +44,34 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kMaxCols = 224;       // N of the MMA: G*HI rounded up to 16
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kMagicBits = 0x48400000u;  // bit pattern of 196608.0f
-constexpr int kCheckWarp = 6;                // epilogue warp that range-checks the key scales
 constexpr int kHalfBar0 = 1;                  // named barriers 1, 2: the four warps of each half
+constexpr int kEpiBar = 3;                    // named barrier 3: all epilogue warps
 constexpr size_t kSmemLimit = 227 * 1024;
 
-// TMEM column map (512 allocated): D[0] at 0, D[1] at 256; scale factors at 224..
-constexpr uint32_t kTmemD1 = 256;
-constexpr uint32_t kTmemSFA0 = 224;   // 4 columns per buffer (x2)
-constexpr uint32_t kTmemSFB = 232;    // 8 columns
-constexpr uint32_t kTmemMagicSFA = 240;
-constexpr uint32_t kTmemMagicSFB = 244;  // 8 columns
+// TMEM column map (512 allocated): NB accumulator buffers of N columns from 0
+// (at most 448 columns), scale factors from column 448.
+constexpr uint32_t kTmemSF = 448;
 
+// Tokens per CTA (prefill): 128 accumulator columns (HI >= 16), so that three
+// buffers fit in TMEM; an even count, split between the two epilogue halves.
 template <int HI>
 struct Geometry {
-  static constexpr int G = kMaxCols / HI < 8 ? kMaxCols / HI : 8;  // tokens per CTA (prefill)
+  static constexpr int G = HI >= 16 ? 128 / HI : 8;
+};
+
+template <int HI, int G>
+struct TileShape {
+  static constexpr int N = ((G * HI + 15) / 16) * 16;      // MMA N (accumulator columns)
+  static constexpr int NB = 448 / N < 8 ? 448 / N : 8;      // accumulator buffers
+  static constexpr uint32_t sfa(int b) { return kTmemSF + 4 * b; }  // key scales, 4 columns each
+  static constexpr uint32_t kSFB = kTmemSF + 32;                    // query scales, 8 columns
+  static constexpr uint32_t kMagicSFA = kTmemSF + 40;              // 4 columns
+  static constexpr uint32_t kMagicSFB = kTmemSF + 44;              // 8 columns
+  static_assert(NB >= 2 && NB * N <= 448, "TMEM budget");
 };
 
 __device__ __forceinline__ int e2m1_times2(uint32_t code) {
@@ -69,45 +83,39 @@ __device__ __forceinline__ int e2m1_times2(uint32_t code) {
 
 }  // namespace
 
-// Head sums of this thread's key lane for the tokens of one half of the group:
-// acc[g] += w2[h] * max(bits(D[g*HI+h]), bits(196608)) over the half's columns,
-// loading up to 64 TMEM columns per wait.  NP partial sums per token break the
-// dependent multiply-add chain when a token has many heads.
-template <int HI, int G, int HALF>
-__device__ __forceinline__ void head_sums(uint32_t dcol, const int* s_w2, uint32_t (&acc)[G]) {
-  constexpr int G0 = (G + 1) / 2;
-  constexpr int c_lo = (HALF ? G0 : 0) * HI;
-  constexpr int c_hi = (HALF ? G : G0) * HI;
+// Head sums of this thread's key lane over the warp's CW accumulator columns
+// (tokens 0..CW/HI-1 of its half): acc[t] += w2[c] * max(bits(D[c]), bits(196608)).
+// The weights sit in registers; TMEM is read 32 columns at a time, each load
+// overlapping the arithmetic on the previous batch.  NP partial sums per token
+// break the dependent multiply-add chain when a token has many heads.
+template <int HI, int CW>
+__device__ __forceinline__ void head_sums(uint32_t dcol, const int (&w)[CW], uint32_t (&acc)[(CW + HI - 1) / HI]) {
+  constexpr int T = (CW + HI - 1) / HI;
   constexpr int NP = HI >= 32 ? 4 : 1;
-  uint32_t part[G][NP];
+  constexpr int NBATCH = (CW + 31) / 32;
+  uint32_t part[T][NP];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int t = 0; t < T; ++t)
 #pragma unroll
-    for (int p = 0; p < NP; ++p) part[g][p] = 0u;
+    for (int p = 0; p < NP; ++p) part[t][p] = 0u;
+  uint32_t v[2][32];
+  if (CW >= 32) tmem_ld32p(dcol, v[0]);
+  else tmem_ld16p(dcol, v[0]);
+  tmem_wait_ld_regs32(v[0]);
 #pragma unroll
-  for (int b0 = c_lo; b0 < c_hi; b0 += 64) {
-    uint32_t v[64];
+  for (int bi = 0; bi < NBATCH; ++bi) {
+    if (bi + 1 < NBATCH) tmem_ld32p(dcol + 32 * (bi + 1), v[(bi + 1) & 1]);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (b0 + 16 * q < c_hi) tmem_ld16p(dcol + b0 + 16 * q, v + 16 * q);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 64; i += 4) {
-      if (b0 + i < c_hi) {
-        const int4 w = *reinterpret_cast<const int4*>(s_w2 + b0 + i);
-        const int ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = b0 + i + q;
-          part[col / HI][col % NP] += (uint32_t)ww[q] * (uint32_t)max((int)v[i + q], (int)kMagicBits);
-        }
-      }
+    for (int i = 0; i < 32; ++i) {
+      const int col = 32 * bi + i;
+      if (col < CW) part[col / HI][col % NP] += (uint32_t)w[col] * (uint32_t)max((int)v[bi & 1][i], (int)kMagicBits);
     }
+    if (bi + 1 < NBATCH) tmem_wait_ld_regs32(v[(bi + 1) & 1]);
   }
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int t = 0; t < T; ++t)
 #pragma unroll
-    for (int p = 0; p < NP; ++p) acc[g] += part[g][p];
+    for (int p = 0; p < NP; ++p) acc[t] += part[t][p];
 }
 
 struct IndexerArgs {
@@ -124,15 +132,16 @@ struct IndexerArgs {
   int check;                // tiles between buffer cut-backs (cap >= k + 128 * check)
   int nsplit;               // key ranges per query group
   int64_t split_tiles;      // 128-key tiles per range
-  int32_t* idx;             // [rows, k]      (nsplit == 1)
-  float* scores;            // [rows, k]      (nsplit == 1, nullable)
-  uint64_t* cand;           // [rows, nsplit, k] keys (nsplit > 1)
+  uint64_t* cand;           // [rows, nsplit, k] selected keys of each key range (unsorted)
+  int* cand_cnt;            // [rows, nsplit]    how many of them are valid
   int* status;
 };
 
 template <int HI, int DI, int G>
 struct IndexerSmem {
-  static constexpr int N = ((G * HI + 15) / 16) * 16;
+  using TS = TileShape<HI, G>;
+  static constexpr int N = TS::N;
+  static constexpr int NB = TS::NB;
   static constexpr int kStages = (G == 1) ? 8 : 4;
   static constexpr int kRowBytes = DI / 2;
   static constexpr int kQBytes = ((N * kRowBytes + 1023) / 1024) * 1024;
@@ -146,55 +155,26 @@ struct IndexerSmem {
   static constexpr size_t off_sumw = off_w2 + (size_t)N * 4;
   static constexpr size_t off_cnt = off_sumw + 64 * 4;
   static constexpr size_t off_thr = off_cnt + 64 * 4;
-  static constexpr size_t off_hist = off_thr + 64 * 8;               // per epilogue warp, kWarpBins ints
-  static constexpr size_t off_sh = off_hist + (size_t)kEpiWarps * topk::kWarpBins * 4;
-  static constexpr size_t off_bar = off_sh + 64;
-  static constexpr size_t off_tslot = off_bar + (2 * kStages + 5) * 8;
+  static constexpr size_t off_hist = off_thr + 64 * 8;  // per token, kWarpBins ints
+  static constexpr size_t off_bar = off_hist + (size_t)G * topk::kWarpBins * 4;
+  static constexpr size_t off_tslot = off_bar + (2 * kStages + 2 * NB + 1) * 8;
   static constexpr size_t off_cand = ((off_tslot + 16 + 15) / 16) * 16;
   static size_t bytes(int cap) { return off_cand + (size_t)G * cap * 8 + 1024; }
 };
-
-// Sort a token's final candidates (cnt <= 32*R) in registers and write idx /
-// scores in rank order, padding with -1 / -inf up to k.
-template <int R>
-__device__ __forceinline__ void write_sorted(const uint64_t* buf, int cnt, const IndexerArgs& a, int64_t r, int lane) {
-  uint64_t v[R];
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    const int e = i * 32 + lane;
-    v[i] = e < cnt ? buf[e] : 0;
-  }
-  topk::warp_sort_regs_desc<R>(v, lane);
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    const int q = i * 32 + lane;
-    if (q < a.k) {
-      int32_t id = -1;
-      float sc = -INFINITY;
-      if (q < cnt) {
-        id = (int32_t)topk::key_index(v[i]);
-        sc = (float)topk::key_score(v[i]) * (1.0f / 128.0f);
-      }
-      a.idx[r * a.k + q] = id;
-      if (a.scores) a.scores[r * a.k + q] = sc;
-    }
-  }
-  // rows beyond 32*R (k > 32*R with cnt <= 32*R) are padding
-  for (int q = 32 * R + lane; q < a.k; q += 32) {
-    a.idx[r * a.k + q] = -1;
-    if (a.scores) a.scores[r * a.k + q] = -INFINITY;
-  }
-}
 
 template <int HI, int DI, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_topk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                         const IndexerArgs a) {
   using L = IndexerSmem<HI, DI, G>;
+  using TS = TileShape<HI, G>;
   constexpr int N = L::N;
+  constexpr int NB = L::NB;
   constexpr int NST = L::kStages;
-  constexpr int KB = DI / 64;  // MMAs of K=64 per tile
-  static_assert(N <= kMaxCols, "N too large");
+  constexpr int KB = DI / 64;            // MMAs of K=64 per tile
+  constexpr bool kAlt = G == 1;          // halves take alternate tiles (else split the tokens)
+  constexpr int G0 = kAlt ? 1 : G / 2;   // tokens per half
+  static_assert(kAlt || (G % 2 == 0 && G0 <= 4 && (G0 * HI) % 16 == 0), "token split between halves");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_q = smem + L::off_q;
@@ -208,11 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L::off_thr);
   int* s_hist = reinterpret_cast<int*>(smem + L::off_hist);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-  uint64_t* full = bar;                 // [NST] producer -> MMA
-  uint64_t* empty = bar + NST;          // [NST] MMA -> producer
-  uint64_t* dfull = bar + 2 * NST;      // [2]   MMA -> epilogue
-  uint64_t* dempty = bar + 2 * NST + 2; // [2]   epilogue -> MMA
-  uint64_t* ready = bar + 2 * NST + 4;  //       epilogue (TMEM scales written) + q tile -> MMA
+  uint64_t* full = bar;                      // [NST] producer -> MMA
+  uint64_t* empty = bar + NST;               // [NST] MMA -> producer
+  uint64_t* dfull = bar + 2 * NST;           // [NB]  MMA -> epilogue
+  uint64_t* dempty = bar + 2 * NST + NB;     // [NB]  epilogue -> MMA
+  uint64_t* ready = bar + 2 * NST + 2 * NB;  //       epilogue (TMEM scales written) + q tile -> MMA
   uint32_t* s_tslot = reinterpret_cast<uint32_t*>(smem + L::off_tslot);
   uint64_t* s_cand = reinterpret_cast<uint64_t*>(smem + L::off_cand);
 
@@ -248,9 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1 + 32);  // TMA transaction arrival + one per producer lane (scales)
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&dfull[b], 1);
-      mbar_init(&dempty[b], kEpiWarps);
+      mbar_init(&dempty[b], kAlt ? kEpiWarps / 2 : kEpiWarps);
     }
     mbar_init(ready, kEpiWarps + 1);
     fence_mbar_init();
@@ -336,34 +316,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(ready, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
       tc_fence_after();
     }
-    const uint32_t sq = smem_u32(s_q);
     const uint32_t layout = DI == 128 ? kSwizzle64 : kSwizzle32;
     const uint32_t sbo = 8 * L::kRowBytes;
+    // descriptors of stage 0 (the address field advances by kABytes/16 and 32 per stage)
+    const uint64_t adesc0 = make_sdesc(smem_u32(s_a), 16, sbo, layout);
+    const uint64_t bdesc0 = make_sdesc(smem_u32(s_q), 16, sbo, layout);
+    const uint64_t sfdesc0 = make_sdesc(smem_u32(s_sf), 16, 128, kSwizzleNone);
+    const uint64_t madesc = make_sdesc(smem_u32(s_ma), 128, 256, kSwizzleNone);
+    const uint64_t mbdesc = make_sdesc(smem_u32(s_mb), 128, 256, kSwizzleNone);
     for (int it = 0; it < ntiles; ++it) {
       const int s = it % NST;
       const uint32_t ph = (it / NST) & 1;
-      const int b = it & 1;
-      const uint32_t dph = (it >> 1) & 1;
+      const int b = it % NB;
+      const uint32_t dph = (it / NB) & 1;
       if (!mbar_wait(&dempty[b], dph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       if (!mbar_wait(&full[s], ph, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
       fence_proxy_async_smem();  // cp.async-written scales -> tcgen05.cp (async proxy)
       tc_fence_after();
       if (elect_one()) {  // issue from a converged warp (much cheaper than a lane-0 branch)
-        const uint32_t d = tbase + (b ? kTmemD1 : 0u);
-        const uint32_t sfa = tbase + kTmemSFA0 + 4 * b;
+        const uint32_t d = tbase + (uint32_t)(b * N);
+        const uint32_t sfa = tbase + TS::sfa(b);
         asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sfa),
-                     "l"(make_sdesc(smem_u32(s_sf + (size_t)s * 512), 16, 128, kSwizzleNone))
+                     "l"(sfdesc0 + (uint64_t)(s * (512 >> 4)))
                      : "memory");
-        const uint32_t sa = smem_u32(s_a + (size_t)s * L::kABytes);
+        const uint64_t adesc = adesc0 + (uint64_t)(s * (L::kABytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
-          mma_mxf4_ss(d, make_sdesc(sa + kk * 32, 16, sbo, layout), make_sdesc(sq + kk * 32, 16, sbo, layout),
+          mma_mxf4_ss(d, adesc + (uint64_t)(kk * 2), bdesc0 + (uint64_t)(kk * 2),
                       idesc_mxf4(128, N, 2 * kk, 2 * kk), sfa | ((uint32_t)(2 * kk) << 30),
-                      (tbase + kTmemSFB) | ((uint32_t)(2 * kk) << 30), kk > 0);
+                      (tbase + TS::kSFB) | ((uint32_t)(2 * kk) << 30), kk > 0);
         }
-        mma_mxf4_ss(d, make_sdesc(smem_u32(s_ma), 128, 256, kSwizzleNone),
-                    make_sdesc(smem_u32(s_mb), 128, 256, kSwizzleNone), idesc_mxf4(128, N, 0, 0),
-                    tbase + kTmemMagicSFA, tbase + kTmemMagicSFB, 1);
+        mma_mxf4_ss(d, madesc, mbdesc, idesc_mxf4(128, N, 0, 0), tbase + TS::kMagicSFA, tbase + TS::kMagicSFB, 1);
         mma_commit(&empty[s]);
         mma_commit(&dfull[b]);
       }
@@ -372,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // =========================== epilogue + selection (warps 2..9)
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;   // which half of the token group
+    const int half = (warp - 2) >> 2;   // which half of the epilogue
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     // scale factors of the query rows and the constant-offset operands (replicated layout)
     if (half == 0) {
@@ -397,130 +380,145 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         w[c] = v;
       }
-      tmem_st4(tbase + lane_base + kTmemSFB, w[0], w[1], w[2], w[3]);
-      tmem_st4(tbase + lane_base + kTmemSFB + 4, w[4], w[5], w[6], w[7]);
-      tmem_st4(tbase + lane_base + kTmemMagicSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      tmem_st4(tbase + lane_base + kTmemMagicSFB, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-      tmem_st4(tbase + lane_base + kTmemMagicSFB + 4, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+      tmem_st4(tbase + lane_base + TS::kSFB, w[0], w[1], w[2], w[3]);
+      tmem_st4(tbase + lane_base + TS::kSFB + 4, w[4], w[5], w[6], w[7]);
+      tmem_st4(tbase + lane_base + TS::kMagicSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      tmem_st4(tbase + lane_base + TS::kMagicSFB, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+      tmem_st4(tbase + lane_base + TS::kMagicSFB + 4, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
       tmem_wait_st();
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(ready);
 
-    // token range of this half (compile-time per instantiation)
-    constexpr int G0 = (G + 1) / 2;
-    static_assert(G == 1 || (G0 * HI) % 16 == 0, "halves must split on a 16-column chunk");
-    const int g_lo = half == 0 ? 0 : G0;
-    const int g_hi = half == 0 ? G0 : G;
-    static_assert(G0 <= 4, "one token per warp of a half");
-    const int my_g = g_lo + quarter;  // token whose buffer this warp maintains
-    int* my_hist = s_hist + (warp - 2) * topk::kWarpBins;
-
-    for (int it = 0; it < ntiles; ++it) {
-      const int b = it & 1;
-      const uint32_t dph = (it >> 1) & 1;
-      if (!mbar_wait(&dfull[b], dph, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
-      tc_fence_after();
-      if (warp == kCheckWarp) {
-        // exactness precondition on this tile's key scales (rows below j_end), read
-        // back from the replicated TMEM copy the MMA used
-        uint32_t sw[4];
-        tmem_ld4(tbase + lane_base + kTmemSFA0 + 4 * b, sw);
-        tmem_wait_ld();
-        const int64_t j0 = j_begin + (int64_t)it * 128;
-        bool bad = false;
+    // tokens of this half and the token whose buffer this warp maintains
+    constexpr int CW = G0 * HI;  // accumulator columns of one half
+    const int g_lo = kAlt ? 0 : half * G0;
+    const int g_hi = g_lo + G0;
+    const int c0 = kAlt ? 0 : half * CW;
+    const int my_g = kAlt ? (warp == 2 ? 0 : G) : g_lo + quarter;
+    int* my_hist = s_hist + (my_g < G ? my_g : 0) * topk::kWarpBins;
+    // per-warp copies of what every tile needs: weights, weight sums, visibility, thresholds
+    int wreg[CW];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (j0 + lane + 32 * c < j_end) {
+    for (int i = 0; i < CW; ++i) wreg[i] = s_w2[c0 + i];
+    uint32_t sumw_magic[G0];
+    int64_t nvis[G0];
+    uint64_t thr[G0];  // running thresholds, refreshed at every meeting
 #pragma unroll
-            for (int q = 0; q < DI / 32; ++q) bad |= ((sw[c] >> (8 * q)) & 255u) - 125u > 3u;
-          }
-        if (bad) report(a.status, CSA_ERR_RANGE);
+    for (int t = 0; t < G0; ++t) {
+      sumw_magic[t] = kMagicBits * (uint32_t)s_sumw[g_lo + t];
+      nvis[t] = kAlt ? tnvis[0] : (half == 0 ? tnvis[t] : tnvis[(G0 + t) % G]);
+      thr[t] = 0;
+    }
+    // meetings for cut-backs: every `check` tiles (rounds of one tile, or of two
+    // alternate tiles) and after the last one
+    const int nrounds = kAlt ? (ntiles + 1) / 2 : ntiles;
+    const int rounds_per_meet = kAlt ? (a.check >= 2 ? a.check / 2 : 1) : a.check;
+    // insertion of a tile is finished one tile later, so that the latency of the
+    // buffer reservation (shared atomic) hides behind the next tile's head sums
+    uint64_t pkey[G0];
+    uint32_t pbal[G0];
+    int pbase[G0];
+#pragma unroll
+    for (int t = 0; t < G0; ++t) {
+      pkey[t] = 0;
+      pbal[t] = 0u;
+      pbase[t] = 0;
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    auto finish_insert = [&]() {
+#pragma unroll
+      for (int t = 0; t < G0; ++t) {
+        if (pbal[t]) {
+          const int bg = __shfl_sync(0xffffffffu, pbase[t], 0);
+          if ((pbal[t] >> lane) & 1u) s_cand[(size_t)(g_lo + t) * cap + bg + __popc(pbal[t] & lt)] = pkey[t];
+        }
+        pbal[t] = 0u;
       }
-      const uint32_t dcol = tbase + lane_base + (b ? kTmemD1 : 0u);
-      uint32_t acc[G];  // arithmetic mod 2^32: the true head sum fits in int32
-#pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = 0u;
-      if (half == 0) head_sums<HI, G, 0>(dcol, s_w2, acc);
-      else head_sums<HI, G, 1>(dcol, s_w2, acc);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&dempty[b]);
+    };
 
-      // insert candidates
-      const int64_t j = j_begin + (int64_t)it * 128 + quarter * 32 + lane;
+    // A wait that timed out (status already recorded) stops this warp's tile work
+    // but not its meetings, so that no partner warp is left at a named barrier.
+    bool dead = false;
+    for (int rd = 0; rd < nrounds; ++rd) {
+      const int it = kAlt ? 2 * rd + half : rd;
+      if (it < ntiles && !dead) dead = !mbar_wait(&dfull[it % NB], (it / NB) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      if (it < ntiles && !dead) {
+        const int b = it % NB;
+        tc_fence_after();
+        // exactness precondition on the key scales: the checking half reads the
+        // scale word of its own key row (lane quarter q, column q of the replicated copy)
+        const bool checker = kAlt || half == 0;
+        uint32_t sfw = 0x7F7F7F7Fu;
+        if (checker) sfw = tmem_ld1(tbase + lane_base + TS::sfa(b) + (uint32_t)quarter);
+        uint32_t acc[G0];  // arithmetic mod 2^32: the true head sum fits in int32
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        if (g < g_lo || g >= g_hi) continue;
-        const int64_t nv = tnvis[g];
-        const int32_t units = (int32_t)(acc[g] - kMagicBits * (uint32_t)s_sumw[g]);
-        const uint64_t key = topk::make_key(units, (uint32_t)j);
-        const bool take = (j < nv) && (j < j_end) && (key >= s_thr[g]);
-        const uint32_t bal = __ballot_sync(0xffffffffu, take);
-        if (bal) {
-          int base = 0;
-          if (lane == 0) base = atomicAdd(&s_cnt[g], __popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (take) s_cand[(size_t)g * cap + base + __popc(bal & ((1u << lane) - 1u))] = key;
+        for (int t = 0; t < G0; ++t) acc[t] = 0u;
+        head_sums<HI, CW>(tbase + lane_base + (uint32_t)(b * N + c0), wreg, acc);
+        tmem_tie(sfw);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dempty[b]);
+        finish_insert();  // previous tile's stores
+        // this tile: keys, ballots and buffer reservations
+        const int64_t j = j_begin + (int64_t)it * 128 + quarter * 32 + lane;
+        const bool jin = j < j_end;
+        if (checker) {
+          bool bad = false;
+#pragma unroll
+          for (int q = 0; q < DI / 32; ++q) bad |= ((sfw >> (8 * q)) & 255u) - 125u > 3u;
+          if (__any_sync(0xffffffffu, bad && jin) && lane == 0) report(a.status, CSA_ERR_RANGE);
+        }
+#pragma unroll
+        for (int t = 0; t < G0; ++t) {
+          pkey[t] = topk::make_key((int32_t)(acc[t] - sumw_magic[t]), (uint32_t)j);
+          pbal[t] = __ballot_sync(0xffffffffu, jin && j < nvis[t] && pkey[t] >= thr[t]);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int t = 0; t < G0; ++t)
+            if (pbal[t]) pbase[t] = atomicAdd(&s_cnt[g_lo + t], __popc(pbal[t]));
         }
       }
-      // every `check` tiles (and after the last one) the half's warps meet; warp
-      // `quarter` then cuts back token g_lo + quarter's buffer if the next `check`
-      // tiles could overflow it (one-pass histogram threshold that keeps >= k)
-      if ((it + 1) % a.check != 0 && it + 1 != ntiles) continue;
-      topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
+      if ((rd + 1) % rounds_per_meet != 0 && rd + 1 != nrounds) continue;
+      // meeting: the warps that insert into a buffer meet; the owner warp cuts it
+      // back if the next `check` tiles could overflow it
+      finish_insert();
+      if (kAlt) topk::named_sync(kEpiBar, kEpiThreads);
+      else topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
       if (my_g < g_hi) {
         uint64_t* buf = s_cand + (size_t)my_g * cap;
         const int cnt = s_cnt[my_g];
         if (cnt > cap - 128 * a.check) {
           int kept;
-          const uint64_t thr = topk::warp_approx_threshold(buf, cnt, a.k, cap - 128 * a.check, my_hist, lane, &kept);
-          const int n = topk::warp_compact_ge(buf, cnt, thr, lane);
+          const uint64_t tq = topk::warp_approx_threshold(buf, cnt, a.k, cap - 128 * a.check, my_hist, lane, &kept);
+          const int n = topk::warp_compact_ge(buf, cnt, tq, lane);
           if (lane == 0) {
             s_cnt[my_g] = n;
-            s_thr[my_g] = thr;
+            s_thr[my_g] = tq;
           }
         }
       }
-      topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
+      if (kAlt) topk::named_sync(kEpiBar, kEpiThreads);
+      else topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
+#pragma unroll
+      for (int t = 0; t < G0; ++t) thr[t] = s_thr[g_lo + t];
     }
 
-    // final exact selection and sort: one warp per token, all tokens in parallel
+    // final exact selection, one warp per token: the k best keys of this key range
+    // go out unsorted; topk_finalize_kernel merges the ranges and sorts
     if (my_g < g_hi && row0 + my_g < a.rows) {
       const int64_t r = row0 + my_g;
       uint64_t* buf = s_cand + (size_t)my_g * cap;
       int cnt = s_cnt[my_g];
       if (cnt > a.k) {
-        const uint64_t thr = topk::warp_select_threshold(buf, cnt, a.k, my_hist, lane);
-        cnt = topk::warp_compact_ge(buf, cnt, thr, lane);
+        const uint64_t tq = topk::warp_select_threshold(buf, cnt, a.k, my_hist, lane);
+        cnt = topk::warp_compact_ge(buf, cnt, tq, lane);
       }
-      if (a.nsplit == 1) {
-        // final order: descending key (the per-range lists of a split search are
-        // merged and sorted by topk_merge_kernel instead)
-        if (cnt <= 512) write_sorted<16>(buf, cnt, a, r, lane);
-        else if (cnt <= 1024) write_sorted<32>(buf, cnt, a, r, lane);
-        else {
-          const int P = topk::next_pow2(cnt);
-          for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
-          __syncwarp();
-          topk::warp_bitonic_desc(buf, P, lane);
-          for (int q = lane; q < a.k; q += 32) {
-            int32_t id = -1;
-            float sc = -INFINITY;
-            if (q < cnt) {
-              const uint64_t key = buf[q];
-              id = (int32_t)topk::key_index(key);
-              sc = (float)topk::key_score(key) * (1.0f / 128.0f);
-            }
-            a.idx[r * a.k + q] = id;
-            if (a.scores) a.scores[r * a.k + q] = sc;
-          }
-        }
-      } else {
-        uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
-        for (int q = lane; q < a.k; q += 32) out[q] = q < cnt ? buf[q] : 0;
-      }
+      uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
+      for (int q = lane; q < cnt; q += 32) out[q] = buf[q];
+      if (lane == 0) a.cand_cnt[r * a.nsplit + split] = cnt;
     }
   }
 
@@ -532,51 +530,93 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the per-range candidate lists of every query row into its final top-k
-// (radix select to k, compaction, bitonic sort).  nsplit*k <= 256*kMergePer.
-constexpr int kMergePer = 40;
-
-__global__ void __launch_bounds__(256) topk_merge_kernel(const uint64_t* __restrict__ cand, int nsplit, int k,
-                                                         int32_t* __restrict__ idx, float* __restrict__ scores,
-                                                         uint64_t* __restrict__ keys_out) {
-  extern __shared__ __align__(16) uint8_t msmem[];
-  const int total = nsplit * k;
-  const int P = topk::next_pow2(total);
-  uint64_t* buf = reinterpret_cast<uint64_t*>(msmem);
-  int* hist = reinterpret_cast<int*>(buf + P);
-  int* sh = hist + 256;
-  const int64_t r = blockIdx.x;
-  const int tid = threadIdx.x;
-  if (tid == 0) sh[8] = 0;
-  __syncthreads();
-  for (int i = tid; i < total; i += 256) {
-    const uint64_t key = cand[(size_t)r * total + i];
-    if (key != 0) buf[atomicAdd(&sh[8], 1)] = key;
+// Final top-k of every query row: merge the per-range lists the indexer wrote,
+// select the k best (exact), sort them (score desc, j asc) and write idx / scores
+// (and the raw keys when asked).  One warp per row, several rows per block, so
+// that many independent warps per SM hide the selection's shared-memory latency.
+template <int R>
+__device__ __forceinline__ void finalize_sorted(const uint64_t* buf, int cnt, int k, int64_t r, int32_t* idx,
+                                                float* scores, uint64_t* keys_out, int lane) {
+  uint64_t v[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int e = lane * R + i;
+    v[i] = e < cnt ? buf[e] : 0;
   }
-  __syncthreads();
-  int cnt = sh[8];
-  __syncthreads();
-  if (cnt > k) {
-    const uint64_t thr = topk::radix_threshold<256>(buf, cnt, k, hist, sh, tid, 1);
-    cnt = topk::compact_ge<256, kMergePer>(buf, cnt, thr, sh + 4, tid, 1);
-  }
-  const int Pk = topk::next_pow2(cnt > 1 ? cnt : 1);
-  for (int i = cnt + tid; i < Pk; i += 256) buf[i] = 0;
-  __syncthreads();
-  topk::bitonic_desc<256>(buf, Pk, tid, 1);
-  for (int q = tid; q < k; q += 256) {
-    int32_t id = -1;
-    float sc = -INFINITY;
-    uint64_t key = 0;
-    if (q < cnt) {
-      key = buf[q];
-      id = (int32_t)topk::key_index(key);
-      sc = (float)topk::key_score(key) * (1.0f / 128.0f);
+  topk::warp_sort_lm_desc<R>(v, lane);
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int q = lane * R + i;
+    if (q < k) {
+      const bool ok = q < cnt;
+      if (idx) idx[r * k + q] = ok ? (int32_t)topk::key_index(v[i]) : -1;
+      if (scores) scores[r * k + q] = ok ? (float)topk::key_score(v[i]) * (1.0f / 128.0f) : -INFINITY;
+      if (keys_out) keys_out[r * k + q] = ok ? v[i] : 0;
     }
-    if (idx) idx[r * k + q] = id;
-    if (scores) scores[r * k + q] = sc;
-    if (keys_out) keys_out[r * k + q] = key;
   }
+  for (int q = 32 * R + lane; q < k; q += 32) {  // k beyond the register tile: padding
+    if (idx) idx[r * k + q] = -1;
+    if (scores) scores[r * k + q] = -INFINITY;
+    if (keys_out) keys_out[r * k + q] = 0;
+  }
+}
+
+__global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __restrict__ cand,
+                                                            const int* __restrict__ cand_cnt, int nsplit, int k,
+                                                            int64_t rows, int32_t* __restrict__ idx,
+                                                            float* __restrict__ scores,
+                                                            uint64_t* __restrict__ keys_out) {
+  extern __shared__ __align__(16) uint8_t fsmem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int64_t r = (int64_t)blockIdx.x * wpb + warp;
+  if (r >= rows) return;
+  const int L = topk::next_pow2(nsplit * k);  // per-warp key capacity (room for the sort padding)
+  uint64_t* buf = reinterpret_cast<uint64_t*>(fsmem) + (size_t)warp * L;
+  int* hist = reinterpret_cast<int*>(reinterpret_cast<uint64_t*>(fsmem) + (size_t)wpb * L) + warp * topk::kWarpBins;
+  int cnt = 0;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const int n = cand_cnt[r * nsplit + sp];
+    const uint64_t* src = cand + ((size_t)r * nsplit + sp) * k;
+    for (int i = lane; i < n; i += 32) buf[cnt + i] = src[i];
+    cnt += n;
+  }
+  __syncwarp();
+  if (cnt > k) {
+    const uint64_t t = topk::warp_select_threshold(buf, cnt, k, hist, lane);
+    cnt = topk::warp_compact_ge(buf, cnt, t, lane);
+  }
+  if (cnt <= 512) {
+    finalize_sorted<16>(buf, cnt, k, r, idx, scores, keys_out, lane);
+  } else if (cnt <= 1024) {
+    finalize_sorted<32>(buf, cnt, k, r, idx, scores, keys_out, lane);
+  } else {
+    const int P = topk::next_pow2(cnt);
+    for (int i = cnt + lane; i < P; i += 32) buf[i] = 0;
+    __syncwarp();
+    topk::warp_bitonic_desc(buf, P, lane);
+    for (int q = lane; q < k; q += 32) {
+      const bool ok = q < cnt;
+      const uint64_t key = ok ? buf[q] : 0;
+      if (idx) idx[r * k + q] = ok ? (int32_t)topk::key_index(key) : -1;
+      if (scores) scores[r * k + q] = ok ? (float)topk::key_score(key) * (1.0f / 128.0f) : -INFINITY;
+      if (keys_out) keys_out[r * k + q] = key;
+    }
+  }
+}
+
+static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, int nsplit, int k, int64_t rows,
+                                   int32_t* idx, float* scores, uint64_t* keys_out, cudaStream_t stream) {
+  const size_t per_warp = (size_t)topk::next_pow2(nsplit * k) * 8 + topk::kWarpBins * 4;
+  int wpb = (int)((kSmemLimit - 1024) / per_warp);
+  if (wpb > 8) wpb = 8;
+  if (wpb < 1) return cudaErrorInvalidConfiguration;
+  const size_t smem = per_warp * wpb;
+  cudaError_t e = cudaFuncSetAttribute(topk_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_finalize_kernel<<<(unsigned)ceil_div(rows, wpb), 32 * wpb, smem, stream>>>(cand, cand_cnt, nsplit, k, rows,
+                                                                                   idx, scores, keys_out);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ host side
@@ -607,7 +647,7 @@ static bool choose_cap(int k, int* cap, int* check) {
   const size_t base = L::bytes(0);
   const int budget = base < kSmemLimit ? (int)((kSmemLimit - base) / (8 * (size_t)G)) & ~127 : 0;
   const int p = topk::next_pow2(k);
-  for (int c = 4; c >= 1; c >>= 1) {
+  for (int c = 4; c >= (G == 1 ? 2 : 1); c >>= 1) {
     const int need = k + 128 * c > p ? k + 128 * c : p;
     if (budget >= need) {
       int want = 4 * k + 128 * c;  // cut-backs rare: room for several k between them
@@ -673,8 +713,8 @@ int indexer_tokens_per_cta(int HI) {
 // Prefill: rows = T, one range per group (direct output).
 cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
                                    const uint8_t* k_codes, const uint8_t* k_scales, int64_t T, int64_t t0, int64_t Nc,
-                                   int HI, int DI, int m, int k, int32_t* idx, float* scores, int* status,
-                                   cudaStream_t stream) {
+                                   int HI, int DI, int m, int k, int32_t* idx, float* scores, uint64_t* cand,
+                                   int* cand_cnt, int* status, cudaStream_t stream) {
   const int G = indexer_tokens_per_cta(HI);
   IndexerArgs a{};
   a.q_scales = q_scales;
@@ -689,14 +729,15 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
   a.k = k;
   a.nsplit = 1;
   a.split_tiles = ceil_div(Nc > 0 ? Nc : 1, 128);
-  a.idx = idx;
-  a.scores = scores;
-  a.cand = nullptr;
+  a.cand = cand;
+  a.cand_cnt = cand_cnt;
   a.status = status;
   dim3 grid((unsigned)ceil_div(T, G), 1);
   const uint8_t* kc = Nc > 0 ? k_codes : q_codes;  // any valid mapping when the cache is empty
-  return DI == 128 ? dispatch_hi<128>(HI, false, q_codes, kc, a, grid, stream)
-                   : dispatch_hi<64>(HI, false, q_codes, kc, a, grid, stream);
+  cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, false, q_codes, kc, a, grid, stream)
+                            : dispatch_hi<64>(HI, false, q_codes, kc, a, grid, stream);
+  if (e != cudaSuccess) return e;
+  return launch_finalize(cand, cand_cnt, 1, k, T, idx, scores, nullptr, stream);
 }
 
 // Decode: rows = B sequences, each with its own cache of Ncap entries and position
@@ -704,8 +745,8 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
 cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
                                   const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
                                   int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
-                                  uint64_t* cand, int32_t* idx, float* scores, uint64_t* keys_out, int* status,
-                                  cudaStream_t stream) {
+                                  uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
+                                  int* status, cudaStream_t stream) {
   IndexerArgs a{};
   a.q_scales = q_scales;
   a.w_codes = w_codes;
@@ -719,21 +760,14 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
   a.k = k;
   a.nsplit = nsplit;
   a.split_tiles = ceil_div(ceil_div(nvis_max > 0 ? nvis_max : 1, nsplit), 128);
-  a.idx = nullptr;
-  a.scores = nullptr;
   a.cand = cand;
+  a.cand_cnt = cand_cnt;
   a.status = status;
   dim3 grid((unsigned)B, (unsigned)nsplit);
   cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, true, q_codes, k_codes, a, grid, stream)
                             : dispatch_hi<64>(HI, true, q_codes, k_codes, a, grid, stream);
   if (e != cudaSuccess) return e;
-  const int total = nsplit * k;
-  const int P = topk::next_pow2(total);
-  const size_t smem = (size_t)P * 8 + 256 * 4 + 64 * 4;
-  e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  topk_merge_kernel<<<B, 256, smem, stream>>>(cand, nsplit, k, idx, scores, keys_out);
-  return cudaGetLastError();
+  return launch_finalize(cand, cand_cnt, nsplit, k, B, idx, scores, keys_out, stream);
 }
 
 }  // namespace csa

@@ -504,6 +504,62 @@ __device__ __forceinline__ void warp_sort_regs_desc(uint64_t (&v)[R], int lane) 
   }
 }
 
+// Lane-major register bitonic sort of 32*R keys, descending: element e = lane*R + r
+// lives in v[r] of lane `lane`.  Strides below R compare registers of one lane
+// (plain ALU), strides of R and more exchange between lanes by shuffles: for
+// R = 16, 15 of the 45 stages shuffle.
+template <int R>
+__device__ __forceinline__ void lm_within_lane(uint64_t (&v)[R], int j, int size, int lane) {
+#define CSA_LM_CASE(J)                                                    \
+  case J:                                                                 \
+    _Pragma("unroll") for (int r = 0; r < R; ++r) {                       \
+      if ((r & J) == 0 && (r | J) < R) {                                  \
+        const bool desc = ((lane * R + r) & size) == 0;                   \
+        const uint64_t x = v[r], y = v[r | J];                            \
+        const bool sw = (x < y) == desc;                                  \
+        v[r] = sw ? y : x;                                                \
+        v[r | J] = sw ? x : y;                                            \
+      }                                                                   \
+    }                                                                     \
+    break;
+  switch (j) {
+    CSA_LM_CASE(1)
+    CSA_LM_CASE(2)
+    CSA_LM_CASE(4)
+    CSA_LM_CASE(8)
+    CSA_LM_CASE(16)
+    CSA_LM_CASE(32)
+    default: break;
+  }
+#undef CSA_LM_CASE
+}
+
+template <int R>
+__device__ __forceinline__ void warp_sort_lm_desc(uint64_t (&v)[R], int lane) {
+  constexpr int P = 32 * R;
+#pragma unroll 1
+  for (int size = 2; size <= P; size <<= 1) {
+#pragma unroll 1
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride < R) {
+        lm_within_lane<R>(v, stride, size, lane);
+      } else {
+        const int ls = stride / R;  // lane distance
+        const bool lower = (lane & ls) == 0;
+        uint64_t y[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) y[r] = __shfl_xor_sync(0xffffffffu, v[r], ls);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const bool desc = ((lane * R + r) & size) == 0;
+          const bool keep_max = lower == desc;
+          v[r] = ((v[r] > y[r]) == keep_max) ? v[r] : y[r];
+        }
+      }
+    }
+  }
+}
+
 __host__ __device__ constexpr int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;

@@ -17,7 +17,7 @@ import math
 
 import torch
 
-from . import csa_compress, csa_indexer_topk, csa_sparse_attn, hca_attn
+from . import csa_compress, csa_indexer_topk, csa_sparse_attn, hca_attn, lib
 
 
 def stack_prefill_chunked(l1, l2, P, chunk, m, k, W, m2, W2, scale=None, out=None, phase_events=None,
@@ -43,7 +43,11 @@ def stack_prefill_chunked(l1, l2, P, chunk, m, k, W, m2, W2, scale=None, out=Non
     O1 = torch.empty_like(Q1)
     Q2 = torch.empty_like(Q1)
     O2 = torch.empty_like(Q1) if out is None else out
-    ws = torch.zeros(1 << 12, dtype=torch.uint8, device=dev)
+    L = lib()
+    HI, dI = l1["qI_scales"].shape[1], l1["qI_scales"].shape[2] * 32
+    ws_bytes = max(L.csa_indexer_topk_workspace_bytes(chunk, T // m, HI, dI, k),
+                   L.csa_sparse_attn_workspace_bytes(chunk, H, d, k, W), L.hca_attn_workspace_bytes(chunk, H, d, W2))
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
 
     def timed(name, fn):
         if phase_events is None:
