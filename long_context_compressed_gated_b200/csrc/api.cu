@@ -114,6 +114,18 @@ int decode_nsplit(int B, int64_t Ncap, int k) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Attention CTAs per decode sequence: enough to fill the GPU, at most one per
+// key tile of the sequence; with more than one, partial outputs go through the
+// workspace and a combine pass.
+int decode_attn_splits(int B, int64_t tiles) {
+  int ns = B > 0 ? 148 / B : 1;
+  if (ns > tiles) ns = (int)tiles;
+  return ns < 1 ? 1 : ns;
+}
+size_t attn_part_bytes(int B, int ns, int H, int d) {
+  return ns > 1 ? align256((size_t)B * ns * H * d * 4) + align256((size_t)B * ns * H * 4) : 0;
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -282,11 +294,12 @@ int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, co
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
-size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int, int, int, int, int k, int) {
+size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int, int, int k, int W) {
   if (B <= 0 || k <= 0) return kWorkspaceHeader;
   const int ns = decode_nsplit(B, Ncap, k);
+  const int nsa = decode_attn_splits(B, ceil_div(k, 128) + window_tiles(W, 1));
   return kWorkspaceHeader + align256((size_t)B * 8) + align256((size_t)B * k * 4) +
-         align256((size_t)B * ns * k * 8) + align256((size_t)B * ns * 4);
+         align256((size_t)B * ns * k * 8) + align256((size_t)B * ns * 4) + attn_part_bytes(B, nsa, H, d);
 }
 
 int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
@@ -322,6 +335,9 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader + align256((size_t)B * 8) +
                                                align256((size_t)B * k * 4));
   int* cand_cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cand) + align256((size_t)B * ns * k * 8));
+  const int nsa = decode_attn_splits(B, ceil_div(k, 128) + window_tiles(W, 1));
+  float* o_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(cand_cnt) + align256((size_t)B * ns * 4));
+  float* lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(o_part) + align256((size_t)B * nsa * H * d * 4));
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = upload_positions(pos_dev, pos, B, s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -360,12 +376,18 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
+  a.nsplit = nsa;
+  a.o_part = o_part;
+  a.lse_part = lse_part;
   e = launch_attention(a, d, (unsigned)B, s);
+  if (e == cudaSuccess && nsa > 1) e = launch_attention_combine(a, B, d, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
-size_t hca_decode_workspace_bytes(int B, int64_t, int, int, int) {
-  return kWorkspaceHeader + align256((size_t)(B > 0 ? B : 0) * 8);
+size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W) {
+  if (B <= 0) return kWorkspaceHeader;
+  const int nsa = decode_attn_splits(B, ceil_div(Ncap, 128) + window_tiles(W, 1));
+  return kWorkspaceHeader + align256((size_t)B * 8) + attn_part_bytes(B, nsa, H, d);
 }
 
 int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
@@ -418,7 +440,12 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
+  a.nsplit = decode_attn_splits(B, ceil_div(Ncap, 128) + window_tiles(W, 1));
+  a.o_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader + align256((size_t)B * 8));
+  a.lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.o_part) +
+                                        align256((size_t)B * a.nsplit * H * d * 4));
   e = launch_attention(a, d, (unsigned)B, s);
+  if (e == cudaSuccess && a.nsplit > 1) e = launch_attention_combine(a, B, d, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 

@@ -215,6 +215,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         s_tiles[nt++] = Tile{kWin, 0, (v + 15) & ~15, v, w0};
       }
     }
+    if (a.nsplit > 1) {
+      // this CTA's share of the sequence's tiles
+      const int tps = (nt + a.nsplit - 1) / a.nsplit;
+      const int first = (int)blockIdx.y * tps;
+      int cnt = nt - first;
+      if (cnt > tps) cnt = tps;
+      if (cnt < 0) cnt = 0;
+      for (int i = 0; i < cnt; ++i) s_tiles[i] = s_tiles[first + i];
+      nt = cnt;
+    }
     misc[0] = nt;
   }
   tc_fence_before();
@@ -487,8 +497,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       l_run = __uint_as_float(v[0]);
     }
     const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
+    const bool part = a.nsplit > 1;
     __nv_bfloat16* orow = nullptr;
-    if (t >= 0) orow = a.O + b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
+    float* part_row = nullptr;
+    if (t >= 0 && !part) orow = a.O + b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
+    if (t >= 0 && part) part_row = a.o_part + ((b * a.nsplit + blockIdx.y) * H + h) * (int64_t)D;
 #pragma unroll
     for (int b0 = 0; b0 < 64; b0 += 32) {
       if (my0 >= D) break;
@@ -499,6 +512,13 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (part_row) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(part_row + my0 + b0 + e) =
+              make_float4(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv,
+                          __uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
       }
       if (orow) {
 #pragma unroll
@@ -516,10 +536,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       // combine the two halves' fp32 row sums
       s_red[half * kRows + row] = l_run32;
       asm volatile("bar.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(kSoftmaxWarps * 32) : "memory");
-      if (half == 0 && t >= 0 && a.lse) {
+      if (half == 0 && t >= 0 && (a.lse || part)) {
         const float l32 = l_run32 + s_red[kRows + row];
         const float lse = l32 > 0.f ? (m_run + log2f(l32)) * 0.69314718055994531f : -INFINITY;
-        a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
+        if (part) a.lse_part[(b * a.nsplit + blockIdx.y) * H + h] = lse;
+        else a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
       }
     }
   }
@@ -563,7 +584,53 @@ static cudaError_t launch_t(const AttnArgs& a, const AttnMaps& maps, unsigned gr
                             cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attention_kernel<D, L><<<grid, kThreads, smem, stream>>>(a, maps);
+  attention_kernel<D, L><<<dim3(grid, a.nsplit > 1 ? a.nsplit : 1), kThreads, smem, stream>>>(a, maps);
+  return cudaGetLastError();
+}
+
+// Merge the split partial outputs of every (sequence, head): one block per sequence.
+template <int D>
+__global__ void __launch_bounds__(256) attention_combine_kernel(const float* __restrict__ o_part,
+                                                                const float* __restrict__ lse_part, int nsplit, int H,
+                                                                __nv_bfloat16* __restrict__ O, int64_t o_batch_stride,
+                                                                float* __restrict__ lse) {
+  const int64_t b = blockIdx.x;
+  constexpr int V = D / 4;  // float4 chunks per row
+  for (int w = threadIdx.x; w < H * V; w += blockDim.x) {
+    const int h = w / V, c = w % V;
+    float mx = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, lse_part[(b * nsplit + s) * H + h]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float sum = 0.f;
+    if (mx > -INFINITY) {
+      for (int s = 0; s < nsplit; ++s) {
+        const float ls = lse_part[(b * nsplit + s) * H + h];
+        if (ls == -INFINITY) continue;
+        const float wt = __expf(ls - mx);
+        const float4 o = reinterpret_cast<const float4*>(o_part + ((b * nsplit + s) * H + h) * (int64_t)D)[c];
+        acc.x += wt * o.x;
+        acc.y += wt * o.y;
+        acc.z += wt * o.z;
+        acc.w += wt * o.w;
+        sum += wt;
+      }
+    }
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    uint2 packed;
+    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(O + b * o_batch_stride + (int64_t)h * D + 4 * c) = packed;
+    if (lse && c == 0) lse[b * H + h] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
+  }
+}
+
+cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream) {
+  if (d == 128)
+    attention_combine_kernel<128><<<B, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, a.O, a.o_batch_stride,
+                                                          a.lse);
+  else
+    attention_combine_kernel<64><<<B, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, a.O, a.o_batch_stride,
+                                                         a.lse);
   return cudaGetLastError();
 }
 
@@ -577,7 +644,7 @@ cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream
       !bf16_map(&maps.vc, a.Vc, a.kc_rows, d, 128) || !bf16_map(&maps.kr, a.Kr, a.raw_rows, d, 128) ||
       !bf16_map(&maps.vr, a.Vr, a.raw_rows, d, 128))
     return cudaErrorInvalidValue;
-  const bool lse = a.lse != nullptr;
+  const bool lse = a.lse != nullptr || a.nsplit > 1;
   if (d == 128)
     return lse ? launch_t<128, true>(a, maps, grid, smem, stream) : launch_t<128, false>(a, maps, grid, smem, stream);
   return lse ? launch_t<64, true>(a, maps, grid, smem, stream) : launch_t<64, false>(a, maps, grid, smem, stream);

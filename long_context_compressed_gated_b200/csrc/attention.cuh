@@ -25,9 +25,17 @@ struct AttnArgs {
   const int64_t* pos;       // device, absolute position of each sequence's new token
   // extents (rows) of the tensors, for the TMA descriptors
   int64_t q_rows, kc_rows, raw_rows;
+  // decode with the key tiles of a sequence spread over nsplit CTAs (grid.y):
+  // each writes its normalised fp32 output and log-sum-exp, merged by
+  // launch_attention_combine.  nsplit = 1: direct bf16 output.
+  int nsplit;
+  float* o_part;    // [B, nsplit, H, d]
+  float* lse_part;  // [B, nsplit, H]
 };
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);
+// O[b,h] = sum_s exp(lse_s - lse) O_s with lse = log sum_s exp(lse_s), as bf16 (+ lse)
+cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream);
 int attention_max_tiles();
 
 }  // namespace csa

@@ -605,8 +605,166 @@ __global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __re
   }
 }
 
+// Block-wide finalize for rows with many candidates (a split decode search):
+// 256 threads per row.  One min/max pass and one 1024-bin histogram over the
+// score range find the bin that holds the k-th key; the keys of that bin are
+// resolved exactly (in-register sort when it holds at most 32, else the warp
+// radix fallback); the k best are compacted, bitonic-sorted and written.
+constexpr int kFinBlock = 256;
+
+__global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const uint64_t* __restrict__ cand,
+                                                                        const int* __restrict__ cand_cnt, int nsplit,
+                                                                        int k, int32_t* __restrict__ idx,
+                                                                        float* __restrict__ scores,
+                                                                        uint64_t* __restrict__ keys_out) {
+  extern __shared__ __align__(16) uint8_t bsmem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t r = blockIdx.x;
+  const int cap = topk::next_pow2(nsplit * k);
+  uint64_t* buf = reinterpret_cast<uint64_t*>(bsmem);    // [cap] gathered candidates
+  uint64_t* sel = buf + cap;                              // [next_pow2(k)] the k best
+  int* hist = reinterpret_cast<int*>(sel + topk::next_pow2(k));  // [kWarpBins]
+  __shared__ int s_off[64];
+  __shared__ uint32_t s_lo[8], s_hi[8];
+  __shared__ int s_bin, s_kept, s_inbin, s_nsel;
+  __shared__ uint64_t s_thr;
+  // gather the per-range lists (offsets by a prefix over the counts)
+  if (tid == 0) {
+    int acc = 0;
+    for (int sp = 0; sp < nsplit; ++sp) {
+      s_off[sp] = acc;
+      acc += cand_cnt[r * nsplit + sp];
+    }
+    s_off[nsplit] = acc;
+    s_nsel = 0;
+  }
+  for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
+  __syncthreads();
+  const int cnt = s_off[nsplit];
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const int n = s_off[sp + 1] - s_off[sp];
+    const uint64_t* src = cand + ((size_t)r * nsplit + sp) * k;
+    for (int i = tid; i < n; i += kFinBlock) buf[s_off[sp] + i] = src[i];
+  }
+  __syncthreads();
+  int nout = cnt;
+  if (cnt > k) {
+    // score range
+    uint32_t lo = 0xFFFFFFFFu, hi = 0;
+    for (int i = tid; i < cnt; i += kFinBlock) {
+      const uint32_t sc = (uint32_t)(buf[i] >> 32);
+      lo = sc < lo ? sc : lo;
+      hi = sc > hi ? sc : hi;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      s_lo[warp] = lo;
+      s_hi[warp] = hi;
+    }
+    __syncthreads();
+    lo = s_lo[0];
+    hi = s_hi[0];
+    for (int w = 1; w < kFinBlock / 32; ++w) {
+      lo = min(lo, s_lo[w]);
+      hi = max(hi, s_hi[w]);
+    }
+    uint64_t thr;
+    if (hi > lo) {
+      const int bits = 32 - __clz(hi - lo);
+      const int shift = bits > 10 ? bits - 10 : 0;
+      for (int i = tid; i < cnt; i += kFinBlock) atomicAdd(&hist[((uint32_t)(buf[i] >> 32) - lo) >> shift], 1);
+      __syncthreads();
+      if (warp == 0) {
+        int bin, kept;
+        topk::warp_hist_cut(hist, k, lane, &bin, &kept);
+        if (lane == 0) {
+          s_bin = bin;
+          s_kept = kept;
+          s_inbin = hist[bin];
+        }
+      }
+      __syncthreads();
+      const int bin = s_bin, in_bin = s_inbin;
+      const int need = k - (s_kept - in_bin);
+      const uint64_t bin_lo = (uint64_t)(lo + ((uint32_t)bin << shift)) << 32;
+      if (need == in_bin) {
+        thr = bin_lo;
+      } else if (in_bin <= 32) {
+        // the boundary bin's keys (at most 32) into `sel`, sorted in registers
+        for (int i = tid; i < cnt; i += kFinBlock) {
+          const uint64_t v = buf[i];
+          if ((int)(((uint32_t)(v >> 32) - lo) >> shift) == bin) sel[atomicAdd(&s_nsel, 1)] = v;
+        }
+        __syncthreads();
+        if (warp == 0) {
+          uint64_t x = lane < in_bin ? sel[lane] : 0;
+          x = topk::warp_sort32_desc(x, lane);
+          const uint64_t t = __shfl_sync(0xffffffffu, x, need - 1);
+          if (lane == 0) s_thr = t;
+        }
+        __syncthreads();
+        thr = s_thr;
+      } else {
+        // heavy ties in the boundary bin: exact radix select over all keys
+        if (warp == 0) {
+          const uint64_t t = topk::warp_exact_threshold(buf, cnt, k, hist, lane);
+          if (lane == 0) s_thr = t;
+        }
+        __syncthreads();
+        thr = s_thr;
+      }
+    } else {
+      // every key has the same score: the order is by index alone
+      if (warp == 0) {
+        const uint64_t t = topk::warp_exact_threshold(buf, cnt, k, hist, lane);
+        if (lane == 0) s_thr = t;
+      }
+      __syncthreads();
+      thr = s_thr;
+    }
+    // the k keys >= thr
+    if (tid == 0) s_nsel = 0;
+    __syncthreads();
+    for (int i = tid; i < cnt; i += kFinBlock) {
+      const uint64_t v = buf[i];
+      if (v >= thr) sel[atomicAdd(&s_nsel, 1)] = v;
+    }
+    __syncthreads();
+    nout = s_nsel;
+  } else {
+    for (int i = tid; i < cnt; i += kFinBlock) sel[i] = buf[i];
+  }
+  const int P = topk::next_pow2(nout > 1 ? nout : 1);
+  for (int i = nout + tid; i < P; i += kFinBlock) sel[i] = 0;
+  __syncthreads();
+  topk::bitonic_desc<kFinBlock>(sel, P, tid, 0);
+  __syncthreads();
+  for (int q = tid; q < k; q += kFinBlock) {
+    const bool ok = q < nout;
+    const uint64_t key = ok ? sel[q] : 0;
+    if (idx) idx[r * k + q] = ok ? (int32_t)topk::key_index(key) : -1;
+    if (scores) scores[r * k + q] = ok ? (float)topk::key_score(key) * (1.0f / 128.0f) : -INFINITY;
+    if (keys_out) keys_out[r * k + q] = key;
+  }
+}
+
 static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, int nsplit, int k, int64_t rows,
                                    int32_t* idx, float* scores, uint64_t* keys_out, cudaStream_t stream) {
+  if (nsplit > 1) {
+    // few rows with many candidates each: a block per row
+    const size_t smem = (size_t)topk::next_pow2(nsplit * k) * 8 + (size_t)topk::next_pow2(k) * 8 + topk::kWarpBins * 4;
+    if (smem > kSmemLimit || nsplit > 63) return cudaErrorInvalidConfiguration;
+    cudaError_t e =
+        cudaFuncSetAttribute(topk_finalize_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_finalize_block_kernel<<<(unsigned)rows, kFinBlock, smem, stream>>>(cand, cand_cnt, nsplit, k, idx, scores,
+                                                                            keys_out);
+    return cudaGetLastError();
+  }
   const size_t per_warp = (size_t)topk::next_pow2(nsplit * k) * 8 + topk::kWarpBins * 4;
   int wpb = (int)((kSmemLimit - 1024) / per_warp);
   if (wpb > 8) wpb = 8;
