@@ -119,6 +119,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // workspace and a combine pass.
 int decode_attn_splits(int B, int64_t tiles) {
   int ns = B > 0 ? 148 / B : 1;
+  if (ns > 16) ns = 16;  // the combine pass merges at most 16 partials
   if (ns > tiles) ns = (int)tiles;
   return ns < 1 ? 1 : ns;
 }

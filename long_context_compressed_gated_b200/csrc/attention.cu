@@ -588,49 +588,66 @@ static cudaError_t launch_t(const AttnArgs& a, const AttnMaps& maps, unsigned gr
   return cudaGetLastError();
 }
 
-// Merge the split partial outputs of every (sequence, head): one block per sequence.
+// Merge the split partial outputs: one warp per (sequence, head), lane c owning
+// dims 4c..4c+3; every partial is loaded before any is combined.
+constexpr int kCombineSplits = 16;
+
 template <int D>
 __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __restrict__ o_part,
                                                                 const float* __restrict__ lse_part, int nsplit, int H,
-                                                                __nv_bfloat16* __restrict__ O, int64_t o_batch_stride,
-                                                                float* __restrict__ lse) {
-  const int64_t b = blockIdx.x;
-  constexpr int V = D / 4;  // float4 chunks per row
-  for (int w = threadIdx.x; w < H * V; w += blockDim.x) {
-    const int h = w / V, c = w % V;
-    float mx = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, lse_part[(b * nsplit + s) * H + h]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float sum = 0.f;
-    if (mx > -INFINITY) {
-      for (int s = 0; s < nsplit; ++s) {
-        const float ls = lse_part[(b * nsplit + s) * H + h];
-        if (ls == -INFINITY) continue;
-        const float wt = __expf(ls - mx);
-        const float4 o = reinterpret_cast<const float4*>(o_part + ((b * nsplit + s) * H + h) * (int64_t)D)[c];
-        acc.x += wt * o.x;
-        acc.y += wt * o.y;
-        acc.z += wt * o.z;
-        acc.w += wt * o.w;
-        sum += wt;
-      }
-    }
-    const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    uint2 packed;
-    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(O + b * o_batch_stride + (int64_t)h * D + 4 * c) = packed;
-    if (lse && c == 0) lse[b * H + h] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
+                                                                int64_t rows, __nv_bfloat16* __restrict__ O,
+                                                                int64_t o_batch_stride, float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (b, h)
+  if (w >= rows) return;
+  const int64_t b = w / H;
+  const int h = (int)(w % H);
+  constexpr int V = D / 4;
+  float ls[kCombineSplits];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < kCombineSplits; ++s) {
+    ls[s] = s < nsplit ? lse_part[(b * nsplit + s) * H + h] : -INFINITY;
+    mx = fmaxf(mx, ls[s]);
   }
+  if (lane >= V) return;
+  float4 o[kCombineSplits];
+#pragma unroll
+  for (int s = 0; s < kCombineSplits; ++s)
+    o[s] = (s < nsplit && ls[s] > -INFINITY)
+               ? reinterpret_cast<const float4*>(o_part + ((b * nsplit + s) * H + h) * (int64_t)D)[lane]
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float sum = 0.f;
+  if (mx > -INFINITY) {
+#pragma unroll
+    for (int s = 0; s < kCombineSplits; ++s) {
+      const float wt = ls[s] > -INFINITY ? __expf(ls[s] - mx) : 0.f;
+      acc.x += wt * o[s].x;
+      acc.y += wt * o[s].y;
+      acc.z += wt * o[s].z;
+      acc.w += wt * o[s].w;
+      sum += wt;
+    }
+  }
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  uint2 packed;
+  packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(O + b * o_batch_stride + (int64_t)h * D + 4 * lane) = packed;
+  if (lse && lane == 0) lse[b * H + h] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
 }
 
 cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream) {
+  if (a.nsplit > kCombineSplits) return cudaErrorInvalidConfiguration;
+  const int64_t rows = (int64_t)B * a.H;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
   if (d == 128)
-    attention_combine_kernel<128><<<B, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, a.O, a.o_batch_stride,
-                                                          a.lse);
+    attention_combine_kernel<128><<<grid, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, rows, a.O,
+                                                             a.o_batch_stride, a.lse);
   else
-    attention_combine_kernel<64><<<B, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, a.O, a.o_batch_stride,
-                                                         a.lse);
+    attention_combine_kernel<64><<<grid, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, rows, a.O,
+                                                            a.o_batch_stride, a.lse);
   return cudaGetLastError();
 }
 

@@ -324,33 +324,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t sfdesc0 = make_sdesc(smem_u32(s_sf), 16, 128, kSwizzleNone);
     const uint64_t madesc = make_sdesc(smem_u32(s_ma), 128, 256, kSwizzleNone);
     const uint64_t mbdesc = make_sdesc(smem_u32(s_mb), 128, 256, kSwizzleNone);
-    for (int it = 0; it < ntiles; ++it) {
-      const int s = it % NST;
-      const uint32_t ph = (it / NST) & 1;
-      const int b = it % NB;
-      const uint32_t dph = (it / NB) & 1;
-      if (!mbar_wait(&dempty[b], dph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
-      if (!mbar_wait(&full[s], ph, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
+    // Tiles go in pairs: the two accumulation chains (scale copy, KB dependent
+    // MMAs, constant offset) interleave, so that the tensor pipe is not bound by
+    // the latency of a single chain.
+    int it = 0;
+    while (it < ntiles) {
+      const int np = it + 1 < ntiles ? 2 : 1;
+      bool ok = true;
+      for (int q = 0; q < np && ok; ++q) {
+        const int t = it + q;
+        ok = mbar_wait(&dempty[t % NB], ((t / NB) & 1) ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT) &&
+             mbar_wait(&full[t % NST], (t / NST) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      }
+      if (!ok) break;
       fence_proxy_async_smem();  // cp.async-written scales -> tcgen05.cp (async proxy)
       tc_fence_after();
       if (elect_one()) {  // issue from a converged warp (much cheaper than a lane-0 branch)
-        const uint32_t d = tbase + (uint32_t)(b * N);
-        const uint32_t sfa = tbase + TS::sfa(b);
-        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sfa),
-                     "l"(sfdesc0 + (uint64_t)(s * (512 >> 4)))
-                     : "memory");
-        const uint64_t adesc = adesc0 + (uint64_t)(s * (L::kABytes >> 4));
+        for (int q = 0; q < np; ++q) {
+          const int t = it + q;
+          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tbase + TS::sfa(t % NB)),
+                       "l"(sfdesc0 + (uint64_t)((t % NST) * (512 >> 4)))
+                       : "memory");
+        }
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
-          mma_mxf4_ss(d, adesc + (uint64_t)(kk * 2), bdesc0 + (uint64_t)(kk * 2),
-                      idesc_mxf4(128, N, 2 * kk, 2 * kk), sfa | ((uint32_t)(2 * kk) << 30),
-                      (tbase + TS::kSFB) | ((uint32_t)(2 * kk) << 30), kk > 0);
+          for (int q = 0; q < np; ++q) {
+            const int t = it + q, b = t % NB, s = t % NST;
+            const uint32_t sfa = tbase + TS::sfa(b);
+            mma_mxf4_ss(tbase + (uint32_t)(b * N), adesc0 + (uint64_t)(s * (L::kABytes >> 4) + kk * 2),
+                        bdesc0 + (uint64_t)(kk * 2), idesc_mxf4(128, N, 2 * kk, 2 * kk),
+                        sfa | ((uint32_t)(2 * kk) << 30), (tbase + TS::kSFB) | ((uint32_t)(2 * kk) << 30), kk > 0);
+          }
         }
-        mma_mxf4_ss(d, madesc, mbdesc, idesc_mxf4(128, N, 0, 0), tbase + TS::kMagicSFA, tbase + TS::kMagicSFB, 1);
-        mma_commit(&empty[s]);
-        mma_commit(&dfull[b]);
+        for (int q = 0; q < np; ++q) {
+          const int t = it + q, b = t % NB;
+          mma_mxf4_ss(tbase + (uint32_t)(b * N), madesc, mbdesc, idesc_mxf4(128, N, 0, 0), tbase + TS::kMagicSFA,
+                      tbase + TS::kMagicSFB, 1);
+          mma_commit(&empty[t % NST]);
+          mma_commit(&dfull[b]);
+        }
       }
       __syncwarp();
+      it += np;
     }
   } else {
     // =========================== epilogue + selection (warps 2..9)
