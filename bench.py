@@ -31,6 +31,14 @@ from long_context_compressed_gated_b200 import inputs  # noqa: E402
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 METRIC = "CSA/HCA prefill tokens/s & TFLOP/s; 1M-ctx decode GB/s; % of B200 roofline"
 FP4_OVER_BF16 = 4.0  # nominal dense ratio (9 vs 2.25 PFLOP/s)
+# DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum) of each phase's
+# kernels on the T=32768 CSA prefill, from the ncu captures summarised under profiles/;
+# to be refreshed whenever those kernels change.
+PHASE_TRAFFIC = {
+    "indexer_topk": (145.440512e6 + 92.454912e6 + 130.384640e6 + 37.054720e6,
+                     "profiles/indexer_topk_csa_prefill_T32768.md (indexer + finalize launches)"),
+    "sparse_attn": (625.381376e6 + 495.227392e6, "profiles/attention_csa_prefill_T32768.md"),
+}
 
 
 def load_peaks():
@@ -477,13 +485,18 @@ def main():
     attn_tf = work["attn_flop"] / (ph["sparse_attn"] * 1e-3) / 1e12
     comp_gbs = work["compress_bytes"] / (ph["compress"] * 1e-3) / 1e9
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    same_cfg = wl.T == inputs.CSA_PREFILL.T
     if dominant == "indexer_topk":
         roof = {"kernel": "indexer_topk", "bound": "tensor", "achieved": idx_tf, "peak": fp4_peak,
-                "unit": "TFLOP/s", "frac": idx_tf / fp4_peak, "traffic": None,
-                "peak_note": "FP4 peak = measured bf16 burst x 4 (nominal dense ratio)"}
+                "unit": "TFLOP/s", "frac": idx_tf / fp4_peak,
+                "traffic": PHASE_TRAFFIC["indexer_topk"][0] if same_cfg else None,
+                "traffic_source": PHASE_TRAFFIC["indexer_topk"][1],
+                "peak_note": "FP4 peak = measured bf16 burst x 4 (nominal dense ratio), %s" % peaks["source"]}
     elif dominant == "sparse_attn":
         roof = {"kernel": "sparse_attn", "bound": "tensor", "achieved": attn_tf, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_tflops"],
+                "traffic": PHASE_TRAFFIC["sparse_attn"][0] if same_cfg else None,
+                "traffic_source": PHASE_TRAFFIC["sparse_attn"][1],
                 "peak_note": "bf16 burst, %s" % peaks["source"]}
     else:
         roof = {"kernel": "compress", "bound": "hbm", "achieved": comp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
