@@ -171,18 +171,26 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   }
   if (tid < 32) reinterpret_cast<uint4*>(s_ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   fence_proxy_async_smem();
-  // compact each token's selected list (drop -1 / out-of-range), one warp per token
+  // compact each token's selected list (drop -1 / out-of-range), one warp per token;
+  // 8 loads per lane are in flight before any is used
   if (idx != nullptr) {
     for (int g = warp; g < ntok; g += kThreads / 32) {
       const int32_t* src = idx + (row_tok0 + g) * a.k;
       int n = 0;
-      for (int base = 0; base < a.k; base += 32) {
-        const int q = base + lane;
-        int32_t j = q < a.k ? src[q] : -1;
-        const bool ok = j >= 0 && j < a.Nc;
-        const uint32_t bal = __ballot_sync(0xffffffffu, ok);
-        if (ok) s_idx[g * a.k + n + __popc(bal & ((1u << lane) - 1u))] = j;
-        n += __popc(bal);
+      for (int base = 0; base < a.k; base += 256) {
+        int32_t jv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int q = base + 32 * u + lane;
+          jv[u] = q < a.k ? __ldg(src + q) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const bool ok = jv[u] >= 0 && jv[u] < a.Nc;
+          const uint32_t bal = __ballot_sync(0xffffffffu, ok);
+          if (ok) s_idx[g * a.k + n + __popc(bal & ((1u << lane) - 1u))] = jv[u];
+          n += __popc(bal);
+        }
       }
       if (lane == 0) misc[2 + g] = n;
     }

@@ -644,22 +644,21 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
   __shared__ int s_bin, s_kept, s_inbin, s_nsel;
   __shared__ uint64_t s_thr;
   // gather the per-range lists (offsets by a prefix over the counts)
+  if (tid < nsplit) s_off[tid + 1] = cand_cnt[r * nsplit + tid];
   if (tid == 0) {
-    int acc = 0;
-    for (int sp = 0; sp < nsplit; ++sp) {
-      s_off[sp] = acc;
-      acc += cand_cnt[r * nsplit + sp];
-    }
-    s_off[nsplit] = acc;
+    s_off[0] = 0;
     s_nsel = 0;
   }
+  __syncthreads();
+  if (tid == 0)
+    for (int sp = 1; sp <= nsplit; ++sp) s_off[sp] += s_off[sp - 1];
   for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
   __syncthreads();
   const int cnt = s_off[nsplit];
-  for (int sp = 0; sp < nsplit; ++sp) {
-    const int n = s_off[sp + 1] - s_off[sp];
-    const uint64_t* src = cand + ((size_t)r * nsplit + sp) * k;
-    for (int i = tid; i < n; i += kFinBlock) buf[s_off[sp] + i] = src[i];
+  // all ranges at once: slot i of the row belongs to range i / k
+  for (int i = tid; i < nsplit * k; i += kFinBlock) {
+    const int sp = i / k, e = i - sp * k;
+    if (e < s_off[sp + 1] - s_off[sp]) buf[s_off[sp] + e] = cand[(size_t)r * nsplit * k + i];
   }
   __syncthreads();
   int nout = cnt;
