@@ -199,9 +199,14 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   if (tid == 0) {
     int nt = 0;
     if (idx != nullptr) {
-      for (int g = 0; g < ntok; ++g) {
-        const int n = misc[2 + g];
-        for (int off = 0; off < n && nt < kMaxTiles; off += kTileKeys) {
+      // the tokens' selected-entry tiles alternate, so that consecutive tiles (in
+      // the two S buffers) keep the softmax warps of both tokens busy
+      int nmax = 0;
+      for (int g = 0; g < ntok; ++g) nmax = misc[2 + g] > nmax ? misc[2 + g] : nmax;
+      for (int off = 0; off < nmax; off += kTileKeys) {
+        for (int g = 0; g < ntok && nt < kMaxTiles; ++g) {
+          const int n = misc[2 + g];
+          if (off >= n) continue;
           const int v = n - off < kTileKeys ? n - off : kTileKeys;
           s_tiles[nt++] = Tile{kSeg, g, (v + 15) & ~15, v, (int64_t)off};
         }
