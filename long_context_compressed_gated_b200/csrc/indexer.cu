@@ -66,7 +66,8 @@ struct Geometry {
 template <int HI, int G>
 struct TileShape {
   static constexpr int N = ((G * HI + 15) / 16) * 16;      // MMA N (accumulator columns)
-  static constexpr int NB = 448 / N < 8 ? 448 / N : 8;      // accumulator buffers
+  static constexpr int NB = G == 1 ? (448 / N >= 8 ? 8 : 4)  // decode: whole barrier groups of 4
+                                   : (448 / N < 8 ? 448 / N : 8);  // accumulator buffers
   static constexpr uint32_t sfa(int b) { return kTmemSF + 4 * b; }  // key scales, 4 columns each
   static constexpr uint32_t kSFB = kTmemSF + 32;                    // query scales, 8 columns
   static constexpr uint32_t kMagicSFA = kTmemSF + 40;              // 4 columns
@@ -142,7 +143,7 @@ struct IndexerSmem {
   using TS = TileShape<HI, G>;
   static constexpr int N = TS::N;
   static constexpr int NB = TS::NB;
-  static constexpr int kStages = (G == 1) ? 8 : 4;
+  static constexpr int kStages = (G == 1) ? 16 : 4;  // decode streams keys from HBM: deeper ring
   static constexpr int kRowBytes = DI / 2;
   static constexpr int kQBytes = ((N * kRowBytes + 1023) / 1024) * 1024;
   static constexpr int kABytes = 128 * kRowBytes;  // multiple of 1024
@@ -173,6 +174,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NST = L::kStages;
   constexpr int KB = DI / 64;            // MMAs of K=64 per tile
   constexpr bool kAlt = G == 1;          // halves take alternate tiles (else split the tokens)
+  // Decode accumulators are narrow (N <= 64): the epilogue re-seeds them with
+  // 196608.0 by tcgen05.st, which is cheaper than the constant-offset MMA there.
+  constexpr bool kSeeded = kAlt;
+  // Barriers cover TPG consecutive tiles (stages / accumulator buffers): decode
+  // waits and commits once per 4 tiles, which the MMA warp's issue rate needs.
+  constexpr int TPG = kAlt ? 4 : 1;
+  constexpr int NSG = NST / TPG, NBG = NB / TPG;  // stage groups, buffer groups
+  static_assert(NST % TPG == 0 && NB % TPG == 0, "barrier groups");
   constexpr int G0 = kAlt ? 1 : G / 2;   // tokens per half
   static_assert(kAlt || (G % 2 == 0 && G0 <= 4 && (G0 * HI) % 16 == 0), "token split between halves");
   extern __shared__ uint8_t smem_raw[];
@@ -188,10 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L::off_thr);
   int* s_hist = reinterpret_cast<int*>(smem + L::off_hist);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-  uint64_t* full = bar;                      // [NST] producer -> MMA
-  uint64_t* empty = bar + NST;               // [NST] MMA -> producer
-  uint64_t* dfull = bar + 2 * NST;           // [NB]  MMA -> epilogue
-  uint64_t* dempty = bar + 2 * NST + NB;     // [NB]  epilogue -> MMA
+  uint64_t* full = bar;                      // [NSG] producer -> MMA
+  uint64_t* empty = bar + NST;               // [NSG] MMA -> producer
+  uint64_t* dfull = bar + 2 * NST;           // [NBG] MMA -> epilogue
+  uint64_t* dempty = bar + 2 * NST + NB;     // [NBG] epilogue -> MMA
   uint64_t* ready = bar + 2 * NST + 2 * NB;  //       epilogue (TMEM scales written) + q tile -> MMA
   uint32_t* s_tslot = reinterpret_cast<uint32_t*>(smem + L::off_tslot);
   uint64_t* s_cand = reinterpret_cast<uint64_t*>(smem + L::off_cand);
@@ -224,13 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- setup
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NSG; ++s) {
       mbar_init(&full[s], 1 + 32);  // TMA transaction arrival + one per producer lane (scales)
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < NB; ++b) {
+    for (int b = 0; b < NBG; ++b) {
       mbar_init(&dfull[b], 1);
-      mbar_init(&dempty[b], kAlt ? kEpiWarps / 2 : kEpiWarps);
+      mbar_init(&dempty[b], TPG * (kAlt ? kEpiWarps / 2 : kEpiWarps));
     }
     mbar_init(ready, kEpiWarps + 1);
     fence_mbar_init();
@@ -274,39 +283,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(ready, N * L::kRowBytes);
       tma_load_2d(s_q, &qmap, ready, 0, (int)(row0 * HI));
     }
-    for (int it = 0; it < ntiles; ++it) {
-      const int s = it % NST;
-      const uint32_t ph = (it / NST) & 1;
-      if (!mbar_wait(&empty[s], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
-      const int64_t j0 = j_begin + (int64_t)it * 128;
-      const int64_t row0k = key_row_base + j0;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], L::kABytes);
-        tma_load_2d(s_a + (size_t)s * L::kABytes, &kmap, &full[s], 0, (int)row0k);
+    for (int g0 = 0; g0 < ntiles; g0 += TPG) {
+      const int gs = (g0 / TPG) % NSG;
+      const uint32_t ph = (g0 / TPG / NSG) & 1;
+      const int nt = ntiles - g0 < TPG ? ntiles - g0 : TPG;
+      if (!mbar_wait(&empty[gs], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&full[gs], (uint32_t)(nt * L::kABytes));
+      for (int u = 0; u < nt; ++u) {
+        const int it = g0 + u, s = it % NST;
+        const int64_t j0 = j_begin + (int64_t)it * 128;
+        const int64_t row0k = key_row_base + j0;
+        if (lane == 0) tma_load_2d(s_a + (size_t)s * L::kABytes, &kmap, &full[gs], 0, (int)row0k);
+        // key scales straight into the tcgen05.cp 32x128b layout: lane l holds the
+        // scale words of rows l, l+32, l+64, l+96 (rows past the tensor read as 0)
+        const uint32_t sdst = smem_u32(s_sf + (size_t)s * 512) + lane * 16;
+        if (DI == 128) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int64_t row = row0k + lane + 32 * c;
+            const bool in = row < a.key_rows;
+            cp_async4(sdst + 4 * c, a.k_scales + (in ? row : 0) * 4, in ? 4u : 0u);
+          }
+        } else {
+          // two scale bytes per row: plain loads, padded to the 4-byte word
+          uint32_t wv[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int64_t row = row0k + lane + 32 * c;
+            wv[c] = row < a.key_rows ? (uint32_t)*reinterpret_cast<const uint16_t*>(a.k_scales + row * 2) | 0x7F7F0000u
+                                     : 0x7F7F7F7Fu;
+          }
+          *reinterpret_cast<uint4*>(s_sf + (size_t)s * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
       }
-      // key scales straight into the tcgen05.cp 32x128b layout: lane l holds the
-      // scale words of rows l, l+32, l+64, l+96 (rows past the tensor read as 0)
-      const uint32_t sdst = smem_u32(s_sf + (size_t)s * 512) + lane * 16;
       if (DI == 128) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int64_t row = row0k + lane + 32 * c;
-          const bool in = row < a.key_rows;
-          cp_async4(sdst + 4 * c, a.k_scales + (in ? row : 0) * 4, in ? 4u : 0u);
-        }
-        cp_async_arrive(&full[s]);
+        cp_async_arrive(&full[gs]);
       } else {
-        // two scale bytes per row: plain loads, padded to the 4-byte word
-        uint32_t wv[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int64_t row = row0k + lane + 32 * c;
-          wv[c] = row < a.key_rows ? (uint32_t)*reinterpret_cast<const uint16_t*>(a.k_scales + row * 2) | 0x7F7F0000u
-                                   : 0x7F7F7F7Fu;
-        }
-        *reinterpret_cast<uint4*>(s_sf + (size_t)s * 512 + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         fence_proxy_async_smem();  // generic-proxy writes -> tcgen05.cp
-        mbar_arrive(&full[s]);
+        mbar_arrive(&full[gs]);
       }
     }
     cp_async_wait_all();
@@ -324,48 +338,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t sfdesc0 = make_sdesc(smem_u32(s_sf), 16, 128, kSwizzleNone);
     const uint64_t madesc = make_sdesc(smem_u32(s_ma), 128, 256, kSwizzleNone);
     const uint64_t mbdesc = make_sdesc(smem_u32(s_mb), 128, 256, kSwizzleNone);
-    // Tiles go in pairs: the two accumulation chains (scale copy, KB dependent
-    // MMAs, constant offset) interleave, so that the tensor pipe is not bound by
-    // the latency of a single chain.
-    int it = 0;
-    while (it < ntiles) {
-      const int np = it + 1 < ntiles ? 2 : 1;
+    // Tiles go in groups of NQ: their accumulation chains (scale copy, KB
+    // dependent MMAs, constant offset) interleave, so that the tensor pipe is not
+    // bound by the latency of a single chain.
+    // One issue unit = UG barrier groups (2 single tiles in prefill, one group of 4
+    // tiles in decode); the tiles' chains interleave.
+    constexpr int UG = TPG == 1 ? 2 : 1;
+    int g0 = 0;
+    while (g0 < ntiles) {
+      const int nt = ntiles - g0 < UG * TPG ? ntiles - g0 : UG * TPG;  // tiles in this unit
       bool ok = true;
-      for (int q = 0; q < np && ok; ++q) {
-        const int t = it + q;
-        ok = mbar_wait(&dempty[t % NB], ((t / NB) & 1) ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT) &&
-             mbar_wait(&full[t % NST], (t / NST) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      for (int t = g0; t < g0 + nt && ok; t += TPG) {
+        const int gi = t / TPG;
+        ok = mbar_wait(&dempty[gi % NBG], ((gi / NBG) & 1) ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT) &&
+             mbar_wait(&full[gi % NSG], (gi / NSG) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       }
       if (!ok) break;
       fence_proxy_async_smem();  // cp.async-written scales -> tcgen05.cp (async proxy)
       tc_fence_after();
       if (elect_one()) {  // issue from a converged warp (much cheaper than a lane-0 branch)
-        for (int q = 0; q < np; ++q) {
-          const int t = it + q;
+        for (int q = 0; q < nt; ++q) {
+          const int t = g0 + q;
           asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tbase + TS::sfa(t % NB)),
                        "l"(sfdesc0 + (uint64_t)((t % NST) * (512 >> 4)))
                        : "memory");
         }
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
-          for (int q = 0; q < np; ++q) {
-            const int t = it + q, b = t % NB, s = t % NST;
+          for (int q = 0; q < nt; ++q) {
+            const int t = g0 + q, b = t % NB, s = t % NST;
             const uint32_t sfa = tbase + TS::sfa(b);
             mma_mxf4_ss(tbase + (uint32_t)(b * N), adesc0 + (uint64_t)(s * (L::kABytes >> 4) + kk * 2),
                         bdesc0 + (uint64_t)(kk * 2), idesc_mxf4(128, N, 2 * kk, 2 * kk),
-                        sfa | ((uint32_t)(2 * kk) << 30), (tbase + TS::kSFB) | ((uint32_t)(2 * kk) << 30), kk > 0);
+                        sfa | ((uint32_t)(2 * kk) << 30), (tbase + TS::kSFB) | ((uint32_t)(2 * kk) << 30),
+                        kSeeded || kk > 0);
           }
         }
-        for (int q = 0; q < np; ++q) {
-          const int t = it + q, b = t % NB;
-          mma_mxf4_ss(tbase + (uint32_t)(b * N), madesc, mbdesc, idesc_mxf4(128, N, 0, 0), tbase + TS::kMagicSFA,
-                      tbase + TS::kMagicSFB, 1);
-          mma_commit(&empty[t % NST]);
-          mma_commit(&dfull[b]);
+        for (int q = 0; q < nt; ++q) {
+          const int t = g0 + q, b = t % NB;
+          if (!kSeeded)
+            mma_mxf4_ss(tbase + (uint32_t)(b * N), madesc, mbdesc, idesc_mxf4(128, N, 0, 0), tbase + TS::kMagicSFA,
+                        tbase + TS::kMagicSFB, 1);
+          if ((t + 1) % TPG == 0 || t + 1 == g0 + nt) {  // the group's last tile: one commit per group
+            mma_commit(&empty[(t / TPG) % NSG]);
+            mma_commit(&dfull[(t / TPG) % NBG]);
+          }
         }
       }
       __syncwarp();
-      it += np;
+      g0 += nt;
     }
   } else {
     // =========================== epilogue + selection (warps 2..9)
@@ -400,6 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st4(tbase + lane_base + TS::kMagicSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       tmem_st4(tbase + lane_base + TS::kMagicSFB, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
       tmem_st4(tbase + lane_base + TS::kMagicSFB + 4, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+      if (kSeeded)
+        for (int c = 0; c < NB * N; c += 4) tmem_st4(tbase + lane_base + (uint32_t)c, kMagicBits, kMagicBits, kMagicBits, kMagicBits);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -456,9 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // A wait that timed out (status already recorded) stops this warp's tile work
     // but not its meetings, so that no partner warp is left at a named barrier.
     bool dead = false;
+    int seen_group = -1;  // barrier group whose accumulators are known complete
     for (int rd = 0; rd < nrounds; ++rd) {
       const int it = kAlt ? 2 * rd + half : rd;
-      if (it < ntiles && !dead) dead = !mbar_wait(&dfull[it % NB], (it / NB) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      if (it < ntiles && !dead && it / TPG != seen_group) {
+        seen_group = it / TPG;
+        dead = !mbar_wait(&dfull[seen_group % NBG], (seen_group / NBG) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      }
       if (it < ntiles && !dead) {
         const int b = it % NB;
         tc_fence_after();
@@ -472,9 +499,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < G0; ++t) acc[t] = 0u;
         head_sums<HI, CW>(tbase + lane_base + (uint32_t)(b * N + c0), wreg, acc);
         tmem_tie(sfw);
+        if (kSeeded) {
+#pragma unroll
+          for (int c = 0; c < N; c += 4)
+            tmem_st4(tbase + lane_base + (uint32_t)(b * N + c), kMagicBits, kMagicBits, kMagicBits, kMagicBits);
+          tmem_wait_st();
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dempty[b]);
+        if (lane == 0) mbar_arrive(&dempty[(it / TPG) % NBG]);
         finish_insert();  // previous tile's stores
         // this tile: keys, ballots and buffer reservations
         const int64_t j = j_begin + (int64_t)it * 128 + quarter * 32 + lane;
