@@ -157,7 +157,8 @@ struct IndexerSmem {
   static constexpr size_t off_cnt = off_sumw + 64 * 4;
   static constexpr size_t off_thr = off_cnt + 64 * 4;
   static constexpr size_t off_hist = off_thr + 64 * 8;  // per token, kWarpBins ints
-  static constexpr size_t off_bar = off_hist + (size_t)G * topk::kWarpBins * 4;
+  static constexpr size_t off_grp = off_hist + (size_t)G * topk::kWarpBins * 4;  // [2][32] ints: group scratch
+  static constexpr size_t off_bar = off_grp + 256;
   static constexpr size_t off_tslot = off_bar + (2 * kStages + 2 * NB + 1) * 8;
   static constexpr size_t off_cand = ((off_tslot + 16 + 15) / 16) * 16;
   static size_t bytes(int cap) { return off_cand + (size_t)G * cap * 8 + 1024; }
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_cnt = reinterpret_cast<int*>(smem + L::off_cnt);
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L::off_thr);
   int* s_hist = reinterpret_cast<int*>(smem + L::off_hist);
+  int* s_grp = reinterpret_cast<int*>(smem + L::off_grp);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* full = bar;                      // [NSG] producer -> MMA
   uint64_t* empty = bar + NST;               // [NSG] MMA -> producer
@@ -432,10 +434,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tokens of this half and the token whose buffer this warp maintains
     constexpr int CW = G0 * HI;  // accumulator columns of one half
     const int g_lo = kAlt ? 0 : half * G0;
-    const int g_hi = g_lo + G0;
     const int c0 = kAlt ? 0 : half * CW;
-    const int my_g = kAlt ? (warp == 2 ? 0 : G) : g_lo + quarter;
-    int* my_hist = s_hist + (my_g < G ? my_g : 0) * topk::kWarpBins;
+    // the warps that insert into the same buffers form a group: one half (prefill)
+    // or all eight epilogue warps (decode); cut-backs and the final selection are
+    // done by the whole group, one buffer at a time
+    constexpr int GNT = kAlt ? kEpiThreads : kEpiThreads / 2;
+    const int gbar = kAlt ? kEpiBar : kHalfBar0 + half;
+    const int gt = kAlt ? tid - 64 : tid - 64 - half * (kEpiThreads / 2);
+    int* gscr = s_grp + (kAlt ? 0 : half) * 32;
     // per-warp copies of what every tile needs: weights, weight sums, visibility, thresholds
     int wreg[CW];
 #pragma unroll
@@ -533,40 +539,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       // meeting: the warps that insert into a buffer meet; the owner warp cuts it
       // back if the next `check` tiles could overflow it
       finish_insert();
-      if (kAlt) topk::named_sync(kEpiBar, kEpiThreads);
-      else topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
-      if (my_g < g_hi) {
-        uint64_t* buf = s_cand + (size_t)my_g * cap;
-        const int cnt = s_cnt[my_g];
+      topk::named_sync(gbar, GNT);
+      for (int t = 0; t < G0; ++t) {  // every warp of the group cuts back each of its buffers
+        const int gg = g_lo + t;
+        uint64_t* buf = s_cand + (size_t)gg * cap;
+        const int cnt = s_cnt[gg];
         if (cnt > cap - 128 * a.check) {
-          int kept;
-          const uint64_t tq = topk::warp_approx_threshold(buf, cnt, a.k, cap - 128 * a.check, my_hist, lane, &kept);
-          const int n = topk::warp_compact_ge(buf, cnt, tq, lane);
-          if (lane == 0) {
-            s_cnt[my_g] = n;
-            s_thr[my_g] = tq;
+          const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, cap - 128 * a.check, false,
+                                                         s_hist + gg * topk::kWarpBins, gscr, gt, gbar);
+          const int n = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
+          if (gt == 0) {
+            s_cnt[gg] = n;
+            s_thr[gg] = tq;
           }
         }
       }
-      if (kAlt) topk::named_sync(kEpiBar, kEpiThreads);
-      else topk::named_sync(kHalfBar0 + half, kEpiThreads / 2);
+      topk::named_sync(gbar, GNT);
 #pragma unroll
       for (int t = 0; t < G0; ++t) thr[t] = s_thr[g_lo + t];
     }
 
-    // final exact selection, one warp per token: the k best keys of this key range
-    // go out unsorted; topk_finalize_kernel merges the ranges and sorts
-    if (my_g < g_hi && row0 + my_g < a.rows) {
-      const int64_t r = row0 + my_g;
-      uint64_t* buf = s_cand + (size_t)my_g * cap;
-      int cnt = s_cnt[my_g];
+    // final exact selection by the group, one buffer at a time: the k best keys of
+    // this key range go out unsorted; topk_finalize_kernel merges the ranges and sorts
+    for (int t = 0; t < G0; ++t) {
+      const int gg = g_lo + t;
+      if (row0 + gg >= a.rows) break;  // uniform over the group
+      const int64_t r = row0 + gg;
+      uint64_t* buf = s_cand + (size_t)gg * cap;
+      int cnt = s_cnt[gg];
       if (cnt > a.k) {
-        const uint64_t tq = topk::warp_select_threshold(buf, cnt, a.k, my_hist, lane);
-        cnt = topk::warp_compact_ge(buf, cnt, tq, lane);
+        const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, s_hist + gg * topk::kWarpBins, gscr,
+                                                       gt, gbar);
+        cnt = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
       }
       uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
-      for (int q = lane; q < cnt; q += 32) out[q] = buf[q];
-      if (lane == 0) a.cand_cnt[r * a.nsplit + split] = cnt;
+      for (int q = gt; q < cnt; q += GNT) out[q] = buf[q];
+      if (gt == 0) a.cand_cnt[r * a.nsplit + split] = cnt;
     }
   }
 

@@ -504,6 +504,142 @@ __device__ __forceinline__ void warp_sort_regs_desc(uint64_t (&v)[R], int lane) 
   }
 }
 
+// ------------------------------------------------------------------ group-cooperative selection
+// NT threads (gt in [0, NT), whole warps) that meet on named barrier `bar` work
+// on one buffer.  `hist` is a shared array of kWarpBins ints, `scr` shared ints
+// (at least 2 * NT/32 + 8).  All threads get the same results.
+
+// Threshold t such that at least `keep` keys of buf[0..cnt) are >= t.  exact:
+// exactly min(keep, cnt) keys.  Approximate (exact = false): all keys of the
+// boundary histogram bin are kept, unless that keeps more than `room`.
+template <int NT>
+__device__ uint64_t group_threshold(const uint64_t* buf, int cnt, int keep, int room, bool exact, int* hist,
+                                    int* scr, int gt, int bar) {
+  constexpr int NW = NT / 32;
+  const int warp = gt >> 5, lane = gt & 31;
+  if (cnt <= keep) return 0;
+  uint64_t* s_thr64 = reinterpret_cast<uint64_t*>(scr + 2 * NW + 4);  // 8-byte aligned slot
+  // score range
+  uint32_t lo = 0xFFFFFFFFu, hi = 0;
+  for (int i = gt; i < cnt; i += NT) {
+    const uint32_t sc = (uint32_t)(buf[i] >> 32);
+    lo = sc < lo ? sc : lo;
+    hi = sc > hi ? sc : hi;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    scr[warp] = (int)lo;
+    scr[NW + warp] = (int)hi;
+  }
+  named_sync(bar, NT);
+  lo = (uint32_t)scr[0];
+  hi = (uint32_t)scr[NW];
+  for (int w = 1; w < NW; ++w) {
+    lo = min(lo, (uint32_t)scr[w]);
+    hi = max(hi, (uint32_t)scr[NW + w]);
+  }
+  const int bits = hi > lo ? 32 - __clz(hi - lo) : 0;
+  const int shift = bits > 10 ? bits - 10 : 0;
+  named_sync(bar, NT);  // scr reused below
+  if (hi > lo) {
+    for (int b = gt; b < kWarpBins; b += NT) hist[b] = 0;
+    named_sync(bar, NT);
+    for (int i = gt; i < cnt; i += NT) atomicAdd(&hist[((uint32_t)(buf[i] >> 32) - lo) >> shift], 1);
+    named_sync(bar, NT);
+    if (warp == 0) {
+      int bin, kept;
+      warp_hist_cut(hist, keep, lane, &bin, &kept);
+      if (lane == 0) {
+        scr[0] = bin;
+        scr[1] = kept;
+        scr[2] = hist[bin];
+      }
+    }
+    named_sync(bar, NT);
+    const int bin = scr[0], kept = scr[1], in_bin = scr[2];
+    const uint64_t bin_lo = (uint64_t)(lo + ((uint32_t)bin << shift)) << 32;
+    const int need = keep - (kept - in_bin);
+    if ((!exact && kept <= room) || need == in_bin) {
+      named_sync(bar, NT);
+      return bin_lo;
+    }
+    if (in_bin <= 32) {
+      // the boundary bin's keys into shared scratch (the histogram is done with), sorted in registers
+      uint64_t* sc = reinterpret_cast<uint64_t*>(hist);
+      if (gt == 0) scr[3] = 0;
+      named_sync(bar, NT);
+      for (int i = gt; i < cnt; i += NT) {
+        const uint64_t v = buf[i];
+        if ((int)(((uint32_t)(v >> 32) - lo) >> shift) == bin) sc[atomicAdd(&scr[3], 1)] = v;
+      }
+      named_sync(bar, NT);
+      if (warp == 0) {
+        uint64_t x = lane < in_bin ? sc[lane] : 0;
+        x = warp_sort32_desc(x, lane);
+        const uint64_t t = __shfl_sync(0xffffffffu, x, need - 1);
+        if (lane == 0) *s_thr64 = t;
+      }
+      named_sync(bar, NT);
+      const uint64_t t = *s_thr64;
+      named_sync(bar, NT);
+      return t;
+    }
+  }
+  // heavy ties: exact radix select by one warp
+  if (warp == 0) {
+    const uint64_t t = warp_exact_threshold(buf, cnt, keep, hist, lane);
+    if (lane == 0) *s_thr64 = t;
+  }
+  named_sync(bar, NT);
+  const uint64_t t = *s_thr64;
+  named_sync(bar, NT);
+  return t;
+}
+
+// In-place compaction of buf[0..cnt) to the keys >= thr (order not kept).  Rounds
+// of U*NT keys: every thread loads its keys of the round before any survivor is
+// written, and survivors only land below the round's end, so nothing unread is
+// overwritten.  Returns the survivor count.
+template <int NT>
+__device__ int group_compact_ge(uint64_t* buf, int cnt, uint64_t thr, int* scr, int gt, int bar) {
+  constexpr int NW = NT / 32, U = 4;
+  const int warp = gt >> 5, lane = gt & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  int out = 0;
+  for (int base = 0; base < cnt; base += U * NT) {
+    uint64_t v[U];
+    uint32_t bal[U];
+    int mine = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * NT + gt;
+      v[u] = i < cnt ? buf[i] : 0;
+      bal[u] = __ballot_sync(0xffffffffu, i < cnt && v[u] >= thr);
+      mine += __popc(bal[u]);
+    }
+    if (lane == 0) scr[warp] = mine;
+    named_sync(bar, NT);
+    int woff = out, total = out;
+    for (int w = 0; w < NW; ++w) {
+      const int c = scr[w];
+      woff += w < warp ? c : 0;
+      total += c;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if ((bal[u] >> lane) & 1u) buf[woff + __popc(bal[u] & lt)] = v[u];
+      woff += __popc(bal[u]);
+    }
+    named_sync(bar, NT);
+    out = total;
+  }
+  return out;
+}
+
 // Lane-major register bitonic sort of 32*R keys, descending: element e = lane*R + r
 // lives in v[r] of lane `lane`.  Strides below R compare registers of one lane
 // (plain ALU), strides of R and more exchange between lanes by shuffles: for
