@@ -665,8 +665,11 @@ __global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __re
 // 256 threads per row.  One min/max pass and one 1024-bin histogram over the
 // score range find the bin that holds the k-th key; the keys of that bin are
 // resolved exactly (in-register sort when it holds at most 32, else the warp
-// radix fallback); the k best are compacted, bitonic-sorted and written.
+// radix fallback); the k best are compacted, sorted (per-warp register sorts
+// merged through shared memory) and written.  The row's keys are loaded 16 per
+// thread at a time, so the gather costs a few memory round trips.
 constexpr int kFinBlock = 256;
+constexpr int kFinSort = 1024;  // keys sorted by the register/shared hybrid sort
 
 __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const uint64_t* __restrict__ cand,
                                                                         const int* __restrict__ cand_cnt, int nsplit,
@@ -678,39 +681,63 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
   const int64_t r = blockIdx.x;
   const int cap = topk::next_pow2(nsplit * k);
   uint64_t* buf = reinterpret_cast<uint64_t*>(bsmem);    // [cap] gathered candidates
-  uint64_t* sel = buf + cap;                              // [next_pow2(k)] the k best
-  int* hist = reinterpret_cast<int*>(sel + topk::next_pow2(k));  // [kWarpBins]
+  const int sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
+  uint64_t* sel = buf + cap;                              // [sel_cap] the k best
+  int* hist = reinterpret_cast<int*>(sel + sel_cap);      // [kWarpBins]
   __shared__ int s_off[64];
   __shared__ uint32_t s_lo[8], s_hi[8];
   __shared__ int s_bin, s_kept, s_inbin, s_nsel;
   __shared__ uint64_t s_thr;
-  // gather the per-range lists (offsets by a prefix over the counts)
+  // gather the per-range lists (offsets by a prefix over the counts).  The loads
+  // of the row are issued kGatherU per thread at a time, so that a row of
+  // nsplit * k keys takes a few memory round trips instead of one per key.
+  constexpr int kGatherU = 16;
+  const int total = nsplit * k;
+  const uint64_t* src = cand + (size_t)r * total;
+  uint64_t v[kGatherU];
+#pragma unroll
+  for (int u = 0; u < kGatherU; ++u) {
+    const int i = u * kFinBlock + tid;
+    v[u] = i < total ? __ldg(src + i) : 0;
+  }
   if (tid < nsplit) s_off[tid + 1] = cand_cnt[r * nsplit + tid];
   if (tid == 0) {
     s_off[0] = 0;
     s_nsel = 0;
   }
+  for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
   __syncthreads();
   if (tid == 0)
     for (int sp = 1; sp <= nsplit; ++sp) s_off[sp] += s_off[sp - 1];
-  for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
   __syncthreads();
   const int cnt = s_off[nsplit];
-  // all ranges at once: slot i of the row belongs to range i / k
-  for (int i = tid; i < nsplit * k; i += kFinBlock) {
-    const int sp = i / k, e = i - sp * k;
-    if (e < s_off[sp + 1] - s_off[sp]) buf[s_off[sp] + e] = cand[(size_t)r * nsplit * k + i];
+  // slot i of the row belongs to range i / k; the valid keys' score range is
+  // taken on the way
+  uint32_t lo = 0xFFFFFFFFu, hi = 0;
+  for (int base = 0; base < total; base += kGatherU * kFinBlock) {
+    if (base > 0) {
+#pragma unroll
+      for (int u = 0; u < kGatherU; ++u) {
+        const int i = base + u * kFinBlock + tid;
+        v[u] = i < total ? __ldg(src + i) : 0;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGatherU; ++u) {
+      const int i = base + u * kFinBlock + tid;
+      if (i < total) {
+        const int sp = i / k, e = i - sp * k;
+        if (e < s_off[sp + 1] - s_off[sp]) {
+          buf[s_off[sp] + e] = v[u];
+          const uint32_t sc = (uint32_t)(v[u] >> 32);
+          lo = sc < lo ? sc : lo;
+          hi = sc > hi ? sc : hi;
+        }
+      }
+    }
   }
-  __syncthreads();
   int nout = cnt;
   if (cnt > k) {
-    // score range
-    uint32_t lo = 0xFFFFFFFFu, hi = 0;
-    for (int i = tid; i < cnt; i += kFinBlock) {
-      const uint32_t sc = (uint32_t)(buf[i] >> 32);
-      lo = sc < lo ? sc : lo;
-      hi = sc > hi ? sc : hi;
-    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -781,12 +808,20 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
       __syncthreads();
       thr = s_thr;
     }
-    // the k keys >= thr
+    // the k keys >= thr, one shared-memory atomic per warp and step
     if (tid == 0) s_nsel = 0;
     __syncthreads();
-    for (int i = tid; i < cnt; i += kFinBlock) {
-      const uint64_t v = buf[i];
-      if (v >= thr) sel[atomicAdd(&s_nsel, 1)] = v;
+    for (int base = 0; base < cnt; base += kFinBlock) {
+      const int i = base + tid;
+      const uint64_t x = i < cnt ? buf[i] : 0;
+      const bool take = i < cnt && x >= thr;
+      const uint32_t mask = __ballot_sync(0xffffffffu, take);
+      if (mask) {
+        int pos = 0;
+        if (lane == 0) pos = atomicAdd(&s_nsel, __popc(mask));
+        pos = __shfl_sync(0xffffffffu, pos, 0);
+        if (take) sel[pos + __popc(mask & ((1u << lane) - 1u))] = x;
+      }
     }
     __syncthreads();
     nout = s_nsel;
@@ -794,10 +829,17 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
     for (int i = tid; i < cnt; i += kFinBlock) sel[i] = buf[i];
   }
   const int P = topk::next_pow2(nout > 1 ? nout : 1);
-  for (int i = nout + tid; i < P; i += kFinBlock) sel[i] = 0;
-  __syncthreads();
-  topk::bitonic_desc<kFinBlock>(sel, P, tid, 0);
-  __syncthreads();
+  if (P <= kFinSort) {
+    // pad to the register sort's fixed size
+    for (int i = nout + tid; i < kFinSort; i += kFinBlock) sel[i] = 0;
+    __syncthreads();
+    topk::block_sort_desc<kFinBlock, kFinSort / kFinBlock>(sel, tid);
+  } else {
+    for (int i = nout + tid; i < P; i += kFinBlock) sel[i] = 0;
+    __syncthreads();
+    topk::bitonic_desc<kFinBlock>(sel, P, tid, 0);
+    __syncthreads();
+  }
   for (int q = tid; q < k; q += kFinBlock) {
     const bool ok = q < nout;
     const uint64_t key = ok ? sel[q] : 0;
@@ -811,7 +853,8 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
                                    int32_t* idx, float* scores, uint64_t* keys_out, cudaStream_t stream) {
   if (nsplit > 1) {
     // few rows with many candidates each: a block per row
-    const size_t smem = (size_t)topk::next_pow2(nsplit * k) * 8 + (size_t)topk::next_pow2(k) * 8 + topk::kWarpBins * 4;
+    const size_t sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
+    const size_t smem = (size_t)topk::next_pow2(nsplit * k) * 8 + sel_cap * 8 + topk::kWarpBins * 4;
     if (smem > kSmemLimit || nsplit > 63) return cudaErrorInvalidConfiguration;
     cudaError_t e =
         cudaFuncSetAttribute(topk_finalize_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

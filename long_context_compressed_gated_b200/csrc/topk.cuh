@@ -696,6 +696,92 @@ __device__ __forceinline__ void warp_sort_lm_desc(uint64_t (&v)[R], int lane) {
   }
 }
 
+// One stage (size, stride) of a bitonic sort, descending overall, on a warp's
+// lane-major chunk of 32*R keys whose first key has index `base` in the whole
+// array (the direction of a pair depends on its global index).  stride < 32*R.
+template <int R>
+__device__ __forceinline__ void lm_stage_at(uint64_t (&v)[R], int size, int stride, int base, int lane) {
+  if (stride < R) {
+    // compile-time register indices per stride (a runtime index would put v in local memory)
+#define CSA_LMA_CASE(J)                                          \
+  case J:                                                        \
+    _Pragma("unroll") for (int r = 0; r < R; ++r) {              \
+      if ((r & J) == 0 && (r | J) < R) {                         \
+        const bool desc = ((base + lane * R + r) & size) == 0;   \
+        const uint64_t x = v[r], y = v[r | J];                   \
+        const bool sw = (x < y) == desc;                         \
+        v[r] = sw ? y : x;                                       \
+        v[r | J] = sw ? x : y;                                   \
+      }                                                          \
+    }                                                            \
+    break;
+    switch (stride) {
+      CSA_LMA_CASE(1)
+      CSA_LMA_CASE(2)
+      CSA_LMA_CASE(4)
+      CSA_LMA_CASE(8)
+      CSA_LMA_CASE(16)
+      default: break;
+    }
+#undef CSA_LMA_CASE
+  } else {
+    const int ls = stride / R;
+    const bool lower = (lane & ls) == 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint64_t y = __shfl_xor_sync(0xffffffffu, v[r], ls);
+      const bool desc = ((base + lane * R + r) & size) == 0;
+      const bool keep_max = lower == desc;
+      v[r] = ((v[r] > y) == keep_max) ? v[r] : y;
+    }
+  }
+}
+
+// Block bitonic sort, descending, of buf[0 .. NT*R) (NT threads, R keys per
+// lane).  Each warp sorts its chunk of 32*R keys in registers; every larger
+// merge runs its strides of 32*R and more as shared-memory compare-exchanges
+// (one barrier each) and its smaller strides in registers again: for 256
+// threads x 4 keys that is 10 barriers instead of one per stage (55).
+template <int NT, int R>
+__device__ void block_sort_desc(uint64_t* buf, int tid) {
+  constexpr int C = 32 * R, P = NT * R;
+  const int lane = tid & 31, base = (tid >> 5) * C;
+  uint64_t v[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) v[r] = buf[base + lane * R + r];
+#pragma unroll 1
+  for (int size = 2; size <= C; size <<= 1)
+#pragma unroll 1
+    for (int stride = size >> 1; stride > 0; stride >>= 1) lm_stage_at<R>(v, size, stride, base, lane);
+#pragma unroll
+  for (int r = 0; r < R; ++r) buf[base + lane * R + r] = v[r];
+  __syncthreads();
+#pragma unroll 1
+  for (int size = 2 * C; size <= P; size <<= 1) {
+#pragma unroll 1
+    for (int stride = size >> 1; stride >= C; stride >>= 1) {
+      for (int i = tid; i < P / 2; i += NT) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = (lo & size) == 0;
+        const uint64_t a = buf[lo], b = buf[hi];
+        if ((a < b) == desc) {
+          buf[lo] = b;
+          buf[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) v[r] = buf[base + lane * R + r];
+#pragma unroll 1
+    for (int stride = C >> 1; stride > 0; stride >>= 1) lm_stage_at<R>(v, size, stride, base, lane);
+#pragma unroll
+    for (int r = 0; r < R; ++r) buf[base + lane * R + r] = v[r];
+    __syncthreads();
+  }
+}
+
 __host__ __device__ constexpr int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;

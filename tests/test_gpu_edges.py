@@ -181,6 +181,30 @@ def test_decode_short_contexts_all_sequences(csa):
         assert_attention_close(O[b:b + 1], o, "decode attention seq %d" % b)
 
 
+def test_decode_k2048_split_search(csa):
+    """Decode with k=2048 over a 64K-token context: the key range is split over
+    several CTAs and the merged selection is larger than the block finalize's
+    register sort, so its shared-memory bitonic path runs."""
+    wl = inputs.Workload("dec_k2048", H=64, d=128, m=4, k=2048, W=128, HI=16, dI=128, batch=2, context=1 << 16,
+                         seed=23)
+    g = inputs.decode_batch(wl)
+    pos = [wl.context - 1, 30000]
+    scale = 1.0 / math.sqrt(wl.d)
+    gc = {k: v.cuda() for k, v in g.items()}
+    O, lse, idx, scores, ws = csa.csa_decode(gc["q"], gc["qI_codes"], gc["qI_scales"], gc["w_codes"], gc["Kc"],
+                                             gc["Vc"], gc["kI_codes"], gc["kI_scales"], gc["Kwin"], gc["Vwin"], pos,
+                                             wl.m, wl.k, scale)
+    assert csa.csa_check_status(ws) == 0
+    for b, t in enumerate(pos):
+        I = oracle.indexer(g["qI_codes"][b:b + 1], g["qI_scales"][b:b + 1], g["w_codes"][b:b + 1], g["kI_codes"][b],
+                           g["kI_scales"][b], t, wl.m)
+        want_idx, want_top = oracle.topk(I, oracle.n_vis([t], wl.m), wl.k)
+        assert_topk_exact(idx[b:b + 1], scores[b:b + 1], want_idx, want_top, "decode k=2048 seq %d" % b)
+        o, l = oracle.attention(g["q"][b:b + 1], g["Kc"][b], g["Vc"][b], g["Kwin"][b], g["Vwin"][b], t, wl.m, wl.W,
+                                scale, sel=want_idx, rows=[0], raw_pos0=t - wl.W + 1)
+        assert_attention_close(O[b:b + 1], o, "decode k=2048 attention seq %d" % b)
+
+
 def test_hca_decode(csa):
     wl = inputs.Workload("hdec", H=64, d=128, m=128, W=128, batch=3, context=1 << 20, seed=22)
     n = wl.context // wl.m
