@@ -152,9 +152,7 @@ struct IndexerSmem {
   static constexpr size_t off_sf = off_a + (size_t)kStages * kABytes;  // key scales, tcgen05.cp layout
   static constexpr size_t off_ma = off_sf + (size_t)kStages * 512;
   static constexpr size_t off_mb = off_ma + 4096;
-  static constexpr size_t off_w2 = off_mb + (size_t)N * 32;
-  static constexpr size_t off_sumw = off_w2 + (size_t)N * 4;
-  static constexpr size_t off_cnt = off_sumw + 64 * 4;
+  static constexpr size_t off_cnt = off_mb + (size_t)N * 32;
   static constexpr size_t off_thr = off_cnt + 64 * 4;
   static constexpr size_t off_hist = off_thr + 64 * 8;  // per token, kWarpBins ints
   static constexpr size_t off_grp = off_hist + (size_t)G * topk::kWarpBins * 4;  // [2][32] ints: group scratch
@@ -192,8 +190,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* s_sf = smem + L::off_sf;
   uint8_t* s_ma = smem + L::off_ma;
   uint8_t* s_mb = smem + L::off_mb;
-  int* s_w2 = reinterpret_cast<int*>(smem + L::off_w2);
-  int* s_sumw = reinterpret_cast<int*>(smem + L::off_sumw);
   int* s_cnt = reinterpret_cast<int*>(smem + L::off_cnt);
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L::off_thr);
   int* s_hist = reinterpret_cast<int*>(smem + L::off_hist);
@@ -255,21 +251,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     reinterpret_cast<uint4*>(s_ma)[i] = make_uint4(0x22222222u, 0x22222222u, 0x22222222u, 0x22222222u);
   for (int i = tid; i < N * 32 / 16; i += kThreads)
     reinterpret_cast<uint4*>(s_mb)[i] = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);
-  for (int c = tid; c < N; c += kThreads) {
-    const int g = c / HI, h = c % HI;
-    const int64_t r = row0 + g;
-    int w2 = 0;
-    if (g < G && r < a.rows) w2 = e2m1_times2(a.w_codes[r * HI + h] & 15u);
-    s_w2[c] = w2;
-  }
   if (tid < G) {
-    int sw = 0;
-    const int64_t r = row0 + tid;
-    if (r < a.rows)
-      for (int h = 0; h < HI; ++h) sw += e2m1_times2(a.w_codes[r * HI + h] & 15u);
-    s_sumw[tid] = sw;
     s_cnt[tid] = 0;
     s_thr[tid] = 0;
+  }
+  // The epilogue warps' global reads (their tokens' head weights; the query
+  // scales, by the first half) are issued here, before the block barrier, so
+  // that their latency overlaps the setup and the first TMA loads.
+  constexpr int CW = G0 * HI;  // accumulator columns of one half
+  const int half = (warp - 2) >> 2;   // which half of the epilogue (warps 2..9)
+  const int g_lo = kAlt ? 0 : half * G0;
+  uint32_t wraw[CW / 4];  // the half's weight codes, four per word (decoded after the barrier)
+  uint32_t qsc[8];
+  if (warp >= 2) {
+    // the half's CW weight codes are consecutive bytes: rows row0+g_lo .. (one
+    // code per head), read as broadcast 32-bit words; rows past the end give code 0
+    const int64_t wb = (row0 + g_lo) * HI;
+#pragma unroll
+    for (int u = 0; u < CW / 4; ++u) {
+      const bool in = row0 + g_lo + (4 * u) / HI < a.rows;
+      wraw[u] = in ? __ldg(reinterpret_cast<const uint32_t*>(a.w_codes + wb) + u) : 0u;
+    }
+    if (half == 0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int rr = lane + 32 * c;  // row (g*HI + h) of the B operand
+        const int g = rr / HI, h = rr % HI;
+        const int64_t r = row0 + g;
+        uint32_t v = 0x7F7F7F7Fu;
+        if (rr < G * HI && r < a.rows) {
+          const uint8_t* p = a.q_scales + (r * HI + h) * (DI / 32);
+          v = DI == 128 ? __ldg(reinterpret_cast<const uint32_t*>(p)) : (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p));
+        }
+        qsc[c] = v;
+      }
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -393,21 +409,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // =========================== epilogue + selection (warps 2..9)
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;   // which half of the epilogue
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     // scale factors of the query rows and the constant-offset operands (replicated layout)
     if (half == 0) {
       uint32_t w[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const int rr = lane + 32 * c;  // row (g*HI + h) of the B operand
-        const int g = rr / HI, h = rr % HI;
-        const int64_t r = row0 + g;
-        uint32_t v = 0x7F7F7F7Fu;
-        if (rr < G * HI && r < a.rows) {
-          const uint8_t* p = a.q_scales + (r * HI + h) * (DI / 32);
-          v = DI == 128 ? *reinterpret_cast<const uint32_t*>(p)
-                        : ((uint32_t)*reinterpret_cast<const uint16_t*>(p) | 0x7F7F0000u);
+        const int rr = lane + 32 * c;
+        const bool live = rr < G * HI && row0 + rr / HI < a.rows;
+        const uint32_t v = DI == 128 || !live ? qsc[c] : qsc[c] | 0x7F7F0000u;
+        if (live) {
           bool bad = false;
 #pragma unroll
           for (int b = 0; b < DI / 32; ++b) {
@@ -432,8 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(ready);
 
     // tokens of this half and the token whose buffer this warp maintains
-    constexpr int CW = G0 * HI;  // accumulator columns of one half
-    const int g_lo = kAlt ? 0 : half * G0;
     const int c0 = kAlt ? 0 : half * CW;
     // the warps that insert into the same buffers form a group: one half (prefill)
     // or all eight epilogue warps (decode); cut-backs and the final selection are
@@ -443,15 +452,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gt = kAlt ? tid - 64 : tid - 64 - half * (kEpiThreads / 2);
     int* gscr = s_grp + (kAlt ? 0 : half) * 32;
     // per-warp copies of what every tile needs: weights, weight sums, visibility, thresholds
-    int wreg[CW];
+    int wreg[CW];  // 2*w of the half's tokens, column order (token-major, then head)
 #pragma unroll
-    for (int i = 0; i < CW; ++i) wreg[i] = s_w2[c0 + i];
+    for (int u = 0; u < CW / 4; ++u)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) wreg[4 * u + q] = e2m1_times2((wraw[u] >> (8 * q)) & 15u);
     uint32_t sumw_magic[G0];
     int64_t nvis[G0];
     uint64_t thr[G0];  // running thresholds, refreshed at every meeting
 #pragma unroll
     for (int t = 0; t < G0; ++t) {
-      sumw_magic[t] = kMagicBits * (uint32_t)s_sumw[g_lo + t];
+      int sw = 0;
+#pragma unroll
+      for (int h = 0; h < HI; ++h) sw += wreg[t * HI + h];
+      sumw_magic[t] = kMagicBits * (uint32_t)sw;
       nvis[t] = kAlt ? tnvis[0] : (half == 0 ? tnvis[t] : tnvis[(G0 + t) % G]);
       thr[t] = 0;
     }
