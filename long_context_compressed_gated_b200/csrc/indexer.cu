@@ -500,11 +500,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // but not its meetings, so that no partner warp is left at a named barrier.
     bool dead = false;
     int seen_group = -1;  // barrier group whose accumulators are known complete
+    // The next tile's accumulator is probed (without blocking) a tile early, right
+    // after this tile's head sums, so that the probe's latency hides behind the
+    // insertion work; the blocking wait runs only when the probe saw it incomplete.
+    bool next_ready = false;
     for (int rd = 0; rd < nrounds; ++rd) {
       const int it = kAlt ? 2 * rd + half : rd;
       if (it < ntiles && !dead && it / TPG != seen_group) {
         seen_group = it / TPG;
-        dead = !mbar_wait(&dfull[seen_group % NBG], (seen_group / NBG) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+        if (!next_ready)
+          dead = !mbar_wait(&dfull[seen_group % NBG], (seen_group / NBG) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
       }
       if (it < ntiles && !dead) {
         const int b = it % NB;
@@ -528,6 +533,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dempty[(it / TPG) % NBG]);
+        {
+          const int itn = kAlt ? it + 2 : it + 1, gn = itn / TPG;
+          next_ready = itn < ntiles && gn != seen_group && mbar_test(&dfull[gn % NBG], (gn / NBG) & 1);
+        }
         finish_insert();  // previous tile's stores
         // this tile: keys, ballots and buffer reservations
         const int64_t j = j_begin + (int64_t)it * 128 + quarter * 32 + lane;
