@@ -926,14 +926,31 @@ static bool choose_cap(int k, int* cap, int* check) {
   const size_t base = L::bytes(0);
   const int budget = base < kSmemLimit ? (int)((kSmemLimit - base) / (8 * (size_t)G)) & ~127 : 0;
   const int p = topk::next_pow2(k);
-  for (int c = 4; c >= (G == 1 ? 2 : 1); c >>= 1) {
+  // capacity for meetings every c tiles: room for c tiles above the cut-back level
+  auto fit = [&](int c, int* cp) {
     const int need = k + 128 * c > p ? k + 128 * c : p;
-    if (budget >= need) {
-      int want = 4 * k + 128 * c;  // cut-backs rare: room for several k between them
-      if (want < 4096) want = 4096;
-      if (want < need) want = need;
-      *cap = (want < budget ? want : budget) & ~127;
-      if (*cap < need) *cap = ((need + 127) / 128) * 128;
+    if (budget < need) return false;
+    int want = 4 * k + 128 * c;  // cut-backs rare: room for several k between them
+    if (want < 4096) want = 4096;
+    if (want < need) want = need;
+    *cp = (want < budget ? want : budget) & ~127;
+    if (*cp < need) *cp = ((need + 127) / 128) * 128;
+    return true;
+  };
+  // Meetings every 8 or 16 tiles when the buffer still leaves 3k keys below the
+  // cut-back level (fewer meetings without more cut-backs); else every 4 or fewer.
+  for (int c = 16; c >= 8; c >>= 1) {
+    int cp;
+    if (fit(c, &cp) && cp - 128 * c >= 3 * k) {
+      *cap = cp;
+      *check = c;
+      return true;
+    }
+  }
+  for (int c = 4; c >= (G == 1 ? 2 : 1); c >>= 1) {
+    int cp;
+    if (fit(c, &cp)) {
+      *cap = cp;
       *check = c;
       return true;
     }
