@@ -154,8 +154,10 @@ struct IndexerSmem {
   static constexpr size_t off_mb = off_ma + 4096;
   static constexpr size_t off_cnt = off_mb + (size_t)N * 32;
   static constexpr size_t off_thr = off_cnt + 64 * 4;
-  static constexpr size_t off_hist = off_thr + 64 * 8;  // per token, kWarpBins ints
-  static constexpr size_t off_grp = off_hist + (size_t)G * topk::kWarpBins * 4;  // [2][32] ints: group scratch
+  // one score histogram per selection group (a half, or all eight epilogue warps in
+  // decode): a group cuts its buffers back one at a time
+  static constexpr size_t off_hist = off_thr + 64 * 8;
+  static constexpr size_t off_grp = off_hist + (size_t)(G == 1 ? 1 : 2) * topk::kWarpBins * 4;  // [2][32] ints
   static constexpr size_t off_bar = off_grp + 256;
   static constexpr size_t off_tslot = off_bar + (2 * kStages + 2 * NB + 1) * 8;
   static constexpr size_t off_cand = ((off_tslot + 16 + 15) / 16) * 16;
@@ -451,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gbar = kAlt ? kEpiBar : kHalfBar0 + half;
     const int gt = kAlt ? tid - 64 : tid - 64 - half * (kEpiThreads / 2);
     int* gscr = s_grp + (kAlt ? 0 : half) * 32;
+    int* ghist = s_hist + (kAlt ? 0 : half) * topk::kWarpBins;
     // per-warp copies of what every tile needs: weights, weight sums, visibility, thresholds
     int wreg[CW];  // 2*w of the half's tokens, column order (token-major, then head)
 #pragma unroll
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cnt = s_cnt[gg];
         if (cnt > cap - 128 * a.check) {
           const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, cap - 128 * a.check, false,
-                                                         s_hist + gg * topk::kWarpBins, gscr, gt, gbar);
+                                                         ghist, gscr, gt, gbar);
           const int n = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
           if (gt == 0) {
             s_cnt[gg] = n;
@@ -591,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* buf = s_cand + (size_t)gg * cap;
       int cnt = s_cnt[gg];
       if (cnt > a.k) {
-        const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, s_hist + gg * topk::kWarpBins, gscr,
+        const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, ghist, gscr,
                                                        gt, gbar);
         cnt = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
       }
