@@ -35,9 +35,9 @@ FP4_OVER_BF16 = 4.0  # nominal dense ratio (9 vs 2.25 PFLOP/s)
 # kernels on the T=32768 CSA prefill, from the ncu captures summarised under profiles/;
 # to be refreshed whenever those kernels change.
 PHASE_TRAFFIC = {
-    "indexer_topk": (146.758400e6 + 92.925952e6 + 130.459648e6 + 37.678080e6,
+    "indexer_topk": (146.680064e6 + 93.195520e6 + 130.341120e6 + 37.730560e6,
                      "profiles/indexer_topk_csa_prefill_T32768.md (indexer + finalize launches)"),
-    "sparse_attn": (626.033664e6 + 495.090432e6, "profiles/attention_csa_prefill_T32768.md"),
+    "sparse_attn": (626.845696e6 + 497.474304e6, "profiles/attention_csa_prefill_T32768.md"),
 }
 
 
