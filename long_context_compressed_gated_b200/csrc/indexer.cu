@@ -688,13 +688,13 @@ __global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __re
 }
 
 // Block-wide finalize for rows with many candidates (a split decode search):
-// 256 threads per row.  One min/max pass and one 1024-bin histogram over the
+// 1024 threads per row.  One min/max pass and one 1024-bin histogram over the
 // score range find the bin that holds the k-th key; the keys of that bin are
 // resolved exactly (in-register sort when it holds at most 32, else the warp
 // radix fallback); the k best are compacted, sorted (per-warp register sorts
 // merged through shared memory) and written.  The row's keys are loaded 16 per
 // thread at a time, so the gather costs a few memory round trips.
-constexpr int kFinBlock = 256;
+constexpr int kFinBlock = 1024;
 constexpr int kFinSort = 1024;  // keys sorted by the register/shared hybrid sort
 
 __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const uint64_t* __restrict__ cand,
@@ -711,7 +711,7 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
   uint64_t* sel = buf + cap;                              // [sel_cap] the k best
   int* hist = reinterpret_cast<int*>(sel + sel_cap);      // [kWarpBins]
   __shared__ int s_off[64];
-  __shared__ uint32_t s_lo[8], s_hi[8];
+  __shared__ uint32_t s_lo[kFinBlock / 32], s_hi[kFinBlock / 32];
   __shared__ int s_bin, s_kept, s_inbin, s_nsel;
   __shared__ uint64_t s_thr;
   // gather the per-range lists (offsets by a prefix over the counts).  The loads
