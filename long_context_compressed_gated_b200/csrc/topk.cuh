@@ -26,89 +26,6 @@ __device__ __forceinline__ int32_t key_score(uint64_t key) {
   return (int32_t)((uint32_t)(key >> 32) ^ 0x80000000u);
 }
 
-// Smallest threshold `thr` such that exactly min(keep, cnt) of buf[0..cnt) satisfy
-// key >= thr (radix select, 8-bit digits from the top, early exit as soon as the
-// selected digit bucket is taken whole).  hist: 256 ints, sh: 4 ints of shared
-// scratch.  Returns 0 when cnt <= keep (everything is kept).
-template <int NT>
-__device__ uint64_t radix_threshold(const uint64_t* buf, int cnt, int keep, int* hist, int* sh, int tid,
-                                    int bar_id) {
-  if (cnt <= keep) return 0;
-  uint64_t prefix = 0, pmask = 0;
-  int need = keep;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
-    named_sync(bar_id, NT);
-    for (int i = tid; i < cnt; i += NT) {
-      const uint64_t key = buf[i];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(int)(key >> shift) & 255], 1);
-    }
-    named_sync(bar_id, NT);
-    if (tid < 32) {
-      // lane l owns digits 255-8l .. 248-8l (descending): exclusive scan across lanes
-      int c[8], tot = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        c[e] = hist[255 - (tid * 8 + e)];
-        tot += c[e];
-      }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += v;
-      }
-      const int excl = incl - tot;
-      if (excl < need && need <= incl) {
-        int cum = excl;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (cum + c[e] >= need) {
-            sh[0] = 255 - (tid * 8 + e);
-            sh[1] = cum;
-            sh[2] = c[e];
-            break;
-          }
-          cum += c[e];
-        }
-      }
-    }
-    named_sync(bar_id, NT);
-    const int d = sh[0], cum_gt = sh[1], hd = sh[2];
-    named_sync(bar_id, NT);  // everyone has read sh before it is rewritten
-    need -= cum_gt;
-    prefix |= (uint64_t)d << shift;
-    pmask |= (uint64_t)255 << shift;
-    if (hd == need) break;
-  }
-  return prefix;
-}
-
-// Keep the keys >= thr of buf[0..cnt) (compacted to the front, any order).
-// Returns the new count. MAXPER bounds the keys per thread (cnt <= NT*MAXPER).
-template <int NT, int MAXPER>
-__device__ int compact_ge(uint64_t* buf, int cnt, uint64_t thr, int* counter, int tid, int bar_id) {
-  uint64_t v[MAXPER];
-#pragma unroll
-  for (int e = 0; e < MAXPER; ++e) {
-    const int i = tid + e * NT;
-    v[e] = i < cnt ? buf[i] : 0;
-  }
-  if (tid == 0) *counter = 0;
-  named_sync(bar_id, NT);
-#pragma unroll
-  for (int e = 0; e < MAXPER; ++e) {
-    if (v[e] != 0 && v[e] >= thr) {
-      const int p = atomicAdd(counter, 1);
-      buf[p] = v[e];
-    }
-  }
-  named_sync(bar_id, NT);
-  const int n = *counter;
-  named_sync(bar_id, NT);
-  return n;
-}
-
 // Sort buf[0..P) descending (P a power of two; pad with zeros beforehand).
 template <int NT>
 __device__ void bitonic_desc(uint64_t* buf, int P, int tid, int bar_id) {
@@ -383,33 +300,6 @@ __device__ uint64_t warp_select_threshold(const uint64_t* buf, int cnt, int keep
   return warp_exact_threshold(buf, cnt, keep, hist, lane);
 }
 
-// One-pass approximate cut: a score threshold keeping at least `keep` keys (all
-// keys of the threshold bin are kept).  Returns the number kept through *kept.
-// Falls back to the exact threshold when ties would keep more than `room`.
-__device__ uint64_t warp_approx_threshold(const uint64_t* buf, int cnt, int keep, int room, int* hist, int lane,
-                                          int* kept_out) {
-  if (cnt <= keep) {
-    *kept_out = cnt;
-    return 0;
-  }
-  uint32_t lo, hi;
-  warp_score_range(buf, cnt, lane, &lo, &hi);
-  if (hi > lo) {
-    const int bits = 32 - __clz(hi - lo);
-    const int shift = bits > 10 ? bits - 10 : 0;
-    warp_score_hist(buf, cnt, lo, shift, hist, lane);
-    int bin, kept;
-    warp_hist_cut(hist, keep, lane, &bin, &kept);
-    __syncwarp();
-    if (kept <= room) {
-      *kept_out = kept;
-      return (uint64_t)(lo + ((uint32_t)bin << shift)) << 32;
-    }
-  }
-  *kept_out = keep;
-  return warp_select_threshold(buf, cnt, keep, hist, lane);
-}
-
 // Sort buf[0..P) descending (P a power of two, padding zeros), one warp.  Each
 // compare-exchange stage loads a batch of pairs per lane before swapping them.
 __device__ void warp_bitonic_desc(uint64_t* buf, int P, int lane) {
@@ -445,61 +335,6 @@ __device__ void warp_bitonic_desc(uint64_t* buf, int P, int lane) {
         }
       }
       __syncwarp();
-    }
-  }
-}
-
-// Register-resident bitonic sort of 32*R keys, descending; element e = r*32 + lane
-// lives in v[r] of lane `lane`.  Strides below 32 exchange across lanes by
-// shuffles, strides of 32 and more swap registers within a lane (the register
-// pair is a compile-time choice per case).  Pad with zeros to fill 32*R.
-template <int R>
-__device__ __forceinline__ void sort_within_lane(uint64_t (&v)[R], int j, int size) {
-  // partner of register r is r ^ j (j = stride / 32, a power of two below R)
-#define CSA_WITHIN_CASE(J)                                                \
-  case J:                                                                 \
-    _Pragma("unroll") for (int r = 0; r < R; ++r) {                       \
-      if ((r & J) == 0 && (r ^ J) < R) {                                  \
-        const bool desc = ((r * 32) & size) == 0;                         \
-        const uint64_t x = v[r], y = v[r ^ J];                            \
-        const bool sw = (x < y) == desc;                                  \
-        v[r] = sw ? y : x;                                                \
-        v[r ^ J] = sw ? x : y;                                            \
-      }                                                                   \
-    }                                                                     \
-    break;
-  switch (j) {
-    CSA_WITHIN_CASE(1)
-    CSA_WITHIN_CASE(2)
-    CSA_WITHIN_CASE(4)
-    CSA_WITHIN_CASE(8)
-    CSA_WITHIN_CASE(16)
-    CSA_WITHIN_CASE(32)
-    default: break;
-  }
-#undef CSA_WITHIN_CASE
-}
-
-template <int R>
-__device__ __forceinline__ void warp_sort_regs_desc(uint64_t (&v)[R], int lane) {
-  constexpr int P = 32 * R;
-#pragma unroll 1
-  for (int size = 2; size <= P; size <<= 1) {
-#pragma unroll 1
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= 32) {
-        sort_within_lane<R>(v, stride >> 5, size);
-      } else {
-        const bool lower = (lane & stride) == 0;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint64_t y = __shfl_xor_sync(0xffffffffu, v[r], stride);
-          const bool desc = (((r << 5) | lane) & size) == 0;
-          const bool keep_max = lower == desc;
-          const bool gt = v[r] > y;
-          v[r] = (gt == keep_max) ? v[r] : y;
-        }
-      }
     }
   }
 }
