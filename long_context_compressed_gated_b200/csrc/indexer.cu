@@ -29,9 +29,10 @@
 //    row, selects its k best and sorts them (score desc, j asc).
 //  * Warp roles: warp 0 TMA producer (key codes; scales by cp.async straight
 //    into the tcgen05.cp layout), warp 1 TMEM allocation and MMA issue, warps
-//    2..9 epilogue + selection.  Key tiles are 4- or 8-stage pipelined; NB
-//    accumulator buffers in TMEM (3 for 128-column groups, 8 for decode) keep
-//    the MMAs ahead of the epilogue.
+//    2..9 epilogue + selection.  Key tiles are pipelined in a 4-stage ring (16
+//    in decode, which streams its keys from HBM); NB accumulator buffers in
+//    TMEM (3 for 128-column groups, 8 for decode) keep the MMAs ahead of the
+//    epilogue.
 #include <cuda.h>
 
 #include "common.cuh"
