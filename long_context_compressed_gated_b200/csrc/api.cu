@@ -109,6 +109,7 @@ int decode_nsplit(int B, int64_t Ncap, int k) {
   if (ns > tiles) ns = (int)tiles;
   const int lim = 256 * 40 / k;  // merge capacity
   if (ns > lim) ns = lim;
+  if (ns > kMaxKeyRanges) ns = kMaxKeyRanges;
   return ns < 1 ? 1 : ns;
 }
 

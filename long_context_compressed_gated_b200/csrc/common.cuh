@@ -31,4 +31,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // Workspace header: status word + padding to 256 bytes.
 constexpr size_t kWorkspaceHeader = 256;
 
+// Most key ranges one decode sequence's indexer search is split into (the
+// block finalize that merges them keeps one prefix entry per range).
+constexpr int kMaxKeyRanges = 63;
+
 }  // namespace csa

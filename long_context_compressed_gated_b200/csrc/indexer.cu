@@ -711,7 +711,7 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
   const int sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
   uint64_t* sel = buf + cap;                              // [sel_cap] the k best
   int* hist = reinterpret_cast<int*>(sel + sel_cap);      // [kWarpBins]
-  __shared__ int s_off[64];
+  __shared__ int s_off[kMaxKeyRanges + 1];
   __shared__ uint32_t s_lo[kFinBlock / 32], s_hi[kFinBlock / 32];
   __shared__ int s_bin, s_kept, s_inbin, s_nsel;
   __shared__ uint64_t s_thr;
@@ -882,7 +882,7 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
     // few rows with many candidates each: a block per row
     const size_t sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
     const size_t smem = (size_t)topk::next_pow2(nsplit * k) * 8 + sel_cap * 8 + topk::kWarpBins * 4;
-    if (smem > kSmemLimit || nsplit > 63) return cudaErrorInvalidConfiguration;
+    if (smem > kSmemLimit || nsplit > kMaxKeyRanges) return cudaErrorInvalidConfiguration;
     cudaError_t e =
         cudaFuncSetAttribute(topk_finalize_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -205,6 +205,31 @@ def test_decode_k2048_split_search(csa):
         assert_attention_close(O[b:b + 1], o, "decode k=2048 attention seq %d" % b)
 
 
+@pytest.mark.parametrize("k,context", [(1024, 1 << 18), (64, 1 << 17)])
+def test_decode_single_sequence_widest_split(csa, k, context):
+    """One sequence over a long context: its key range is split over the most
+    CTAs the merge allows (10 ranges at k = 1024; at k = 64 the SM count would give
+    148 and the range limit of the block finalize, 63, applies)."""
+    wl = inputs.Workload("dec_b1", H=64, d=128, m=4, k=k, W=128, HI=16, dI=128, batch=1, context=context,
+                         seed=24 + k)
+    g = inputs.decode_batch(wl)
+    pos = [wl.context - 1]
+    scale = 1.0 / math.sqrt(wl.d)
+    gc = {key: v.cuda() for key, v in g.items()}
+    O, lse, idx, scores, ws = csa.csa_decode(gc["q"], gc["qI_codes"], gc["qI_scales"], gc["w_codes"], gc["Kc"],
+                                             gc["Vc"], gc["kI_codes"], gc["kI_scales"], gc["Kwin"], gc["Vwin"], pos,
+                                             wl.m, wl.k, scale)
+    assert csa.csa_check_status(ws) == 0
+    t = pos[0]
+    I = oracle.indexer(g["qI_codes"], g["qI_scales"], g["w_codes"], g["kI_codes"][0], g["kI_scales"][0], t, wl.m)
+    want_idx, want_top = oracle.topk(I, oracle.n_vis([t], wl.m), wl.k)
+    assert_topk_exact(idx, scores, want_idx, want_top, "decode B=1 k=%d" % k)
+    o, l = oracle.attention(g["q"], g["Kc"][0], g["Vc"][0], g["Kwin"][0], g["Vwin"][0], t, wl.m, wl.W, scale,
+                            sel=want_idx, rows=[0], raw_pos0=t - wl.W + 1)
+    assert_attention_close(O, o, "decode B=1 k=%d attention" % k)
+    np.testing.assert_allclose(lse.cpu().numpy(), l, atol=2e-3)
+
+
 def test_hca_decode(csa):
     wl = inputs.Workload("hdec", H=64, d=128, m=128, W=128, batch=3, context=1 << 20, seed=22)
     n = wl.context // wl.m
