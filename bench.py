@@ -34,6 +34,8 @@ FP4_OVER_BF16 = 4.0  # nominal dense ratio (9 vs 2.25 PFLOP/s)
 # DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum) of each phase's
 # kernels on the T=32768 CSA prefill, from the ncu captures summarised under profiles/;
 # to be refreshed whenever those kernels change.
+E2E_CHUNKS = 16  # query chunks of the pipelined end-to-end step
+
 PHASE_TRAFFIC = {
     "indexer_topk": (146.680064e6 + 93.195520e6 + 130.341120e6 + 37.730560e6,
                      "profiles/indexer_topk_csa_prefill_T32768.md (indexer + finalize launches)"),
@@ -219,25 +221,64 @@ def run_csa_prefill(csa, wl, steps, warmup, dist_on, rank):
     ms = t0.elapsed_time(t1) / steps
     status = csa.csa_check_status(ws)
     phases = timer.per_phase_ms()
-    # e2e through the public API with host buffers: H2D of the step's inputs, D2H of O
+    # e2e through the public API with host buffers: H2D of the step's inputs, D2H of O.
+    # The step is pipelined over query chunks on three streams: the inputs every
+    # chunk needs (K, V, Z, B, the indexer keys) go first and are compressed; then
+    # chunk c's queries are copied in while chunk c-1 is scored and attended, and
+    # chunk c-1's output is copied out (chunked calls give the unchunked result).
     host = {k: v.cpu().pin_memory() for k, v in d.items() if k != "B_hca"}
     O_host = torch.empty(O.shape, dtype=O.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = O.numel() * O.element_size()
     dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    shared = ("K", "V", "Z", "B", "kI_codes", "kI_scales")
+    per_row = [k for k in host if k not in shared]  # query-row tensors: Q, qI codes / scales, w
+    n_chunks = E2E_CHUNKS if T % E2E_CHUNKS == 0 and (T // E2E_CHUNKS) % wl.m == 0 else 1
+    C = T // n_chunks
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_step():
-        for k, v in host.items():
-            dev[k].copy_(v, non_blocking=True)
-        csa.csa_compress(dev["K"], dev["V"], dev["Z"], dev["B"], wl.m, Kc=Kc, Vc=Vc)
-        csa.csa_indexer_topk(dev["qI_codes"], dev["qI_scales"], dev["w_codes"], dev["kI_codes"], dev["kI_scales"],
-                             wl.m, wl.k, idx=idx, want_scores=False, workspace=ws)
-        csa.csa_sparse_attn(dev["Q"], Kc, Vc, idx, dev["K"], dev["V"], wl.W, scale, O=O, want_lse=False,
-                            workspace=ws)
-        O_host.copy_(O, non_blocking=True)
+        main = torch.cuda.current_stream()
+        for s_ in (s_in, s_comp, s_out):
+            s_.wait_stream(main)
+        ev_shared = torch.cuda.Event()
+        ev_in = [torch.cuda.Event() for _ in range(n_chunks)]
+        ev_done = [torch.cuda.Event() for _ in range(n_chunks)]
+        with torch.cuda.stream(s_in):
+            for k in shared:
+                dev[k].copy_(host[k], non_blocking=True)
+            ev_shared.record()
+            for c in range(n_chunks):
+                sl = slice(c * C, (c + 1) * C)
+                for k in per_row:
+                    dev[k][sl].copy_(host[k][sl], non_blocking=True)
+                ev_in[c].record()
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_shared)
+            csa.csa_compress(dev["K"], dev["V"], dev["Z"], dev["B"], wl.m, Kc=Kc, Vc=Vc)
+            for c in range(n_chunks):
+                t0c = c * C
+                sl = slice(t0c, t0c + C)
+                e1 = (t0c + C) // wl.m
+                s_comp.wait_event(ev_in[c])
+                csa.csa_indexer_topk(dev["qI_codes"][sl], dev["qI_scales"][sl], dev["w_codes"][sl],
+                                     dev["kI_codes"][:e1], dev["kI_scales"][:e1], wl.m, wl.k, t0=t0c, idx=idx[sl],
+                                     want_scores=False, workspace=ws)
+                csa.csa_sparse_attn(dev["Q"][sl], Kc[:e1], Vc[:e1], idx[sl], dev["K"][: t0c + C],
+                                    dev["V"][: t0c + C], wl.W, scale, t0=t0c, O=O[sl], want_lse=False, workspace=ws)
+                ev_done[c].record()
+        with torch.cuda.stream(s_out):
+            for c in range(n_chunks):
+                sl = slice(c * C, (c + 1) * C)
+                s_out.wait_event(ev_done[c])
+                O_host[sl].copy_(O[sl], non_blocking=True)
+        for s_ in (s_in, s_comp, s_out):
+            main.wait_stream(s_)
 
+    O_dev_ref = O.clone()  # output of the device-resident (timed) path, same inputs
     e2e_step()
     barrier(dist_on)
+    e2e_matches = bool(torch.equal(O_host, O_dev_ref.cpu()))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     n_e2e = max(1, min(steps, 3))
@@ -249,7 +290,7 @@ def run_csa_prefill(csa, wl, steps, warmup, dist_on, rank):
     e2e_ms = e0.elapsed_time(e1) / n_e2e
     del dev, host
     return {"ms": ms, "phases": phases, "status": status, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launches_per_step": 3}
+            "launches_per_step": 3, "e2e_chunks": n_chunks, "e2e_matches": e2e_matches}
 
 
 def run_hca_prefill(csa, wl, steps, warmup):
@@ -528,7 +569,8 @@ def main():
                     "sparse_attn_ms": ph["sparse_attn"], "sparse_attn_tflops": attn_tf,
                     "sparse_attn_frac_bf16": attn_tf / peaks["bf16_tflops"]},
         "e2e": {"value": job_throughput(wl.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
-                "d2h_bytes_per_step": res["d2h"]},
+                "d2h_bytes_per_step": res["d2h"], "pipelined_chunks": res["e2e_chunks"],
+                "output_equals_device_path": res["e2e_matches"]},
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": sampler.summary(),
         "device_status": res["status"],
