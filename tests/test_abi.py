@@ -85,3 +85,35 @@ def test_zero_sized_calls_are_no_ops(lib):
     assert lib.csa_compress(fake, fake, fake, fake, 0, 128, 4, fake, fake, None) == 0
     assert lib.csa_indexer_topk(fake, fake, fake, fake, fake, 0, 0, 0, 16, 128, 4, 8, fake, None, fake, 256,
                                 None) == 0
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+def _decode_workspace(B, Ncap, H, d, k, W):
+    """The decode workspace layout: a 256-byte status header, positions [B] i64,
+    the merged selection [B,k] i32, each key range's candidate keys [B,ns,k] u64
+    and counts [B,ns] i32, and split-attention partials [B,nsa,H,d] f32 + [B,nsa,H]
+    f32 when a sequence's attention is split.  ns: key ranges per sequence (one
+    wave of one-CTA-per-SM blocks, at most one per 128-key tile, at most what one
+    finalize block merges, at most 63); nsa: attention splits (one wave, at most
+    16, at most one per key tile)."""
+    ns = max(1, min(148 // B, -(-Ncap // 128), 256 * 40 // k, 63))
+    tiles = -(-k // 128) + (-(-W // 128) if W > 0 else 0)
+    nsa = max(1, min(148 // B, 16, tiles))
+    part = _align256(B * nsa * H * d * 4) + _align256(B * nsa * H * 4) if nsa > 1 else 0
+    return 256 + _align256(B * 8) + _align256(B * k * 4) + _align256(B * ns * k * 8) + _align256(B * ns * 4) + part
+
+
+@pytest.mark.parametrize("B,Ncap,k,W", [
+    (16, 262144, 1024, 128),   # the 1M-context decode: 9 key ranges per sequence
+    (1, 65536, 1024, 128),     # one sequence: the merge limit (10 ranges at k = 1024)
+    (1, 32768, 64, 128),       # one sequence, small k: the 63-range limit
+    (4, 1024, 64, 32),         # short cache: one range per 128-key tile
+    (64, 262144, 512, 0),      # many sequences, no window
+])
+def test_decode_workspace_follows_the_split_rule(lib, B, Ncap, k, W):
+    H, d = 64, 128
+    got = lib.csa_decode_workspace_bytes(B, Ncap, H, d, 16, 128, k, W)
+    assert got == _decode_workspace(B, Ncap, H, d, k, W)
