@@ -30,7 +30,7 @@ from long_context_compressed_gated_b200 import inputs  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 METRIC = "CSA/HCA prefill tokens/s & TFLOP/s; 1M-ctx decode GB/s; % of B200 roofline"
-FP4_OVER_BF16 = 4.0  # nominal dense ratio (9 vs 2.25 PFLOP/s)
+NOMINAL_FP4_TFLOPS = 9000.0  # NVIDIA's dense FP4 figure for B200 (context only)
 # DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum) of each phase's
 # kernels on the T=32768 CSA prefill, from the ncu captures summarised under profiles/;
 # to be refreshed whenever those kernels change.
@@ -51,6 +51,52 @@ def load_peaks():
                 "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------- tensor-pipe peaks
+def measure_tensor_peaks(csa, sustained_s=0.0, sampler=None):
+    """The MXFP4 and bf16 ceilings of this GPU's tensor pipe: csa_peak_mma (one
+    CTA per SM, back-to-back tcgen05.mma on shared-memory operands), each launch
+    ~20 ms, best of 10 (burst); with sustained_s > 0 also a back-to-back run of
+    that many seconds per kind (mean rate)."""
+    out = {}
+    for kind, name in ((1, "mxf4"), (0, "bf16")):
+        probe = 4096
+        fl, ws = csa.csa_peak_mma(kind, probe)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fl, ws = csa.csa_peak_mma(kind, probe, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        per_iter_ms = e0.elapsed_time(e1) / probe
+        iters = max(1024, int(20.0 / max(per_iter_ms, 1e-9)))
+        best = 0.0
+        for _ in range(10):
+            e0.record()
+            fl, ws = csa.csa_peak_mma(kind, iters, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            best = max(best, fl / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+        rec = {"burst_tflops": best, "iters_per_cta": iters}
+        if sustained_s > 0:
+            n = max(1, int(sustained_s * 1000 / 20))
+            if sampler is not None:
+                sampler.start()
+            e0.record()
+            for _ in range(n):
+                fl, ws = csa.csa_peak_mma(kind, iters, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if sampler is not None:
+                sampler.stop()
+                rec["clocks"] = sampler.summary()
+                sampler.samples = []
+            rec["sustained_tflops"] = fl * n / (e0.elapsed_time(e1) * 1e-3) / 1e12
+            rec["sustained_s"] = e0.elapsed_time(e1) * 1e-3
+        rec["status"] = csa.csa_check_status(ws)
+        out[name] = rec
+    return out
 
 
 # ----------------------------------------------------------------- algorithmic work
@@ -290,7 +336,8 @@ def run_csa_prefill(csa, wl, steps, warmup, dist_on, rank):
     e2e_ms = e0.elapsed_time(e1) / n_e2e
     del dev, host
     return {"ms": ms, "phases": phases, "status": status, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launches_per_step": 3, "e2e_chunks": n_chunks, "e2e_matches": e2e_matches}
+            "launches_per_step": 4,  # compress, indexer, top-k finalize, attention
+            "e2e_chunks": n_chunks, "e2e_matches": e2e_matches}
 
 
 def run_hca_prefill(csa, wl, steps, warmup):
@@ -388,37 +435,133 @@ def run_stack(csa, wl, steps, warmup):
 
 
 # ----------------------------------------------------------------- CPU oracle (reference arm / baseline)
-def oracle_sample(wl, seconds=12.0, max_rows=4096):
-    """Time the CPU oracle on a bounded sample of the CSA prefill workload: the
-    compression of every block, then indexer + top-k + attention for sampled
-    query rows, until about `seconds` have passed. Returns tokens/s and details."""
+def _boundary_rows(wl):
+    """Rows every CPU sample includes: 0, m-1, m, W-1, W, the rows where the
+    visible count reaches k, and T-1."""
+    r = {0, wl.m - 1, wl.m, wl.W - 1, wl.W, wl.k * wl.m - 1, wl.k * wl.m, wl.T - 1}
+    return sorted(x for x in r if 0 <= x < wl.T)
+
+
+class OracleCSA:
+    """The CPU oracle on the CSA prefill workload: compression of every block
+    once, then indexer + top-k + attention for batches of query rows (boundary
+    rows first, then a seeded permutation)."""
+
+    def __init__(self, wl):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.d = inputs.prefill_layer(wl)
+        self.scale = 1.0 / math.sqrt(wl.d)
+        self.nthreads = oracle.default_threads()
+        t = time.perf_counter()
+        Kc64, Vc64 = oracle.compress(self.d["K"], self.d["V"], self.d["Z"], self.d["B"], wl.m, self.nthreads)
+        self.Kcw, self.Vcw = oracle.to_bf16_words(Kc64), oracle.to_bf16_words(Vc64)
+        self.t_comp = time.perf_counter() - t
+        b = _boundary_rows(wl)
+        rest = np.random.default_rng(0).permutation(wl.T)
+        self.order = np.concatenate([np.array(b, np.int64), rest[~np.isin(rest, b)]])
+        self.done = 0
+
+    def rows(self, n):
+        r = np.sort(self.order[self.done:self.done + n])
+        self.done += len(r)
+        return r
+
+    def run_rows(self, rows):
+        o, d, wl = self.oracle, self.d, self.wl
+        I = o.indexer(d["qI_codes"], d["qI_scales"], d["w_codes"], d["kI_codes"], d["kI_scales"], 0, wl.m, rows,
+                      self.nthreads)
+        sel, _ = o.topk(I, o.n_vis(rows, wl.m), wl.k, self.nthreads)
+        o.attention(d["Q"], self.Kcw, self.Vcw, d["K"], d["V"], 0, wl.m, wl.W, self.scale, sel=sel, rows=rows,
+                    nthreads=self.nthreads)
+
+    def timed(self, seconds, batch=None):
+        """Rows processed in about `seconds`; returns (rows, seconds)."""
+        batch = batch or max(8, self.nthreads)
+        n, t_rows = 0, 0.0
+        while t_rows < seconds and self.done < self.wl.T:
+            r = self.rows(batch)
+            t1 = time.perf_counter()
+            self.run_rows(r)
+            t_rows += time.perf_counter() - t1
+            n += len(r)
+        return n, t_rows
+
+
+def oracle_sample(wl, seconds=8.0):
+    """Time the CPU oracle on a bounded sample of the CSA prefill workload and
+    extrapolate the full step as compress + T * (time per row)."""
+    oc = OracleCSA(wl)
+    n, t_rows = oc.timed(seconds)
+    total_s = oc.t_comp + t_rows / n * wl.T
+    return {"tokens_per_s": wl.T / total_s, "rows": n, "seconds": oc.t_comp + t_rows, "cores": oc.nthreads,
+            "sample": "compression of all %d blocks + indexer/top-k/attention of %d query rows of %d (the boundary "
+                      "rows %s, then seeded random rows; %.1f s of CPU time); full step extrapolated as compress + "
+                      "T x time per row" % (wl.T // wl.m, n, wl.T, _boundary_rows(wl), oc.t_comp + t_rows)}
+
+
+def oracle_other_configs():
+    """The oracle on the other workloads: the tiny layer and the 1M-context decode
+    in full, the HCA prefill and the two-layer stack on seeded rows that include
+    the boundary rows (time per row and an extrapolated full time, so labelled)."""
     import oracle
+    out = {}
+    nth = oracle.default_threads()
+    # tiny CSA + HCA layer, in full
+    wl = inputs.TINY
     d = inputs.prefill_layer(wl)
-    scale = 1.0 / math.sqrt(wl.d)
-    nthreads = oracle.default_threads()
-    t_start = time.perf_counter()
-    Kc64, Vc64 = oracle.compress(d["K"], d["V"], d["Z"], d["B"], wl.m, nthreads)
-    Kcw, Vcw = oracle.to_bf16_words(Kc64), oracle.to_bf16_words(Vc64)
-    t_comp = time.perf_counter() - t_start
-    rng = np.random.default_rng(0)
-    order = rng.permutation(wl.T)
-    done, t_rows, batch = 0, 0.0, max(8, nthreads)
-    while t_rows < seconds and done < max_rows:
-        rows = np.sort(order[done:done + batch])
-        t1 = time.perf_counter()
-        I = oracle.indexer(d["qI_codes"], d["qI_scales"], d["w_codes"], d["kI_codes"], d["kI_scales"], 0, wl.m,
-                           rows, nthreads)
-        sel, _ = oracle.topk(I, oracle.n_vis(rows, wl.m), wl.k, nthreads)
-        oracle.attention(d["Q"], Kcw, Vcw, d["K"], d["V"], 0, wl.m, wl.W, scale, sel=sel, rows=rows,
-                         nthreads=nthreads)
-        t_rows += time.perf_counter() - t1
-        done += len(rows)
-    per_row = t_rows / done
-    total_s = t_comp + per_row * wl.T  # extrapolated full step
-    return {"tokens_per_s": wl.T / total_s, "rows": done, "seconds": t_comp + t_rows, "cores": nthreads,
-            "sample": "compression of all %d blocks + indexer/top-k/attention of %d uniformly sampled query rows "
-                      "of %d (%.1f s of CPU time); full step extrapolated as compress + T * per-row"
-                      % (wl.T // wl.m, done, wl.T, t_comp + t_rows)}
+    sc = 1.0 / math.sqrt(wl.d)
+    t = time.perf_counter()
+    oracle.csa_layer(d, wl.m, wl.k, wl.W, sc, nthreads=nth)
+    K2, V2 = oracle.compress(d["K"], d["V"], d["Z"], d["B_hca"], wl.m_hca, nth)
+    oracle.attention(d["Q"], oracle.to_bf16_words(K2), oracle.to_bf16_words(V2), d["K"], d["V"], 0, wl.m_hca,
+                     wl.W_hca, sc, nthreads=nth)
+    out[wl.name] = {"seconds": time.perf_counter() - t, "scope": "full (CSA and HCA layer, all %d rows)" % wl.T}
+    # 1M-context decode, all 16 sequences, generated on the GPU and copied to the host
+    wl = inputs.CSA_DECODE
+    g = inputs.decode_batch(wl, device="cuda")
+    h = {k: v.cpu() for k, v in g.items()}
+    del g
+    torch.cuda.empty_cache()
+    sc = 1.0 / math.sqrt(wl.d)
+    t = time.perf_counter()
+    pos = wl.context - 1
+
+    def one_sequence(b):  # one query row per sequence: the sequences go to separate threads
+        I = oracle.indexer(h["qI_codes"][b:b + 1], h["qI_scales"][b:b + 1], h["w_codes"][b:b + 1], h["kI_codes"][b],
+                           h["kI_scales"][b], pos, wl.m, nthreads=1)
+        sel, _ = oracle.topk(I, oracle.n_vis([pos], wl.m), wl.k, 1)
+        oracle.attention(h["q"][b:b + 1], h["Kc"][b], h["Vc"][b], h["Kwin"][b], h["Vwin"][b], pos, wl.m, wl.W, sc,
+                         sel=sel, rows=[0], raw_pos0=pos - wl.W + 1, nthreads=1)
+
+    import concurrent.futures as cf
+    with cf.ThreadPoolExecutor(max_workers=min(nth, wl.batch)) as ex:
+        list(ex.map(one_sequence, range(wl.batch)))
+    dt = time.perf_counter() - t
+    out[wl.name] = {"seconds": dt, "us_per_step": dt * 1e6, "threads": min(nth, wl.batch),
+                    "scope": "full (16 sequences, one step, a thread per sequence)"}
+    del h
+    # HCA prefill, 128 rows
+    wl = inputs.HCA_PREFILL
+    d = inputs.prefill_layer(wl, with_indexer=False)
+    sc = 1.0 / math.sqrt(wl.d)
+    t = time.perf_counter()
+    K2, V2 = oracle.compress(d["K"], d["V"], d["Z"], d["B_hca"], wl.m_hca, nth)
+    t_comp = time.perf_counter() - t
+    rows = np.array(sorted(set([0, wl.m_hca - 1, wl.m_hca, wl.W_hca - 1, wl.W_hca, wl.T - 1]) |
+                           set(np.random.default_rng(2).choice(wl.T, 122, replace=False).tolist())), np.int64)
+    t = time.perf_counter()
+    oracle.attention(d["Q"], oracle.to_bf16_words(K2), oracle.to_bf16_words(V2), d["K"], d["V"], 0, wl.m_hca,
+                     wl.W_hca, sc, rows=rows, nthreads=nth)
+    per_row = (time.perf_counter() - t) / len(rows)
+    out[wl.name] = {"rows": len(rows), "s_per_row": per_row, "compress_s": t_comp,
+                    "extrapolated_full_s": t_comp + per_row * wl.T,
+                    "tokens_per_s_extrapolated": wl.T / (t_comp + per_row * wl.T),
+                    "scope": "compression of all blocks + attention of %d rows incl. boundary rows; extrapolated"
+                             % len(rows)}
+    del d
+    return out
 
 
 EXTRA_CASES = ("hca_prefill", "csa_decode", "stack")
@@ -469,7 +612,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the HCA and decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default="all", choices=("all", "csa_prefill") + EXTRA_CASES,
+    ap.add_argument("--case", default="all", choices=("all", "csa_prefill", "peaks") + EXTRA_CASES,
                     help="all: the CSA prefill line plus the other workloads; csa_prefill: that line alone; "
                          "otherwise one other workload alone, on one GPU (for profiling)")
     ap.add_argument("--T", type=int, default=None,
@@ -487,15 +630,35 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        r = oracle_sample(wl, seconds=max(5.0, 4.0 * args.steps / max(1, args.steps)))
-        v = r["tokens_per_s"]
+        # each step = one bounded sample of the workload's query rows (a budget that
+        # keeps the whole --steps K --warmup W run within a few minutes); the value
+        # is the workload's tokens/s extrapolated from the rows done per second
+        oc = OracleCSA(wl)
+        budget = min(8.0, 150.0 / max(1, args.steps + args.warmup))
+        for _ in range(args.warmup):
+            oc.timed(budget / 4)
+        step_s, rows_done = [], 0
+        for _ in range(args.steps):
+            n, t_rows = oc.timed(budget)
+            if n == 0:
+                break
+            step_s.append(t_rows)
+            rows_done += n
+        t_rows = sum(step_s)
+        per_row = t_rows / max(1, rows_done)
+        v = wl.T / (oc.t_comp + per_row * wl.T)
+        sample = ("each step: indexer/top-k/attention of a batch of query rows for ~%.1f s (boundary rows %s first, "
+                  "then seeded random rows); %d rows over %d steps; compression of all %d blocks (%.2f s) once; "
+                  "tokens/s extrapolated as T / (compress + T x time per row)"
+                  % (budget, _boundary_rows(wl), rows_done, len(step_s), wl.T // wl.m, oc.t_comp))
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.T / v,
+                "steps": len(step_s), "warmup": args.warmup,
+                "ms_per_step": 1000.0 * t_rows / max(1, len(step_s)), "rows_per_step": rows_done / max(1, len(step_s)),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "d": wl.d, "m": wl.m,
                                                  "k": wl.k, "W": wl.W, "HI": wl.HI, "dI": wl.dI},
-                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
-                                 "sample": r["sample"]},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oc.nthreads, "kind": "oracle",
+                                 "sample": sample},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -509,6 +672,18 @@ def main():
     import long_context_compressed_gated_b200 as csa
     csa.lib()
     peaks = load_peaks()
+    if args.case == "peaks":
+        if rank == 0:
+            sm = ClockSampler(local)
+            print(json.dumps({"case": "peaks", "tensor_peaks": measure_tensor_peaks(csa, sustained_s=4.0, sampler=sm),
+                              "cublas_bf16_measured": peaks}), flush=True)
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return
+    tensor_peaks = measure_tensor_peaks(csa)
+    peaks["mxf4_tflops"] = tensor_peaks["mxf4"]["burst_tflops"]
+    peaks["mxf4_source"] = "measured: csa_peak_mma loop, best of 10"
+    peaks["bf16_mma_loop_tflops"] = tensor_peaks["bf16"]["burst_tflops"]
     if args.case in EXTRA_CASES:
         if rank == 0:
             print(json.dumps({"case": args.case, "workloads": run_extra(args.case, csa, peaks, args.steps,
@@ -536,14 +711,15 @@ def main():
     idx_tf = work["indexer_flop"] / (ph["indexer_topk"] * 1e-3) / 1e12
     attn_tf = work["attn_flop"] / (ph["sparse_attn"] * 1e-3) / 1e12
     comp_gbs = work["compress_bytes"] / (ph["compress"] * 1e-3) / 1e9
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    fp4_peak = peaks["mxf4_tflops"]
     same_cfg = wl.T == inputs.CSA_PREFILL.T
     if dominant == "indexer_topk":
         roof = {"kernel": "indexer_topk", "bound": "tensor", "achieved": idx_tf, "peak": fp4_peak,
                 "unit": "TFLOP/s", "frac": idx_tf / fp4_peak,
                 "traffic": PHASE_TRAFFIC["indexer_topk"][0] if same_cfg else None,
                 "traffic_source": PHASE_TRAFFIC["indexer_topk"][1],
-                "peak_note": "FP4 peak = measured bf16 burst x 4 (nominal dense ratio), %s" % peaks["source"]}
+                "peak_note": "measured kind::mxf4 peak (tcgen05 MMA loop on this GPU, burst, best of 10); "
+                             "NVIDIA's dense FP4 figure %.0f TFLOP/s for context" % NOMINAL_FP4_TFLOPS}
     elif dominant == "sparse_attn":
         roof = {"kernel": "sparse_attn", "bound": "tensor", "achieved": attn_tf, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_tflops"],
@@ -575,12 +751,15 @@ def main():
         "clocks": sampler.summary(),
         "device_status": res["status"],
         "peaks": peaks,
+        "tensor_peaks": tensor_peaks,
         "workloads": extra,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = oracle_sample(wl, seconds=12.0)
+        r = oracle_sample(wl, seconds=8.0)
         line["cpu_baseline"] = {"value": r["tokens_per_s"], "unit": "tokens/s", "cores": r["cores"],
                                 "kind": "oracle", "sample": r["sample"]}
+        if args.case == "all" and not args.no_extra:
+            line["cpu_baseline"]["other_workloads"] = oracle_other_configs()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:

@@ -68,6 +68,12 @@ typedef enum {
   CSA_ERR_RANGE = -7              /* (status word) MXFP4 scale outside [125,128] */
 } csa_status_t;
 
+/* Element type of an attention output O (the o_dtype argument). */
+typedef enum {
+  CSA_BF16 = 0, /* IEEE bfloat16, round to nearest even of the fp32 result */
+  CSA_F32 = 1   /* the fp32 result itself (no output rounding; 2x the bytes) */
+} csa_dtype_t;
+
 /* Human-readable text of a status code (static storage). */
 const char* csa_status_string(int status);
 /* The cudaError_t of the last CSA_ERR_CUDA on this host thread (0 if none). */
@@ -76,8 +82,40 @@ int csa_last_cuda_error(void);
 int csa_version(void);
 
 /* Reads the device status word at the start of `workspace` (synchronously on
- * `stream`) and clears it.  Returns CSA_OK or the first device-side error. */
+ * `stream`) and clears it.  Returns CSA_OK or the first device-side error.
+ * While the word holds CSA_ERR_DEVICE_TIMEOUT, kernels given that workspace
+ * skip their work (their outputs are then unspecified) instead of waiting out
+ * every deadline again: clear it before reusing the workspace. */
 int csa_check_status(void* workspace, csa_stream_t stream);
+
+/* Test hook for the device-side timeout path (no counterpart on the pages).
+ * Every wait of a kernel on another part of the same kernel is bounded
+ * (~0.14 s of SM clock); when a wait runs out, the kernel records
+ * CSA_ERR_DEVICE_TIMEOUT in the status word, lets the copies it already
+ * started land, frees its tensor memory and returns, so the context stays
+ * usable.  csa_debug_inject(CSA_FAULT_INDEXER_STALL) makes the NEXT indexer
+ * launch in this process (csa_indexer_topk or the indexer of csa_decode) skip
+ * its first key-tile copy, so its MMA and epilogue waits run out; the launch
+ * then reports CSA_ERR_DEVICE_TIMEOUT through csa_check_status.  No memory is
+ * touched out of bounds.  The code is consumed by that launch.  Returns CSA_OK,
+ * or CSA_ERR_INVALID_ARG for an unknown code. */
+enum { CSA_FAULT_NONE = 0, CSA_FAULT_INDEXER_STALL = 1 };
+int csa_debug_inject(int code);
+
+/* ---------------------------------------------------------------- measurement
+ * Tensor-pipe ceiling of this GPU, the roofline denominator of the indexer's
+ * MXFP4 contraction (m.youleyou.com/wenzhang/2906406.html section 1 puts the
+ * indexer's query-key path on MXFP4) and, for calibration against a library
+ * GEMM, of bf16.  Enqueues `ctas` CTAs (one per SM: pass the SM count) that each
+ * issue `iters` back-to-back tcgen05.mma instructions of shape 128 x 240 on
+ * operands resident in shared memory (kind::mxf4.block_scale.block32 with K = 64
+ * for CSA_PEAK_MXF4, kind::f16 on bf16 with K = 16 for CSA_PEAK_BF16).  *flops
+ * (nullable) receives the work of the launch, 2*128*240*K*iters*ctas; time it
+ * with events on `stream`.  workspace: >= 256 bytes for the status word.
+ * iters >= 2, ctas >= 1. */
+enum { CSA_PEAK_BF16 = 0, CSA_PEAK_MXF4 = 1 };
+int csa_peak_mma(int kind, int64_t iters, int ctas, void* workspace, size_t workspace_bytes, double* flops,
+                 csa_stream_t stream);
 
 /* ---------------------------------------------------------------- compress
  * Softmax-gated per-channel pooling of every complete block of m tokens
@@ -90,6 +128,25 @@ int csa_check_status(void* workspace, csa_stream_t stream);
  * No workspace. */
 int csa_compress(const void* K, const void* V, const void* Z, const float* B, int64_t T, int d, int m, void* Kc,
                  void* Vc, csa_stream_t stream);
+
+/* ---------------------------------------------------------------- MXFP4 quantiser
+ * bf16 -> MXFP4, the operand format of the indexer's query-key path
+ * (m.youleyou.com/wenzhang/2906406.html section 1: MXFP4 on the indexer's QK
+ * path; ferris-liu.github.io ... deepseek-v4, engineering layer: FP4 on the
+ * indexer).  The pages give no scale rule; this is the OCP MX conversion.  For
+ * every block of 32 consecutive elements of a row of x [rows, n] bf16:
+ *   X = floor(log2 max|x|) - 2 (an all-zero block: X = -127), clamped to
+ *   [-127, 127]; with mode CSA_MX_INDEXER clamped to [-2, 1] instead, so that
+ *   the scale bytes meet the indexer's exact range 125..128 (blocks with
+ *   max|x| >= 12 then saturate, small ones round more coarsely);
+ *   scales[r, b] = X + 127; codes: E2M1 nearest to x / 2^X, ties to the even
+ *   code, magnitudes above 6 saturate to 6, the sign is kept (-0 is code 8);
+ *   element 2i in the low nibble of byte i of codes [rows, n/2].
+ * A block holding an Inf or NaN gets scale byte 255 and zero codes.
+ * n % 32 == 0.  Deterministic; no workspace. */
+enum { CSA_MX_OCP = 0, CSA_MX_INDEXER = 1 };
+int csa_mxfp4_quantize(const void* x, int64_t rows, int n, int mode, uint8_t* codes, uint8_t* scales,
+                       csa_stream_t stream);
 
 /* ---------------------------------------------------------------- indexer + top-k
  * Lightning indexer on MXFP4 fused with the causal top-k (ifanr repost,
@@ -117,25 +174,31 @@ int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const ui
  *   Kc, Vc [Nc, d] bf16 compressed entries; idx [T, k] int32 (-1 = none)
  *   Kraw, Vraw : raw K/V rows indexed by ABSOLUTE position (row s at
  *          Kraw + s*d); rows max(0, t0-W+1) .. t0+T-1 must be readable.
- *   O      [T, H, d] bf16 output; lse [T, H] float natural-log sum of exp of
- *          the scaled logits (may be NULL).
+ *   O      [T, H, d] output of element type o_dtype (CSA_BF16 or CSA_F32; any
+ *          other value is CSA_ERR_INVALID_ARG); lse [T, H] float natural-log sum
+ *          of exp of the scaled logits (may be NULL).
  * One joint softmax over the selected entries and the window; scale is the
  * logit multiplier (> 0; 1/sqrt(d) for the usual reading).  A row with an empty key
  * set gets O = 0, lse = -inf.  H in {4, 8, 16, 32, 64, 128}, d in {64, 128},
- * 1 <= k <= 2048, 0 <= W <= 1024. */
+ * 1 <= k <= 2048, 0 <= W <= 1024, and (128/H) * ceil(k/128) <= 512 (the
+ * selected-entry tiles of one 128-row block; shared memory may bind first for
+ * small H with large k, reported as CSA_ERR_UNSUPPORTED_SHAPE). */
 size_t csa_sparse_attn_workspace_bytes(int64_t T, int H, int d, int k, int W);
 int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t* idx, const void* Kraw,
                     const void* Vraw, int64_t T, int64_t t0, int64_t Nc, int H, int d, int k, int W, float scale,
-                    void* O, float* lse, void* workspace, size_t workspace_bytes, csa_stream_t stream);
+                    void* O, int o_dtype, float* lse, void* workspace, size_t workspace_bytes,
+                    csa_stream_t stream);
 
 /* ---------------------------------------------------------------- HCA attention
  * Dense attention over every visible compressed entry plus the window
  * (blog.nickys.cn/?p=150 "2. HCA").  Same layouts as csa_sparse_attn without
- * idx; entries j < min(Nc, floor((t+1)/m)) are visible to position t. */
+ * idx; entries j < min(Nc, floor((t+1)/m)) are visible to position t.  The
+ * number of visible entries is not limited (dense tiles are generated, not
+ * listed). */
 size_t hca_attn_workspace_bytes(int64_t T, int H, int d, int W);
 int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, const void* Vraw, int64_t T, int64_t t0,
-             int64_t Nc, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
-             size_t workspace_bytes, csa_stream_t stream);
+             int64_t Nc, int H, int d, int m, int W, float scale, void* O, int o_dtype, float* lse,
+             void* workspace, size_t workspace_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------- decode
  * One new token per sequence against a compressed KV cache (the decode case of
@@ -147,39 +210,43 @@ int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, co
  *   kI_codes [B, Ncap, dI/2]          kI_scales [B, Ncap, dI/32]
  *   Kwin, Vwin [B, W, d] bf16: raw K/V of positions pos[b]-W+1 .. pos[b]
  *            (newest last; rows for negative positions are ignored)
- *   O [B, H, d] bf16; lse [B, H] float (nullable); idx [B, k] int32 and
+ *   O [B, H, d] of element type o_dtype; lse [B, H] float (nullable); idx [B, k] int32 and
  *   scores [B, k] float (both nullable) receive the selection.
  * Entries j < min(Ncap, floor((pos[b]+1)/m)) are visible. */
 size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int HI, int dI, int k, int W);
 int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
                const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
                const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
-               int W, float scale, void* O, float* lse, int32_t* idx, float* scores, void* workspace,
+               int W, float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
                size_t workspace_bytes, csa_stream_t stream);
 
 /* HCA decode: dense over every visible cached entry plus the window. */
 size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W);
 int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
-               int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
-               size_t workspace_bytes, csa_stream_t stream);
+               int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, int o_dtype, float* lse,
+               void* workspace, size_t workspace_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------- decode without allocation
- * csa_decode for callers that cannot allocate device memory: code recording a
- * CUDA graph (an allocation would break the capture), serving loops that ban
- * allocator calls on the hot path, and embedders that own every buffer and hand
- * the library nothing else.  The pages describe no such interface; it exists
+ * csa_decode for callers that cannot allocate device memory: serving loops
+ * that forbid allocator calls once they are running, embedders that own every
+ * buffer and hand the library nothing else, and code running where a
+ * cudaMalloc is not allowed.  The pages describe no such interface; it exists
  * only for these callers.
- * Same arguments and results as csa_decode, minus the workspace: the scratch
- * lives in one static 8 MiB device array inside libcsa.so that every GPU loading
- * the library keeps until the process exits.  Calls whose
+ * Same arguments and results as csa_decode (O in bf16), minus the workspace:
+ * the scratch lives in one static 8 MiB device array inside libcsa.so that
+ * every GPU loading the library keeps until the process exits.  Calls whose
  * csa_decode_workspace_bytes() exceeds 8 MiB are rejected with
- * CSA_ERR_WORKSPACE (B = 16, k = 1024 fits for any cache length).
+ * CSA_ERR_WORKSPACE; with H <= 64 at d = 128, B = 16 sequences with k = 1024
+ * fit for any cache length (at H = 128 the split attention partials alone need
+ * more).
+ * The positions pos[] are read on the host during the call, like csa_decode.
  * The first call on a device looks up the array's device address (a runtime
- * call, once per device, with that device current); make that first call
- * before capturing a stream into a graph.  All calls on a device share the
- * array, so calls that can overlap on the GPU (different streams, no ordering
- * between them) race with each other; issue them on one stream or order them.
- * The call clears the array's status word itself.  status_out (device int,
+ * query, once per device, with that device current) and keeps it for the life
+ * of the process: it assumes the runtime's primary context of that device and
+ * no cudaDeviceReset in between.  All calls on a device share the array, so
+ * calls that can overlap on the GPU (different streams, no ordering between
+ * them) race with each other; issue them on one stream or order them.  The
+ * call clears the array's status word itself.  status_out (device int,
  * nullable) receives the device status word of the call (CSA_OK, or
  * CSA_ERR_DEVICE_TIMEOUT / CSA_ERR_RANGE) in stream order.
  * Allocates nothing: no cudaMalloc/cudaFree, no allocating library routine. */

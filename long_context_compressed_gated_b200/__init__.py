@@ -43,18 +43,21 @@ def lib():
             "csa_last_cuda_error": ([], I),
             "csa_version": ([], I),
             "csa_check_status": ([P, P], I),
+            "csa_debug_inject": ([I], I),
+            "csa_mxfp4_quantize": ([P, I64, I, I, P, P, P], I),
+            "csa_peak_mma": ([I, I64, I, P, SZ, P, P], I),
             "csa_compress": ([P, P, P, P, I64, I, I, P, P, P], I),
             "csa_indexer_topk_workspace_bytes": ([I64, I64, I, I, I], SZ),
             "csa_indexer_topk": ([P, P, P, P, P, I64, I64, I64, I, I, I, I, P, P, P, SZ, P], I),
             "csa_sparse_attn_workspace_bytes": ([I64, I, I, I, I], SZ),
-            "csa_sparse_attn": ([P, P, P, P, P, P, I64, I64, I64, I, I, I, I, F, P, P, P, SZ, P], I),
+            "csa_sparse_attn": ([P, P, P, P, P, P, I64, I64, I64, I, I, I, I, F, P, I, P, P, SZ, P], I),
             "hca_attn_workspace_bytes": ([I64, I, I, I], SZ),
-            "hca_attn": ([P, P, P, P, P, I64, I64, I64, I, I, I, I, F, P, P, P, SZ, P], I),
+            "hca_attn": ([P, P, P, P, P, I64, I64, I64, I, I, I, I, F, P, I, P, P, SZ, P], I),
             "csa_decode_workspace_bytes": ([I, I64, I, I, I, I, I, I], SZ),
-            "csa_decode": ([P, P, P, P, P, P, P, P, P, P, P, I, I64, I, I, I, I, I, I, I, F, P, P, P, P, P, SZ, P],
-                           I),
+            "csa_decode": ([P, P, P, P, P, P, P, P, P, P, P, I, I64, I, I, I, I, I, I, I, F, P, I, P, P, P, P, SZ,
+                            P], I),
             "hca_decode_workspace_bytes": ([I, I64, I, I, I], SZ),
-            "hca_decode": ([P, P, P, P, P, P, I, I64, I, I, I, I, F, P, P, P, SZ, P], I),
+            "hca_decode": ([P, P, P, P, P, P, I, I64, I, I, I, I, F, P, I, P, P, SZ, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -70,6 +73,18 @@ def csa_status_string(code):
 
 def csa_version():
     return lib().csa_version()
+
+
+_ODTYPE = {torch.bfloat16: 0, torch.float32: 1}  # csa_dtype_t
+
+
+def _out(O, like, shape, out_dtype, name="O"):
+    """Output tensor of the given dtype (bf16 or fp32): allocated when O is None."""
+    if out_dtype not in _ODTYPE:
+        raise TypeError("%s dtype must be torch.bfloat16 or torch.float32" % name)
+    if O is None:
+        return torch.empty(shape, dtype=out_dtype, device=like.device)
+    return _dev(O, out_dtype, name)
 
 
 def _ptr(t):
@@ -112,6 +127,38 @@ def csa_check_status(workspace):
     return lib().csa_check_status(_ptr(workspace), _stream())
 
 
+def csa_peak_mma(kind, iters, ctas=None, workspace=None):
+    """Enqueue the tensor-pipe peak loop (kind 0 = bf16, 1 = MXFP4) on the current
+    stream; returns (flops of the launch, workspace).  ctas defaults to the SM count."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    ws = _workspace(256, dev, workspace)
+    fl = ctypes.c_double(0.0)
+    _check(lib().csa_peak_mma(int(kind), int(iters), int(ctas), _ptr(ws), ws.numel(), ctypes.byref(fl), _stream()),
+           "csa_peak_mma")
+    return fl.value, ws
+
+
+MX_OCP, MX_INDEXER = 0, 1
+
+
+def csa_mxfp4_quantize(x, mode=MX_OCP, codes=None, scales=None):
+    """bf16 [..., n] (n % 32 == 0) -> MXFP4 (codes uint8 [..., n/2], scales uint8
+    [..., n/32]).  mode MX_INDEXER keeps the scale bytes in 125..128."""
+    _dev(x, torch.bfloat16, "x")
+    n = x.shape[-1]
+    rows = x.numel() // n if n else 0
+    lead = tuple(x.shape[:-1])
+    codes = torch.empty(lead + (n // 2,), dtype=torch.uint8, device=x.device) if codes is None else \
+        _dev(codes, torch.uint8, "codes")
+    scales = torch.empty(lead + (n // 32,), dtype=torch.uint8, device=x.device) if scales is None else \
+        _dev(scales, torch.uint8, "scales")
+    _check(lib().csa_mxfp4_quantize(_ptr(x), rows, n, int(mode), _ptr(codes), _ptr(scales), _stream()),
+           "csa_mxfp4_quantize")
+    return codes, scales
+
+
 def csa_compress(K, V, Z, B, m, Kc=None, Vc=None):
     """Gated pooling of every complete block of m tokens. K,V,Z [T,d] bf16, B [m,d] f32.
     Returns (Kc, Vc) [T//m, d] bf16."""
@@ -139,6 +186,8 @@ def csa_indexer_topk(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, m, k, t0
     idx = torch.empty(T, k, dtype=torch.int32, device=dev) if idx is None else _dev(idx, torch.int32, "idx")
     if want_scores and scores is None:
         scores = torch.empty(T, k, dtype=torch.float32, device=dev)
+    elif scores is not None:
+        _dev(scores, torch.float32, "scores")
     ws = _workspace(lib().csa_indexer_topk_workspace_bytes(T, Nc, HI, dI, k), dev, workspace)
     _check(lib().csa_indexer_topk(_ptr(qI_codes), _ptr(qI_scales), _ptr(w_codes), _ptr(kI_codes), _ptr(kI_scales),
                                   T, t0, Nc, HI, dI, m, k, _ptr(idx), _ptr(scores), _ptr(ws), ws.numel(),
@@ -146,40 +195,46 @@ def csa_indexer_topk(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, m, k, t0
     return idx, scores, ws
 
 
-def csa_sparse_attn(Q, Kc, Vc, idx, Kraw, Vraw, W, scale, t0=0, O=None, lse=None, want_lse=True, workspace=None):
-    """CSA attention over the selected entries plus the raw window. Returns (O, lse, workspace)."""
+def csa_sparse_attn(Q, Kc, Vc, idx, Kraw, Vraw, W, scale, t0=0, O=None, lse=None, want_lse=True, workspace=None,
+                    out_dtype=torch.bfloat16):
+    """CSA attention over the selected entries plus the raw window. Returns (O, lse, workspace).
+    out_dtype: torch.bfloat16 (default) or torch.float32 for O."""
     _dev(Q, torch.bfloat16, "Q", 3), _dev(Kc, torch.bfloat16, "Kc", 2), _dev(Vc, torch.bfloat16, "Vc", 2)
     _dev(idx, torch.int32, "idx", 2), _dev(Kraw, torch.bfloat16, "Kraw", 2), _dev(Vraw, torch.bfloat16, "Vraw", 2)
     T, H, d = Q.shape
     k = idx.shape[1]
     dev = Q.device
-    O = torch.empty_like(Q) if O is None else _dev(O, torch.bfloat16, "O")
+    O = _out(O, Q, Q.shape, out_dtype)
     if want_lse and lse is None:
         lse = torch.empty(T, H, dtype=torch.float32, device=dev)
     ws = _workspace(lib().csa_sparse_attn_workspace_bytes(T, H, d, k, W), dev, workspace)
     _check(lib().csa_sparse_attn(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(idx), _ptr(Kraw), _ptr(Vraw), T, t0,
-                                 Kc.shape[0], H, d, k, W, float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
-                                 _stream()), "csa_sparse_attn")
+                                 Kc.shape[0], H, d, k, W, float(scale), _ptr(O), _ODTYPE[out_dtype], _ptr(lse),
+                                 _ptr(ws), ws.numel(), _stream()), "csa_sparse_attn")
     return O, lse, ws
 
 
-def hca_attn(Q, Kc, Vc, Kraw, Vraw, m, W, scale, t0=0, O=None, lse=None, want_lse=True, workspace=None):
-    """HCA attention over every visible compressed entry plus the raw window. Returns (O, lse, workspace)."""
+def hca_attn(Q, Kc, Vc, Kraw, Vraw, m, W, scale, t0=0, O=None, lse=None, want_lse=True, workspace=None,
+             out_dtype=torch.bfloat16):
+    """HCA attention over every visible compressed entry plus the raw window. Returns (O, lse, workspace).
+    out_dtype: torch.bfloat16 (default) or torch.float32 for O."""
     _dev(Q, torch.bfloat16, "Q", 3), _dev(Kc, torch.bfloat16, "Kc", 2), _dev(Vc, torch.bfloat16, "Vc", 2)
     _dev(Kraw, torch.bfloat16, "Kraw", 2), _dev(Vraw, torch.bfloat16, "Vraw", 2)
     T, H, d = Q.shape
     dev = Q.device
-    O = torch.empty_like(Q) if O is None else _dev(O, torch.bfloat16, "O")
+    O = _out(O, Q, Q.shape, out_dtype)
     if want_lse and lse is None:
         lse = torch.empty(T, H, dtype=torch.float32, device=dev)
     ws = _workspace(lib().hca_attn_workspace_bytes(T, H, d, W), dev, workspace)
     _check(lib().hca_attn(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(Kraw), _ptr(Vraw), T, t0, Kc.shape[0], H, d, m, W,
-                          float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(), _stream()), "hca_attn")
+                          float(scale), _ptr(O), _ODTYPE[out_dtype], _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+           "hca_attn")
     return O, lse, ws
 
 
 def csa_decode(q, qI_codes, qI_scales, w_codes, Kc, Vc, kI_codes, kI_scales, Kwin, Vwin, pos, m, k, scale,
-               O=None, lse=None, idx=None, scores=None, want_lse=True, want_sel=True, workspace=None):
+               O=None, lse=None, idx=None, scores=None, want_lse=True, want_sel=True, workspace=None,
+               out_dtype=torch.bfloat16):
     """One new token per sequence against its compressed cache (indexer, top-k,
     sparse + window attention). pos: list of absolute positions (host).
     Returns (O [B,H,d], lse, idx [B,k], scores [B,k], workspace)."""
@@ -193,7 +248,7 @@ def csa_decode(q, qI_codes, qI_scales, w_codes, Kc, Vc, kI_codes, kI_scales, Kwi
     Ncap = Kc.shape[1]
     W = Kwin.shape[1]
     dev = q.device
-    O = torch.empty_like(q) if O is None else _dev(O, torch.bfloat16, "O")
+    O = _out(O, q, q.shape, out_dtype)
     if want_lse and lse is None:
         lse = torch.empty(B, H, dtype=torch.float32, device=dev)
     if want_sel:
@@ -203,23 +258,25 @@ def csa_decode(q, qI_codes, qI_scales, w_codes, Kc, Vc, kI_codes, kI_scales, Kwi
     ws = _workspace(lib().csa_decode_workspace_bytes(B, Ncap, H, d, HI, dI, k, W), dev, workspace)
     _check(lib().csa_decode(_ptr(q), _ptr(qI_codes), _ptr(qI_scales), _ptr(w_codes), _ptr(Kc), _ptr(Vc),
                             _ptr(kI_codes), _ptr(kI_scales), _ptr(Kwin), _ptr(Vwin), posa, B, Ncap, H, d, HI, dI,
-                            m, k, W, float(scale), _ptr(O), _ptr(lse), _ptr(idx), _ptr(scores), _ptr(ws),
-                            ws.numel(), _stream()), "csa_decode")
+                            m, k, W, float(scale), _ptr(O), _ODTYPE[out_dtype], _ptr(lse), _ptr(idx),
+                            _ptr(scores), _ptr(ws), ws.numel(), _stream()), "csa_decode")
     return O, lse, idx, scores, ws
 
 
-def hca_decode(q, Kc, Vc, Kwin, Vwin, pos, m, scale, O=None, lse=None, want_lse=True, workspace=None):
+def hca_decode(q, Kc, Vc, Kwin, Vwin, pos, m, scale, O=None, lse=None, want_lse=True, workspace=None,
+               out_dtype=torch.bfloat16):
     """HCA decode: one token per sequence, dense over its visible cache + window."""
     _dev(q, torch.bfloat16, "q", 3), _dev(Kc, torch.bfloat16, "Kc", 3), _dev(Vc, torch.bfloat16, "Vc", 3)
     _dev(Kwin, torch.bfloat16, "Kwin", 3), _dev(Vwin, torch.bfloat16, "Vwin", 3)
     B, H, d = q.shape
     Ncap, W = Kc.shape[1], Kwin.shape[1]
     dev = q.device
-    O = torch.empty_like(q) if O is None else _dev(O, torch.bfloat16, "O")
+    O = _out(O, q, q.shape, out_dtype)
     if want_lse and lse is None:
         lse = torch.empty(B, H, dtype=torch.float32, device=dev)
     posa = (ctypes.c_int64 * B)(*[int(p) for p in pos])
     ws = _workspace(lib().hca_decode_workspace_bytes(B, Ncap, H, d, W), dev, workspace)
     _check(lib().hca_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Kwin), _ptr(Vwin), posa, B, Ncap, H, d, m, W,
-                            float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(), _stream()), "hca_decode")
+                            float(scale), _ptr(O), _ODTYPE[out_dtype], _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+           "hca_decode")
     return O, lse, ws

@@ -23,8 +23,11 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
                                   int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
                                   uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
                                   int* status, cudaStream_t stream);
-
-
+int inject_fault(int code);
+cudaError_t launch_mxfp4_quantize(const void* x, int64_t nblocks, int mode, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t stream);
+cudaError_t launch_peak_mma(int kind, long long iters, int ctas, int* status, cudaStream_t stream);
+double peak_mma_flops(int kind, long long iters, int ctas);
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -99,11 +102,25 @@ cudaError_t upload_positions(int64_t* dst, const int64_t* host, int B, cudaStrea
   return cudaGetLastError();
 }
 
+// Streaming multiprocessors of the current device (queried once per device).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+bool valid_odtype(int t) { return t == CSA_BF16 || t == CSA_F32; }
+
 // decode workspace: [header][pos B*8][idx B*k*4][cand B*nsplit*k*8]
 // Key ranges per decode row: as many as fill the GPU in one wave of
 // one-CTA-per-SM indexer blocks (a second partial wave would double the time).
 int decode_nsplit(int B, int64_t Ncap, int k) {
-  int sms = 148;
+  const int sms = sm_count();
   int ns = B > 0 ? sms / B : 1;
   const int64_t tiles = ceil_div(Ncap > 0 ? Ncap : 1, 128);
   if (ns > tiles) ns = (int)tiles;
@@ -119,7 +136,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // key tile of the sequence; with more than one, partial outputs go through the
 // workspace and a combine pass.
 int decode_attn_splits(int B, int64_t tiles) {
-  int ns = B > 0 ? 148 / B : 1;
+  int ns = B > 0 ? sm_count() / B : 1;
   if (ns > 16) ns = 16;  // the combine pass merges at most 16 partials
   if (ns > tiles) ns = (int)tiles;
   return ns < 1 ? 1 : ns;
@@ -151,7 +168,22 @@ const char* csa_status_string(int status) {
 
 int csa_last_cuda_error(void) { return g_last_cuda_error; }
 
-int csa_version(void) { return 100; }
+int csa_version(void) { return 200; }
+
+int csa_peak_mma(int kind, int64_t iters, int ctas, void* workspace, size_t workspace_bytes, double* flops,
+                 csa_stream_t stream) {
+  if ((kind != CSA_PEAK_BF16 && kind != CSA_PEAK_MXF4) || iters < 2 || ctas < 1) return CSA_ERR_INVALID_ARG;
+  int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
+  if (rc) return rc;
+  if (flops) *flops = peak_mma_flops(kind, iters, ctas);
+  cudaError_t e = launch_peak_mma(kind, iters, ctas, status_word(workspace), (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+int csa_debug_inject(int code) {
+  if (code != CSA_FAULT_NONE && code != CSA_FAULT_INDEXER_STALL) return CSA_ERR_INVALID_ARG;
+  return inject_fault(code);
+}
 
 int csa_check_status(void* workspace, csa_stream_t stream) {
   if (workspace == nullptr) return CSA_ERR_WORKSPACE;
@@ -176,6 +208,16 @@ int csa_compress(const void* K, const void* V, const void* Z, const float* B, in
   int rc = check_ptrs(K, V, Z, B, Kc, Vc);
   if (rc) return rc;
   cudaError_t e = launch_compress(K, V, Z, B, T, d, m, Kc, Vc, (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+int csa_mxfp4_quantize(const void* x, int64_t rows, int n, int mode, uint8_t* codes, uint8_t* scales,
+                       csa_stream_t stream) {
+  if (rows < 0 || n <= 0 || n % 32 != 0 || (mode != CSA_MX_OCP && mode != CSA_MX_INDEXER)) return CSA_ERR_INVALID_ARG;
+  if (rows == 0) return CSA_OK;
+  int rc = check_ptrs(x, codes, scales);
+  if (rc) return rc;
+  cudaError_t e = launch_mxfp4_quantize(x, rows * (n / 32), mode, codes, scales, (cudaStream_t)stream);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
@@ -211,12 +253,13 @@ size_t csa_sparse_attn_workspace_bytes(int64_t, int, int, int, int) { return kWo
 
 int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t* idx, const void* Kraw,
                     const void* Vraw, int64_t T, int64_t t0, int64_t Nc, int H, int d, int k, int W, float scale,
-                    void* O, float* lse, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
-  if (T < 0 || t0 < 0 || Nc < 0 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f))
+                    void* O, int o_dtype, float* lse, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  if (T < 0 || t0 < 0 || Nc < 0 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f) ||
+      !valid_odtype(o_dtype))
     return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   const int gq = 128 / H;
-  if (gq * ceil_div(k, 128) + window_tiles(W, gq) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
+  if (gq * ceil_div(k, 128) > attention_max_seg_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
   int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
   if (rc) return rc;
   if (T == 0) return CSA_OK;
@@ -241,7 +284,8 @@ int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t
   a.m = 1;
   a.W = W;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.O = static_cast<__nv_bfloat16*>(O);
+  a.O = O;
+  a.o_f32 = o_dtype == CSA_F32;
   a.lse = lse;
   a.status = status_word(workspace);
   a.q_rows = T * H;
@@ -254,14 +298,13 @@ int csa_sparse_attn(const void* Q, const void* Kc, const void* Vc, const int32_t
 size_t hca_attn_workspace_bytes(int64_t, int, int, int) { return kWorkspaceHeader; }
 
 int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, const void* Vraw, int64_t T, int64_t t0,
-             int64_t Nc, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
+             int64_t Nc, int H, int d, int m, int W, float scale, void* O, int o_dtype, float* lse, void* workspace,
              size_t workspace_bytes, csa_stream_t stream) {
-  if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f)) return CSA_ERR_INVALID_ARG;
+  if (T < 0 || t0 < 0 || Nc < 0 || m < 1 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f) ||
+      !valid_odtype(o_dtype))
+    return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   const int gq = 128 / H;
-  int64_t nv = n_visible(t0 + T - 1, m);
-  if (nv > Nc) nv = Nc;
-  if (ceil_div(nv, 128) + window_tiles(W, gq) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
   int rc = check_ws(workspace, workspace_bytes, kWorkspaceHeader);
   if (rc) return rc;
   if (T == 0) return CSA_OK;
@@ -286,7 +329,8 @@ int hca_attn(const void* Q, const void* Kc, const void* Vc, const void* Kraw, co
   a.m = m;
   a.W = W;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.O = static_cast<__nv_bfloat16*>(O);
+  a.O = O;
+  a.o_f32 = o_dtype == CSA_F32;
   a.lse = lse;
   a.status = status_word(workspace);
   a.q_rows = T * H;
@@ -307,13 +351,13 @@ size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int, int, i
 int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
                const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
                const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
-               int W, float scale, void* O, float* lse, int32_t* idx, float* scores, void* workspace,
+               int W, float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
                size_t workspace_bytes, csa_stream_t stream) {
-  if (B < 0 || Ncap < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f))
+  if (B < 0 || Ncap < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f) ||
+      !valid_odtype(o_dtype))
     return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128) || !valid_HI(HI) || (dI != 64 && dI != 128))
     return CSA_ERR_UNSUPPORTED_SHAPE;
-  if (ceil_div(k, 128) + window_tiles(W, 1) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
   int rc = check_ws(workspace, workspace_bytes, csa_decode_workspace_bytes(B, Ncap, H, d, HI, dI, k, W));
   if (rc) return rc;
   if (B == 0) return CSA_OK;
@@ -367,7 +411,8 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   a.m = m;
   a.W = W;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.O = static_cast<__nv_bfloat16*>(O);
+  a.O = O;
+  a.o_f32 = o_dtype == CSA_F32;
   a.lse = lse;
   a.status = status_word(workspace);
   a.q_batch_stride = (int64_t)H * d;
@@ -393,9 +438,11 @@ size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W) {
 }
 
 int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
-               int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, float* lse, void* workspace,
-               size_t workspace_bytes, csa_stream_t stream) {
-  if (B < 0 || Ncap < 0 || m < 1 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f)) return CSA_ERR_INVALID_ARG;
+               int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, int o_dtype, float* lse,
+               void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  if (B < 0 || Ncap < 0 || m < 1 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f) ||
+      !valid_odtype(o_dtype))
+    return CSA_ERR_INVALID_ARG;
   if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   int rc = check_ws(workspace, workspace_bytes, hca_decode_workspace_bytes(B, Ncap, H, d, W));
   if (rc) return rc;
@@ -408,7 +455,6 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
     if (nv > Ncap) nv = Ncap;
     if (nv > nvis_max) nvis_max = nv;
   }
-  if (ceil_div(nvis_max, 128) + window_tiles(W, 1) > attention_max_tiles()) return CSA_ERR_UNSUPPORTED_SHAPE;
   rc = check_ptrs(q, O);
   if (rc) return rc;
   if (Ncap > 0 && (rc = check_ptrs(Kc, Vc))) return rc;
@@ -431,7 +477,8 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
   a.m = m;
   a.W = W;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.O = static_cast<__nv_bfloat16*>(O);
+  a.O = O;
+  a.o_f32 = o_dtype == CSA_F32;
   a.lse = lse;
   a.status = status_word(workspace);
   a.q_batch_stride = (int64_t)H * d;

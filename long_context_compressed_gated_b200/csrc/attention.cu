@@ -41,7 +41,10 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr int kTileKeys = 128;
-constexpr int kMaxTiles = 80;
+// Selected-entry (SEG) tiles of one CTA are listed in shared memory (4 bytes
+// each); dense (HCA) and window tiles are computed from their index, so their
+// number is not limited by the list.
+constexpr int kMaxSegTiles = 512;
 constexpr int kSoftmaxWarps = 8, kLoaderWarps = 4;
 constexpr int kLoaderThreads = kLoaderWarps * 32;
 constexpr int kMmaWarp = kSoftmaxWarps + kLoaderWarps;
@@ -55,6 +58,32 @@ struct Tile {
   int type, owner, width, valid;  // valid: keys of the tile that exist (<= width)
   int64_t base;                   // SEG: offset in the token's list; HCA: j0; WIN: w0
 };
+
+// A CTA's tile list: nseg listed SEG tiles, then nhca dense tiles of the visible
+// prefix (nv_hca entries), then nwin window tiles from position win_lo; the CTA
+// works on tiles [first, first + count) of that list.
+struct TileList {
+  int nseg, nhca, nwin, first, count, pad;
+  int64_t nv_hca, win_lo, win_hi;  // win_hi: last window position (inclusive)
+};
+
+__device__ __forceinline__ Tile tile_at(const TileList& L, const uint32_t* seg, int i) {
+  i += L.first;
+  if (i < L.nseg) {
+    const uint32_t p = seg[i];
+    return Tile{kSeg, (int)(p & 0xFFu), (int)((p >> 16) & 0xFFu), (int)(p >> 24), (int64_t)((p >> 8) & 0xFFu) * kTileKeys};
+  }
+  i -= L.nseg;
+  if (i < L.nhca) {
+    const int64_t j0 = (int64_t)i * kTileKeys;
+    const int v = (int)(L.nv_hca - j0 < kTileKeys ? L.nv_hca - j0 : kTileKeys);
+    return Tile{kHca, 0, (v + 15) & ~15, v, j0};
+  }
+  i -= L.nhca;
+  const int64_t w0 = L.win_lo + (int64_t)i * kTileKeys;
+  const int v = (int)(L.win_hi - w0 + 1 < kTileKeys ? L.win_hi - w0 + 1 : kTileKeys);
+  return Tile{kWin, 0, (v + 15) & ~15, v, w0};
+}
 
 // 2^x with the SFU (ex2.approx, ~2 ulp; -inf -> +0).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -93,8 +122,9 @@ struct AttnSmem {
   static constexpr size_t off_k = off_q + kTileBytes;      // 2 stages
   static constexpr size_t off_v = off_k + 2 * kTileBytes;  // 2 stages
   static constexpr size_t off_p = off_v + 2 * kTileBytes;  // 128 x 128 bf16
-  static constexpr size_t off_tiles = off_p + 2 * kHalf;
-  static constexpr size_t off_bar = off_tiles + kMaxTiles * sizeof(Tile);
+  static constexpr size_t off_tiles = off_p + 2 * kHalf;               // SEG tiles, packed
+  static constexpr size_t off_list = off_tiles + kMaxSegTiles * 4;      // TileList
+  static constexpr size_t off_bar = off_list + 64;
   static constexpr size_t off_misc = off_bar + 16 * 8;
   static constexpr size_t off_ones = off_misc + 256;       // 16 x 16 bf16 ones (row-sum MMA operand)
   static constexpr size_t off_red = off_ones + 512;        // [2][128] floats: partial fp32 row sums
@@ -115,7 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   uint8_t* s_k = smem + L::off_k;
   uint8_t* s_v = smem + L::off_v;
   uint8_t* s_p = smem + L::off_p;
-  Tile* s_tiles = reinterpret_cast<Tile*>(smem + L::off_tiles);
+  uint32_t* s_seg = reinterpret_cast<uint32_t*>(smem + L::off_tiles);
+  TileList* s_list = reinterpret_cast<TileList*>(smem + L::off_list);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* q_full = bar + 0;
   uint64_t* k_full = bar + 1;   // [2]
@@ -126,7 +157,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   uint64_t* s_free = bar + 11;  // [2]
   uint64_t* p_full = bar + 13;
   uint64_t* pv_done = bar + 14;
-  int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [0] ntiles, [1] tmem, [2..] seg counts
+  uint64_t* mma_fin = bar + 15;  // every issued MMA complete (before TMEM is freed)
+  int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [0] ntiles, [1] tmem, [2..33] seg counts
+  volatile int* s_abort = misc + 48;  // set by the first wait that timed out; every role then stops
   uint8_t* s_ones = smem + L::off_ones;
   float* s_red = reinterpret_cast<float*>(smem + L::off_red);
   int* s_idx = reinterpret_cast<int*>(smem + L::off_idx);
@@ -149,6 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   };
   const int ntok = (int)((T - row_tok0) < GQ ? (T - row_tok0) : GQ);
   const int64_t t_first = token_pos(0), t_last = token_pos(ntok - 1);
+  // A bounded wait of an earlier CTA (or kernel on this workspace) gave up: skip
+  // the work instead of waiting out every deadline again.
+  const int status_at_entry = tid == 0 ? *reinterpret_cast<volatile int*>(a.status) : 0;
 
   // ---- setup: barriers, TMEM, selected-index lists, tile list
   if (tid == 0) {
@@ -163,6 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     }
     mbar_init(p_full, kSoftmaxWarps);
     mbar_init(pv_done, 1);
+    mbar_init(mma_fin, 1);
+    *s_abort = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -197,37 +235,39 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   }
   __syncthreads();
   if (tid == 0) {
-    int nt = 0;
+    TileList tl{};
+    int nseg = 0;
     if (idx != nullptr) {
       // the tokens' selected-entry tiles alternate, so that consecutive tiles (in
       // the two S buffers) keep the softmax warps of both tokens busy
       int nmax = 0;
       for (int g = 0; g < ntok; ++g) nmax = misc[2 + g] > nmax ? misc[2 + g] : nmax;
       for (int off = 0; off < nmax; off += kTileKeys) {
-        for (int g = 0; g < ntok && nt < kMaxTiles; ++g) {
+        for (int g = 0; g < ntok && nseg < kMaxSegTiles; ++g) {
           const int n = misc[2 + g];
           if (off >= n) continue;
           const int v = n - off < kTileKeys ? n - off : kTileKeys;
-          s_tiles[nt++] = Tile{kSeg, g, (v + 15) & ~15, v, (int64_t)off};
+          s_seg[nseg++] = (uint32_t)g | ((uint32_t)(off / kTileKeys) << 8) | ((uint32_t)((v + 15) & ~15) << 16) |
+                          ((uint32_t)v << 24);
         }
       }
     } else {
       int64_t nv = n_visible(t_last, a.m);
       if (nv > a.Nc) nv = a.Nc;
-      for (int64_t j0 = 0; j0 < nv && nt < kMaxTiles; j0 += kTileKeys) {
-        const int v = (int)(nv - j0 < kTileKeys ? nv - j0 : kTileKeys);
-        s_tiles[nt++] = Tile{kHca, 0, (v + 15) & ~15, v, j0};
-      }
+      tl.nv_hca = nv > 0 ? nv : 0;
+      tl.nhca = (int)ceil_div(tl.nv_hca, kTileKeys);
     }
+    tl.nseg = nseg;
     if (a.W > 0 && ntok > 0) {
       int64_t w_lo = t_first - a.W + 1;
       if (w_lo < raw_lo) w_lo = raw_lo;
       if (w_lo < 0) w_lo = 0;
-      for (int64_t w0 = w_lo; w0 <= t_last && nt < kMaxTiles; w0 += kTileKeys) {
-        const int v = (int)(t_last - w0 + 1 < kTileKeys ? t_last - w0 + 1 : kTileKeys);
-        s_tiles[nt++] = Tile{kWin, 0, (v + 15) & ~15, v, w0};
-      }
+      tl.win_lo = w_lo;
+      tl.win_hi = t_last;
+      tl.nwin = t_last >= w_lo ? (int)ceil_div(t_last - w_lo + 1, kTileKeys) : 0;
     }
+    int nt = tl.nseg + tl.nhca + tl.nwin;
+    tl.first = 0;
     if (a.nsplit > 1) {
       // this CTA's share of the sequence's tiles
       const int tps = (nt + a.nsplit - 1) / a.nsplit;
@@ -235,9 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       int cnt = nt - first;
       if (cnt > tps) cnt = tps;
       if (cnt < 0) cnt = 0;
-      for (int i = 0; i < cnt; ++i) s_tiles[i] = s_tiles[first + i];
+      tl.first = first < nt ? first : 0;
       nt = cnt;
     }
+    if (status_at_entry == CSA_ERR_DEVICE_TIMEOUT) nt = 0;
+    tl.count = nt;
+    *s_list = tl;
     misc[0] = nt;
   }
   tc_fence_before();
@@ -245,6 +288,14 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   tc_fence_after();
   const int ntiles = misc[0];
   const uint32_t tbase = (uint32_t)misc[1];
+  const TileList tlist = *s_list;
+  // Bounded wait that also stops once any role of this CTA has given up.
+  auto wait = [&](uint64_t* b_, uint32_t ph) -> bool {
+    if (*s_abort) return false;
+    if (mbar_wait(b_, ph, a.status, CSA_ERR_DEVICE_TIMEOUT)) return true;
+    *s_abort = 1;
+    return false;
+  };
   constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
 
   if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
@@ -252,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     const int lt = tid - kSoftmaxWarps * 32;                 // 0..127
     const int64_t kc_base = decode ? b * a.Nc : 0;           // first compressed row of this sequence
     const int64_t raw_base = decode ? b * (int64_t)a.W : 0;  // first raw row of this sequence
-    if (lt == 0) {
+    if (lt == 0 && ntiles > 0) {
       prefetch_tmap(&maps.q);
       mbar_arrive_expect_tx(q_full, HALVES * kHalfBytes);
       const int qrow = (int)(decode ? b * H : row_tok0 * H);
@@ -264,15 +315,22 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     constexpr int RSTEP = kLoaderThreads / CH;
     const int c = lt % CH, r0 = lt / CH;
     const uint32_t dst_lane = (uint32_t)((c >> 3) * kHalfBytes + r0 * 128 + (((c & 7) ^ (r0 & 7)) << 4));
-    for (int i = 0; i < ntiles; ++i) {
-      const Tile tl = s_tiles[i];
+    // TMA loads this thread has armed and not yet seen consumed: [K/V][stage] parity
+    int armed[2][2] = {{-1, -1}, {-1, -1}};
+    bool live = true;
+    for (int i = 0; i < ntiles && live; ++i) {
+      const Tile tl = tile_at(tlist, s_seg, i);
       const int st = i & 1;
       const uint32_t ph = (i >> 1) & 1;
       for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
         uint64_t* empty = which ? &v_empty[st] : &k_empty[st];
         uint64_t* fullb = which ? &v_full[st] : &k_full[st];
         uint8_t* dst = (which ? s_v : s_k) + (size_t)st * L::kTileBytes;
-        if (!mbar_wait(empty, ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
+        if (!wait(empty, ph ^ 1)) {
+          live = false;
+          break;
+        }
+        armed[which][st] = -1;  // the stage's previous load was consumed
         if (tl.type == kSeg) {
           const int* sel = s_idx + tl.owner * a.k + (int)tl.base;
           const __nv_bfloat16* src0 = (which ? Vc : Kc) + c * 8;
@@ -290,26 +348,33 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
             const int row = (int)(tl.type == kHca ? kc_base + tl.base : raw_base + (tl.base - raw_lo));
             mbar_arrive_expect_tx(fullb, HALVES * kHalfBytes);
             for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(dst + hf * kHalfBytes, m, fullb, hf * 64, row);
+            armed[which][st] = (int)ph;
           }
           mbar_arrive(fullb);
         }
       }
     }
     cp_async_wait_all();
+    // after an abort, wait (bounded) for the TMA loads still landing in shared memory
+    if (lt == 0) {
+      for (int w = 0; w < 2; ++w)
+        for (int st = 0; st < 2; ++st)
+          if (armed[w][st] >= 0) mbar_wait(w ? &v_full[st] : &k_full[st], (uint32_t)armed[w][st]);
+      if (ntiles > 0) mbar_wait(q_full, 0);
+    }
   } else if (warp == kMmaWarp) {
     // =========================== MMA issuer
-    if (ntiles > 0) mbar_wait(q_full, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
+    bool live = ntiles > 0 && wait(q_full, 0);
     tc_fence_after();
     const uint32_t sq = smem_u32(s_q), sp = smem_u32(s_p);
-    auto issue_s = [&](int i) {
+    auto issue_s = [&](int i) -> bool {
       const int st = i & 1;
       const uint32_t ph = (i >> 1) & 1;
-      mbar_wait(&k_full[st], ph, a.status, CSA_ERR_DEVICE_TIMEOUT);
-      mbar_wait(&s_free[st], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      if (!wait(&k_full[st], ph) || !wait(&s_free[st], ph ^ 1)) return false;
       fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tcgen05 (async proxy) reads
       tc_fence_after();
       if (elect_one()) {  // converged-warp issue
-        const int width = s_tiles[i].width;
+        const int width = tile_at(tlist, s_seg, i).width;
         const uint32_t sk = smem_u32(s_k + (size_t)st * L::kTileBytes);
         const uint32_t d = tbase + (st ? kTmemS1 : kTmemS0);
 #pragma unroll
@@ -322,18 +387,18 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         mma_commit(&k_empty[st]);
       }
       __syncwarp();
+      return true;
     };
-    if (ntiles > 0) issue_s(0);
-    if (ntiles > 1) issue_s(1);
+    if (live && ntiles > 0) live = issue_s(0);
+    if (live && ntiles > 1) live = issue_s(1);
     const uint64_t ones = make_sdesc(smem_u32(s_ones), 128, 256, kSwizzleNone);
-    for (int i = 0; i < ntiles; ++i) {
+    for (int i = 0; i < ntiles && live; ++i) {
       const int st = i & 1;
-      mbar_wait(p_full, i & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
-      mbar_wait(&v_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      if (!wait(p_full, i & 1) || !wait(&v_full[st], (i >> 1) & 1)) break;
       fence_proxy_async_smem();
       tc_fence_after();
       if (elect_one()) {
-        const int width = s_tiles[i].width;
+        const int width = tile_at(tlist, s_seg, i).width;
         const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
         for (int ks = 0; ks < width / 16; ++ks) {
           const uint32_t aoff = (uint32_t)((ks >> 2) * kHalfBytes + (ks & 3) * 32);
@@ -348,8 +413,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         mma_commit(&v_empty[st]);
       }
       __syncwarp();
-      if (i + 2 < ntiles) issue_s(i + 2);
+      if (i + 2 < ntiles && !issue_s(i + 2)) break;
     }
+    // every MMA this warp issued has completed before TMEM is freed
+    if (elect_one()) mma_commit(mma_fin);
+    __syncwarp();
+    mbar_wait(mma_fin, 0);
   } else {
     // =========================== softmax (warps 0..7): row = TMEM lane, columns [64*half, +64)
     const int quarter = warp & 3, half = warp >> 2;
@@ -363,9 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     const int my0 = half * 64;     // first column this warp turns into probabilities
     float m_run = -INFINITY, l_run32 = 0.f;
     const uint32_t prow = smem_u32(s_p) + (uint32_t)(half * kHalfBytes + row * 128);
+    bool live = true;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
-      const Tile tl = s_tiles[i];
+      const Tile tl = tile_at(tlist, s_seg, i);
       int lo = 0, hi = 0;
       if (t >= 0) {
         if (tl.type == kSeg) {
@@ -384,7 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const int width = tl.width;
       const bool warp_any = __any_sync(0xffffffffu, hi > lo);
       const bool warp_full = __all_sync(0xffffffffu, lo == 0 && hi == width);
-      mbar_wait(&s_full[st], (i >> 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      if (!wait(&s_full[st], (i >> 1) & 1)) {
+        live = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t scol = tbase + lane_base + (st ? kTmemS1 : kTmemS0);
       // pass 1: row maximum of the raw logits over the visible range (all columns)
@@ -453,7 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       if (lane == 0) mbar_arrive(&s_free[st]);
       // wait until PV of the previous tile finished: P buffer free, O stable
       if (i > 0) {
-        mbar_wait(pv_done, (i - 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+        if (!wait(pv_done, (i - 1) & 1)) {
+          live = false;
+          break;
+        }
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
@@ -501,8 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     }
     // epilogue: O / l, with l the row sum of the bf16 weights (tensor-core P x ones)
     float l_run = 0.f;
-    if (ntiles > 0) {
-      mbar_wait(pv_done, (ntiles - 1) & 1, a.status, CSA_ERR_DEVICE_TIMEOUT);
+    const bool have_o = ntiles > 0 && live && wait(pv_done, (ntiles - 1) & 1);
+    if (have_o) {
       tc_fence_after();
       uint32_t v[16];
       tmem_ld16p(tbase + lane_base + kTmemO + D, v);
@@ -512,14 +588,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
     const bool part = a.nsplit > 1;
     __nv_bfloat16* orow = nullptr;
-    float* part_row = nullptr;
-    if (t >= 0 && !part) orow = a.O + b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
+    float* part_row = nullptr;  // fp32 rows: a split's partial output, or O itself when o_f32
+    const int64_t o_off = b * a.o_batch_stride + ((row_tok0 + g) * H + h) * (int64_t)D;
+    if (t >= 0 && !part && !a.o_f32) orow = static_cast<__nv_bfloat16*>(a.O) + o_off;
+    if (t >= 0 && !part && a.o_f32) part_row = static_cast<float*>(a.O) + o_off;
     if (t >= 0 && part) part_row = a.o_part + ((b * a.nsplit + blockIdx.y) * H + h) * (int64_t)D;
 #pragma unroll
     for (int b0 = 0; b0 < 64; b0 += 32) {
       if (my0 >= D) break;
       uint32_t v[32];
-      if (ntiles > 0) {
+      if (have_o) {
         tmem_ld32p(tbase + lane_base + kTmemO + my0 + b0, v);
         tmem_wait_ld();
       } else {
@@ -572,7 +650,7 @@ size_t attention_smem_bytes(int d, int idx_entries) {
   return d == 128 ? AttnSmem<128>::bytes(idx_entries) : AttnSmem<64>::bytes(idx_entries);
 }
 
-int attention_max_tiles() { return kMaxTiles; }
+int attention_max_seg_tiles() { return kMaxSegTiles; }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -608,7 +686,7 @@ constexpr int kCombineSplits = 16;
 template <int D>
 __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __restrict__ o_part,
                                                                 const float* __restrict__ lse_part, int nsplit, int H,
-                                                                int64_t rows, __nv_bfloat16* __restrict__ O,
+                                                                int64_t rows, void* __restrict__ O, int o_f32,
                                                                 int64_t o_batch_stride, float* __restrict__ lse) {
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (b, h)
@@ -644,10 +722,16 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __r
     }
   }
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
-  uint2 packed;
-  packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-  packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-  *reinterpret_cast<uint2*>(O + b * o_batch_stride + (int64_t)h * D + 4 * lane) = packed;
+  const int64_t off = b * o_batch_stride + (int64_t)h * D + 4 * lane;
+  if (o_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(O) + off) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  } else {
+    uint2 packed;
+    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(O) + off) = packed;
+  }
   if (lse && lane == 0) lse[b * H + h] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
 }
 
@@ -657,10 +741,10 @@ cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream
   const unsigned grid = (unsigned)((rows + 7) / 8);
   if (d == 128)
     attention_combine_kernel<128><<<grid, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, rows, a.O,
-                                                             a.o_batch_stride, a.lse);
+                                                             a.o_f32, a.o_batch_stride, a.lse);
   else
     attention_combine_kernel<64><<<grid, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, rows, a.O,
-                                                            a.o_batch_stride, a.lse);
+                                                            a.o_f32, a.o_batch_stride, a.lse);
   return cudaGetLastError();
 }
 

@@ -17,7 +17,8 @@ struct AttnArgs {
   int64_t T, t0, Nc, raw_lo;
   int H, k, m, W;
   float scale_log2;         // softmax scale * log2(e)
-  __nv_bfloat16* O;         // [T, H, d]
+  void* O;                  // [T, H, d] bf16, or fp32 when o_f32
+  int o_f32;                // 1: O is written as fp32 (no bf16 rounding of the result)
   float* lse;               // [T, H] natural-log normaliser, nullable
   int* status;              // device status word
   // decode (pos != null): one sequence per CTA, batch strides in elements
@@ -36,6 +37,6 @@ struct AttnArgs {
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);
 // O[b,h] = sum_s exp(lse_s - lse) O_s with lse = log sum_s exp(lse_s), as bf16 (+ lse)
 cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream);
-int attention_max_tiles();
+int attention_max_seg_tiles();
 
 }  // namespace csa

@@ -35,6 +35,8 @@
 //    epilogue.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "topk.cuh"
@@ -137,6 +139,7 @@ struct IndexerArgs {
   uint64_t* cand;           // [rows, nsplit, k] selected keys of each key range (unsorted)
   int* cand_cnt;            // [rows, nsplit]    how many of them are valid
   int* status;
+  int fault;                // test hook (csa_debug_inject): 1 = the producer skips its first stage group
 };
 
 template <int HI, int DI, int G>
@@ -160,7 +163,7 @@ struct IndexerSmem {
   static constexpr size_t off_hist = off_thr + 64 * 8;
   static constexpr size_t off_grp = off_hist + (size_t)(G == 1 ? 1 : 2) * topk::kWarpBins * 4;  // [2][32] ints
   static constexpr size_t off_bar = off_grp + 256;
-  static constexpr size_t off_tslot = off_bar + (2 * kStages + 2 * NB + 1) * 8;
+  static constexpr size_t off_tslot = off_bar + (2 * kStages + 2 * NB + 2) * 8;
   static constexpr size_t off_cand = ((off_tslot + 16 + 15) / 16) * 16;
   static size_t bytes(int cap) { return off_cand + (size_t)G * cap * 8 + 1024; }
 };
@@ -203,12 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* dfull = bar + 2 * NST;           // [NBG] MMA -> epilogue
   uint64_t* dempty = bar + 2 * NST + NB;     // [NBG] epilogue -> MMA
   uint64_t* ready = bar + 2 * NST + 2 * NB;  //       epilogue (TMEM scales written) + q tile -> MMA
+  uint64_t* mma_fin = ready + 1;             //       every issued MMA complete (before TMEM is freed)
   uint32_t* s_tslot = reinterpret_cast<uint32_t*>(smem + L::off_tslot);
   uint64_t* s_cand = reinterpret_cast<uint64_t*>(smem + L::off_cand);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cap = a.cap;
   const bool decode = a.pos != nullptr;
+  // A bounded wait of an earlier CTA on this workspace gave up: skip the work
+  // (read now, used after the setup, so the load overlaps it).
+  const int status_at_entry = *reinterpret_cast<volatile int*>(a.status);
 
   // ---- which tokens and which key range
   const int64_t grp = decode ? blockIdx.x : (int64_t)(gridDim.x - 1 - blockIdx.x);  // heavy groups first
@@ -230,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t j_begin = (int64_t)split * a.split_tiles * 128;
   int64_t j_end = j_begin + a.split_tiles * 128;
   if (j_end > nvis_max) j_end = nvis_max;
-  const int ntiles = j_end > j_begin ? (int)ceil_div(j_end - j_begin, 128) : 0;
+  const int ntiles_all = j_end > j_begin ? (int)ceil_div(j_end - j_begin, 128) : 0;
 
   // ---- setup
   if (tid == 0) {
@@ -243,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&dempty[b], TPG * (kAlt ? kEpiWarps / 2 : kEpiWarps));
     }
     mbar_init(ready, kEpiWarps + 1);
+    mbar_init(mma_fin, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -295,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *s_tslot;
+  const int ntiles = status_at_entry == CSA_ERR_DEVICE_TIMEOUT ? 0 : ntiles_all;
 
   if (warp == 0) {
     // =========================== producer
@@ -304,11 +313,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(ready, N * L::kRowBytes);
       tma_load_2d(s_q, &qmap, ready, 0, (int)(row0 * HI));
     }
+    // the phase of each stage group's last fill not yet seen consumed (-1: none)
+    int armed[NSG];
+#pragma unroll
+    for (int q = 0; q < NSG; ++q) armed[q] = -1;
+    bool aborted = false;
     for (int g0 = 0; g0 < ntiles; g0 += TPG) {
+      if (a.fault == 1 && g0 == 0) continue;  // injected: stage group 0 is never filled
       const int gs = (g0 / TPG) % NSG;
       const uint32_t ph = (g0 / TPG / NSG) & 1;
       const int nt = ntiles - g0 < TPG ? ntiles - g0 : TPG;
-      if (!mbar_wait(&empty[gs], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) break;
+      if (!mbar_wait(&empty[gs], ph ^ 1, a.status, CSA_ERR_DEVICE_TIMEOUT)) {
+        aborted = true;
+        break;
+      }
+#pragma unroll
+      for (int q = 0; q < NSG; ++q)
+        if (q == gs) armed[q] = (int)ph;
       if (lane == 0) mbar_arrive_expect_tx(&full[gs], (uint32_t)(nt * L::kABytes));
       for (int u = 0; u < nt; ++u) {
         const int it = g0 + u, s = it % NST;
@@ -345,10 +366,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     cp_async_wait_all();
+    // wait (bounded) for the copies still landing in shared memory: none in a
+    // run that went through, the unconsumed ones after an abort
+#pragma unroll
+    for (int q = 0; q < NSG; ++q)
+      if (armed[q] >= 0) mbar_wait(&full[q], (uint32_t)armed[q]);
+    if (ntiles > 0) mbar_wait(ready, 0);
+    (void)aborted;
   } else if (warp == 1) {
     // =========================== MMA issuer
+    bool live = true;
     if (ntiles > 0) {
-      mbar_wait(ready, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
+      live = mbar_wait(ready, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
       tc_fence_after();
     }
     const uint32_t layout = DI == 128 ? kSwizzle64 : kSwizzle32;
@@ -365,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One issue unit = UG barrier groups (2 single tiles in prefill, one group of 4
     // tiles in decode); the tiles' chains interleave.
     constexpr int UG = TPG == 1 ? 2 : 1;
-    int g0 = 0;
+    int g0 = live ? 0 : ntiles;
     while (g0 < ntiles) {
       const int nt = ntiles - g0 < UG * TPG ? ntiles - g0 : UG * TPG;  // tiles in this unit
       bool ok = true;
@@ -409,6 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       g0 += nt;
     }
+    // every MMA (and scale copy) this warp issued has completed before TMEM is freed
+    if (elect_one()) mma_commit(mma_fin);
+    __syncwarp();
+    mbar_wait(mma_fin, 0, a.status, CSA_ERR_DEVICE_TIMEOUT);
   } else {
     // =========================== epilogue + selection (warps 2..9)
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
@@ -922,6 +955,14 @@ static bool make_u8_map(CUtensorMap* m, const void* base, int64_t rows, int row_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Test hook: a fault code set by csa_debug_inject() and taken by the next indexer launch.
+static std::atomic<int> g_injected_fault{0};
+static int take_injected_fault() { return g_injected_fault.exchange(0); }
+int inject_fault(int code) {
+  g_injected_fault.store(code);
+  return 0;
+}
+
 // Candidate capacity per token: whatever shared memory is left (cut-backs are
 // rarer the larger it is), at least k + 128*check and a power of two >= k.
 template <int HI, int DI, int G>
@@ -965,6 +1006,7 @@ static bool choose_cap(int k, int* cap, int* check) {
 template <int HI, int DI, int G>
 static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, IndexerArgs a, dim3 grid,
                               cudaStream_t stream) {
+  a.fault = take_injected_fault();
   using L = IndexerSmem<HI, DI, G>;
   CUtensorMap qmap, kmap;
   if (!make_u8_map(&qmap, q_codes, a.rows * HI, DI / 2, L::N)) return cudaErrorInvalidValue;

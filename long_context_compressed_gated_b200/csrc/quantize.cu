@@ -1,0 +1,88 @@
+// quantize.cu - bf16 activations -> MXFP4, the operand format of the indexer's
+// query-key contraction (m.youleyou.com/wenzhang/2906406.html section 1 and
+// ferris-liu.github.io ... deepseek-v4 "engineering": the indexer's QK path
+// runs in FP4).  The pages give no scale rule; this follows the OCP MX
+// conversion: per block of 32 consecutive elements
+//   X = floor(log2 max|x|) - 2,  scale byte = X + 127 (E8M0),
+//   code = E2M1 nearest to x / 2^X, ties to the even code, |.| > 6 -> 6, sign kept.
+// mode CSA_MX_INDEXER clamps X to [-2, 1] (scale bytes 125..128), the range in
+// which the indexer's exact fixed-point head sum holds.
+//
+// HBM-bound: one thread per 32-element block reads its 64 bytes with four
+// 16-byte loads and writes 16 bytes of codes and one scale byte.
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+// E2M1 magnitude code of y >= 0 (y exact in fp32): the number of rounding
+// boundaries y has passed.  The boundaries are the midpoints between the
+// magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; a midpoint itself goes to the even
+// code, hence ">" where the lower neighbour is even and ">=" where it is odd.
+__device__ __forceinline__ uint32_t e2m1_magnitude_code(float y) {
+  return (uint32_t)(y > 0.25f) + (uint32_t)(y >= 0.75f) + (uint32_t)(y > 1.25f) + (uint32_t)(y >= 1.75f) +
+         (uint32_t)(y > 2.5f) + (uint32_t)(y >= 3.5f) + (uint32_t)(y > 5.0f);
+}
+
+__global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const uint4* __restrict__ x, int64_t nblocks, int mode,
+                                                             uint4* __restrict__ codes,
+                                                             uint8_t* __restrict__ scales) {
+  const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (blk >= nblocks) return;
+  uint32_t w[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = __ldg(x + blk * 4 + q);
+    w[4 * q] = u.x;
+    w[4 * q + 1] = u.y;
+    w[4 * q + 2] = u.z;
+    w[4 * q + 3] = u.w;
+  }
+  // max |x| over the block on the bf16 magnitude bits (an order-preserving
+  // integer for finite values); an exponent field of all ones is Inf or NaN
+  uint32_t amax_bits = 0;
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
+    finite &= (lo < 0x7F80u) & (hi < 0x7F80u);
+    amax_bits = max(amax_bits, max(lo, hi));
+  }
+  if (!finite) {
+    codes[blk] = make_uint4(0u, 0u, 0u, 0u);
+    scales[blk] = 255;
+    return;
+  }
+  int X = -127;
+  if (amax_bits != 0) {
+    int e;
+    frexpf(__uint_as_float(amax_bits << 16), &e);  // amax = f * 2^e, f in [0.5, 1)
+    X = e - 3;                                     // floor(log2 amax) - 2
+  }
+  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  if (mode == CSA_MX_INDEXER) X = X < -2 ? -2 : (X > 1 ? 1 : X);
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t b = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
+    const float y = ldexpf(__uint_as_float((b & 0x7FFFu) << 16), -X);  // exact: a power-of-two scaling
+    const uint32_t code = ((b >> 12) & 8u) | e2m1_magnitude_code(y);
+    out[i >> 3] |= code << (4 * (i & 7));
+  }
+  codes[blk] = make_uint4(out[0], out[1], out[2], out[3]);
+  scales[blk] = (uint8_t)(X + 127);
+}
+
+}  // namespace
+
+cudaError_t launch_mxfp4_quantize(const void* x, int64_t nblocks, int mode, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t stream) {
+  if (nblocks == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)ceil_div(nblocks, 256);
+  mxfp4_quantize_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(x), nblocks, mode,
+                                                  reinterpret_cast<uint4*>(codes), scales);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

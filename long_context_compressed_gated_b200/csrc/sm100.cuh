@@ -9,9 +9,10 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-// Deadline of a bounded wait, in SM clock cycles (~2 s at 2 GHz).
+// Deadline of a bounded wait, in SM clock cycles (2^28: ~0.14 s at 1.965 GHz,
+// thousands of times the longest wait of a working pipeline).
 #ifndef CSA_WAIT_CYCLES
-#define CSA_WAIT_CYCLES (1ll << 32)
+#define CSA_WAIT_CYCLES (1ll << 28)
 #endif
 
 namespace csa {

@@ -21,14 +21,16 @@ from . import csa_compress, csa_indexer_topk, csa_sparse_attn, hca_attn, lib
 
 
 def stack_prefill_chunked(l1, l2, P, chunk, m, k, W, m2, W2, scale=None, out=None, phase_events=None,
-                          return_o1=False):
+                          return_o1=False, idx_out=None, scores_out=None):
     """Run the two-layer stack over all T tokens in chunks of `chunk`.
 
     l1: dict with Q [T,H,d], K, V, Z [T,d], B [m,d], qI_codes [T,HI,dI/2],
         qI_scales [T,HI,dI/32], w_codes [T,HI], kI_codes [T/m,dI/2], kI_scales.
     l2: dict with K, V, Z [T,d], B [m2,d].   P: [d,d] bf16.
     Returns O2 [T,H,d] (and O1 when return_o1).  phase_events: optional list that
-    receives (name, start_event, end_event) per phase for timing.
+    receives (name, start_event, end_event) per phase for timing.  idx_out [T,k]
+    int32 / scores_out [T,k] f32 (optional): keep every chunk's layer-1 selection
+    (the indexer writes its rows there instead of a per-chunk buffer).
     """
     Q1 = l1["Q"]
     T, H, d = Q1.shape
@@ -39,7 +41,7 @@ def stack_prefill_chunked(l1, l2, P, chunk, m, k, W, m2, W2, scale=None, out=Non
     Vc1 = torch.empty_like(Kc1)
     Kc2 = torch.empty(T // m2, d, dtype=torch.bfloat16, device=dev)
     Vc2 = torch.empty_like(Kc2)
-    idx = torch.empty(chunk, k, dtype=torch.int32, device=dev)
+    idx_chunk = torch.empty(chunk, k, dtype=torch.int32, device=dev) if idx_out is None else None
     O1 = torch.empty_like(Q1)
     Q2 = torch.empty_like(Q1)
     O2 = torch.empty_like(Q1) if out is None else out
@@ -64,12 +66,15 @@ def stack_prefill_chunked(l1, l2, P, chunk, m, k, W, m2, W2, scale=None, out=Non
         sl = slice(t0, t0 + chunk)
         b1, e1 = t0 // m, (t0 + chunk) // m
         b2, e2 = t0 // m2, (t0 + chunk) // m2
+        idx = idx_chunk if idx_out is None else idx_out[sl]
+        sc = None if scores_out is None else scores_out[sl]
         # layer 1 (CSA)
         timed("compress", lambda: csa_compress(l1["K"][sl], l1["V"][sl], l1["Z"][sl], l1["B"], m, Kc=Kc1[b1:e1],
                                                Vc=Vc1[b1:e1]))
         timed("indexer_topk", lambda: csa_indexer_topk(l1["qI_codes"][sl], l1["qI_scales"][sl], l1["w_codes"][sl],
                                                        l1["kI_codes"][:e1], l1["kI_scales"][:e1], m, k, t0=t0,
-                                                       idx=idx, want_scores=False, workspace=ws))
+                                                       idx=idx, scores=sc, want_scores=sc is not None,
+                                                       workspace=ws))
         timed("sparse_attn", lambda: csa_sparse_attn(Q1[sl], Kc1[:e1], Vc1[:e1], idx, l1["K"][: t0 + chunk],
                                                      l1["V"][: t0 + chunk], W, scale, t0=t0, O=O1[sl],
                                                      want_lse=False, workspace=ws))

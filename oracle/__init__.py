@@ -15,7 +15,11 @@ marshals numpy arrays through ctypes and composes the steps:
   topk            -- k largest visible I[t,j], ties -> smaller j, pad -1 / -inf
   attention       -- one joint softmax over selected (or all visible) compressed
                      entries and the raw window [max(0,t-W+1), t]
-  csa_decode/hca_decode -- the same steps for one new token per sequence
+  mxfp4_quantize  -- bf16 -> MXFP4 by the OCP MX scale rule (E8M0 per 32, E2M1
+                     nearest with ties to even, saturating)
+  csa_layer       -- compress, indexer, top-k and attention composed for rows
+Decode is the same steps for one query row at the sequence's position; the
+tests compose it from these functions.
 
 Parity status of each function is stated in its docstring; every function here
 is pinned by tests/test_oracle_*.py against hand-worked values, closed forms,
@@ -44,6 +48,7 @@ def lib():
         L.oracle_attention.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_long, ctypes.c_int, P,
                                        ctypes.c_int, P, P, ctypes.c_long, ctypes.c_long, ctypes.c_long, P,
                                        ctypes.c_long, ctypes.c_double, P, P, ctypes.c_int]
+        L.oracle_mxfp4_quantize.argtypes = [P, ctypes.c_long, ctypes.c_int, ctypes.c_int, P, P]
         L.oracle_e2m1_value.argtypes = [ctypes.c_int]
         L.oracle_e2m1_value.restype = ctypes.c_double
         L.oracle_e8m0_value.argtypes = [ctypes.c_int]
@@ -182,6 +187,23 @@ def csa_layer(inp, m, k, W, scale, rows=None, Kc=None, Vc=None, nthreads=None):
     O, lse = attention(inp["Q"], Kc, Vc, inp["K"], inp["V"], 0, m, W, scale, sel=idx, rows=rows, nthreads=nthreads)
     out.update(idx=idx, top=top, O=O, lse=lse, I=I)
     return out
+
+
+def mxfp4_quantize(x, mode=0):
+    """bf16 [rows, n] -> (codes uint8 [rows, n/2], scales uint8 [rows, n/32]) by
+    the OCP MX rule: per 32-element block X = floor(log2 max|x|) - 2, codes the
+    E2M1 values nearest to x / 2^X (ties to even, saturating at 6, sign kept).
+    mode 1 clamps X to [-2, 1] (scale bytes 125..128)."""
+    xa = _u16(x)
+    shape = xa.shape
+    n = shape[-1]
+    rows = int(np.prod(shape[:-1])) if len(shape) > 1 else 1
+    xa = np.ascontiguousarray(xa.reshape(rows, n))
+    codes = np.zeros((rows, n // 2), np.uint8)
+    scales = np.zeros((rows, n // 32), np.uint8)
+    rc = lib().oracle_mxfp4_quantize(_p(xa), rows, n, mode, _p(codes), _p(scales))
+    assert rc == 0
+    return codes.reshape(shape[:-1] + (n // 2,)), scales.reshape(shape[:-1] + (n // 32,))
 
 
 def to_bf16_words(x):

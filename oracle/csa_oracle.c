@@ -360,3 +360,77 @@ int oracle_attention(const uint16_t* Q, int H, int d, const uint16_t* Kc, const 
   parallel_rows(attn_row, &x, nrows, nthreads);
   return 0;
 }
+
+/* ------------------------------------------------------------------ MXFP4 quantiser
+ * bf16 activations -> MXFP4 (the indexer's query-key operands; the pages put
+ * the indexer's QK path on MXFP4 but give no scale rule).  Reading taken, the
+ * OCP MX conversion: for every block of 32 consecutive elements of a row,
+ *   X = floor(log2(max_i |x_i|)) - 2        (2 = exponent of E2M1's largest
+ *                                            value 6 = 1.5 * 2^2)
+ *   scale byte = X + 127 (E8M0), code_i = E2M1 nearest to x_i / 2^X, ties to
+ *   the even code, magnitudes above 6 saturated to 6, sign kept (-0 allowed).
+ * Mode 0 keeps X in the E8M0 range [-127, 127] (an all-zero block gets X =
+ * -127); mode 1 clamps X to [-2, 1] (scale bytes 125..128, the range in which
+ * the GPU indexer's exact fixed-point head sum holds), which saturates blocks
+ * with max |x| >= 12 and flushes small ones more coarsely.  A block holding a
+ * NaN or an infinity gets scale byte 255 (NaN) and zero codes.
+ * Layouts: x [rows, n] bf16 (n % 32 == 0) -> codes [rows, n/2] (element 2i in
+ * the low nibble of byte i), scales [rows, n/32].
+ */
+static int e2m1_round_magnitude(double y) {
+  /* nearest of the eight E2M1 magnitudes (decoded from the bit fields), ties to
+   * the even code; y >= 6 saturates to 6 */
+  if (y >= 6.0) return 7;
+  int best = 0;
+  double bestd = fabs(y - oracle_e2m1_value(0));
+  for (int c = 1; c < 8; ++c) {
+    double dd = fabs(y - oracle_e2m1_value(c));
+    if (dd < bestd || (dd == bestd && (c & 1) == 0)) {
+      best = c;
+      bestd = dd;
+    }
+  }
+  return best;
+}
+
+int oracle_mxfp4_quantize(const uint16_t* x, long rows, int n, int mode, uint8_t* codes, uint8_t* scales) {
+  if (!x || !codes || !scales || rows < 0 || n <= 0 || n % 32 || (mode != 0 && mode != 1)) return -1;
+  for (long r = 0; r < rows; ++r) {
+    for (int b = 0; b < n / 32; ++b) {
+      const uint16_t* blk = x + r * n + b * 32;
+      double amax = 0;
+      int finite = 1;
+      for (int i = 0; i < 32; ++i) {
+        double v = bf16_value(blk[i]);
+        if (!isfinite(v)) finite = 0;
+        else if (fabs(v) > amax) amax = fabs(v);
+      }
+      uint8_t* crow = codes + r * (n / 2) + b * 16;
+      if (!finite) {
+        scales[r * (n / 32) + b] = 255;
+        memset(crow, 0, 16);
+        continue;
+      }
+      int X;
+      if (amax == 0) {
+        X = -127;
+      } else {
+        int e;
+        frexp(amax, &e); /* amax = f * 2^e, f in [0.5, 1): floor(log2 amax) = e - 1 */
+        X = (e - 1) - 2;
+      }
+      if (X < -127) X = -127;
+      if (X > 127) X = 127;
+      if (mode == 1) X = X < -2 ? -2 : (X > 1 ? 1 : X);
+      scales[r * (n / 32) + b] = (uint8_t)(X + 127);
+      for (int i = 0; i < 32; ++i) {
+        double v = bf16_value(blk[i]);
+        int sign = signbit(v) ? 8 : 0;
+        int code = sign | e2m1_round_magnitude(fabs(v) / ldexp(1.0, X));
+        if (i % 2 == 0) crow[i / 2] = (uint8_t)code;
+        else crow[i / 2] |= (uint8_t)(code << 4);
+      }
+    }
+  }
+  return 0;
+}

@@ -50,11 +50,17 @@ def assert_within_bf16_ulp(got_bf16, exact_f64, what, slack=None):
 
 
 def assert_attention_close(got_bf16, want_f64, what):
+    """Spec tolerance on an attention output (bf16 or fp32 tensor); prints the
+    margins used (max |O|, max-abs and rel-Frobenius as fractions of the bound)."""
     got = bf16_to_f64(got_bf16)
     want = np.asarray(want_f64, np.float64)
     diff = got - want
     max_abs = float(np.abs(diff).max()) if diff.size else 0.0
     fro = float(np.linalg.norm(diff) / max(np.linalg.norm(want), 1e-30)) if diff.size else 0.0
+    omax = float(np.abs(want).max()) if want.size else 0.0
+    print("[margin] %s (%s): max|O| %.3f, max-abs %.3e (%.0f%% of bound), rel-Fro %.3e (%.0f%% of bound)" % (
+        what, str(getattr(got_bf16, "dtype", "?")).replace("torch.", ""), omax, max_abs,
+        100 * max_abs / ATTN_MAX_ABS, fro, 100 * fro / ATTN_REL_FRO))
     assert max_abs <= ATTN_MAX_ABS and fro <= ATTN_REL_FRO, "%s: max-abs %.3e (<= %.0e), rel-Frobenius %.3e (<= %.0e)" % (
         what, max_abs, ATTN_MAX_ABS, fro, ATTN_REL_FRO)
     return max_abs, fro

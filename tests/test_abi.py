@@ -67,17 +67,25 @@ def test_host_side_validation_rejects_bad_arguments(lib):
                                 None) == -5
     # attention: window too large, bad H
     assert lib.csa_sparse_attn(fake, fake, fake, fake, fake, fake, 8, 0, 8, 64, 128, 16, 5000,
-                               ctypes.c_float(0.1), fake, None, ws, 256, None) == -1
+                               ctypes.c_float(0.1), fake, 0, None, ws, 256, None) == -1
     assert lib.csa_sparse_attn(fake, fake, fake, fake, fake, fake, 8, 0, 8, 48, 128, 16, 64,
-                               ctypes.c_float(0.1), fake, None, ws, 256, None) == -3
-    assert lib.hca_attn(fake, fake, fake, fake, fake, 8, 0, 8, 64, 128, 0, 64, ctypes.c_float(0.1), fake, None,
+                               ctypes.c_float(0.1), fake, 0, None, ws, 256, None) == -3
+    assert lib.hca_attn(fake, fake, fake, fake, fake, 8, 0, 8, 64, 128, 0, 64, ctypes.c_float(0.1), fake, 0, None,
                         ws, 256, None) == -1
+    # output element type other than CSA_BF16 (0) / CSA_F32 (1)
+    assert lib.csa_sparse_attn(fake, fake, fake, fake, fake, fake, 8, 0, 8, 64, 128, 16, 64,
+                               ctypes.c_float(0.1), fake, 2, None, ws, 256, None) == -1
+    assert lib.hca_attn(fake, fake, fake, fake, fake, 8, 0, 8, 64, 128, 4, 64, ctypes.c_float(0.1), fake, -1, None,
+                        ws, 256, None) == -1
+    # selected-entry tiles of one block beyond the list: H = 4 gives 32 tokens x 16 tiles at k = 2048
+    assert lib.csa_sparse_attn(fake, fake, fake, fake, fake, fake, 8, 0, 8, 4, 128, 2048, 64,
+                               ctypes.c_float(0.1), fake, 0, None, ws, 256, None) == -3
     # decode: workspace smaller than required
     need = lib.csa_decode_workspace_bytes(4, 1024, 64, 128, 16, 128, 64, 32)
     assert need > 256
     pos = (ctypes.c_int64 * 4)(10, 20, 30, 40)
     assert lib.csa_decode(fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, pos, 4, 1024, 64, 128, 16, 128,
-                          4, 64, 32, ctypes.c_float(0.1), fake, None, None, None, ws, 256, None) == -5
+                          4, 64, 32, ctypes.c_float(0.1), fake, 0, None, None, None, ws, 256, None) == -5
 
 
 def test_zero_sized_calls_are_no_ops(lib):
@@ -117,3 +125,8 @@ def test_decode_workspace_follows_the_split_rule(lib, B, Ncap, k, W):
     H, d = 64, 128
     got = lib.csa_decode_workspace_bytes(B, Ncap, H, d, 16, 128, k, W)
     assert got == _decode_workspace(B, Ncap, H, d, k, W)
+
+
+def test_debug_inject_rejects_unknown_codes(lib):
+    assert lib.csa_debug_inject(99) == -1
+    assert lib.csa_debug_inject(0) == 0

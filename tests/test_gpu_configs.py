@@ -68,6 +68,11 @@ def test_csa_prefill_full_size_sampled(csa):
         O_want[i], lse_want[i] = o[0], l[0]
     assert_attention_close(O[torch.from_numpy(rows).cuda()], O_want, "CSA prefill attention (sampled rows)")
     np.testing.assert_allclose(lse[torch.from_numpy(rows).cuda()].cpu().numpy(), lse_want, atol=2e-3)
+    # the same call with an fp32 output: no bf16 rounding of the result
+    O32, _, ws = csa.csa_sparse_attn(g["Q"], from_words(Kcw, "cuda"), from_words(Vcw, "cuda"), sel_all, g["K"],
+                                     g["V"], wl.W, scale, out_dtype=torch.float32, want_lse=False)
+    assert csa.csa_check_status(ws) == 0
+    assert_attention_close(O32[torch.from_numpy(rows).cuda()], O_want, "CSA prefill attention (sampled rows)")
 
 
 def test_hca_prefill_full_size_sampled(csa):
@@ -93,6 +98,10 @@ def test_hca_prefill_full_size_sampled(csa):
         O_want[i], lse_want[i] = o[0], l[0]
     assert_attention_close(O[torch.from_numpy(rows).cuda()], O_want, "HCA prefill attention (sampled rows)")
     np.testing.assert_allclose(lse[torch.from_numpy(rows).cuda()].cpu().numpy(), lse_want, atol=2e-3)
+    O32, _, ws = csa.hca_attn(g["Q"], from_words(Kcw, "cuda"), from_words(Vcw, "cuda"), g["K"], g["V"], wl.m_hca,
+                              wl.W_hca, scale, out_dtype=torch.float32, want_lse=False)
+    assert csa.csa_check_status(ws) == 0
+    assert_attention_close(O32[torch.from_numpy(rows).cuda()], O_want, "HCA prefill attention (sampled rows)")
 
 
 def test_csa_decode_1m_context_sampled_sequences(csa):
@@ -104,6 +113,11 @@ def test_csa_decode_1m_context_sampled_sequences(csa):
                                              g["kI_codes"], g["kI_scales"], g["Kwin"], g["Vwin"], pos, wl.m, wl.k,
                                              scale)
     assert csa.csa_check_status(ws) == 0
+    O32, _, idx32, _, ws = csa.csa_decode(g["q"], g["qI_codes"], g["qI_scales"], g["w_codes"], g["Kc"], g["Vc"],
+                                          g["kI_codes"], g["kI_scales"], g["Kwin"], g["Vwin"], pos, wl.m, wl.k,
+                                          scale, out_dtype=torch.float32, want_lse=False)
+    assert csa.csa_check_status(ws) == 0
+    assert torch.equal(idx32, idx)
     for b in (0, 9):
         t = pos[b]
         I = oracle.indexer(g["qI_codes"][b:b + 1].cpu(), g["qI_scales"][b:b + 1].cpu(), g["w_codes"][b:b + 1].cpu(),
@@ -114,4 +128,5 @@ def test_csa_decode_1m_context_sampled_sequences(csa):
                                 g["Vwin"][b].cpu(), t, wl.m, wl.W, scale, sel=want_idx, rows=[0],
                                 raw_pos0=t - wl.W + 1)
         assert_attention_close(O[b:b + 1], o, "decode attention seq %d" % b)
+        assert_attention_close(O32[b:b + 1], o, "decode attention seq %d" % b)
         np.testing.assert_allclose(lse[b:b + 1].cpu().numpy(), l, atol=2e-3)

@@ -259,3 +259,70 @@ def test_compress_edges(csa, T, d, m):
     assert Kc.shape[0] == T // m
     assert_within_bf16_ulp(Kc, Kx, "Kc", fp32_pool_slack(K, m))
     assert_within_bf16_ulp(Vc, Vx, "Vc", fp32_pool_slack(V, m))
+
+
+def test_hca_attention_many_visible_entries(csa):
+    """A dense block over ~12.5K visible entries (98 key tiles of 128): dense
+    tiles are generated from their index, so no tile list bounds the count."""
+    T, t0, H, d, m, W = 64, 200000, 64, 128, 16, 128
+    Nc = (t0 + T) // m
+    Q, Kc, Vc = _attn_inputs(T, H, d, Nc, seed=77)
+    Kraw, Vraw = _raw_kv(t0 + T, d, seed=78)
+    scale = 1.0 / math.sqrt(d)
+    O, lse, ws = csa.hca_attn(Q.cuda(), Kc.cuda(), Vc.cuda(), Kraw.cuda(), Vraw.cuda(), m, W, scale, t0=t0,
+                              out_dtype=torch.float32)
+    assert csa.csa_check_status(ws) == 0
+    O_want, lse_want = oracle.attention(Q, Kc, Vc, Kraw, Vraw, t0, m, W, scale)
+    assert_attention_close(O, O_want, "HCA over %d entries" % Nc)
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_want, atol=2e-3)
+
+
+def test_large_outputs_need_the_fp32_output(csa):
+    """A peaked softmax (queries scaled by 10) over V ~ N(0, 1.25^2) gives |O| of 4
+    and more: there one bf16 half-ulp (2^-6) alone is above the 1e-2 bound, so
+    the fp32 output is the one held to the tolerance; the bf16 output must be
+    the round-to-nearest-even of that same fp32 result.  (V much wider than the
+    workloads' N(0,1) would not do: the bf16 rounding of the softmax weights
+    before the PV product, 2^-9 relative, then exceeds the bound by itself.)"""
+    T, t0, H, d, m, k, W = 256, 0, 64, 128, 4, 64, 128
+    Nc = (t0 + T) // m
+    Q, Kc, Vc = _attn_inputs(T, H, d, Nc, seed=91)
+    Kraw, Vraw = _raw_kv(t0 + T, d, seed=92)
+    Q = (Q.float() * 10).to(torch.bfloat16)
+    Vc = (Vc.float() * 1.25).to(torch.bfloat16)
+    Vraw = (Vraw.float() * 1.25).to(torch.bfloat16)
+    rng = np.random.default_rng(93)
+    sel = np.full((T, k), -1, np.int32)
+    for r in range(T):
+        nv = (t0 + r + 1) // m
+        c = rng.choice(nv, size=min(k, nv), replace=False) if nv else []
+        sel[r, : len(c)] = c
+    scale = 1.0 / math.sqrt(d)
+    O_want, _ = oracle.attention(Q, Kc, Vc, Kraw, Vraw, t0, m, W, scale, sel=sel)
+    assert np.abs(O_want).max() >= 4.0
+    O32, _, ws = csa.csa_sparse_attn(Q.cuda(), Kc.cuda(), Vc.cuda(), torch.from_numpy(sel).cuda(), Kraw.cuda(),
+                                     Vraw.cuda(), W, scale, t0=t0, out_dtype=torch.float32)
+    assert csa.csa_check_status(ws) == 0
+    assert_attention_close(O32, O_want, "sparse attention, peaked softmax, |O| >= 4")
+    O16, _, ws = csa.csa_sparse_attn(Q.cuda(), Kc.cuda(), Vc.cuda(), torch.from_numpy(sel).cuda(), Kraw.cuda(),
+                                     Vraw.cuda(), W, scale, t0=t0, out_dtype=torch.bfloat16)
+    assert torch.equal(O16, O32.to(torch.bfloat16))
+
+
+def test_hca_decode_fp32_output(csa):
+    wl = inputs.Workload("hdec32", H=64, d=128, m=128, W=128, batch=2, context=1 << 18, seed=29)
+    n = wl.context // wl.m
+    gen = torch.Generator().manual_seed(29)
+    f = lambda *s: torch.randn(*s, generator=gen).to(torch.bfloat16)
+    q, Kc, Vc = f(wl.batch, wl.H, wl.d), f(wl.batch, n, wl.d), f(wl.batch, n, wl.d)
+    Kw, Vw = f(wl.batch, wl.W, wl.d), f(wl.batch, wl.W, wl.d)
+    pos = [wl.context - 1, 70000]
+    scale = 1.0 / math.sqrt(wl.d)
+    O, lse, ws = csa.hca_decode(q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), pos, wl.m, scale,
+                                out_dtype=torch.float32)
+    assert csa.csa_check_status(ws) == 0
+    assert O.dtype == torch.float32
+    for b, t in enumerate(pos):
+        o, l = oracle.attention(q[b:b + 1], Kc[b], Vc[b], Kw[b], Vw[b], t, wl.m, wl.W, scale, rows=[0],
+                                raw_pos0=t - wl.W + 1)
+        assert_attention_close(O[b:b + 1], o, "HCA decode fp32 seq %d" % b)

@@ -14,7 +14,7 @@ import torch
 import oracle
 from long_context_compressed_gated_b200 import inputs
 from long_context_compressed_gated_b200.stack import stack_inputs, stack_prefill_chunked
-from tests.parity import assert_attention_close, from_words, sample_rows
+from tests.parity import assert_attention_close, assert_topk_exact, from_words, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -86,13 +86,41 @@ def test_small_stack_against_oracle():
     assert_attention_close(torch.cat(got), O2x, "stack layer 2 per layer (sampled rows)")
 
 
+def _stack_indexer_rows(wl):
+    """Rows of the full stack whose layer-1 selection is checked bit for bit: in
+    every chunk its first row, the rows either side of the chunk start, its last
+    row and two seeded rows; the rows where the visible count crosses k; T-1."""
+    rows = {wl.k * wl.m - 2, wl.k * wl.m - 1, wl.k * wl.m, wl.k * wl.m + wl.m, wl.T - 1}
+    rng = np.random.default_rng(404)
+    for c in range(wl.T // wl.chunk):
+        s0 = c * wl.chunk
+        rows.update({s0, s0 + 1, s0 - 1, s0 + wl.chunk - 1})
+        rows.update(int(x) for x in rng.integers(s0, s0 + wl.chunk, size=2))
+    return np.array(sorted(r for r in rows if 0 <= r < wl.T), dtype=np.int64)
+
+
 def test_full_size_stack_sampled():
     """The T=262144 stack in 16384-token chunks (64 x 128, CSA m=4 k=1024, HCA
-    m'=128, indexer 16 x 128), oracle on sampled rows from several chunks."""
+    m'=128, indexer 16 x 128).  The layer-1 indexer scores and top-k indices of
+    the chunked calls are compared bit for bit with the oracle on rows of every
+    chunk (up to 65536 visible entries); the attention outputs on sampled rows."""
     wl = inputs.STACK
     l1, l2, P = stack_inputs(wl, device="cuda")
-    O2, O1 = stack_prefill_chunked(l1, l2, P, wl.chunk, wl.m, wl.k, wl.W, wl.m_hca, wl.W_hca, return_o1=True)
+    idx_all = torch.empty(wl.T, wl.k, dtype=torch.int32, device="cuda")
+    sc_all = torch.empty(wl.T, wl.k, dtype=torch.float32, device="cuda")
+    O2, O1 = stack_prefill_chunked(l1, l2, P, wl.chunk, wl.m, wl.k, wl.W, wl.m_hca, wl.W_hca, return_o1=True,
+                                   idx_out=idx_all, scores_out=sc_all)
     torch.cuda.synchronize()
+    irows = _stack_indexer_rows(wl)
+    hI = {k: l1[k].cpu() for k in ("qI_codes", "qI_scales", "w_codes", "kI_codes", "kI_scales")}
+    I = oracle.indexer(hI["qI_codes"], hI["qI_scales"], hI["w_codes"], hI["kI_codes"], hI["kI_scales"], 0, wl.m,
+                       irows)
+    want_idx, want_top = oracle.topk(I, oracle.n_vis(irows, wl.m), wl.k)
+    del I
+    sel = torch.from_numpy(irows).cuda()
+    assert_topk_exact(idx_all[sel], sc_all[sel], want_idx, want_top,
+                      "stack layer-1 indexer, %d rows of all %d chunks" % (len(irows), wl.T // wl.chunk))
+    del idx_all, sc_all
     rows = np.array([0, 4095, 16383, 16384, 16385, 70000, 131071, 200000, wl.T - 1], dtype=np.int64)
     h1 = {k: v.cpu() for k, v in l1.items() if k != "Q"}
     h1["Q"] = l1["Q"][torch.from_numpy(rows).cuda()].cpu()

@@ -57,7 +57,8 @@ def test_indexer_topk_exact(lib, data):
     assert_topk_exact(idx, scores, want_idx, want_top, "tiny indexer")
 
 
-def test_sparse_attention_against_oracle(lib, data):
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_sparse_attention_against_oracle(lib, data, out_dtype):
     scale = 1.0 / math.sqrt(WL.d)
     Kc64, Vc64 = oracle.compress(data["K"], data["V"], data["Z"], data["B"], WL.m)
     Kcw, Vcw = oracle.to_bf16_words(Kc64), oracle.to_bf16_words(Vc64)
@@ -67,21 +68,24 @@ def test_sparse_attention_against_oracle(lib, data):
     O_want, lse_want = oracle.attention(data["Q"], Kcw, Vcw, data["K"], data["V"], 0, WL.m, WL.W, scale, sel=sel)
     g = _cuda(data)
     O, lse, ws = lib.csa_sparse_attn(g["Q"], from_words(Kcw, "cuda"), from_words(Vcw, "cuda"),
-                                     torch.from_numpy(sel).cuda(), g["K"], g["V"], WL.W, scale)
+                                     torch.from_numpy(sel).cuda(), g["K"], g["V"], WL.W, scale, out_dtype=out_dtype)
     assert lib.csa_check_status(ws) == 0
+    assert O.dtype == out_dtype
     assert_attention_close(O, O_want, "tiny CSA attention")
     np.testing.assert_allclose(lse.cpu().numpy(), lse_want, atol=2e-3)
 
 
-def test_hca_attention_against_oracle(lib, data):
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_hca_attention_against_oracle(lib, data, out_dtype):
     scale = 1.0 / math.sqrt(WL.d)
     Kc64, Vc64 = oracle.compress(data["K"], data["V"], data["Z"], data["B_hca"], WL.m_hca)
     Kcw, Vcw = oracle.to_bf16_words(Kc64), oracle.to_bf16_words(Vc64)
     O_want, lse_want = oracle.attention(data["Q"], Kcw, Vcw, data["K"], data["V"], 0, WL.m_hca, WL.W_hca, scale)
     g = _cuda(data)
     O, lse, ws = lib.hca_attn(g["Q"], from_words(Kcw, "cuda"), from_words(Vcw, "cuda"), g["K"], g["V"], WL.m_hca,
-                              WL.W_hca, scale)
+                              WL.W_hca, scale, out_dtype=out_dtype)
     assert lib.csa_check_status(ws) == 0
+    assert O.dtype == out_dtype
     assert_attention_close(O, O_want, "tiny HCA attention")
     np.testing.assert_allclose(lse.cpu().numpy(), lse_want, atol=2e-3)
 

@@ -1,10 +1,11 @@
 """csa_decode_noalloc: the decode entry point for callers that cannot allocate
-device memory (graph capture, allocator-free serving loops, embedders that own
-every buffer).  It keeps its scratch in a static device array inside the
-library.  Checked through the C ABI against csa_decode with a caller workspace,
-on two calls in a row (the shared scratch keeps the previous call's contents).
-This file sorts last so that a run stopping at the first failure has already
-run every other test."""
+device memory (serving loops that forbid allocator calls once running,
+embedders that own every buffer).  It keeps its scratch in a static device
+array inside the library.  Checked through the C ABI against csa_decode with a
+caller workspace, on two calls in a row (the shared scratch keeps the previous
+call's contents), and checked to leave torch's allocator untouched.  This file
+sorts last so that a run stopping at the first failure has already run every
+other test."""
 import ctypes
 import math
 
@@ -52,12 +53,15 @@ def test_noalloc_matches_workspace_decode_twice():
         idx = torch.full_like(idx_ref, -7)
         sc = torch.full_like(sc_ref, float("nan"))
         status = torch.full((1,), 12345, dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+        allocated = torch.cuda.memory_allocated()
         rc = L.csa_decode_noalloc(_p(g["q"]), _p(g["qI_codes"]), _p(g["qI_scales"]), _p(g["w_codes"]), _p(g["Kc"]),
                                   _p(g["Vc"]), _p(g["kI_codes"]), _p(g["kI_scales"]), _p(g["Kwin"]), _p(g["Vwin"]),
                                   posa, B, g["Kc"].shape[1], H, d, wl.HI, wl.dI, wl.m, wl.k, wl.W, scale, _p(O),
                                   _p(lse), _p(idx), _p(sc), _p(status), stream)
         assert rc == 0, csa.csa_status_string(rc)
         torch.cuda.synchronize()
+        assert torch.cuda.memory_allocated() == allocated  # nothing went through torch's allocator
         assert int(status.item()) == 0
         np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref.cpu().numpy())
         np.testing.assert_array_equal(sc.cpu().numpy(), sc_ref.cpu().numpy())
@@ -65,14 +69,16 @@ def test_noalloc_matches_workspace_decode_twice():
         np.testing.assert_allclose(lse.cpu().numpy(), lse_ref.cpu().numpy(), atol=2e-3)
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+@pytest.mark.parametrize("B,H,k", [
+    (1024, 64, 2048),  # many sequences with a large k
+    (16, 128, 1024),   # 128 heads: the split attention partials alone exceed the scratch
+])
+def test_noalloc_rejects_problems_beyond_its_scratch(B, H, k):
     csa, L = _lib()
-    # B = 1024 sequences with k = 2048 need more than the 8 MiB static scratch
-    B = 1024
-    need = csa.lib().csa_decode_workspace_bytes(B, 1 << 20, 64, 128, 16, 128, 2048, 128)
+    need = csa.lib().csa_decode_workspace_bytes(B, 1 << 18, H, 128, 16, 128, k, 128)
     assert need > (8 << 20)
     fake = ctypes.c_void_p(0x1000)
-    posa = (ctypes.c_int64 * B)(*([(1 << 22) - 1] * B))
-    rc = L.csa_decode_noalloc(fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, posa, B, 1 << 20, 64,
-                              128, 16, 128, 4, 2048, 128, 0.088, fake, None, None, None, None, None)
+    posa = (ctypes.c_int64 * B)(*([(1 << 20) - 1] * B))
+    rc = L.csa_decode_noalloc(fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, posa, B, 1 << 18, H,
+                              128, 16, 128, 4, k, 128, 0.088, fake, None, None, None, None, None)
     assert rc == -5  # CSA_ERR_WORKSPACE
