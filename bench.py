@@ -336,7 +336,7 @@ def run_csa_prefill(csa, wl, steps, warmup, dist_on, rank):
     e2e_ms = e0.elapsed_time(e1) / n_e2e
     del dev, host
     return {"ms": ms, "phases": phases, "status": status, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launches_per_step": 4,  # compress, indexer, top-k finalize, attention
+            "launches_per_step": 3,  # compress, indexer (selection sorted in the kernel), attention
             "e2e_chunks": n_chunks, "e2e_matches": e2e_matches}
 
 
@@ -432,6 +432,37 @@ def run_stack(csa, wl, steps, warmup):
     for name, e0, e1 in events:
         phases[name] = phases.get(name, 0.0) + e0.elapsed_time(e1) / steps
     return {"ms": t0.elapsed_time(t1) / steps, "phases": phases}
+
+
+class _OneRank:
+    """The all-gather of a single rank (no process group)."""
+    rank, world = 0, 1
+
+    def all_gather(self, flat):
+        return [flat]
+
+
+def run_sharded_stack(csa, wl, steps, warmup, dist_on, rank, world):
+    """The two-layer stack of ONE sequence token-sharded over the ranks (zig-zag
+    chunks, one all-gather of compressed entries + halos per layer): strong
+    scaling, the job's time is its slowest rank's."""
+    from long_context_compressed_gated_b200.sharded import ShardedPrefill, TorchComm, shard_inputs
+    from long_context_compressed_gated_b200.stack import stack_inputs
+    l1, l2, P = stack_inputs(wl, device="cuda")
+    sp = ShardedPrefill(wl.T, world, wl.m, wl.k, wl.W, wl.m_hca, wl.W_hca)
+    x = shard_inputs(l1, l2, P, rank, world, wl.T, wl.m)
+    comm = TorchComm() if dist_on else _OneRank()
+    for _ in range(warmup):
+        sp.run(x, comm)
+    barrier(dist_on)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        sp.run(x, comm)
+    t1.record()
+    barrier(dist_on)
+    return max_over_ranks(t0.elapsed_time(t1) / steps, dist_on)
 
 
 # ----------------------------------------------------------------- CPU oracle (reference arm / baseline)
@@ -612,7 +643,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the HCA and decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default="all", choices=("all", "csa_prefill", "peaks") + EXTRA_CASES,
+    ap.add_argument("--case", default="all", choices=("all", "csa_prefill", "peaks", "sharded_stack") + EXTRA_CASES,
                     help="all: the CSA prefill line plus the other workloads; csa_prefill: that line alone; "
                          "otherwise one other workload alone, on one GPU (for profiling)")
     ap.add_argument("--T", type=int, default=None,
@@ -684,6 +715,18 @@ def main():
     peaks["mxf4_tflops"] = tensor_peaks["mxf4"]["burst_tflops"]
     peaks["mxf4_source"] = "measured: csa_peak_mma loop, best of 10"
     peaks["bf16_mma_loop_tflops"] = tensor_peaks["bf16"]["burst_tflops"]
+    if args.case == "sharded_stack":
+        wls = inputs.STACK if args.T is None else __import__("dataclasses").replace(inputs.STACK, T=args.T)
+        ms = run_sharded_stack(csa, wls, args.steps, args.warmup, dist_on, rank, world)
+        if rank == 0:
+            print(json.dumps({"case": "sharded_stack", "metric": METRIC, "value": wls.T / (ms * 1e-3),
+                              "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": ms, "scaling": "strong",
+                              "config": {"workload": wls.name, "T": wls.T, "parallelism": "token-sharded zig-zag, "
+                                         "one all-gather of compressed entries + halos per layer"}}), flush=True)
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return
     if args.case in EXTRA_CASES:
         if rank == 0:
             print(json.dumps({"case": args.case, "workloads": run_extra(args.case, csa, peaks, args.steps,

@@ -148,6 +148,17 @@ enum { CSA_MX_OCP = 0, CSA_MX_INDEXER = 1 };
 int csa_mxfp4_quantize(const void* x, int64_t rows, int n, int mode, uint8_t* codes, uint8_t* scales,
                        csa_stream_t stream);
 
+/* MXFP8 for the compressed K/V cache (ferris-liu.github.io ... deepseek-v4,
+ * engineering layer: the KV cache mixes BF16 and FP8 storage; read here as the
+ * compressed entries in FP8 and the raw window in BF16).  For every block of 32
+ * consecutive elements of a row of x [rows, n] bf16: X = floor(log2 max|x|) - 8
+ * (an all-zero block: -127), clamped to [-127, 127]; scales[r, b] = X + 127
+ * (E8M0); codes[r, i] = E4M3 (OCP: bias 7, no infinity) nearest to x / 2^X, ties
+ * to even, saturating at +-448, sign kept.  An Inf/NaN block gets scale 255 and
+ * zero codes.  codes [rows, n] u8, scales [rows, n/32] u8; n % 32 == 0.  Every
+ * code times its scale is exactly a bf16 value (4 significant bits). */
+int csa_mxfp8_quantize(const void* x, int64_t rows, int n, uint8_t* codes, uint8_t* scales, csa_stream_t stream);
+
 /* ---------------------------------------------------------------- indexer + top-k
  * Lightning indexer on MXFP4 fused with the causal top-k (ifanr repost,
  * attention section; blog.nickys.cn/?p=150 "1. CSA").
@@ -220,11 +231,58 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
                int W, float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
                size_t workspace_bytes, csa_stream_t stream);
 
+/* csa_decode over a compressed cache stored in MXFP8 (ferris-liu.github.io ...
+ * deepseek-v4, engineering layer: the KV cache mixes BF16 and FP8 storage; here
+ * the compressed entries are FP8 and the window BF16).  Kc_codes / Vc_codes
+ * [B, Ncap, d] E4M3 bytes and Kc_scales / Vc_scales [B, Ncap, d/32] E8M0 bytes,
+ * as csa_mxfp8_quantize writes them; every other argument as csa_decode.  The
+ * selected entries are dequantised exactly to bf16 as they are gathered, so the
+ * result equals csa_decode over the dequantised cache bit for bit; the gathered
+ * bytes halve.  Workspace: csa_decode_workspace_bytes(). */
+int csa_decode_fp8(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                   const uint8_t* Kc_codes, const uint8_t* Kc_scales, const uint8_t* Vc_codes, const uint8_t* Vc_scales,
+                   const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin, const void* Vwin,
+                   const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k, int W,
+                   float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
+                   size_t workspace_bytes, csa_stream_t stream);
+
 /* HCA decode: dense over every visible cached entry plus the window. */
 size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W);
 int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,
                int B, int64_t Ncap, int H, int d, int m, int W, float scale, void* O, int o_dtype, float* lse,
                void* workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------- decode cache maintenance
+ * One new token per sequence enters the decode state that csa_decode /
+ * hca_decode read (blog.nickys.cn/?p=150 "1. CSA" / "2. HCA": every m tokens
+ * become one compressed entry, and the sliding window keeps the latest raw
+ * tokens; ferris-liu.github.io ... deepseek-v4 section 3: the compressed cache
+ * of a 1M-token context).  For sequence b, the token at absolute position
+ * pos[b] (host array) with raw K_new[b], V_new[b] and gate logits Z_new[b]
+ * ([B, d] bf16 each):
+ *   - the window Kwin/Vwin [B, W, d] (newest last) moves up one row and the
+ *     token becomes row W-1, so after the call it holds pos-W+1 .. pos;
+ *   - if the token ends a block ((pos+1) % m == 0), entry j = (pos+1)/m - 1 of
+ *     Kc/Vc [B, Ncap, d] is written by the gated pooling of the block's m
+ *     tokens with bias Bias [m, d] f32 -- bit for bit the entry csa_compress
+ *     computes from the same tokens -- and the caller's indexer key of that
+ *     entry, kI_codes_new [B, dI/2] / kI_scales_new [B, dI/32], is copied to
+ *     kI_codes [B, Ncap, dI/2] / kI_scales [B, Ncap, dI/32] (how an entry's
+ *     indexer key is derived from its tokens is not on the pages);
+ *   - otherwise the token's K/V/Z are staged in slot pos % m of Kblk/Vblk/Zblk
+ *     [B, m, d] bf16 (the caller's buffers; a block's earlier tokens must have
+ *     been appended by earlier calls, or staged by the caller).
+ * Call it before csa_decode for the same position.  The four kI pointers are
+ * all given or all NULL (hca_decode_append passes NULL).  A sequence whose
+ * block completes at j >= Ncap is CSA_ERR_INVALID_ARG.  d in {64, 128};
+ * m <= 4096 with m <= 8 or m % 8 == 0; 0 <= W <= 1024.  No workspace. */
+int csa_decode_append(const void* K_new, const void* V_new, const void* Z_new, const float* Bias,
+                      const uint8_t* kI_codes_new, const uint8_t* kI_scales_new, const int64_t* pos, int B,
+                      int64_t Ncap, int d, int dI, int m, int W, void* Kwin, void* Vwin, void* Kblk, void* Vblk,
+                      void* Zblk, void* Kc, void* Vc, uint8_t* kI_codes, uint8_t* kI_scales, csa_stream_t stream);
+int hca_decode_append(const void* K_new, const void* V_new, const void* Z_new, const float* Bias, const int64_t* pos,
+                      int B, int64_t Ncap, int d, int m, int W, void* Kwin, void* Vwin, void* Kblk, void* Vblk,
+                      void* Zblk, void* Kc, void* Vc, csa_stream_t stream);
 
 /* ---------------------------------------------------------------- decode without allocation
  * csa_decode for callers that cannot allocate device memory: serving loops

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "CsaError", "lib", "csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode",
-    "hca_decode", "csa_check_status", "csa_status_string", "csa_version", "LIB_PATH",
+    "hca_decode", "csa_check_status", "csa_status_string", "csa_version", "LIB_PATH", "csa_decode_append",
+    "hca_decode_append", "csa_mxfp4_quantize", "csa_mxfp8_quantize", "csa_decode_fp8", "csa_peak_mma",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
@@ -44,7 +45,10 @@ def lib():
             "csa_version": ([], I),
             "csa_check_status": ([P, P], I),
             "csa_debug_inject": ([I], I),
+            "csa_decode_append": ([P, P, P, P, P, P, P, I, I64, I, I, I, I, P, P, P, P, P, P, P, P, P, P], I),
+            "hca_decode_append": ([P, P, P, P, P, I, I64, I, I, I, P, P, P, P, P, P, P, P], I),
             "csa_mxfp4_quantize": ([P, I64, I, I, P, P, P], I),
+            "csa_mxfp8_quantize": ([P, I64, I, P, P, P], I),
             "csa_peak_mma": ([I, I64, I, P, SZ, P, P], I),
             "csa_compress": ([P, P, P, P, I64, I, I, P, P, P], I),
             "csa_indexer_topk_workspace_bytes": ([I64, I64, I, I, I], SZ),
@@ -56,6 +60,8 @@ def lib():
             "csa_decode_workspace_bytes": ([I, I64, I, I, I, I, I, I], SZ),
             "csa_decode": ([P, P, P, P, P, P, P, P, P, P, P, I, I64, I, I, I, I, I, I, I, F, P, I, P, P, P, P, SZ,
                             P], I),
+            "csa_decode_fp8": ([P, P, P, P, P, P, P, P, P, P, P, P, P, I, I64, I, I, I, I, I, I, I, F, P, I, P, P, P,
+                                P, SZ, P], I),
             "hca_decode_workspace_bytes": ([I, I64, I, I, I], SZ),
             "hca_decode": ([P, P, P, P, P, P, I, I64, I, I, I, I, F, P, I, P, P, SZ, P], I),
         }
@@ -156,6 +162,21 @@ def csa_mxfp4_quantize(x, mode=MX_OCP, codes=None, scales=None):
         _dev(scales, torch.uint8, "scales")
     _check(lib().csa_mxfp4_quantize(_ptr(x), rows, n, int(mode), _ptr(codes), _ptr(scales), _stream()),
            "csa_mxfp4_quantize")
+    return codes, scales
+
+
+def csa_mxfp8_quantize(x, codes=None, scales=None):
+    """bf16 [..., n] (n % 32 == 0) -> MXFP8 (E4M3 codes uint8 [..., n], E8M0 scales
+    uint8 [..., n/32]): the FP8 form of the compressed K/V cache."""
+    _dev(x, torch.bfloat16, "x")
+    n = x.shape[-1]
+    rows = x.numel() // n if n else 0
+    lead = tuple(x.shape[:-1])
+    codes = torch.empty(lead + (n,), dtype=torch.uint8, device=x.device) if codes is None else \
+        _dev(codes, torch.uint8, "codes")
+    scales = torch.empty(lead + (n // 32,), dtype=torch.uint8, device=x.device) if scales is None else \
+        _dev(scales, torch.uint8, "scales")
+    _check(lib().csa_mxfp8_quantize(_ptr(x), rows, n, _ptr(codes), _ptr(scales), _stream()), "csa_mxfp8_quantize")
     return codes, scales
 
 
@@ -263,6 +284,38 @@ def csa_decode(q, qI_codes, qI_scales, w_codes, Kc, Vc, kI_codes, kI_scales, Kwi
     return O, lse, idx, scores, ws
 
 
+def csa_decode_fp8(q, qI_codes, qI_scales, w_codes, Kc_codes, Kc_scales, Vc_codes, Vc_scales, kI_codes, kI_scales,
+                   Kwin, Vwin, pos, m, k, scale, O=None, lse=None, idx=None, scores=None, want_lse=True,
+                   want_sel=True, workspace=None, out_dtype=torch.bfloat16):
+    """csa_decode over an MXFP8 compressed cache: Kc/Vc codes [B,Ncap,d] uint8 (E4M3)
+    and scales [B,Ncap,d/32] uint8 (E8M0).  Returns (O, lse, idx, scores, workspace)."""
+    _dev(q, torch.bfloat16, "q", 3), _dev(qI_codes, torch.uint8, "qI_codes", 3)
+    _dev(qI_scales, torch.uint8, "qI_scales", 3), _dev(w_codes, torch.uint8, "w_codes", 2)
+    for t, n in ((Kc_codes, "Kc_codes"), (Kc_scales, "Kc_scales"), (Vc_codes, "Vc_codes"), (Vc_scales, "Vc_scales"),
+                 (kI_codes, "kI_codes"), (kI_scales, "kI_scales")):
+        _dev(t, torch.uint8, n, 3)
+    _dev(Kwin, torch.bfloat16, "Kwin", 3), _dev(Vwin, torch.bfloat16, "Vwin", 3)
+    B, H, d = q.shape
+    HI, dI = qI_codes.shape[1], qI_codes.shape[2] * 2
+    Ncap = Kc_codes.shape[1]
+    W = Kwin.shape[1]
+    dev = q.device
+    O = _out(O, q, q.shape, out_dtype)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    if want_sel:
+        idx = torch.empty(B, k, dtype=torch.int32, device=dev) if idx is None else idx
+        scores = torch.empty(B, k, dtype=torch.float32, device=dev) if scores is None else scores
+    posa = (ctypes.c_int64 * B)(*[int(p) for p in pos])
+    ws = _workspace(lib().csa_decode_workspace_bytes(B, Ncap, H, d, HI, dI, k, W), dev, workspace)
+    _check(lib().csa_decode_fp8(_ptr(q), _ptr(qI_codes), _ptr(qI_scales), _ptr(w_codes), _ptr(Kc_codes),
+                                _ptr(Kc_scales), _ptr(Vc_codes), _ptr(Vc_scales), _ptr(kI_codes), _ptr(kI_scales),
+                                _ptr(Kwin), _ptr(Vwin), posa, B, Ncap, H, d, HI, dI, m, k, W, float(scale), _ptr(O),
+                                _ODTYPE[out_dtype], _ptr(lse), _ptr(idx), _ptr(scores), _ptr(ws), ws.numel(),
+                                _stream()), "csa_decode_fp8")
+    return O, lse, idx, scores, ws
+
+
 def hca_decode(q, Kc, Vc, Kwin, Vwin, pos, m, scale, O=None, lse=None, want_lse=True, workspace=None,
                out_dtype=torch.bfloat16):
     """HCA decode: one token per sequence, dense over its visible cache + window."""
@@ -280,3 +333,37 @@ def hca_decode(q, Kc, Vc, Kwin, Vwin, pos, m, scale, O=None, lse=None, want_lse=
                             float(scale), _ptr(O), _ODTYPE[out_dtype], _ptr(lse), _ptr(ws), ws.numel(), _stream()),
            "hca_decode")
     return O, lse, ws
+
+
+def csa_decode_append(K_new, V_new, Z_new, B, pos, Kwin, Vwin, Kblk, Vblk, Zblk, Kc, Vc, kI_codes_new=None,
+                      kI_scales_new=None, kI_codes=None, kI_scales=None):
+    """Append one token per sequence to the decode state (window, block staging,
+    and on block completion the compressed entry and its indexer key), in place.
+    K_new/V_new/Z_new [Bseq,d] bf16; B [m,d] f32; pos: host positions of the new
+    tokens; Kwin/Vwin [Bseq,W,d]; Kblk/Vblk/Zblk [Bseq,m,d]; Kc/Vc [Bseq,Ncap,d];
+    kI_* (all or none): the completed entry's MXFP4 key [Bseq,dI/2]/[Bseq,dI/32]
+    and the cache's key tensors [Bseq,Ncap,dI/2]/[Bseq,Ncap,dI/32]."""
+    for t, n in ((K_new, "K_new"), (V_new, "V_new"), (Z_new, "Z_new"), (Kwin, "Kwin"), (Vwin, "Vwin"),
+                 (Kblk, "Kblk"), (Vblk, "Vblk"), (Zblk, "Zblk"), (Kc, "Kc"), (Vc, "Vc")):
+        _dev(t, torch.bfloat16, n)
+    _dev(B, torch.float32, "B", 2)
+    nb, d = K_new.shape
+    m = Kblk.shape[1]
+    W = Kwin.shape[1]
+    Ncap = Kc.shape[1]
+    posa = (ctypes.c_int64 * nb)(*[int(p) for p in pos])
+    dI = 0
+    if kI_codes is not None:
+        for t, n in ((kI_codes_new, "kI_codes_new"), (kI_scales_new, "kI_scales_new"), (kI_codes, "kI_codes"),
+                     (kI_scales, "kI_scales")):
+            _dev(t, torch.uint8, n)
+        dI = kI_codes.shape[-1] * 2
+    _check(lib().csa_decode_append(_ptr(K_new), _ptr(V_new), _ptr(Z_new), _ptr(B), _ptr(kI_codes_new),
+                                   _ptr(kI_scales_new), posa, nb, Ncap, d, dI, m, W, _ptr(Kwin), _ptr(Vwin),
+                                   _ptr(Kblk), _ptr(Vblk), _ptr(Zblk), _ptr(Kc), _ptr(Vc), _ptr(kI_codes),
+                                   _ptr(kI_scales), _stream()), "csa_decode_append")
+
+
+def hca_decode_append(K_new, V_new, Z_new, B, pos, Kwin, Vwin, Kblk, Vblk, Zblk, Kc, Vc):
+    """csa_decode_append without indexer keys (the HCA layer's cache, ratio m')."""
+    csa_decode_append(K_new, V_new, Z_new, B, pos, Kwin, Vwin, Kblk, Vblk, Zblk, Kc, Vc)

@@ -8,6 +8,7 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "compress.cuh"
 
 namespace csa {
 
@@ -24,7 +25,14 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
                                   uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
                                   int* status, cudaStream_t stream);
 int inject_fault(int code);
+cudaError_t launch_decode_append(const void* Kn, const void* Vn, const void* Zn, const float* Bias,
+                                 const uint8_t* kIc_new, const uint8_t* kIs_new, const int64_t* pos, int B,
+                                 int64_t Ncap, int d, int dI, int m, int W, void* Kwin, void* Vwin, void* Kblk,
+                                 void* Vblk, void* Zblk, void* Kc, void* Vc, uint8_t* kIc, uint8_t* kIs,
+                                 cudaStream_t stream);
 cudaError_t launch_mxfp4_quantize(const void* x, int64_t nblocks, int mode, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t stream);
+cudaError_t launch_mxfp8_quantize(const void* x, int64_t nblocks, uint8_t* codes, uint8_t* scales,
                                   cudaStream_t stream);
 cudaError_t launch_peak_mma(int kind, long long iters, int ctas, int* status, cudaStream_t stream);
 double peak_mma_flops(int kind, long long iters, int ctas);
@@ -221,12 +229,18 @@ int csa_mxfp4_quantize(const void* x, int64_t rows, int n, int mode, uint8_t* co
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
-// Indexer workspace: status header, then per query row the k selected keys
-// (uint64) and their count, which the finalize pass sorts into idx / scores.
-size_t csa_indexer_topk_workspace_bytes(int64_t T, int64_t, int, int, int k) {
-  if (T <= 0 || k <= 0) return kWorkspaceHeader;
-  return kWorkspaceHeader + align256((size_t)T * k * 8) + align256((size_t)T * 4);
+int csa_mxfp8_quantize(const void* x, int64_t rows, int n, uint8_t* codes, uint8_t* scales, csa_stream_t stream) {
+  if (rows < 0 || n <= 0 || n % 32 != 0) return CSA_ERR_INVALID_ARG;
+  if (rows == 0) return CSA_OK;
+  int rc = check_ptrs(x, codes, scales);
+  if (rc) return rc;
+  cudaError_t e = launch_mxfp8_quantize(x, rows * (n / 32), codes, scales, (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
+
+// Indexer workspace: the status header only (each CTA selects, sorts and writes
+// its rows' top-k itself).
+size_t csa_indexer_topk_workspace_bytes(int64_t, int64_t, int, int, int) { return kWorkspaceHeader; }
 
 int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
                      const uint8_t* kI_codes, const uint8_t* kI_scales, int64_t T, int64_t t0, int64_t Nc, int HI,
@@ -241,11 +255,8 @@ int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const ui
   if (rc) return rc;
   if (Nc > 0 && (rc = check_ptrs(kI_codes, kI_scales))) return rc;
   if ((rc = check_opt(scores))) return rc;
-  uint8_t* w = static_cast<uint8_t*>(workspace);
-  uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader);
-  int* cand_cnt = reinterpret_cast<int*>(w + kWorkspaceHeader + align256((size_t)T * k * 8));
   cudaError_t e = launch_indexer_prefill(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, T, t0, Nc, HI, dI, m, k,
-                                         idx, scores, cand, cand_cnt, status_word(workspace), (cudaStream_t)stream);
+                                         idx, scores, nullptr, nullptr, status_word(workspace), (cudaStream_t)stream);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
@@ -348,11 +359,13 @@ size_t csa_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int, int, i
          align256((size_t)B * ns * k * 8) + align256((size_t)B * ns * 4) + attn_part_bytes(B, nsa, H, d);
 }
 
-int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
-               const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
-               const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
-               int W, float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
-               size_t workspace_bytes, csa_stream_t stream) {
+static int decode_impl(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                       const void* Kc, const void* Vc, const uint8_t* kc8, const uint8_t* kc8s, const uint8_t* vc8,
+                       const uint8_t* vc8s, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
+                       const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m,
+                       int k, int W, float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores,
+                       void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  const bool fp8 = kc8 != nullptr;
   if (B < 0 || Ncap < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 || !(std::isfinite(scale) && scale > 0.f) ||
       !valid_odtype(o_dtype))
     return CSA_ERR_INVALID_ARG;
@@ -371,7 +384,9 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   }
   rc = check_ptrs(q, qI_codes, qI_scales, w_codes, O);
   if (rc) return rc;
-  if (Ncap > 0 && (rc = check_ptrs(Kc, Vc, kI_codes, kI_scales))) return rc;
+  if (Ncap > 0 && (rc = check_ptrs(kI_codes, kI_scales))) return rc;
+  if (Ncap > 0 && !fp8 && (rc = check_ptrs(Kc, Vc))) return rc;
+  if (Ncap > 0 && fp8 && (rc = check_ptrs(kc8, kc8s, vc8, vc8s))) return rc;
   if (W > 0 && (rc = check_ptrs(Kwin, Vwin))) return rc;
   if ((rc = check_opt(lse)) || (rc = check_opt(idx)) || (rc = check_opt(scores))) return rc;
   const int ns = decode_nsplit(B, Ncap, k);
@@ -398,8 +413,14 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   }
   AttnArgs a{};
   a.Q = static_cast<const __nv_bfloat16*>(q);
-  a.Kc = static_cast<const __nv_bfloat16*>(Ncap > 0 ? Kc : q);
-  a.Vc = static_cast<const __nv_bfloat16*>(Ncap > 0 ? Vc : q);
+  a.Kc = static_cast<const __nv_bfloat16*>(Ncap > 0 && !fp8 ? Kc : q);  // (FP8: the maps are unused)
+  a.Vc = static_cast<const __nv_bfloat16*>(Ncap > 0 && !fp8 ? Vc : q);
+  if (fp8 && Ncap > 0) {
+    a.kc8 = kc8;
+    a.kc8_scales = kc8s;
+    a.vc8 = vc8;
+    a.vc8_scales = vc8s;
+  }
   a.idx = sel;
   a.Kr = static_cast<const __nv_bfloat16*>(W > 0 ? Kwin : q);
   a.Vr = static_cast<const __nv_bfloat16*>(W > 0 ? Vwin : q);
@@ -421,7 +442,7 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
   a.q_rows = (int64_t)B * H;
-  a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
+  a.kc_rows = Ncap > 0 && !fp8 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
   a.nsplit = nsa;
   a.o_part = o_part;
@@ -429,6 +450,66 @@ int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales,
   e = launch_attention(a, d, (unsigned)B, s);
   if (e == cudaSuccess && nsa > 1) e = launch_attention_combine(a, B, d, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+int csa_decode(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+               const void* Kc, const void* Vc, const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin,
+               const void* Vwin, const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k,
+               int W, float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
+               size_t workspace_bytes, csa_stream_t stream) {
+  return decode_impl(q, qI_codes, qI_scales, w_codes, Kc, Vc, nullptr, nullptr, nullptr, nullptr, kI_codes, kI_scales,
+                     Kwin, Vwin, pos, B, Ncap, H, d, HI, dI, m, k, W, scale, O, o_dtype, lse, idx, scores, workspace,
+                     workspace_bytes, stream);
+}
+
+int csa_decode_fp8(const void* q, const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                   const uint8_t* Kc_codes, const uint8_t* Kc_scales, const uint8_t* Vc_codes, const uint8_t* Vc_scales,
+                   const uint8_t* kI_codes, const uint8_t* kI_scales, const void* Kwin, const void* Vwin,
+                   const int64_t* pos, int B, int64_t Ncap, int H, int d, int HI, int dI, int m, int k, int W,
+                   float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
+                   size_t workspace_bytes, csa_stream_t stream) {
+  if (Ncap > 0 && (Kc_codes == nullptr || Kc_scales == nullptr || Vc_codes == nullptr || Vc_scales == nullptr))
+    return CSA_ERR_INVALID_ARG;
+  static const uint8_t kNone = 0;  // marks the MXFP8 path when the cache is empty
+  return decode_impl(q, qI_codes, qI_scales, w_codes, nullptr, nullptr, Kc_codes ? Kc_codes : &kNone, Kc_scales,
+                     Vc_codes, Vc_scales, kI_codes, kI_scales, Kwin, Vwin, pos, B, Ncap, H, d, HI, dI, m, k, W, scale,
+                     O, o_dtype, lse, idx, scores, workspace, workspace_bytes, stream);
+}
+
+int csa_decode_append(const void* K_new, const void* V_new, const void* Z_new, const float* Bias,
+                      const uint8_t* kI_codes_new, const uint8_t* kI_scales_new, const int64_t* pos, int B,
+                      int64_t Ncap, int d, int dI, int m, int W, void* Kwin, void* Vwin, void* Kblk, void* Vblk,
+                      void* Zblk, void* Kc, void* Vc, uint8_t* kI_codes, uint8_t* kI_scales, csa_stream_t stream) {
+  if (B < 0 || Ncap < 0 || m < 1 || m > 4096 || W < 0 || W > 1024) return CSA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int L, S;
+  pool_shape(d, m, &L, &S);
+  if (m % L != 0) return CSA_ERR_UNSUPPORTED_SHAPE;
+  const bool with_ki = kI_codes_new || kI_scales_new || kI_codes || kI_scales;
+  if (with_ki && (dI != 64 && dI != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return CSA_OK;
+  if (pos == nullptr) return CSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0) return CSA_ERR_INVALID_ARG;
+    if ((pos[b] + 1) % m == 0 && (pos[b] + 1) / m > Ncap) return CSA_ERR_INVALID_ARG;  // no slot for the entry
+  }
+  int rc = check_ptrs(K_new, V_new, Z_new, Bias, Kblk, Vblk, Zblk);
+  if (rc) return rc;
+  if (Ncap > 0 && (rc = check_ptrs(Kc, Vc))) return rc;
+  if (W > 0 && (rc = check_ptrs(Kwin, Vwin))) return rc;
+  if (with_ki && (rc = check_ptrs(kI_codes_new, kI_scales_new, kI_codes, kI_scales))) return rc;
+  cudaError_t e = launch_decode_append(K_new, V_new, Z_new, Bias, with_ki ? kI_codes_new : nullptr,
+                                       with_ki ? kI_scales_new : nullptr, pos, B, Ncap, d, dI, m, W, Kwin, Vwin, Kblk,
+                                       Vblk, Zblk, Kc, Vc, with_ki ? kI_codes : nullptr,
+                                       with_ki ? kI_scales : nullptr, (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+int hca_decode_append(const void* K_new, const void* V_new, const void* Z_new, const float* Bias, const int64_t* pos,
+                      int B, int64_t Ncap, int d, int m, int W, void* Kwin, void* Vwin, void* Kblk, void* Vblk,
+                      void* Zblk, void* Kc, void* Vc, csa_stream_t stream) {
+  return csa_decode_append(K_new, V_new, Z_new, Bias, nullptr, nullptr, pos, B, Ncap, d, 0, m, W, Kwin, Vwin, Kblk,
+                           Vblk, Zblk, Kc, Vc, nullptr, nullptr, stream);
 }
 
 size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W) {

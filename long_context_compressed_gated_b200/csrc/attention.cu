@@ -29,6 +29,8 @@
 // PV of tile i still reads V.
 #include <cuda.h>
 
+#include <cuda_fp16.h>
+
 #include "attention.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
@@ -105,6 +107,22 @@ __device__ __forceinline__ float2 scale_sub2(float a, float b, float c, float m)
   float2 r;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(y));
   return r;
+}
+
+// Eight E4M3 codes times the block scale 2^(sbyte-127) as eight bf16 values (exact:
+// an E4M3 value has 4 significant bits and the scale is a power of two).
+__device__ __forceinline__ uint4 dequant_e4m3x8(uint2 c, uint32_t sbyte) {
+  const float s = __uint_as_float(sbyte == 0 ? 0x00400000u : ((sbyte & 0xFFu) << 23));  // 2^(sbyte-127)
+  uint32_t r[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint16_t pair = (uint16_t)(((q < 2 ? c.x : c.y) >> (16 * (q & 1))) & 0xFFFFu);
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+    r[q] = pack_bf16x2(f.x * s, f.y * s);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 }  // namespace
@@ -331,7 +349,27 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
           break;
         }
         armed[which][st] = -1;  // the stage's previous load was consumed
-        if (tl.type == kSeg) {
+        if (tl.type == kSeg && a.kc8 != nullptr) {
+          // MXFP8 entries: 8 codes + their block scale per thread and row, dequantised
+          const int* sel = s_idx + tl.owner * a.k + (int)tl.base;
+          const uint8_t* codes = (which ? a.vc8 : a.kc8) + kc_base * D + c * 8;
+          const uint8_t* scl = (which ? a.vc8_scales : a.kc8_scales) + kc_base * (D / 32) + c / 4;
+          const uint32_t d0 = smem_u32(dst) + dst_lane;
+          for (int x = r0; x < tl.width; x += RSTEP) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (x < tl.valid) {
+              const int j = sel[x];
+              const uint2 cw = __ldg(reinterpret_cast<const uint2*>(codes + (int64_t)j * D));
+              v = dequant_e4m3x8(cw, __ldg(scl + (int64_t)j * (D / 32)));
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d0 + (uint32_t)(x - r0) * 128), "r"(v.x),
+                         "r"(v.y), "r"(v.z), "r"(v.w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();  // generic-proxy stores -> tcgen05 (async proxy) reads
+          mbar_arrive(fullb);
+          if (lt == 0) mbar_arrive(fullb);
+        } else if (tl.type == kSeg) {
           const int* sel = s_idx + tl.owner * a.k + (int)tl.base;
           const __nv_bfloat16* src0 = (which ? Vc : Kc) + c * 8;
           const uint32_t d0 = smem_u32(dst) + dst_lane;

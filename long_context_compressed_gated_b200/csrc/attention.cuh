@@ -32,6 +32,10 @@ struct AttnArgs {
   int nsplit;
   float* o_part;    // [B, nsplit, H, d]
   float* lse_part;  // [B, nsplit, H]
+  // compressed entries in MXFP8 (decode): E4M3 codes [rows, d] and E8M0 scales
+  // [rows, d/32]; when set, the selected rows are dequantised (exactly) into the
+  // bf16 tiles instead of copied from Kc / Vc
+  const uint8_t *kc8, *kc8_scales, *vc8, *vc8_scales;
 };
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);

@@ -138,6 +138,8 @@ struct IndexerArgs {
   int64_t split_tiles;      // 128-key tiles per range
   uint64_t* cand;           // [rows, nsplit, k] selected keys of each key range (unsorted)
   int* cand_cnt;            // [rows, nsplit]    how many of them are valid
+  int32_t* idx;             // prefill (one key range): [rows, k] written directly, sorted
+  float* scores;            // nullable
   int* status;
   int fault;                // test hook (csa_debug_inject): 1 = the producer skips its first stage group
 };
@@ -522,6 +524,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       pbase[t] = 0;
     }
     const uint32_t lt = (1u << lane) - 1u;
+    // keys held in fixed slots (no cut-back yet): the visible ones among the first n of the range
+    auto fixed_count = [&](int64_t nv, int64_t n) -> int {
+      int64_t lim = nv < j_end ? nv : j_end;
+      lim -= j_begin;
+      if (lim > n) lim = n;
+      return lim > 0 ? (int)lim : 0;
+    };
     auto finish_insert = [&]() {
 #pragma unroll
       for (int t = 0; t < G0; ++t) {
@@ -587,7 +596,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int t = 0; t < G0; ++t) {
           pkey[t] = topk::make_key((int32_t)(acc[t] - sumw_magic[t]), (uint32_t)j);
-          pbal[t] = __ballot_sync(0xffffffffu, jin && j < nvis[t] && pkey[t] >= thr[t]);
+          const bool vis = jin && j < nvis[t];
+          if (thr[t] == 0) {
+            // no cut-back yet: every visible key is kept, in its fixed slot (the
+            // visible keys of a tile are a prefix of it, so the slots stay dense)
+            if (vis) s_cand[(size_t)(g_lo + t) * cap + (size_t)it * 128 + quarter * 32 + lane] = pkey[t];
+          } else {
+            pbal[t] = __ballot_sync(0xffffffffu, vis && pkey[t] >= thr[t]);
+          }
         }
         if (lane == 0) {
 #pragma unroll
@@ -600,10 +616,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // back if the next `check` tiles could overflow it
       finish_insert();
       topk::named_sync(gbar, GNT);
+      const int tiles_done = min(ntiles, kAlt ? 2 * (rd + 1) : rd + 1);
       for (int t = 0; t < G0; ++t) {  // every warp of the group cuts back each of its buffers
         const int gg = g_lo + t;
         uint64_t* buf = s_cand + (size_t)gg * cap;
-        const int cnt = s_cnt[gg];
+        const int cnt = thr[t] == 0 ? fixed_count(nvis[t], (int64_t)tiles_done * 128) : s_cnt[gg];
         if (cnt > cap - 128 * a.check) {
           const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, cap - 128 * a.check, false,
                                                          ghist, gscr, gt, gbar);
@@ -626,11 +643,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row0 + gg >= a.rows) break;  // uniform over the group
       const int64_t r = row0 + gg;
       uint64_t* buf = s_cand + (size_t)gg * cap;
-      int cnt = s_cnt[gg];
+      int cnt = thr[t] == 0 ? fixed_count(nvis[t], (int64_t)ntiles * 128) : s_cnt[gg];
       if (cnt > a.k) {
         const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, ghist, gscr,
                                                        gt, gbar);
         cnt = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
+      }
+      if (!kAlt && a.idx != nullptr) {
+        // one key range per row: these are the row's k best; sort them (score
+        // desc, j asc) and write idx / scores directly
+        const int P = topk::next_pow2(a.k) > 128 ? topk::next_pow2(a.k) : 128;
+        for (int q = cnt + gt; q < P; q += GNT) buf[q] = 0;
+        topk::named_sync(gbar, GNT);
+        if constexpr (GNT == 128) {
+          switch (P / 128) {
+            case 1: topk::group_sort_desc<128, 1>(buf, gt, gbar); break;
+            case 2: topk::group_sort_desc<128, 2>(buf, gt, gbar); break;
+            case 4: topk::group_sort_desc<128, 4>(buf, gt, gbar); break;
+            case 8: topk::group_sort_desc<128, 8>(buf, gt, gbar); break;
+            default: topk::group_sort_desc<128, 16>(buf, gt, gbar); break;
+          }
+        }
+        for (int q = gt; q < a.k; q += GNT) {
+          const uint64_t key = buf[q];  // 0: padding (fewer than k visible entries)
+          a.idx[r * a.k + q] = key ? (int32_t)topk::key_index(key) : -1;
+          if (a.scores) a.scores[r * a.k + q] = key ? (float)topk::key_score(key) * (1.0f / 128.0f) : -INFINITY;
+        }
+        topk::named_sync(gbar, GNT);  // the buffer is reused by the next token of the group
+        continue;
       }
       uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
       for (int q = gt; q < cnt; q += GNT) out[q] = buf[q];
@@ -1073,13 +1113,13 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
   a.split_tiles = ceil_div(Nc > 0 ? Nc : 1, 128);
   a.cand = cand;
   a.cand_cnt = cand_cnt;
+  a.idx = idx;  // one key range per row: the indexer sorts and writes the selection itself
+  a.scores = scores;
   a.status = status;
   dim3 grid((unsigned)ceil_div(T, G), 1);
   const uint8_t* kc = Nc > 0 ? k_codes : q_codes;  // any valid mapping when the cache is empty
-  cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, false, q_codes, kc, a, grid, stream)
-                            : dispatch_hi<64>(HI, false, q_codes, kc, a, grid, stream);
-  if (e != cudaSuccess) return e;
-  return launch_finalize(cand, cand_cnt, 1, k, T, idx, scores, nullptr, stream);
+  return DI == 128 ? dispatch_hi<128>(HI, false, q_codes, kc, a, grid, stream)
+                   : dispatch_hi<64>(HI, false, q_codes, kc, a, grid, stream);
 }
 
 // Decode: rows = B sequences, each with its own cache of Ncap entries and position

@@ -74,7 +74,75 @@ __global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const uint4* __rest
   scales[blk] = (uint8_t)(X + 127);
 }
 
+// Two floats -> two E4M3 bytes (round to nearest even, saturating at +-448), a in
+// the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// MXFP8 for the compressed K/V cache: per block of 32 elements X = floor(log2
+// max|x|) - 8 (448 = 1.75 * 2^8 is E4M3's largest value), scale byte X + 127,
+// codes E4M3(x / 2^X).  One thread per block: 64 bytes in, 32 + 1 out.
+__global__ void __launch_bounds__(256) mxfp8_quantize_kernel(const uint4* __restrict__ x, int64_t nblocks,
+                                                             uint4* __restrict__ codes,
+                                                             uint8_t* __restrict__ scales) {
+  const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (blk >= nblocks) return;
+  uint32_t w[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = __ldg(x + blk * 4 + q);
+    w[4 * q] = u.x;
+    w[4 * q + 1] = u.y;
+    w[4 * q + 2] = u.z;
+    w[4 * q + 3] = u.w;
+  }
+  uint32_t amax_bits = 0;
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
+    finite &= (lo < 0x7F80u) & (hi < 0x7F80u);
+    amax_bits = max(amax_bits, max(lo, hi));
+  }
+  if (!finite) {
+    codes[blk * 2] = make_uint4(0u, 0u, 0u, 0u);
+    codes[blk * 2 + 1] = make_uint4(0u, 0u, 0u, 0u);
+    scales[blk] = 255;
+    return;
+  }
+  int X = -127;
+  if (amax_bits != 0) {
+    int e;
+    frexpf(__uint_as_float(amax_bits << 16), &e);
+    X = e - 9;  // floor(log2 amax) - 8
+  }
+  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  uint32_t out[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    // elements 4q .. 4q+3 (words 2q, 2q+1)
+    const float a0 = ldexpf(bf16_lo(w[2 * q]), -X), a1 = ldexpf(bf16_hi(w[2 * q]), -X);
+    const float a2 = ldexpf(bf16_lo(w[2 * q + 1]), -X), a3 = ldexpf(bf16_hi(w[2 * q + 1]), -X);
+    out[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
+  }
+  codes[blk * 2] = make_uint4(out[0], out[1], out[2], out[3]);
+  codes[blk * 2 + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+  scales[blk] = (uint8_t)(X + 127);
+}
+
 }  // namespace
+
+cudaError_t launch_mxfp8_quantize(const void* x, int64_t nblocks, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t stream) {
+  if (nblocks == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)ceil_div(nblocks, 256);
+  mxfp8_quantize_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(x), nblocks,
+                                                  reinterpret_cast<uint4*>(codes), scales);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mxfp4_quantize(const void* x, int64_t nblocks, int mode, uint8_t* codes, uint8_t* scales,
                                   cudaStream_t stream) {

@@ -17,6 +17,8 @@ marshals numpy arrays through ctypes and composes the steps:
                      entries and the raw window [max(0,t-W+1), t]
   mxfp4_quantize  -- bf16 -> MXFP4 by the OCP MX scale rule (E8M0 per 32, E2M1
                      nearest with ties to even, saturating)
+  mxfp8_quantize  -- bf16 -> MXFP8 (E4M3 + E8M0 per 32) for the FP8 compressed
+                     cache; mxfp8_dequantize decodes it
   csa_layer       -- compress, indexer, top-k and attention composed for rows
 Decode is the same steps for one query row at the sequence's position; the
 tests compose it from these functions.
@@ -49,6 +51,9 @@ def lib():
                                        ctypes.c_int, P, P, ctypes.c_long, ctypes.c_long, ctypes.c_long, P,
                                        ctypes.c_long, ctypes.c_double, P, P, ctypes.c_int]
         L.oracle_mxfp4_quantize.argtypes = [P, ctypes.c_long, ctypes.c_int, ctypes.c_int, P, P]
+        L.oracle_mxfp8_quantize.argtypes = [P, ctypes.c_long, ctypes.c_int, P, P]
+        L.oracle_e4m3_value.argtypes = [ctypes.c_int]
+        L.oracle_e4m3_value.restype = ctypes.c_double
         L.oracle_e2m1_value.argtypes = [ctypes.c_int]
         L.oracle_e2m1_value.restype = ctypes.c_double
         L.oracle_e8m0_value.argtypes = [ctypes.c_int]
@@ -204,6 +209,35 @@ def mxfp4_quantize(x, mode=0):
     rc = lib().oracle_mxfp4_quantize(_p(xa), rows, n, mode, _p(codes), _p(scales))
     assert rc == 0
     return codes.reshape(shape[:-1] + (n // 2,)), scales.reshape(shape[:-1] + (n // 32,))
+
+
+def mxfp8_quantize(x):
+    """bf16 [rows, n] -> (E4M3 codes uint8 [rows, n], E8M0 scales uint8 [rows, n/32])
+    by the OCP MX rule: per 32-element block X = floor(log2 max|x|) - 8, codes the
+    E4M3 values nearest to x / 2^X (ties to even, saturating at 448, sign kept)."""
+    xa = _u16(x)
+    shape = xa.shape
+    n = shape[-1]
+    rows = int(np.prod(shape[:-1])) if len(shape) > 1 else 1
+    xa = np.ascontiguousarray(xa.reshape(rows, n))
+    codes = np.zeros((rows, n), np.uint8)
+    scales = np.zeros((rows, n // 32), np.uint8)
+    rc = lib().oracle_mxfp8_quantize(_p(xa), rows, n, _p(codes), _p(scales))
+    assert rc == 0
+    return codes.reshape(shape), scales.reshape(shape[:-1] + (n // 32,))
+
+
+def e4m3_value(code):
+    return lib().oracle_e4m3_value(int(code))
+
+
+def mxfp8_dequantize(codes, scales):
+    """E4M3 codes [..., n] and E8M0 scales [..., n/32] -> float64 values."""
+    c = np.asarray(codes.cpu().numpy() if hasattr(codes, "cpu") else codes)
+    s = np.asarray(scales.cpu().numpy() if hasattr(scales, "cpu") else scales)
+    table = np.array([e4m3_value(i) for i in range(256)])
+    sv = np.array([e8m0_value(b) for b in range(256)])
+    return table[c] * np.repeat(sv[s], 32, axis=-1)
 
 
 def to_bf16_words(x):

@@ -434,3 +434,76 @@ int oracle_mxfp4_quantize(const uint16_t* x, long rows, int n, int mode, uint8_t
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------ MXFP8 (E4M3) cache quantiser
+ * The compressed K/V cache in FP8 (ferris-liu.github.io ... deepseek-v4,
+ * engineering layer: the KV cache mixes BF16 and FP8 storage).  Reading taken:
+ * compressed entries in E4M3 with one E8M0 scale per 32 channels (OCP MX), the
+ * raw window in bf16.  Per block of 32 elements:
+ *   X = floor(log2 max|x|) - 8      (8 = exponent of E4M3's largest value
+ *                                    448 = 1.75 * 2^8), clamped to [-127, 127];
+ *   scale byte = X + 127; code = E4M3 nearest to x / 2^X, ties to the even
+ *   code, magnitudes above 448 saturated to 448, sign kept.
+ * An all-zero block gets X = -127; a block with Inf/NaN gets scale byte 255 and
+ * zero codes.  E4M3 (OCP): sign, 4 exponent bits (bias 7), 3 mantissa bits;
+ * exponent field 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN (never
+ * produced), so the largest magnitude is 1.75 * 2^8.
+ */
+double oracle_e4m3_value(int code) {
+  int s = (code >> 7) & 1, e = (code >> 3) & 15, mbits = code & 7;
+  if (e == 15 && mbits == 7) return NAN;
+  double mag = (e == 0) ? ldexp(mbits / 8.0, -6) : ldexp(1.0 + mbits / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+static int e4m3_round_magnitude(double y) {
+  /* nearest of the 127 finite non-negative E4M3 magnitudes (codes 0..126),
+   * ties to the even code; y above 448 saturates to 448 (code 126) */
+  if (y >= 448.0) return 126;
+  int best = 0;
+  double bestd = fabs(y - oracle_e4m3_value(0));
+  for (int c = 1; c < 127; ++c) {
+    double dd = fabs(y - oracle_e4m3_value(c));
+    if (dd < bestd || (dd == bestd && (c & 1) == 0)) {
+      best = c;
+      bestd = dd;
+    }
+  }
+  return best;
+}
+
+int oracle_mxfp8_quantize(const uint16_t* x, long rows, int n, uint8_t* codes, uint8_t* scales) {
+  if (!x || !codes || !scales || rows < 0 || n <= 0 || n % 32) return -1;
+  for (long r = 0; r < rows; ++r) {
+    for (int b = 0; b < n / 32; ++b) {
+      const uint16_t* blk = x + r * n + b * 32;
+      double amax = 0;
+      int finite = 1;
+      for (int i = 0; i < 32; ++i) {
+        double v = bf16_value(blk[i]);
+        if (!isfinite(v)) finite = 0;
+        else if (fabs(v) > amax) amax = fabs(v);
+      }
+      uint8_t* crow = codes + r * n + b * 32;
+      if (!finite) {
+        scales[r * (n / 32) + b] = 255;
+        memset(crow, 0, 32);
+        continue;
+      }
+      int X = -127;
+      if (amax > 0) {
+        int e;
+        frexp(amax, &e);
+        X = (e - 1) - 8;
+      }
+      if (X < -127) X = -127;
+      if (X > 127) X = 127;
+      scales[r * (n / 32) + b] = (uint8_t)(X + 127);
+      for (int i = 0; i < 32; ++i) {
+        double v = bf16_value(blk[i]);
+        crow[i] = (uint8_t)((signbit(v) ? 0x80 : 0) | e4m3_round_magnitude(fabs(v) / ldexp(1.0, X)));
+      }
+    }
+  }
+  return 0;
+}
