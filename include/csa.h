@@ -246,6 +246,46 @@ int csa_decode_fp8(const void* q, const uint8_t* qI_codes, const uint8_t* qI_sca
                    float scale, void* O, int o_dtype, float* lse, int32_t* idx, float* scores, void* workspace,
                    size_t workspace_bytes, csa_stream_t stream);
 
+/* ---------------------------------------------------------------- split-cache decode
+ * One sequence's compressed cache split over several GPUs by entry ranges (the
+ * decode case of blog.nickys.cn/?p=150 "1. CSA": the indexer's top-k over all
+ * visible entries, then attention over the selection plus the window).  Rank r
+ * holds entries [j_base, j_base + Nloc) of each sequence and runs:
+ *   1. csa_decode_search: its slice's k best as exact 64-bit keys, keys [B, k]
+ *      u64 (score << 32 | ~j, j the GLOBAL entry; 0 = none, after the valid
+ *      ones), over the visible entries j < floor((pos+1)/m);
+ *   2. (all-gather of the keys; every rank then holds [B, L, k])
+ *   3. csa_topk_merge: the exact top-k of the L lists per sequence, in rank
+ *      order (score desc, j asc), idx [B, k] int32 (global, -1 padding),
+ *      scores [B, k] f32 (nullable), keys_out [B, k] (nullable); identical on
+ *      every rank;
+ *   4. csa_decode_attend: attention over the selected entries that lie in its
+ *      slice (others are skipped) plus the window (pass W = 0 except on the
+ *      rank holding the newest tokens), O (o_dtype; pass CSA_F32 for merging)
+ *      and lse [B, H] (required for merging);
+ *   5. (all-gather of O and lse) csa_attn_combine: O = sum_r exp(lse_r - lse) O_r.
+ * Layouts as csa_decode, with Kc/Vc/kI the rank's slice [B, Nloc, .].  The result
+ * equals csa_decode on the whole cache: idx/scores bit for bit, O within the
+ * attention tolerance (fp32 partials merged in a different order).
+ * Workspaces: csa_decode_search_workspace_bytes(B, Nloc, k),
+ * csa_topk_merge_workspace_bytes(B, L), and for csa_decode_attend
+ * csa_decode_workspace_bytes(B, Nloc, H, d, HI, dI, k, W).  1 <= L <= 63 lists,
+ * L <= 16 partials. */
+size_t csa_decode_search_workspace_bytes(int B, int64_t Nloc, int k);
+int csa_decode_search(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                      const uint8_t* kI_codes, const uint8_t* kI_scales, const int64_t* pos, int B, int64_t Nloc,
+                      int64_t j_base, int HI, int dI, int m, int k, uint64_t* keys, void* workspace,
+                      size_t workspace_bytes, csa_stream_t stream);
+size_t csa_topk_merge_workspace_bytes(int B, int L);
+int csa_topk_merge(const uint64_t* keys, int B, int L, int k, int32_t* idx, float* scores, uint64_t* keys_out,
+                   void* workspace, size_t workspace_bytes, csa_stream_t stream);
+int csa_decode_attend(const void* q, const void* Kc, const void* Vc, const int32_t* idx, int64_t j_base,
+                      const void* Kwin, const void* Vwin, const int64_t* pos, int B, int64_t Nloc, int H, int d, int m,
+                      int k, int W, float scale, void* O, int o_dtype, float* lse, void* workspace,
+                      size_t workspace_bytes, csa_stream_t stream);
+int csa_attn_combine(const float* O_parts, const float* lse_parts, int L, int B, int H, int d, void* O, int o_dtype,
+                     float* lse, csa_stream_t stream);
+
 /* HCA decode: dense over every visible cached entry plus the window. */
 size_t hca_decode_workspace_bytes(int B, int64_t Ncap, int H, int d, int W);
 int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, const void* Vwin, const int64_t* pos,

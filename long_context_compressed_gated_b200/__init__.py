@@ -17,6 +17,7 @@ __all__ = [
     "CsaError", "lib", "csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode",
     "hca_decode", "csa_check_status", "csa_status_string", "csa_version", "LIB_PATH", "csa_decode_append",
     "hca_decode_append", "csa_mxfp4_quantize", "csa_mxfp8_quantize", "csa_decode_fp8", "csa_peak_mma",
+    "csa_decode_search", "csa_topk_merge", "csa_decode_attend", "csa_attn_combine",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
@@ -63,6 +64,12 @@ def lib():
             "csa_decode_fp8": ([P, P, P, P, P, P, P, P, P, P, P, P, P, I, I64, I, I, I, I, I, I, I, F, P, I, P, P, P,
                                 P, SZ, P], I),
             "hca_decode_workspace_bytes": ([I, I64, I, I, I], SZ),
+            "csa_decode_search_workspace_bytes": ([I, I64, I], SZ),
+            "csa_decode_search": ([P, P, P, P, P, P, I, I64, I64, I, I, I, I, P, P, SZ, P], I),
+            "csa_topk_merge_workspace_bytes": ([I, I], SZ),
+            "csa_topk_merge": ([P, I, I, I, P, P, P, P, SZ, P], I),
+            "csa_decode_attend": ([P, P, P, P, I64, P, P, P, I, I64, I, I, I, I, I, F, P, I, P, P, SZ, P], I),
+            "csa_attn_combine": ([P, P, I, I, I, I, P, I, P, P], I),
             "hca_decode": ([P, P, P, P, P, P, I, I64, I, I, I, I, F, P, I, P, P, SZ, P], I),
         }
         for name, (args, res) in sig.items():
@@ -367,3 +374,64 @@ def csa_decode_append(K_new, V_new, Z_new, B, pos, Kwin, Vwin, Kblk, Vblk, Zblk,
 def hca_decode_append(K_new, V_new, Z_new, B, pos, Kwin, Vwin, Kblk, Vblk, Zblk, Kc, Vc):
     """csa_decode_append without indexer keys (the HCA layer's cache, ratio m')."""
     csa_decode_append(K_new, V_new, Z_new, B, pos, Kwin, Vwin, Kblk, Vblk, Zblk, Kc, Vc)
+
+
+def csa_decode_search(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, pos, m, k, j_base=0, keys=None,
+                      workspace=None):
+    """The k best entries of a cache slice (global indices j_base + local) as exact
+    uint64 keys [B, k] (torch.int64 storage; 0 = none).  Returns (keys, workspace)."""
+    B, HI, half = qI_codes.shape
+    dI = half * 2
+    Nloc = kI_codes.shape[1]
+    dev = qI_codes.device
+    keys = torch.empty(B, k, dtype=torch.int64, device=dev) if keys is None else _dev(keys, torch.int64, "keys")
+    posa = (ctypes.c_int64 * B)(*[int(p) for p in pos])
+    ws = _workspace(lib().csa_decode_search_workspace_bytes(B, Nloc, k), dev, workspace)
+    _check(lib().csa_decode_search(_ptr(qI_codes), _ptr(qI_scales), _ptr(w_codes), _ptr(kI_codes), _ptr(kI_scales),
+                                   posa, B, Nloc, int(j_base), HI, dI, m, k, _ptr(keys), _ptr(ws), ws.numel(),
+                                   _stream()), "csa_decode_search")
+    return keys, ws
+
+
+def csa_topk_merge(keys, k, idx=None, scores=None, workspace=None):
+    """keys [B, L, k] (int64 storage of the uint64 keys) -> (idx [B,k], scores [B,k])."""
+    _dev(keys, torch.int64, "keys", 3)
+    B, L, kk = keys.shape
+    assert kk == k
+    dev = keys.device
+    idx = torch.empty(B, k, dtype=torch.int32, device=dev) if idx is None else idx
+    scores = torch.empty(B, k, dtype=torch.float32, device=dev) if scores is None else scores
+    ws = _workspace(lib().csa_topk_merge_workspace_bytes(B, L), dev, workspace)
+    _check(lib().csa_topk_merge(_ptr(keys), B, L, k, _ptr(idx), _ptr(scores), None, _ptr(ws), ws.numel(), _stream()),
+           "csa_topk_merge")
+    return idx, scores
+
+
+def csa_decode_attend(q, Kc, Vc, idx, Kwin, Vwin, pos, m, W, scale, j_base=0, O=None, lse=None,
+                      out_dtype=torch.float32, workspace=None):
+    """Attention over the selected entries inside a cache slice [B, Nloc, d] (+ the
+    window when W > 0).  Returns (O, lse) for merging with csa_attn_combine."""
+    B, H, d = q.shape
+    Nloc = Kc.shape[1]
+    k = idx.shape[1]
+    dev = q.device
+    O = _out(O, q, q.shape, out_dtype)
+    lse = torch.empty(B, H, dtype=torch.float32, device=dev) if lse is None else lse
+    posa = (ctypes.c_int64 * B)(*[int(p) for p in pos])
+    ws = _workspace(lib().csa_decode_workspace_bytes(B, Nloc, H, d, 16, 128, k, W), dev, workspace)
+    _check(lib().csa_decode_attend(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(idx), int(j_base), _ptr(Kwin) if W else None,
+                                   _ptr(Vwin) if W else None, posa, B, Nloc, H, d, m, k, W, float(scale), _ptr(O),
+                                   _ODTYPE[out_dtype], _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+           "csa_decode_attend")
+    return O, lse
+
+
+def csa_attn_combine(O_parts, lse_parts, out_dtype=torch.bfloat16, O=None, lse=None):
+    """O_parts [L, B, H, d] f32, lse_parts [L, B, H] f32 -> (O [B, H, d], lse [B, H])."""
+    _dev(O_parts, torch.float32, "O_parts", 4), _dev(lse_parts, torch.float32, "lse_parts", 3)
+    L, B, H, d = O_parts.shape
+    O = _out(O, O_parts, (B, H, d), out_dtype)
+    lse = torch.empty(B, H, dtype=torch.float32, device=O_parts.device) if lse is None else lse
+    _check(lib().csa_attn_combine(_ptr(O_parts), _ptr(lse_parts), L, B, H, d, _ptr(O), _ODTYPE[out_dtype], _ptr(lse),
+                                  _stream()), "csa_attn_combine")
+    return O, lse

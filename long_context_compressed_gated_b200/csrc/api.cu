@@ -23,7 +23,9 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
                                   const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
                                   int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
                                   uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
-                                  int* status, cudaStream_t stream);
+                                  int* status, cudaStream_t stream, int64_t j_base);
+cudaError_t launch_topk_merge(const uint64_t* keys, int rows, int lists, int k, int* cnt, int32_t* idx,
+                              float* scores, uint64_t* keys_out, cudaStream_t stream);
 int inject_fault(int code);
 cudaError_t launch_decode_append(const void* Kn, const void* Vn, const void* Zn, const float* Bias,
                                  const uint8_t* kIc_new, const uint8_t* kIs_new, const int64_t* pos, int B,
@@ -238,9 +240,12 @@ int csa_mxfp8_quantize(const void* x, int64_t rows, int n, uint8_t* codes, uint8
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
-// Indexer workspace: the status header only (each CTA selects, sorts and writes
-// its rows' top-k itself).
-size_t csa_indexer_topk_workspace_bytes(int64_t, int64_t, int, int, int) { return kWorkspaceHeader; }
+// Indexer workspace: status header, then per query row the k selected keys
+// (uint64) and their count, which the finalize pass sorts into idx / scores.
+size_t csa_indexer_topk_workspace_bytes(int64_t T, int64_t, int, int, int k) {
+  if (T <= 0 || k <= 0) return kWorkspaceHeader;
+  return kWorkspaceHeader + align256((size_t)T * k * 8) + align256((size_t)T * 4);
+}
 
 int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
                      const uint8_t* kI_codes, const uint8_t* kI_scales, int64_t T, int64_t t0, int64_t Nc, int HI,
@@ -255,8 +260,11 @@ int csa_indexer_topk(const uint8_t* qI_codes, const uint8_t* qI_scales, const ui
   if (rc) return rc;
   if (Nc > 0 && (rc = check_ptrs(kI_codes, kI_scales))) return rc;
   if ((rc = check_opt(scores))) return rc;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader);
+  int* cand_cnt = reinterpret_cast<int*>(w + kWorkspaceHeader + align256((size_t)T * k * 8));
   cudaError_t e = launch_indexer_prefill(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, T, t0, Nc, HI, dI, m, k,
-                                         idx, scores, nullptr, nullptr, status_word(workspace), (cudaStream_t)stream);
+                                         idx, scores, cand, cand_cnt, status_word(workspace), (cudaStream_t)stream);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
@@ -405,7 +413,7 @@ static int decode_impl(const void* q, const uint8_t* qI_codes, const uint8_t* qI
   int32_t* sel = idx ? idx : idx_ws;
   if (Ncap > 0) {
     e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, nvis_max, Ncap, HI, dI,
-                              m, k, ns, cand, cand_cnt, sel, scores, nullptr, status_word(workspace), s);
+                              m, k, ns, cand, cand_cnt, sel, scores, nullptr, status_word(workspace), s, 0);
     if (e != cudaSuccess) return cuda_fail(e);
   } else {
     e = cudaMemsetAsync(sel, 0xFF, (size_t)B * k * 4, s);
@@ -474,6 +482,144 @@ int csa_decode_fp8(const void* q, const uint8_t* qI_codes, const uint8_t* qI_sca
   return decode_impl(q, qI_codes, qI_scales, w_codes, nullptr, nullptr, Kc_codes ? Kc_codes : &kNone, Kc_scales,
                      Vc_codes, Vc_scales, kI_codes, kI_scales, Kwin, Vwin, pos, B, Ncap, H, d, HI, dI, m, k, W, scale,
                      O, o_dtype, lse, idx, scores, workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------- split-cache decode pieces
+size_t csa_decode_search_workspace_bytes(int B, int64_t Nloc, int k) {
+  if (B <= 0 || k <= 0) return kWorkspaceHeader;
+  const int ns = decode_nsplit(B, Nloc, k);
+  return kWorkspaceHeader + align256((size_t)B * 8) + align256((size_t)B * k * 4) + align256((size_t)B * ns * k * 8) +
+         align256((size_t)B * ns * 4);
+}
+
+int csa_decode_search(const uint8_t* qI_codes, const uint8_t* qI_scales, const uint8_t* w_codes,
+                      const uint8_t* kI_codes, const uint8_t* kI_scales, const int64_t* pos, int B, int64_t Nloc,
+                      int64_t j_base, int HI, int dI, int m, int k, uint64_t* keys, void* workspace,
+                      size_t workspace_bytes, csa_stream_t stream) {
+  if (B < 0 || Nloc < 0 || j_base < 0 || m < 1 || k < 1 || k > 2048) return CSA_ERR_INVALID_ARG;
+  if (!valid_HI(HI) || (dI != 64 && dI != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, csa_decode_search_workspace_bytes(B, Nloc, k));
+  if (rc) return rc;
+  if (B == 0) return CSA_OK;
+  if (pos == nullptr) return CSA_ERR_INVALID_ARG;
+  int64_t nvis_max = 0;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0) return CSA_ERR_INVALID_ARG;
+    int64_t nv = n_visible(pos[b], m) - j_base;
+    if (nv > Nloc) nv = Nloc;
+    if (nv > nvis_max) nvis_max = nv;
+  }
+  rc = check_ptrs(qI_codes, qI_scales, w_codes, keys);
+  if (rc) return rc;
+  if (Nloc > 0 && (rc = check_ptrs(kI_codes, kI_scales))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (Nloc == 0 || nvis_max <= 0) {
+    cudaError_t e = cudaMemsetAsync(keys, 0, (size_t)B * k * 8, s);
+    return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+  }
+  const int ns = decode_nsplit(B, Nloc, k);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int64_t* pos_dev = reinterpret_cast<int64_t*>(w + kWorkspaceHeader);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader + align256((size_t)B * 8) +
+                                               align256((size_t)B * k * 4));
+  int* cand_cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cand) + align256((size_t)B * ns * k * 8));
+  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  if (e == cudaSuccess)
+    e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, nvis_max, Nloc, HI, dI,
+                              m, k, ns, cand, cand_cnt, nullptr, nullptr, keys, status_word(workspace), s, j_base);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+size_t csa_topk_merge_workspace_bytes(int B, int L) {
+  return kWorkspaceHeader + align256((size_t)(B > 0 ? B : 0) * (L > 0 ? L : 0) * 4);
+}
+
+int csa_topk_merge(const uint64_t* keys, int B, int L, int k, int32_t* idx, float* scores, uint64_t* keys_out,
+                   void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  if (B < 0 || L < 1 || L > kMaxKeyRanges || k < 1 || k > 2048) return CSA_ERR_INVALID_ARG;
+  int rc = check_ws(workspace, workspace_bytes, csa_topk_merge_workspace_bytes(B, L));
+  if (rc) return rc;
+  if (B == 0) return CSA_OK;
+  if ((rc = check_ptrs(keys, idx))) return rc;
+  if ((rc = check_opt(scores)) || (rc = check_opt(keys_out))) return rc;
+  int* cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
+  cudaError_t e = launch_topk_merge(keys, B, L, k, cnt, idx, scores, keys_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+int csa_decode_attend(const void* q, const void* Kc, const void* Vc, const int32_t* idx, int64_t j_base,
+                      const void* Kwin, const void* Vwin, const int64_t* pos, int B, int64_t Nloc, int H, int d, int m,
+                      int k, int W, float scale, void* O, int o_dtype, float* lse, void* workspace,
+                      size_t workspace_bytes, csa_stream_t stream) {
+  if (B < 0 || Nloc < 0 || j_base < 0 || m < 1 || k < 1 || k > 2048 || W < 0 || W > 1024 ||
+      !(std::isfinite(scale) && scale > 0.f) || !valid_odtype(o_dtype))
+    return CSA_ERR_INVALID_ARG;
+  if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_ws(workspace, workspace_bytes, csa_decode_workspace_bytes(B, Nloc, H, d, 16, 128, k, W));
+  if (rc) return rc;
+  if (B == 0) return CSA_OK;
+  if (pos == nullptr) return CSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (pos[b] < 0) return CSA_ERR_INVALID_ARG;
+  if ((rc = check_ptrs(q, idx, O))) return rc;
+  if (Nloc > 0 && (rc = check_ptrs(Kc, Vc))) return rc;
+  if (W > 0 && (rc = check_ptrs(Kwin, Vwin))) return rc;
+  if ((rc = check_opt(lse))) return rc;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int64_t* pos_dev = reinterpret_cast<int64_t*>(w + kWorkspaceHeader);
+  const int ns = decode_nsplit(B, Nloc, k);
+  uint8_t* part_base = w + kWorkspaceHeader + align256((size_t)B * 8) + align256((size_t)B * k * 4) +
+                       align256((size_t)B * ns * k * 8) + align256((size_t)B * ns * 4);
+  const int nsa = decode_attn_splits(B, ceil_div(k, 128) + window_tiles(W, 1));
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  AttnArgs a{};
+  a.Q = static_cast<const __nv_bfloat16*>(q);
+  a.Kc = static_cast<const __nv_bfloat16*>(Nloc > 0 ? Kc : q);
+  a.Vc = static_cast<const __nv_bfloat16*>(Nloc > 0 ? Vc : q);
+  a.idx = idx;
+  a.idx_base = j_base;
+  a.Kr = static_cast<const __nv_bfloat16*>(W > 0 ? Kwin : q);
+  a.Vr = static_cast<const __nv_bfloat16*>(W > 0 ? Vwin : q);
+  a.T = 1;
+  a.Nc = Nloc;
+  a.H = H;
+  a.k = k;
+  a.m = m;
+  a.W = W;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = O;
+  a.o_f32 = o_dtype == CSA_F32;
+  a.lse = lse;
+  a.status = status_word(workspace);
+  a.q_batch_stride = (int64_t)H * d;
+  a.kc_batch_stride = Nloc * d;
+  a.raw_batch_stride = (int64_t)W * d;
+  a.o_batch_stride = (int64_t)H * d;
+  a.pos = pos_dev;
+  a.q_rows = (int64_t)B * H;
+  a.kc_rows = Nloc > 0 ? (int64_t)B * Nloc : 1;
+  a.raw_rows = W > 0 ? (int64_t)B * W : 1;
+  a.nsplit = nsa;
+  a.o_part = reinterpret_cast<float*>(part_base);
+  a.lse_part = reinterpret_cast<float*>(part_base + align256((size_t)B * nsa * H * d * 4));
+  e = launch_attention(a, d, (unsigned)B, s);
+  if (e == cudaSuccess && nsa > 1) e = launch_attention_combine(a, B, d, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
+}
+
+int csa_attn_combine(const float* O_parts, const float* lse_parts, int L, int B, int H, int d, void* O, int o_dtype,
+                     float* lse, csa_stream_t stream) {
+  if (L < 1 || L > kMaxCombineParts || B < 0 || !valid_odtype(o_dtype)) return CSA_ERR_INVALID_ARG;
+  if (!valid_H(H) || (d != 64 && d != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return CSA_OK;
+  int rc = check_ptrs(O_parts, lse_parts, O);
+  if (rc) return rc;
+  if ((rc = check_opt(lse))) return rc;
+  cudaError_t e = launch_combine(O_parts, lse_parts, L, B, H, d, O, o_dtype == CSA_F32, (int64_t)H * d, lse, 1, B,
+                                 (cudaStream_t)stream);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
 int csa_decode_append(const void* K_new, const void* V_new, const void* Z_new, const float* Bias,

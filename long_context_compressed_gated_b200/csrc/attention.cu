@@ -16,14 +16,16 @@
 //
 // Per tile: S = Q K^T (tcgen05 kind::f16, M=128, N=width, fp32 in TMEM), online
 // softmax, P (bf16) to shared memory, O += P V (tcgen05, V as an MN-major
-// operand) and l += P 1 (row sums of the same bf16 weights, tensor core), with
-// O and l accumulated in TMEM.  Warp roles:
-//   warps 0..7   softmax: two warps per TMEM lane quarter, each owning 64 of the
-//                128 columns of a tile (the row maximum is taken over all columns
-//                by both warps, so they agree without exchanging data);
+// operand).  The two halves of a tile's keys (columns 0..63 and 64..127) are
+// softmaxed by different warps, each with its own running maximum and fp32 row
+// sum, and accumulate into their own output accumulators O_A / O_B in TMEM; the
+// halves combine once after the last tile (O = (O_A 2^(mA-m) + O_B 2^(mB-m)) / l),
+// so no warp waits for the other half inside the tile loop.  Warp roles:
+//   warps 0..7   softmax: two warps per TMEM lane quarter, one per key half;
 //   warps 8..11  loaders: 16-byte cp.async gathers of selected rows into
-//                128B-swizzled tiles; contiguous tiles (HCA, window) and Q come
-//                in whole 128-row boxes by TMA;
+//                128B-swizzled tiles (MXFP8 rows dequantised on the way);
+//                contiguous tiles (HCA, window) and Q come in whole 128-row
+//                boxes by TMA;
 //   warp 12      TMEM allocation and MMA issue.
 // K and V have separate double-buffered rings, so S of tile i+2 can start while
 // PV of tile i still reads V.
@@ -94,6 +96,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32x2 add.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long x, y, z;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(z));
+  return r;
+}
+
 // (a*c - m, b*c - m) with one packed fp32x2 fma.
 __device__ __forceinline__ float2 scale_sub2(float a, float b, float c, float m) {
   unsigned long long x, y;
@@ -144,9 +157,8 @@ struct AttnSmem {
   static constexpr size_t off_list = off_tiles + kMaxSegTiles * 4;      // TileList
   static constexpr size_t off_bar = off_list + 64;
   static constexpr size_t off_misc = off_bar + 16 * 8;
-  static constexpr size_t off_ones = off_misc + 256;       // 16 x 16 bf16 ones (row-sum MMA operand)
-  static constexpr size_t off_red = off_ones + 512;        // [2][128] floats: partial fp32 row sums
-  static constexpr size_t off_idx = off_red + 1024;
+  static constexpr size_t off_red = off_misc + 256;        // [2][128][4] (max, sums) of the two halves
+  static constexpr size_t off_idx = off_red + 4096;
   static size_t bytes(int idx_entries) { return off_idx + (size_t)idx_entries * 4 + 1024; }
 };
 
@@ -178,7 +190,6 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   uint64_t* mma_fin = bar + 15;  // every issued MMA complete (before TMEM is freed)
   int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [0] ntiles, [1] tmem, [2..33] seg counts
   volatile int* s_abort = misc + 48;  // set by the first wait that timed out; every role then stops
-  uint8_t* s_ones = smem + L::off_ones;
   float* s_red = reinterpret_cast<float*>(smem + L::off_red);
   int* s_idx = reinterpret_cast<int*>(smem + L::off_idx);
 
@@ -225,7 +236,6 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     tmem_alloc(reinterpret_cast<uint32_t*>(&misc[1]), 512);
     tmem_relinquish();
   }
-  if (tid < 32) reinterpret_cast<uint4*>(s_ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   fence_proxy_async_smem();
   // compact each token's selected list (drop -1 / out-of-range), one warp per token;
   // 8 loads per lane are in flight before any is used
@@ -242,9 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const bool ok = jv[u] >= 0 && jv[u] < a.Nc;
+          const int64_t jl = (int64_t)jv[u] - a.idx_base;  // row of this (slice of the) cache
+          const bool ok = jv[u] >= 0 && jl >= 0 && jl < a.Nc;
           const uint32_t bal = __ballot_sync(0xffffffffu, ok);
-          if (ok) s_idx[g * a.k + n + __popc(bal & ((1u << lane) - 1u))] = jv[u];
+          if (ok) s_idx[g * a.k + n + __popc(bal & ((1u << lane) - 1u))] = (int)jl;
           n += __popc(bal);
         }
       }
@@ -314,7 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     *s_abort = 1;
     return false;
   };
-  constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+  // TMEM columns: S double buffer, then the two halves' output accumulators
+  constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemOA = 256, kTmemOB = 256 + D;
 
   if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
     // =========================== loaders: Q and contiguous tiles by TMA, selected rows by cp.async
@@ -429,28 +441,29 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     };
     if (live && ntiles > 0) live = issue_s(0);
     if (live && ntiles > 1) live = issue_s(1);
-    const uint64_t ones = make_sdesc(smem_u32(s_ones), 128, 256, kSwizzleNone);
+    bool o_written[2] = {false, false};  // O_A / O_B hold data (else the first PV MMA initialises)
     for (int i = 0; i < ntiles && live; ++i) {
       const int st = i & 1;
       if (!wait(p_full, i & 1) || !wait(&v_full[st], (i >> 1) & 1)) break;
       fence_proxy_async_smem();
       tc_fence_after();
+      const int width = tile_at(tlist, s_seg, i).width;
       if (elect_one()) {
-        const int width = tile_at(tlist, s_seg, i).width;
         const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
         for (int ks = 0; ks < width / 16; ++ks) {
-          const uint32_t aoff = (uint32_t)((ks >> 2) * kHalfBytes + (ks & 3) * 32);
+          const int hf = ks >> 2;  // key half: 0 -> O_A, 1 -> O_B
+          const uint32_t aoff = (uint32_t)(hf * kHalfBytes + (ks & 3) * 32);
           const uint64_t pdesc = make_sdesc(sp + aoff, 16, 1024, kSwizzle128);
-          const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
-          mma_bf16_ss(tbase + kTmemO, pdesc, make_sdesc(sv + ks * 2048, kHalfBytes, 1024, kSwizzle128),
-                      idesc_bf16(128, D, 0, 1), acc);
-          // row sums of the same bf16 weights: P x ones -> 16 columns after O
-          mma_bf16_ss(tbase + kTmemO + D, pdesc, ones, idesc_bf16(128, 16, 0, 0), acc);
+          const uint32_t acc = (o_written[hf] || (ks & 3) > 0) ? 1u : 0u;
+          mma_bf16_ss(tbase + (hf ? kTmemOB : kTmemOA), pdesc,
+                      make_sdesc(sv + ks * 2048, kHalfBytes, 1024, kSwizzle128), idesc_bf16(128, D, 0, 1), acc);
         }
         mma_commit(pv_done);
         mma_commit(&v_empty[st]);
       }
       __syncwarp();
+      o_written[0] = true;
+      if (width > 64) o_written[1] = true;
       if (i + 2 < ntiles && !issue_s(i + 2)) break;
     }
     // every MMA this warp issued has completed before TMEM is freed
@@ -458,7 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     __syncwarp();
     mbar_wait(mma_fin, 0);
   } else {
-    // =========================== softmax (warps 0..7): row = TMEM lane, columns [64*half, +64)
+    // =========================== softmax (warps 0..7): row = TMEM lane, key columns [64*half, +64)
+    // Each half keeps its own running maximum, its own fp32 row sum and its own
+    // output accumulator (O_A for keys 0..63 of every tile, O_B for 64..127), so
+    // the two halves never wait for each other inside the tile loop; they combine
+    // once, after the last tile.
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;
     const int g = row / H, h = row % H;
@@ -467,8 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     if (nvis > a.Nc) nvis = a.Nc;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float c = a.scale_log2;  // > 0: max of raw logits * c = max of scaled logits
-    const int my0 = half * 64;     // first column this warp turns into probabilities
-    float m_run = -INFINITY, l_run32 = 0.f;
+    const int my0 = half * 64;     // first key column of this half
+    const uint32_t o_mine = tbase + lane_base + (half ? kTmemOB : kTmemOA);
+    float m_run = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f);  // running row sum of the bf16 weights (two partial sums)
+  float2 u2 = make_float2(0.f, 0.f);  // the same of the unrounded weights (for the log-sum-exp)
     const uint32_t prow = smem_u32(s_p) + (uint32_t)(half * kHalfBytes + row * 128);
     bool live = true;
     for (int i = 0; i < ntiles; ++i) {
@@ -489,36 +509,34 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
           hi = (int)(h0 > l0 ? h0 : l0);
         }
       }
+      // this half's part of the visible range
+      lo = lo > my0 ? lo : my0;
+      hi = hi < my0 + 64 ? hi : my0 + 64;
       const int width = tl.width;
-      const bool warp_any = __any_sync(0xffffffffu, hi > lo);
-      const bool warp_full = __all_sync(0xffffffffu, lo == 0 && hi == width);
+      const bool warp_any = my0 < width && __any_sync(0xffffffffu, hi > lo);
+      const bool warp_full = __all_sync(0xffffffffu, lo == my0 && hi == my0 + 64);
       if (!wait(&s_full[st], (i >> 1) & 1)) {
         live = false;
         break;
       }
       tc_fence_after();
-      const uint32_t scol = tbase + lane_base + (st ? kTmemS1 : kTmemS0);
-      // pass 1: row maximum of the raw logits over the visible range (all columns)
+      const uint32_t scol = tbase + lane_base + (st ? kTmemS1 : kTmemS0) + my0;
+      // pass 1: maximum of this half's visible raw logits
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (warp_any) {
 #pragma unroll
-        for (int c0 = 0; c0 < kTileKeys; c0 += 32) {
-          if (c0 < width) {
+        for (int b0 = 0; b0 < 64; b0 += 32) {
+          if (my0 + b0 < width) {
             uint32_t v[32];
-            tmem_ld32p(scol + c0, v);
+            tmem_ld32p(scol + b0, v);
             tmem_wait_ld();
+            if (warp_full) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              if (c0 + 16 * q < width) {
-                if (warp_full) {
+              for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
+            } else {
 #pragma unroll
-                  for (int e = 16 * q; e < 16 * q + 16; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
-                } else {
-#pragma unroll
-                  for (int e = 16 * q; e < 16 * q + 16; ++e)
-                    if (c0 + e >= lo && c0 + e < hi) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
-                }
-              }
+              for (int e = 0; e < 32; ++e)
+                if (my0 + b0 + e >= lo && my0 + b0 + e < hi) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
             }
           }
         }
@@ -527,17 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const bool raise = mt > m_run + kRescaleSlack || (m_run == -INFINITY && mt > -INFINITY);
       const float m_new = raise ? mt : m_run;
       const float alpha = raise ? exp2f(m_run - m_new) : 1.0f;  // exp2(-inf) = 0 on the first raise
-      // pass 2: p = 2^(s*c - m) over this warp's 64 columns, packed to bf16 pairs
+      // pass 2: p = 2^(s*c - m) over this half's 64 columns, packed to bf16 pairs
       uint32_t pk[32];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 ps = make_float2(0.f, 0.f), pu = make_float2(0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < 32; ++q) pk[q] = 0u;
-      if (warp_any && my0 < width) {
+      if (warp_any) {
 #pragma unroll
         for (int b0 = 0; b0 < 64; b0 += 32) {
           if (my0 + b0 < width) {
             uint32_t v[32];
-            tmem_ld32p(scol + my0 + b0, v);
+            tmem_ld32p(scol + b0, v);
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -551,8 +569,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
                     p0 = (x >= lo && x < hi) ? p0 : 0.f;
                     p1 = (x + 1 >= lo && x + 1 < hi) ? p1 : 0.f;
                   }
-                  if (WANT_LSE) ls[(e >> 1) & 3] += p0 + p1;
-                  pk[(b0 + e) / 2] = pack_bf16x2(p0, p1);
+                  const uint32_t pw = pack_bf16x2(p0, p1);
+                  pk[(b0 + e) / 2] = pw;
+                  // the row sum of the same bf16 weights the PV product uses, so that
+                  // numerator and denominator see identical P
+                  ps = add2(ps, make_float2(bf16_lo(pw), bf16_hi(pw)));
+                  if (WANT_LSE) pu = add2(pu, make_float2(p0, p1));
                 }
               }
             }
@@ -571,32 +593,23 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
-        // rescale this warp's half of O (and, for half 0, the row-sum columns)
+        // rescale this half's output accumulator (all D columns)
         const float sc = (raise && i > 0) ? alpha : 1.0f;
-        if (my0 < D) {
-#pragma unroll
-          for (int b0 = 0; b0 < 64; b0 += 32) {
-            uint32_t v[32];
-            tmem_ld32p(tbase + lane_base + kTmemO + my0 + b0, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
-            tmem_st32p(tbase + lane_base + kTmemO + my0 + b0, v);
-          }
-        }
-        if (half == 0) {
-          uint32_t v[16];
-          tmem_ld16p(tbase + lane_base + kTmemO + D, v);
+#pragma unroll 1
+        for (int b0 = 0; b0 < D; b0 += 32) {
+          uint32_t v[32];
+          tmem_ld32p(o_mine + b0, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
-          tmem_st16p(tbase + lane_base + kTmemO + D, v);
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * sc);
+          tmem_st32p(o_mine + b0, v);
         }
         tmem_wait_st();
       }
-      if (WANT_LSE) l_run32 = l_run32 * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+      l2 = make_float2(l2.x * alpha + ps.x, l2.y * alpha + ps.y);
+      if (WANT_LSE) u2 = make_float2(u2.x * alpha + pu.x, u2.y * alpha + pu.y);
       m_run = m_new;
-      // store this warp's half of the P row (K-major, 128B swizzle)
+      // store this half's P row (K-major, 128B swizzle)
       if (my0 < width) {
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
@@ -613,17 +626,21 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // epilogue: O / l, with l the row sum of the bf16 weights (tensor-core P x ones)
-    float l_run = 0.f;
+    // epilogue: the two halves' (max, sum) meet once; O = (O_A f_A + O_B f_B) / l
     const bool have_o = ntiles > 0 && live && wait(pv_done, (ntiles - 1) & 1);
-    if (have_o) {
-      tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16p(tbase + lane_base + kTmemO + D, v);
-      tmem_wait_ld();
-      l_run = __uint_as_float(v[0]);
-    }
-    const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
+    if (have_o) tc_fence_after();
+    const float l_mine = have_o ? l2.x + l2.y : 0.f;
+    *reinterpret_cast<float4*>(s_red + 4 * (half * kRows + row)) =
+        make_float4(m_run, l_mine, have_o ? u2.x + u2.y : 0.f, 0.f);
+    asm volatile("bar.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(kSoftmaxWarps * 32) : "memory");
+    const float4 ra = *reinterpret_cast<const float4*>(s_red + 4 * row);
+    const float4 rb = *reinterpret_cast<const float4*>(s_red + 4 * (kRows + row));
+    const float mA = ra.x, lA = ra.y, mB = rb.x, lB = rb.y;
+    const float mm = fmaxf(mA, mB);
+    const float fA = lA > 0.f ? exp2f(mA - mm) : 0.f, fB = lB > 0.f ? exp2f(mB - mm) : 0.f;
+    const float l_all = lA * fA + lB * fB;
+    const float inv = l_all > 0.f ? 1.0f / l_all : 0.f;
+    const float wA = fA * inv, wB = fB * inv;
     const bool part = a.nsplit > 1;
     __nv_bfloat16* orow = nullptr;
     float* part_row = nullptr;  // fp32 rows: a split's partial output, or O itself when o_f32
@@ -631,46 +648,47 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     if (t >= 0 && !part && !a.o_f32) orow = static_cast<__nv_bfloat16*>(a.O) + o_off;
     if (t >= 0 && !part && a.o_f32) part_row = static_cast<float*>(a.O) + o_off;
     if (t >= 0 && part) part_row = a.o_part + ((b * a.nsplit + blockIdx.y) * H + h) * (int64_t)D;
+#pragma unroll 1
+    for (int b0 = 0; b0 < 64; b0 += 16) {
+      if (my0 >= D) break;  // d = 64: half 1 has no output columns
+      float o[16];
 #pragma unroll
-    for (int b0 = 0; b0 < 64; b0 += 32) {
-      if (my0 >= D) break;
-      uint32_t v[32];
+      for (int e = 0; e < 16; ++e) o[e] = 0.f;
       if (have_o) {
-        tmem_ld32p(tbase + lane_base + kTmemO + my0 + b0, v);
+        uint32_t va[16], vb[16];
+        tmem_ld16p(tbase + lane_base + kTmemOA + my0 + b0, va);
+        tmem_ld16p(tbase + lane_base + kTmemOB + my0 + b0, vb);
         tmem_wait_ld();
-      } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0u;
+        for (int e = 0; e < 16; ++e) {
+          // an accumulator that never received a key holds no data: weight 0 exactly
+          const float x = wA != 0.f ? __uint_as_float(va[e]) * wA : 0.f;
+          o[e] = wB != 0.f ? fmaf(__uint_as_float(vb[e]), wB, x) : x;
+        }
       }
       if (part_row) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(part_row + my0 + b0 + e) =
-              make_float4(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv,
-                          __uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(part_row + my0 + b0 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
       }
       if (orow) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 o;
-          o.x = pack_bf16x2(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
-          o.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
-          o.z = pack_bf16x2(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
-          o.w = pack_bf16x2(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + my0 + b0 + e) = o;
+        for (int e = 0; e < 16; e += 8) {
+          uint4 ov;
+          ov.x = pack_bf16x2(o[e], o[e + 1]);
+          ov.y = pack_bf16x2(o[e + 2], o[e + 3]);
+          ov.z = pack_bf16x2(o[e + 4], o[e + 5]);
+          ov.w = pack_bf16x2(o[e + 6], o[e + 7]);
+          *reinterpret_cast<uint4*>(orow + my0 + b0 + e) = ov;
         }
       }
     }
-    if (WANT_LSE) {
-      // combine the two halves' fp32 row sums
-      s_red[half * kRows + row] = l_run32;
-      asm volatile("bar.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(kSoftmaxWarps * 32) : "memory");
-      if (half == 0 && t >= 0 && (a.lse || part)) {
-        const float l32 = l_run32 + s_red[kRows + row];
-        const float lse = l32 > 0.f ? (m_run + log2f(l32)) * 0.69314718055994531f : -INFINITY;
-        if (part) a.lse_part[(b * a.nsplit + blockIdx.y) * H + h] = lse;
-        else a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
-      }
+    if (WANT_LSE && half == 0 && t >= 0 && (a.lse || part)) {
+      // the log-sum-exp of the unrounded weights
+      const float u_all = ra.z * fA + rb.z * fB;
+      const float lse = u_all > 0.f ? (mm + log2f(u_all)) * 0.69314718055994531f : -INFINITY;
+      if (part) a.lse_part[(b * a.nsplit + blockIdx.y) * H + h] = lse;
+      else a.lse[b * (decode ? H : 0) + (row_tok0 + g) * H + h] = lse;
     }
   }
 
@@ -721,11 +739,14 @@ static cudaError_t launch_t(const AttnArgs& a, const AttnMaps& maps, unsigned gr
 // dims 4c..4c+3; every partial is loaded before any is combined.
 constexpr int kCombineSplits = 16;
 
+// Partial s of sequence b is at row (b * sb + s * ss) of the partials ([B, nsplit]
+// order: sb = nsplit, ss = 1; [nsplit, B] order: sb = 1, ss = B).
 template <int D>
 __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __restrict__ o_part,
                                                                 const float* __restrict__ lse_part, int nsplit, int H,
                                                                 int64_t rows, void* __restrict__ O, int o_f32,
-                                                                int64_t o_batch_stride, float* __restrict__ lse) {
+                                                                int64_t o_batch_stride, float* __restrict__ lse,
+                                                                int64_t sb, int64_t ss) {
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (b, h)
   if (w >= rows) return;
@@ -736,7 +757,7 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __r
   float mx = -INFINITY;
 #pragma unroll
   for (int s = 0; s < kCombineSplits; ++s) {
-    ls[s] = s < nsplit ? lse_part[(b * nsplit + s) * H + h] : -INFINITY;
+    ls[s] = s < nsplit ? lse_part[(b * sb + s * ss) * H + h] : -INFINITY;
     mx = fmaxf(mx, ls[s]);
   }
   if (lane >= V) return;
@@ -744,7 +765,7 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __r
 #pragma unroll
   for (int s = 0; s < kCombineSplits; ++s)
     o[s] = (s < nsplit && ls[s] > -INFINITY)
-               ? reinterpret_cast<const float4*>(o_part + ((b * nsplit + s) * H + h) * (int64_t)D)[lane]
+               ? reinterpret_cast<const float4*>(o_part + ((b * sb + s * ss) * H + h) * (int64_t)D)[lane]
                : make_float4(0.f, 0.f, 0.f, 0.f);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float sum = 0.f;
@@ -773,17 +794,25 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __r
   if (lse && lane == 0) lse[b * H + h] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
 }
 
-cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream) {
-  if (a.nsplit > kCombineSplits) return cudaErrorInvalidConfiguration;
-  const int64_t rows = (int64_t)B * a.H;
+cudaError_t launch_combine(const float* o_part, const float* lse_part, int nsplit, int B, int H, int d, void* O,
+                           int o_f32, int64_t o_batch_stride, float* lse, int64_t sb, int64_t ss,
+                           cudaStream_t stream) {
+  if (nsplit > kCombineSplits) return cudaErrorInvalidConfiguration;
+  const int64_t rows = (int64_t)B * H;
   const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (rows == 0) return cudaSuccess;
   if (d == 128)
-    attention_combine_kernel<128><<<grid, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, rows, a.O,
-                                                             a.o_f32, a.o_batch_stride, a.lse);
+    attention_combine_kernel<128><<<grid, 256, 0, stream>>>(o_part, lse_part, nsplit, H, rows, O, o_f32,
+                                                             o_batch_stride, lse, sb, ss);
   else
-    attention_combine_kernel<64><<<grid, 256, 0, stream>>>(a.o_part, a.lse_part, a.nsplit, a.H, rows, a.O,
-                                                            a.o_f32, a.o_batch_stride, a.lse);
+    attention_combine_kernel<64><<<grid, 256, 0, stream>>>(o_part, lse_part, nsplit, H, rows, O, o_f32,
+                                                            o_batch_stride, lse, sb, ss);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream) {
+  return launch_combine(a.o_part, a.lse_part, a.nsplit, B, a.H, d, a.O, a.o_f32, a.o_batch_stride, a.lse, a.nsplit, 1,
+                        stream);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream) {

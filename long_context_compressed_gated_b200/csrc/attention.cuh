@@ -12,6 +12,7 @@ struct AttnArgs {
   const __nv_bfloat16* Kc;  // [Nc, d] compressed keys (decode: per-sequence cache)
   const __nv_bfloat16* Vc;
   const int32_t* idx;       // [T, k] selected entries (CSA) or null (HCA)
+  int64_t idx_base;         // idx holds global entry numbers; Kc row r is entry idx_base + r
   const __nv_bfloat16* Kr;  // raw K rows, row 0 at absolute position raw_lo
   const __nv_bfloat16* Vr;
   int64_t T, t0, Nc, raw_lo;
@@ -42,5 +43,11 @@ cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream
 // O[b,h] = sum_s exp(lse_s - lse) O_s with lse = log sum_s exp(lse_s), as bf16 (+ lse)
 cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream);
 int attention_max_seg_tiles();
+// Merge nsplit normalised fp32 partial outputs with their log-sum-exps (partial s
+// of sequence b at row b*sb + s*ss): O = sum_s exp(lse_s - lse) O_s, lse = log sum exp.
+cudaError_t launch_combine(const float* o_part, const float* lse_part, int nsplit, int B, int H, int d, void* O,
+                           int o_f32, int64_t o_batch_stride, float* lse, int64_t sb, int64_t ss,
+                           cudaStream_t stream);
+constexpr int kMaxCombineParts = 16;
 
 }  // namespace csa

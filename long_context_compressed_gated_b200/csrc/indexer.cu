@@ -136,10 +136,9 @@ struct IndexerArgs {
   int check;                // tiles between buffer cut-backs (cap >= k + 128 * check)
   int nsplit;               // key ranges per query group
   int64_t split_tiles;      // 128-key tiles per range
+  int64_t j_base;           // decode over a slice of the cache: global index of its entry 0
   uint64_t* cand;           // [rows, nsplit, k] selected keys of each key range (unsorted)
   int* cand_cnt;            // [rows, nsplit]    how many of them are valid
-  int32_t* idx;             // prefill (one key range): [rows, k] written directly, sorted
-  float* scores;            // nullable
   int* status;
   int fault;                // test hook (csa_debug_inject): 1 = the producer skips its first stage group
 };
@@ -230,7 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t r = row0 + g;
     int64_t t = -1;
     if (r < a.rows) t = decode ? a.pos[r] : a.t0 + r;
-    int64_t nv = n_visible(t, a.m);
+    int64_t nv = n_visible(t, a.m) - a.j_base;  // entries of this (slice of the) cache visible to t
+    if (nv < 0) nv = 0;
     if (nv > a.Nc) nv = a.Nc;
     tnvis[g] = nv;
     if (nv > nvis_max) nvis_max = nv;
@@ -524,6 +524,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       pbase[t] = 0;
     }
     const uint32_t lt = (1u << lane) - 1u;
+    // entries visible to token gg of the group (recomputed where a loop over the
+    // tokens is not unrolled, so that no register array is indexed at run time)
+    auto token_nvis = [&](int gg) -> int64_t {
+      const int64_t r = row0 + gg;
+      if (r >= a.rows) return 0;
+      int64_t nv = n_visible(decode ? a.pos[r] : a.t0 + r, a.m) - a.j_base;
+      if (nv < 0) nv = 0;
+      return nv > a.Nc ? a.Nc : nv;
+    };
     // keys held in fixed slots (no cut-back yet): the visible ones among the first n of the range
     auto fixed_count = [&](int64_t nv, int64_t n) -> int {
       int64_t lim = nv < j_end ? nv : j_end;
@@ -561,8 +570,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = it % NB;
         tc_fence_after();
         // exactness precondition on the key scales: the checking half reads the
-        // scale word of its own key row (lane quarter q, column q of the replicated copy)
-        const bool checker = kAlt || half == 0;
+        // scale word of its own key row (lane quarter q, column q of the replicated
+        // copy).  In prefill every CTA reads the same entries and block 0 (the
+        // heaviest group, heavy groups first) reads every entry any CTA reads, so
+        // it checks for all; in decode each CTA checks its own key range.
+        const bool checker = kAlt || (half == 0 && blockIdx.x == 0);
         uint32_t sfw = 0x7F7F7F7Fu;
         if (checker) sfw = tmem_ld1(tbase + lane_base + TS::sfa(b) + (uint32_t)quarter);
         uint32_t acc[G0];  // arithmetic mod 2^32: the true head sum fits in int32
@@ -595,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int t = 0; t < G0; ++t) {
-          pkey[t] = topk::make_key((int32_t)(acc[t] - sumw_magic[t]), (uint32_t)j);
+          pkey[t] = topk::make_key((int32_t)(acc[t] - sumw_magic[t]), (uint32_t)(j + a.j_base));
           const bool vis = jin && j < nvis[t];
           if (thr[t] == 0) {
             // no cut-back yet: every visible key is kept, in its fixed slot (the
@@ -620,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < G0; ++t) {  // every warp of the group cuts back each of its buffers
         const int gg = g_lo + t;
         uint64_t* buf = s_cand + (size_t)gg * cap;
-        const int cnt = thr[t] == 0 ? fixed_count(nvis[t], (int64_t)tiles_done * 128) : s_cnt[gg];
+        const int cnt = s_thr[gg] == 0 ? fixed_count(token_nvis(gg), (int64_t)tiles_done * 128) : s_cnt[gg];
         if (cnt > cap - 128 * a.check) {
           const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, cap - 128 * a.check, false,
                                                          ghist, gscr, gt, gbar);
@@ -643,34 +655,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row0 + gg >= a.rows) break;  // uniform over the group
       const int64_t r = row0 + gg;
       uint64_t* buf = s_cand + (size_t)gg * cap;
-      int cnt = thr[t] == 0 ? fixed_count(nvis[t], (int64_t)ntiles * 128) : s_cnt[gg];
+      int cnt = s_thr[gg] == 0 ? fixed_count(token_nvis(gg), (int64_t)ntiles * 128) : s_cnt[gg];
       if (cnt > a.k) {
         const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, ghist, gscr,
                                                        gt, gbar);
         cnt = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
-      }
-      if (!kAlt && a.idx != nullptr) {
-        // one key range per row: these are the row's k best; sort them (score
-        // desc, j asc) and write idx / scores directly
-        const int P = topk::next_pow2(a.k) > 128 ? topk::next_pow2(a.k) : 128;
-        for (int q = cnt + gt; q < P; q += GNT) buf[q] = 0;
-        topk::named_sync(gbar, GNT);
-        if constexpr (GNT == 128) {
-          switch (P / 128) {
-            case 1: topk::group_sort_desc<128, 1>(buf, gt, gbar); break;
-            case 2: topk::group_sort_desc<128, 2>(buf, gt, gbar); break;
-            case 4: topk::group_sort_desc<128, 4>(buf, gt, gbar); break;
-            case 8: topk::group_sort_desc<128, 8>(buf, gt, gbar); break;
-            default: topk::group_sort_desc<128, 16>(buf, gt, gbar); break;
-          }
-        }
-        for (int q = gt; q < a.k; q += GNT) {
-          const uint64_t key = buf[q];  // 0: padding (fewer than k visible entries)
-          a.idx[r * a.k + q] = key ? (int32_t)topk::key_index(key) : -1;
-          if (a.scores) a.scores[r * a.k + q] = key ? (float)topk::key_score(key) * (1.0f / 128.0f) : -INFINITY;
-        }
-        topk::named_sync(gbar, GNT);  // the buffer is reused by the next token of the group
-        continue;
       }
       uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
       for (int q = gt; q < cnt; q += GNT) out[q] = buf[q];
@@ -975,6 +964,33 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
   return cudaGetLastError();
 }
 
+// Valid keys of each candidate list (nonzero keys first, zero padding after):
+// one warp per list.
+__global__ void __launch_bounds__(256) count_keys_kernel(const uint64_t* __restrict__ keys, int64_t lists, int k,
+                                                         int* __restrict__ cnt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t l = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (l >= lists) return;
+  int n = 0;
+  for (int q = lane; q < k; q += 32) n += __popc(__ballot_sync(0xffffffffu, keys[l * k + q] != 0));
+  if (lane == 0) cnt[l] = n;
+}
+
+cudaError_t launch_topk_merge(const uint64_t* keys, int rows, int lists, int k, int* cnt, int32_t* idx,
+                              float* scores, uint64_t* keys_out, cudaStream_t stream) {
+  const int64_t nl = (int64_t)rows * lists;
+  if (nl > 0) {
+    count_keys_kernel<<<(unsigned)ceil_div(nl, 8), 256, 0, stream>>>(keys, nl, k, cnt);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (lists == 1) {
+    // one list per row: the warp-per-row pass
+    return launch_finalize(keys, cnt, 1, k, rows, idx, scores, keys_out, stream);
+  }
+  return launch_finalize(keys, cnt, lists, k, rows, idx, scores, keys_out, stream);
+}
+
 // ------------------------------------------------------------------ host side
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1113,13 +1129,15 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
   a.split_tiles = ceil_div(Nc > 0 ? Nc : 1, 128);
   a.cand = cand;
   a.cand_cnt = cand_cnt;
-  a.idx = idx;  // one key range per row: the indexer sorts and writes the selection itself
-  a.scores = scores;
   a.status = status;
   dim3 grid((unsigned)ceil_div(T, G), 1);
   const uint8_t* kc = Nc > 0 ? k_codes : q_codes;  // any valid mapping when the cache is empty
-  return DI == 128 ? dispatch_hi<128>(HI, false, q_codes, kc, a, grid, stream)
-                   : dispatch_hi<64>(HI, false, q_codes, kc, a, grid, stream);
+  cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, false, q_codes, kc, a, grid, stream)
+                            : dispatch_hi<64>(HI, false, q_codes, kc, a, grid, stream);
+  if (e != cudaSuccess) return e;
+  // a sorting pass per row (one warp each; many rows per SM) is cheaper than
+  // sorting inside the indexer CTA, where the sort would sit on the CTA's tail
+  return launch_finalize(cand, cand_cnt, 1, k, T, idx, scores, nullptr, stream);
 }
 
 // Decode: rows = B sequences, each with its own cache of Ncap entries and position
@@ -1128,8 +1146,9 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
                                   const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
                                   int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
                                   uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
-                                  int* status, cudaStream_t stream) {
+                                  int* status, cudaStream_t stream, int64_t j_base) {
   IndexerArgs a{};
+  a.j_base = j_base;
   a.q_scales = q_scales;
   a.w_codes = w_codes;
   a.k_scales = k_scales;

@@ -617,48 +617,6 @@ __device__ void block_sort_desc(uint64_t* buf, int tid) {
   }
 }
 
-// The same sort for a group of NT threads (whole warps, gt in [0, NT)) that
-// meets on named barrier `bar`: buf[0 .. NT*R) descending.
-template <int NT, int R>
-__device__ __noinline__ void group_sort_desc(uint64_t* buf, int gt, int bar) {
-  constexpr int C = 32 * R, P = NT * R;
-  const int lane = gt & 31, base = (gt >> 5) * C;
-  uint64_t v[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) v[r] = buf[base + lane * R + r];
-#pragma unroll 1
-  for (int size = 2; size <= C; size <<= 1)
-#pragma unroll 1
-    for (int stride = size >> 1; stride > 0; stride >>= 1) lm_stage_at<R>(v, size, stride, base, lane);
-#pragma unroll
-  for (int r = 0; r < R; ++r) buf[base + lane * R + r] = v[r];
-  named_sync(bar, NT);
-#pragma unroll 1
-  for (int size = 2 * C; size <= P; size <<= 1) {
-#pragma unroll 1
-    for (int stride = size >> 1; stride >= C; stride >>= 1) {
-      for (int i = gt; i < P / 2; i += NT) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint64_t a = buf[lo], b = buf[hi];
-        if ((a < b) == desc) {
-          buf[lo] = b;
-          buf[hi] = a;
-        }
-      }
-      named_sync(bar, NT);
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) v[r] = buf[base + lane * R + r];
-#pragma unroll 1
-    for (int stride = C >> 1; stride > 0; stride >>= 1) lm_stage_at<R>(v, size, stride, base, lane);
-#pragma unroll
-    for (int r = 0; r < R; ++r) buf[base + lane * R + r] = v[r];
-    named_sync(bar, NT);
-  }
-}
-
 __host__ __device__ constexpr int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;

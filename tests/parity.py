@@ -22,15 +22,42 @@ def from_words(w, device):
     return torch.from_numpy(np.ascontiguousarray(w).view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def fp32_pool_slack(x_bf16, m):
-    """Error bound of an fp32 weighted mean over blocks of m rows: (m + 8) * 2^-24
-    * max |x| in the block, per (block, channel).  When the weighted sum cancels,
-    this absolute error can exceed one bf16 ulp of the (small) result."""
+def _pool_shape(d, m):
+    """Rows per thread L and slices S of the GPU pooling of one block (the launch
+    rule of the compression kernel: L = min(m, 8), doubled while (d/8) * (m/L) >
+    256 threads)."""
+    L = m if m <= 8 else 8
+    while (d // 8) * (m // L) > 256:
+        L *= 2
+    return L, m // L
+
+
+def fp32_pool_slack(x_bf16, m, Z, B):
+    """Worst-case absolute error of the fp32 gated pooling, per (block, channel),
+    with u = 2^-24, X = max |x| over the block, G = max |z + b| over the block,
+    and the kernel's L rows per slice and S slices:
+      every weight exp(g_i - M) carries a relative error of at most
+        u*G (rounding of z + b) + (L + S) * (2*u*G + 4*u)
+      (each of the at most L-1 in-slice rescales and S-1 slice merges multiplies
+      it by one more exp of a rounded difference: 2uG for the difference, 4u for
+      expf's 2-ulp bound); a relative weight error eta moves a weighted mean by at
+      most 2*eta*X; the m-term sums of numerator and denominator plus the L
+      rescale products add (m + L) * u * X each; the division and the final
+      product 2*u*X.  Total:
+        u * X * (2*G*(1 + 2*(L+S)) + 8*(L+S) + 2*(m+L) + 2).
+    When the weighted sum cancels, this can exceed one bf16 ulp of the (small)
+    result; otherwise the bf16 ulp dominates."""
     xf = x_bf16.detach().float().cpu().double().numpy() if hasattr(x_bf16, "detach") else oracle.bf16_words_to_f64(x_bf16)
+    zf = Z.detach().float().cpu().double().numpy() if hasattr(Z, "detach") else oracle.bf16_words_to_f64(Z)
+    bf = B.detach().float().cpu().double().numpy() if hasattr(B, "detach") else np.asarray(B, np.float64)
     T, d = xf.shape
     nb = T // m
-    blk = np.abs(xf[: nb * m]).reshape(nb, m, d).max(axis=1)
-    return (m + 8) * 2.0 ** -24 * blk
+    X = np.abs(xf[: nb * m]).reshape(nb, m, d).max(axis=1)
+    g = zf[: nb * m].reshape(nb, m, d) + bf[None, :, :]
+    G = np.abs(g).max(axis=1)
+    L, S = _pool_shape(d, m)
+    u = 2.0 ** -24
+    return u * X * (2 * G * (1 + 2 * (L + S)) + 8 * (L + S) + 2 * (m + L) + 2)
 
 
 def assert_within_bf16_ulp(got_bf16, exact_f64, what, slack=None):

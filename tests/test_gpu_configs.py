@@ -44,8 +44,8 @@ def test_csa_prefill_full_size_sampled(csa):
     rows = sample_rows(wl.T, 24, special, seed=11)
     # compression of every block
     Kx, Vx = oracle.compress(h["K"], h["V"], h["Z"], h["B"], wl.m)
-    assert_within_bf16_ulp(Kc, Kx, "Kc", fp32_pool_slack(h["K"], wl.m))
-    assert_within_bf16_ulp(Vc, Vx, "Vc", fp32_pool_slack(h["V"], wl.m))
+    assert_within_bf16_ulp(Kc, Kx, "Kc", fp32_pool_slack(h["K"], wl.m, h["Z"], h["B"]))
+    assert_within_bf16_ulp(Vc, Vx, "Vc", fp32_pool_slack(h["V"], wl.m, h["Z"], h["B"]))
     # indexer + top-k on sampled rows
     I = oracle.indexer(h["qI_codes"], h["qI_scales"], h["w_codes"], h["kI_codes"], h["kI_scales"], 0, wl.m, rows)
     want_idx, want_top = oracle.topk(I, oracle.n_vis(rows, wl.m), wl.k)
@@ -82,8 +82,8 @@ def test_hca_prefill_full_size_sampled(csa):
     h = _host(g, ["K", "V", "Z", "B_hca"])
     Kx, Vx = oracle.compress(h["K"], h["V"], h["Z"], h["B_hca"], wl.m_hca)
     Kc, Vc = csa.csa_compress(g["K"], g["V"], g["Z"], g["B_hca"], wl.m_hca)
-    assert_within_bf16_ulp(Kc, Kx, "HCA Kc", fp32_pool_slack(h["K"], wl.m_hca))
-    assert_within_bf16_ulp(Vc, Vx, "HCA Vc", fp32_pool_slack(h["V"], wl.m_hca))
+    assert_within_bf16_ulp(Kc, Kx, "HCA Kc", fp32_pool_slack(h["K"], wl.m_hca, h["Z"], h["B_hca"]))
+    assert_within_bf16_ulp(Vc, Vx, "HCA Vc", fp32_pool_slack(h["V"], wl.m_hca, h["Z"], h["B_hca"]))
     Kcw, Vcw = oracle.to_bf16_words(Kx), oracle.to_bf16_words(Vx)
     O, lse, ws = csa.hca_attn(g["Q"], from_words(Kcw, "cuda"), from_words(Vcw, "cuda"), g["K"], g["V"], wl.m_hca,
                               wl.W_hca, scale)

@@ -42,8 +42,8 @@ def test_compress_csa_and_hca(lib, data):
         Kc, Vc = lib.csa_compress(g["K"], g["V"], g["Z"], g[B], m)
         torch.cuda.synchronize()
         Kx, Vx = oracle.compress(data["K"], data["V"], data["Z"], data[B], m)
-        assert_within_bf16_ulp(Kc, Kx, "Kc m=%d" % m, fp32_pool_slack(data["K"], m))
-        assert_within_bf16_ulp(Vc, Vx, "Vc m=%d" % m, fp32_pool_slack(data["V"], m))
+        assert_within_bf16_ulp(Kc, Kx, "Kc m=%d" % m, fp32_pool_slack(data["K"], m, data["Z"], data[B]))
+        assert_within_bf16_ulp(Vc, Vx, "Vc m=%d" % m, fp32_pool_slack(data["V"], m, data["Z"], data[B]))
 
 
 def test_indexer_topk_exact(lib, data):
