@@ -229,3 +229,79 @@ class EmulatedRanks:
         parts2 = [sp.hca_parts(x) for x in xs]
         O2 = [sp.hca_attend(x, parts2, q) for x, q in zip(xs, Q2)]
         return O2, O1
+
+
+# ------------------------------------------------------------------ split-cache decode
+class SplitCacheDecode:
+    """Decode of B sequences whose compressed caches are split over the ranks by
+    entry ranges: rank r holds entries [j_base, j_base + Nloc) of every sequence,
+    the last rank also the raw window (the newest tokens).  Per step:
+
+      1. search     the k best entries of the rank's slice, as exact 64-bit keys
+                    with global entry numbers (csa_decode_search);
+      2. exchange   all-gather of the keys ([L, B, k]);
+      3. merge      the exact top-k of the L lists, identical on every rank
+                    (csa_topk_merge);
+      4. attend     attention over the selected entries inside the slice, plus
+                    the window on the last rank: an fp32 partial output and its
+                    log-sum-exp (csa_decode_attend);
+      5. exchange   all-gather of the partials, then their log-sum-exp combine
+                    (csa_attn_combine).
+
+    x: dict with q [B,H,d], qI_codes, qI_scales, w_codes, Kc, Vc [B,Nloc,d] (the
+    slice), kI_codes [B,Nloc,dI/2], kI_scales, Kwin, Vwin [B,W,d], pos (host list),
+    j_base, has_window.  The result equals csa_decode on the whole cache: the
+    selection bit for bit, O within the attention tolerance.
+    """
+
+    def __init__(self, m, k, W, scale, ops=None):
+        self.m, self.k, self.W, self.scale = m, k, W, scale
+        if ops is None:
+            import long_context_compressed_gated_b200 as ops
+        self.ops = ops
+
+    def search(self, x):
+        keys, _ = self.ops.csa_decode_search(x["qI_codes"], x["qI_scales"], x["w_codes"], x["kI_codes"],
+                                             x["kI_scales"], x["pos"], self.m, self.k, j_base=x["j_base"])
+        return keys
+
+    def merge(self, gathered_keys):
+        return self.ops.csa_topk_merge(torch.stack(gathered_keys, dim=1), self.k)
+
+    def attend(self, x, idx):
+        W = self.W if x["has_window"] else 0
+        return self.ops.csa_decode_attend(x["q"], x["Kc"], x["Vc"], idx, x["Kwin"], x["Vwin"], x["pos"], self.m, W,
+                                          self.scale, j_base=x["j_base"])
+
+    def combine(self, gathered_O, gathered_lse, out_dtype=torch.float32):
+        return self.ops.csa_attn_combine(torch.stack(gathered_O), torch.stack(gathered_lse), out_dtype=out_dtype)
+
+    def run(self, x, comm, out_dtype=torch.float32):
+        """One decode step on this rank; returns (O, lse, idx, scores), the same on every rank."""
+        keys = self.search(x)
+        idx, scores = self.merge(comm.all_gather(keys))
+        O_r, lse_r = self.attend(x, idx)
+        O, lse = self.combine(comm.all_gather(O_r), comm.all_gather(lse_r), out_dtype)
+        return O, lse, idx, scores
+
+
+def split_cache(batch, rank, world):
+    """The rank's slice of full decode inputs (for tests and benchmarks): entries
+    [r*N/G, (r+1)*N/G) of every sequence's cache; the last rank keeps the window."""
+    N = batch["Kc"].shape[1]
+    lo, hi = rank * N // world, (rank + 1) * N // world
+    x = {k: batch[k] for k in ("q", "qI_codes", "qI_scales", "w_codes", "Kwin", "Vwin")}
+    for key in ("Kc", "Vc", "kI_codes", "kI_scales"):
+        x[key] = batch[key][:, lo:hi].contiguous()
+    x["j_base"] = lo
+    x["has_window"] = rank == world - 1
+    return x
+
+
+def emulated_split_decode(dec, xs, out_dtype=torch.float32):
+    """All ranks' steps in one process (one GPU): the all-gathers are lists."""
+    keys = [dec.search(x) for x in xs]
+    merged = [dec.merge(keys) for _ in xs]
+    parts = [dec.attend(x, m[0]) for x, m in zip(xs, merged)]
+    O, lse = dec.combine([p[0] for p in parts], [p[1] for p in parts], out_dtype)
+    return O, lse, merged[0][0], merged[0][1]

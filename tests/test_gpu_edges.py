@@ -329,3 +329,27 @@ def test_hca_decode_fp32_output(csa):
         o, l = oracle.attention(q[b:b + 1], Kc[b], Vc[b], Kw[b], Vw[b], t, wl.m, wl.W, scale, rows=[0],
                                 raw_pos0=t - wl.W + 1)
         assert_attention_close(O[b:b + 1], o, "HCA decode fp32 seq %d" % b)
+
+
+@pytest.mark.parametrize("HI,dI", [(4, 64), (32, 128), (64, 128)])
+def test_decode_indexer_head_counts(csa, HI, dI):
+    """Decode with 4, 32 and 64 indexer heads: the 16-warp epilogue (four groups
+    taking turns on the key tiles) and, at 64 heads, the 8-warp one."""
+    wl = inputs.Workload("dec_hi", H=64, d=128, m=4, k=256, W=64, HI=HI, dI=dI, batch=3, context=1 << 16,
+                         seed=90 + HI)
+    g = inputs.decode_batch(wl)
+    pos = [wl.context - 1, 40000, 777]
+    scale = 1.0 / math.sqrt(wl.d)
+    gc = {key: v.cuda() for key, v in g.items()}
+    O, lse, idx, scores, ws = csa.csa_decode(gc["q"], gc["qI_codes"], gc["qI_scales"], gc["w_codes"], gc["Kc"],
+                                             gc["Vc"], gc["kI_codes"], gc["kI_scales"], gc["Kwin"], gc["Vwin"], pos,
+                                             wl.m, wl.k, scale, out_dtype=torch.float32)
+    assert csa.csa_check_status(ws) == 0
+    for b, t in enumerate(pos):
+        I = oracle.indexer(g["qI_codes"][b:b + 1], g["qI_scales"][b:b + 1], g["w_codes"][b:b + 1], g["kI_codes"][b],
+                           g["kI_scales"][b], t, wl.m)
+        want_idx, want_top = oracle.topk(I, oracle.n_vis([t], wl.m), wl.k)
+        assert_topk_exact(idx[b:b + 1], scores[b:b + 1], want_idx, want_top, "decode HI=%d seq %d" % (HI, b))
+        o, _ = oracle.attention(g["q"][b:b + 1], g["Kc"][b], g["Vc"][b], g["Kwin"][b], g["Vwin"][b], t, wl.m, wl.W,
+                                scale, sel=want_idx, rows=[0], raw_pos0=t - wl.W + 1)
+        assert_attention_close(O[b:b + 1], o, "decode HI=%d attention seq %d" % (HI, b))

@@ -37,3 +37,32 @@ def test_emulated_ranks_equal_the_single_gpu_stack(wl, world):
             if c in (0, 2 * world - 1):
                 assert_attention_close(O2[r][c], O2_ref[sl].float().cpu().double().numpy(),
                                        "layer 2, chunk %d of %d ranks" % (c, world))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_split_cache_decode_emulated_ranks(world):
+    """Split-cache decode with the ranks emulated on one GPU, against csa_decode
+    over the whole cache: selection bit for bit, output within the tolerance."""
+    import math
+    import long_context_compressed_gated_b200 as csa
+    from long_context_compressed_gated_b200.sharded import SplitCacheDecode, emulated_split_decode, split_cache
+    wl = inputs.Workload("split_dec", H=64, d=128, m=4, k=1024, W=128, HI=16, dI=128, batch=4, context=1 << 18,
+                         seed=62)
+    g = {key: v.cuda() for key, v in inputs.decode_batch(wl).items()}
+    pos = [wl.context - 1, 200000, 70001, 4100]
+    scale = 1.0 / math.sqrt(wl.d)
+    O_ref, lse_ref, idx_ref, sc_ref, ws = csa.csa_decode(g["q"], g["qI_codes"], g["qI_scales"], g["w_codes"], g["Kc"],
+                                                         g["Vc"], g["kI_codes"], g["kI_scales"], g["Kwin"], g["Vwin"],
+                                                         pos, wl.m, wl.k, scale, out_dtype=torch.float32)
+    assert csa.csa_check_status(ws) == 0
+    dec = SplitCacheDecode(wl.m, wl.k, wl.W, scale)
+    xs = []
+    for r in range(world):
+        x = split_cache(g, r, world)
+        x["pos"] = pos
+        xs.append(x)
+    O, lse, idx, sc = emulated_split_decode(dec, xs)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_ref) and torch.equal(sc, sc_ref)
+    assert_attention_close(O, O_ref.double().cpu().numpy(), "split-cache decode over %d ranks" % world)
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_ref.cpu().numpy(), atol=1e-4)

@@ -104,3 +104,49 @@ def test_emulated_ranks_equal_torch_ranks_on_cpu():
         for c in chunks_of(r, world):
             got = O1e[r][c].contiguous().view(torch.int16).numpy().view(np.uint16)
             np.testing.assert_array_equal(got, O1w[c * C:(c + 1) * C])
+
+
+# ------------------------------------------------------------------ split-cache decode on two gloo ranks
+DEC = inputs.Workload("split_dec_small", H=4, d=64, m=4, k=16, W=32, HI=4, dI=64, batch=2, context=4096, seed=61)
+
+
+def _decode_rank_main(rank, world, port, outdir):
+    import torch.distributed as dist
+    from long_context_compressed_gated_b200.sharded import SplitCacheDecode, split_cache
+    from tests import oracle_ops
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank, world_size=world)
+    try:
+        batch = inputs.decode_batch(DEC)
+        batch["pos"] = [DEC.context - 1, 3000]
+        dec = SplitCacheDecode(DEC.m, DEC.k, DEC.W, 1.0 / math.sqrt(DEC.d), ops=oracle_ops)
+        x = split_cache(batch, rank, world)
+        x["pos"] = batch["pos"]
+        O, lse, idx, sc = dec.run(x, TorchComm())
+        torch.save({"O": O, "idx": idx}, os.path.join(outdir, "dec%d.pt" % rank))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_cache_decode_on_two_gloo_ranks():
+    """Each rank searches its half of the cache; one all-gather of candidates, an
+    identical merge, attention over its own selected entries (+ the window on the
+    last rank), an all-gather of the partial outputs and their log-sum-exp combine:
+    equal to the oracle's decode over the whole cache."""
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_decode_rank_main, args=(world, _free_port(), d), nprocs=world, join=True,
+                           start_method="spawn")
+        res = [torch.load(os.path.join(d, "dec%d.pt" % r)) for r in range(world)]
+    batch = inputs.decode_batch(DEC)
+    pos = [DEC.context - 1, 3000]
+    scale = 1.0 / math.sqrt(DEC.d)
+    for b, t in enumerate(pos):
+        I = oracle.indexer(batch["qI_codes"][b:b + 1], batch["qI_scales"][b:b + 1], batch["w_codes"][b:b + 1],
+                           batch["kI_codes"][b], batch["kI_scales"][b], t, DEC.m)
+        want_idx, _ = oracle.topk(I, oracle.n_vis([t], DEC.m), DEC.k)
+        o, _ = oracle.attention(batch["q"][b:b + 1], batch["Kc"][b], batch["Vc"][b], batch["Kwin"][b],
+                                batch["Vwin"][b], t, DEC.m, DEC.W, scale, sel=want_idx, rows=[0],
+                                raw_pos0=t - DEC.W + 1)
+        for r in range(world):
+            np.testing.assert_array_equal(res[r]["idx"][b].numpy(), want_idx[0])
+            np.testing.assert_allclose(res[r]["O"][b].numpy(), o[0], atol=1e-5)
