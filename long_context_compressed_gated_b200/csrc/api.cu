@@ -56,6 +56,18 @@ EncodeFn get_encode_fn() {
   return fn;
 }
 
+// Streaming multiprocessors of the current device (queried once per device).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
 namespace {
 
 thread_local int g_last_cuda_error = 0;
@@ -112,17 +124,6 @@ cudaError_t upload_positions(int64_t* dst, const int64_t* host, int B, cudaStrea
   return cudaGetLastError();
 }
 
-// Streaming multiprocessors of the current device (queried once per device).
-int sm_count() {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
-  if (dev < 64 && cached[dev] > 0) return cached[dev];
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  if (dev < 64) cached[dev] = n;
-  return n;
-}
 
 bool valid_odtype(int t) { return t == CSA_BF16 || t == CSA_F32; }
 
@@ -209,11 +210,8 @@ int csa_compress(const void* K, const void* V, const void* Z, const float* B, in
                  void* Vc, csa_stream_t stream) {
   if (T < 0 || m < 1) return CSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return CSA_ERR_UNSUPPORTED_SHAPE;
-  // rows per thread L and slices S = m / L with (d/8) * S <= 256 threads per block
-  const int CG = d / 8;
-  int L = m <= 8 ? m : 8;
-  while ((int64_t)CG * (m / L) > 256) L *= 2;
-  if (m % L != 0 || m > 4096) return CSA_ERR_UNSUPPORTED_SHAPE;
+  // m <= 8 or a multiple of 8 up to 512: the pooling's slices then tile a block
+  if (m > 512 || (m > 8 && m % 8 != 0)) return CSA_ERR_UNSUPPORTED_SHAPE;
   if (T / m == 0) return CSA_OK;
   int rc = check_ptrs(K, V, Z, B, Kc, Vc);
   if (rc) return rc;
@@ -628,9 +626,7 @@ int csa_decode_append(const void* K_new, const void* V_new, const void* Z_new, c
                       void* Zblk, void* Kc, void* Vc, uint8_t* kI_codes, uint8_t* kI_scales, csa_stream_t stream) {
   if (B < 0 || Ncap < 0 || m < 1 || m > 4096 || W < 0 || W > 1024) return CSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return CSA_ERR_UNSUPPORTED_SHAPE;
-  int L, S;
-  pool_shape(d, m, &L, &S);
-  if (m % L != 0) return CSA_ERR_UNSUPPORTED_SHAPE;
+  if (m > 8 && m % 8 != 0) return CSA_ERR_UNSUPPORTED_SHAPE;
   const bool with_ki = kI_codes_new || kI_scales_new || kI_codes || kI_scales;
   if (with_ki && (dI != 64 && dI != 128)) return CSA_ERR_UNSUPPORTED_SHAPE;
   if (B == 0) return CSA_OK;

@@ -24,8 +24,8 @@ namespace csa {
 
 namespace {
 
-constexpr int kAppendThreads = 256;
-constexpr int kChunksPerThread = 16;  // 16-byte chunks each thread holds per shift round
+constexpr int kMinThreads = 256;      // at least; more when the pooling group of a block is larger
+constexpr int kChunksPerThread = 4;   // 16-byte chunks each thread holds per shift round
 constexpr int kMaxSeqPerLaunch = 64;
 
 struct AppendPos {
@@ -44,10 +44,12 @@ struct AppendArgs {
   uint8_t *kIc, *kIs;                 // [B, Ncap, dI/2], [B, Ncap, dI/32] or null
 };
 
-__global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(const AppendArgs a, const AppendPos P,
-                                                                       int b0) {
-  __shared__ Gate8 sh[kAppendThreads];
-  const int tid = threadIdx.x;
+// blockDim.x = max(256, the pooling group of a block); shared memory:
+// kGateWords floats per thread for the slice merge.
+__global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const AppendArgs a, const AppendPos P,
+                                                                        int b0) {
+  extern __shared__ __align__(16) float sh_gate[];
+  const int tid = threadIdx.x, nthr = blockDim.x;
   const int64_t b = b0 + blockIdx.x;
   const int64_t pos = P.v[blockIdx.x];
   const int d = a.d, CH = d / 8;  // 16-byte chunks per row
@@ -59,12 +61,12 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(const App
   if (a.W > 0) {
     uint4* kw = reinterpret_cast<uint4*>(a.Kwin + b * (int64_t)a.W * d);
     uint4* vw = reinterpret_cast<uint4*>(a.Vwin + b * (int64_t)a.W * d);
-    const int R = kAppendThreads * kChunksPerThread / (2 * CH);  // rows per round
+    const int R = nthr * kChunksPerThread / (2 * CH);  // rows per round
     for (int r0 = 1; r0 < a.W; r0 += R) {
       uint4 v[kChunksPerThread];
 #pragma unroll
       for (int u = 0; u < kChunksPerThread; ++u) {
-        const int c = u * kAppendThreads + tid;  // chunk of the round: [matrix][row][chunk]
+        const int c = u * nthr + tid;  // chunk of the round: [matrix][row][chunk]
         const int mat = c / (R * CH), rr = (c / CH) % R, ch = c % CH;
         const int row = r0 + rr;
         if (row < a.W) v[u] = (mat ? vw : kw)[(int64_t)row * CH + ch];
@@ -72,7 +74,7 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(const App
       __syncthreads();
 #pragma unroll
       for (int u = 0; u < kChunksPerThread; ++u) {
-        const int c = u * kAppendThreads + tid;
+        const int c = u * nthr + tid;
         const int mat = c / (R * CH), rr = (c / CH) % R, ch = c % CH;
         const int row = r0 + rr;
         if (row < a.W) (mat ? vw : kw)[(int64_t)(row - 1) * CH + ch] = v[u];
@@ -90,9 +92,9 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(const App
   const int64_t blk_base = b * (int64_t)a.m * d;
   if (slot == a.m - 1) {
     const int64_t j = (pos + 1) / a.m - 1;
-    const int tpb = CH * a.S;
-    pool_block(a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.Bias, d, a.L, a.S, tid,
-               tid < tpb, true, sh, a.Kc + (b * a.Ncap + j) * d, a.Vc + (b * a.Ncap + j) * d);
+    const int tpb = (d / kPoolChan) * a.S;
+    pool_block<true>(a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.Bias, d, a.L, a.S, tid, tid,
+               nthr, tid < tpb, true, sh_gate, a.Kc + (b * a.Ncap + j) * d, a.Vc + (b * a.Ncap + j) * d);
     if (a.kIc != nullptr) {
       const int cb = a.dI / 2, sb = a.dI / 32;
       if (tid < cb / 4)
@@ -137,11 +139,19 @@ cudaError_t launch_decode_append(const void* Kn, const void* Vn, const void* Zn,
   a.Vc = static_cast<__nv_bfloat16*>(Vc);
   a.kIc = kIc;
   a.kIs = kIs;
+  const int tpb = (d / kPoolChan) * a.S;
+  const int threads = tpb > kMinThreads ? tpb : kMinThreads;
+  const size_t smem = (size_t)threads * kGateWords * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPoolMaxThreads * kGateWords * (int)sizeof(float));
+    if (e != cudaSuccess) return e;
+  }
   for (int b0 = 0; b0 < B; b0 += kMaxSeqPerLaunch) {
     AppendPos P{};
     const int n = B - b0 < kMaxSeqPerLaunch ? B - b0 : kMaxSeqPerLaunch;
     for (int i = 0; i < n; ++i) P.v[i] = pos[b0 + i];
-    decode_append_kernel<<<n, kAppendThreads, 0, stream>>>(a, P, b0);
+    decode_append_kernel<<<n, threads, smem, stream>>>(a, P, b0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

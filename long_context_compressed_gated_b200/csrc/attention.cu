@@ -367,16 +367,31 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
           const uint8_t* codes = (which ? a.vc8 : a.kc8) + kc_base * D + c * 8;
           const uint8_t* scl = (which ? a.vc8_scales : a.kc8_scales) + kc_base * (D / 32) + c / 4;
           const uint32_t d0 = smem_u32(dst) + dst_lane;
-          for (int x = r0; x < tl.width; x += RSTEP) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (x < tl.valid) {
-              const int j = sel[x];
-              const uint2 cw = __ldg(reinterpret_cast<const uint2*>(codes + (int64_t)j * D));
-              v = dequant_e4m3x8(cw, __ldg(scl + (int64_t)j * (D / 32)));
+          // eight rows' loads are in flight before any of them is converted
+          for (int x0 = r0; x0 < tl.width; x0 += 8 * RSTEP) {
+            uint2 cw[8];
+            uint32_t sb[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int x = x0 + u * RSTEP;
+              cw[u] = make_uint2(0u, 0u);
+              sb[u] = 0u;
+              if (x < tl.valid) {
+                const int j = sel[x];
+                cw[u] = __ldg(reinterpret_cast<const uint2*>(codes + (int64_t)j * D));
+                sb[u] = __ldg(scl + (int64_t)j * (D / 32));
+              }
             }
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d0 + (uint32_t)(x - r0) * 128), "r"(v.x),
-                         "r"(v.y), "r"(v.z), "r"(v.w)
-                         : "memory");
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int x = x0 + u * RSTEP;
+              if (x < tl.width) {
+                const uint4 v = x < tl.valid ? dequant_e4m3x8(cw[u], sb[u]) : make_uint4(0u, 0u, 0u, 0u);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d0 + (uint32_t)(x - r0) * 128),
+                             "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                             : "memory");
+              }
+            }
           }
           fence_proxy_async_smem();  // generic-proxy stores -> tcgen05 (async proxy) reads
           mbar_arrive(fullb);

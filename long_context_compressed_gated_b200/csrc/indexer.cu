@@ -47,9 +47,18 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kEpiWarps = 8;
-constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kThreads = 64 + kEpiThreads;
+// Epilogue warps: 8 in prefill (two halves of four, one per TMEM lane quarter,
+// owning half of the group's tokens each); 16 in decode with up to 32 indexer
+// heads (four groups of four that take turns on the key tiles, so that four
+// tiles' epilogues are in flight; with 64 heads the weights need the registers of
+// the 8-warp layout, where two groups take turns).
+template <int HI, int G>
+struct Epi {
+  static constexpr int kWarps = (G == 1 && HI <= 32) ? 16 : 8;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kGroups = kWarps / 4;  // 4-warp groups (one warp per lane quarter)
+  static constexpr int kBlock = 64 + kThreads;
+};
 constexpr uint32_t kMagicBits = 0x48400000u;  // bit pattern of 196608.0f
 constexpr int kHalfBar0 = 1;                  // named barriers 1, 2: the four warps of each half
 constexpr int kEpiBar = 3;                    // named barrier 3: all epilogue warps
@@ -170,7 +179,7 @@ struct IndexerSmem {
 };
 
 template <int HI, int DI, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
     indexer_topk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                         const IndexerArgs a) {
   using L = IndexerSmem<HI, DI, G>;
@@ -189,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NSG = NST / TPG, NBG = NB / TPG;  // stage groups, buffer groups
   static_assert(NST % TPG == 0 && NB % TPG == 0, "barrier groups");
   constexpr int G0 = kAlt ? 1 : G / 2;   // tokens per half
+  constexpr int kEpiWarps = Epi<HI, G>::kWarps, kEpiThreads = Epi<HI, G>::kThreads, kThreads = Epi<HI, G>::kBlock;
+  constexpr int NQ = Epi<HI, G>::kGroups;    // decode: groups that take turns on the tiles
   static_assert(kAlt || (G % 2 == 0 && G0 <= 4 && (G0 * HI) % 16 == 0), "token split between halves");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < NBG; ++b) {
       mbar_init(&dfull[b], 1);
-      mbar_init(&dempty[b], TPG * (kAlt ? kEpiWarps / 2 : kEpiWarps));
+      mbar_init(&dempty[b], TPG * (kAlt ? 4 : kEpiWarps));  // the warps that read a tile
     }
     mbar_init(ready, kEpiWarps + 1);
     mbar_init(mma_fin, 1);
@@ -510,8 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // meetings for cut-backs: every `check` tiles (rounds of one tile, or of two
     // alternate tiles) and after the last one
-    const int nrounds = kAlt ? (ntiles + 1) / 2 : ntiles;
-    const int rounds_per_meet = kAlt ? (a.check >= 2 ? a.check / 2 : 1) : a.check;
+    const int nrounds = kAlt ? (ntiles + NQ - 1) / NQ : ntiles;
+    const int rounds_per_meet = kAlt ? (a.check >= NQ ? a.check / NQ : 1) : a.check;
     // insertion of a tile is finished one tile later, so that the latency of the
     // buffer reservation (shared atomic) hides behind the next tile's head sums
     uint64_t pkey[G0];
@@ -560,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // insertion work; the blocking wait runs only when the probe saw it incomplete.
     bool next_ready = false;
     for (int rd = 0; rd < nrounds; ++rd) {
-      const int it = kAlt ? 2 * rd + half : rd;
+      const int it = kAlt ? NQ * rd + half : rd;
       if (it < ntiles && !dead && it / TPG != seen_group) {
         seen_group = it / TPG;
         if (!next_ready)
@@ -592,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&dempty[(it / TPG) % NBG]);
         {
-          const int itn = kAlt ? it + 2 : it + 1, gn = itn / TPG;
+          const int itn = kAlt ? it + NQ : it + 1, gn = itn / TPG;
           next_ready = itn < ntiles && gn != seen_group && mbar_test(&dfull[gn % NBG], (gn / NBG) & 1);
         }
         finish_insert();  // previous tile's stores
@@ -628,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // back if the next `check` tiles could overflow it
       finish_insert();
       topk::named_sync(gbar, GNT);
-      const int tiles_done = min(ntiles, kAlt ? 2 * (rd + 1) : rd + 1);
+      const int tiles_done = min(ntiles, kAlt ? NQ * (rd + 1) : rd + 1);
       for (int t = 0; t < G0; ++t) {  // every warp of the group cuts back each of its buffers
         const int gg = g_lo + t;
         uint64_t* buf = s_cand + (size_t)gg * cap;
@@ -1048,7 +1059,7 @@ static bool choose_cap(int k, int* cap, int* check) {
       return true;
     }
   }
-  for (int c = 4; c >= (G == 1 ? 2 : 1); c >>= 1) {
+  for (int c = 4; c >= (G == 1 ? Epi<HI, G>::kGroups : 1); c >>= 1) {
     int cp;
     if (fit(c, &cp)) {
       *cap = cp;
@@ -1073,7 +1084,7 @@ static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, In
   auto kern = indexer_topk_kernel<HI, DI, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(qmap, kmap, a);
+  kern<<<grid, Epi<HI, G>::kBlock, smem, stream>>>(qmap, kmap, a);
   return cudaGetLastError();
 }
 

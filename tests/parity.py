@@ -24,10 +24,10 @@ def from_words(w, device):
 
 def _pool_shape(d, m):
     """Rows per thread L and slices S of the GPU pooling of one block (the launch
-    rule of the compression kernel: L = min(m, 8), doubled while (d/8) * (m/L) >
-    256 threads)."""
-    L = m if m <= 8 else 8
-    while (d // 8) * (m // L) > 256:
+    rule of the compression kernel: L = m up to 8, else 4, doubled while
+    (d/4) * (m/L) > 512 threads)."""
+    L = m if m <= 8 else 4
+    while (d // 4) * (m // L) > 512:
         L *= 2
     return L, m // L
 
@@ -38,9 +38,10 @@ def fp32_pool_slack(x_bf16, m, Z, B):
     and the kernel's L rows per slice and S slices:
       every weight exp(g_i - M) carries a relative error of at most
         u*G (rounding of z + b) + (L + S) * (2*u*G + 4*u)
-      (each of the at most L-1 in-slice rescales and S-1 slice merges multiplies
-      it by one more exp of a rounded difference: 2uG for the difference, 4u for
-      expf's 2-ulp bound); a relative weight error eta moves a weighted mean by at
+      (each of the at most L-1 in-slice rescales and of the slice merges on its
+      path - ceil(log2 S) <= S-1 in the kernel's pairwise tree - multiplies it by
+      one more exp of a rounded difference: 2uG for the difference, 4u for expf's
+      2-ulp bound); a relative weight error eta moves a weighted mean by at
       most 2*eta*X; the m-term sums of numerator and denominator plus the L
       rescale products add (m + L) * u * X each; the division and the final
       product 2*u*X.  Total:
