@@ -595,7 +595,7 @@ def oracle_other_configs():
     return out
 
 
-EXTRA_CASES = ("hca_prefill", "csa_decode", "stack", "fp8_decode", "append", "quantize")
+EXTRA_CASES = ("hca_prefill", "csa_decode", "stack", "fp8_decode", "append", "quantize", "compress")
 
 
 def _event_ms(fn, reps, warmup=3):
@@ -673,6 +673,25 @@ def run_quantize(csa, steps):
     return out
 
 
+def run_compress(csa, wl, steps):
+    """The gated compression of the HCA prefill workload alone (m' = 128, 131072
+    tokens: 100 MB of K, V, Z).  The inputs fit in L2, so every step first
+    overwrites a 256 MB buffer; its own time, measured alone, is subtracted."""
+    d = inputs.prefill_layer(wl, device="cuda", with_indexer=False, with_q=False)
+    Kc = torch.empty(wl.T // wl.m_hca, wl.d, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        flush.zero_()
+        csa.csa_compress(d["K"], d["V"], d["Z"], d["B_hca"], wl.m_hca, Kc=Kc, Vc=Vc)
+
+    reps = max(20, steps)
+    ms = _event_ms(step, reps) - _event_ms(lambda: flush.zero_(), reps)
+    by = 3 * wl.T * wl.d * 2 + 2 * (wl.T // wl.m_hca) * wl.d * 2 + wl.m_hca * wl.d * 4
+    return {"ms": ms, "bytes": by}
+
+
 def run_extra(name, csa, peaks, steps, warmup, T=None):
     """One of the workloads reported under "workloads" (T overrides its length)."""
     import dataclasses
@@ -707,6 +726,12 @@ def run_extra(name, csa, peaks, steps, warmup, T=None):
         r = run_append(csa, inputs.CSA_DECODE, steps)
         return {"csa_decode_append_B16": {"us_per_step": r["us_per_step"], "bytes": r["bytes"],
                                           "gbs": r["bytes"] / (r["us_per_step"] * 1e-6) / 1e9}}
+    if name == "compress":
+        w2 = inputs.HCA_PREFILL if T is None else dataclasses.replace(inputs.HCA_PREFILL, T=T)
+        r = run_compress(csa, w2, steps)
+        gbs = r["bytes"] / (r["ms"] * 1e-3) / 1e9
+        return {"compress_hca_T%d_m%d" % (w2.T, w2.m_hca): {"ms": r["ms"], "bytes": r["bytes"], "gbs": gbs,
+                                                           "frac_hbm": gbs / peaks["hbm_gbs"], "l2": "flushed"}}
     if name == "quantize":
         return {"quantize": {k: dict(v, frac_hbm=v["gbs"] / peaks["hbm_gbs"]) for k, v in run_quantize(csa, steps).items()}}
     if name == "stack":

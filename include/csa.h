@@ -252,11 +252,13 @@ int csa_decode_fp8(const void* q, const uint8_t* qI_codes, const uint8_t* qI_sca
  * visible entries, then attention over the selection plus the window).  Rank r
  * holds entries [j_base, j_base + Nloc) of each sequence and runs:
  *   1. csa_decode_search: its slice's k best as exact 64-bit keys, keys [B, k]
- *      u64 (score << 32 | ~j, j the GLOBAL entry; 0 = none, after the valid
- *      ones), over the visible entries j < floor((pos+1)/m);
+ *      u64 (score << 32 | ~j, j the GLOBAL entry) in rank order (score desc,
+ *      j asc; 0 = none, after the valid ones), over the visible entries
+ *      j < floor((pos+1)/m);
  *   2. (all-gather of the keys; every rank then holds [B, L, k])
- *   3. csa_topk_merge: the exact top-k of the L lists per sequence, in rank
- *      order (score desc, j asc), idx [B, k] int32 (global, -1 padding),
+ *   3. csa_topk_merge: the exact top-k of the L lists per sequence (each list
+ *      in rank order, as csa_decode_search writes it), in rank order (score
+ *      desc, j asc), idx [B, k] int32 (global, -1 padding),
  *      scores [B, k] f32 (nullable), keys_out [B, k] (nullable); identical on
  *      every rank;
  *   4. csa_decode_attend: attention over the selected entries that lie in its

@@ -45,7 +45,7 @@ struct AppendArgs {
 };
 
 // blockDim.x = max(256, the pooling group of a block); shared memory:
-// kGateWords floats per thread for the slice merge.
+// pool_smem_bytes (the staged rows of the pooling, then its merge slots).
 __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const AppendArgs a, const AppendPos P,
                                                                         int b0) {
   extern __shared__ __align__(16) float sh_gate[];
@@ -92,9 +92,29 @@ __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const Ap
   const int64_t blk_base = b * (int64_t)a.m * d;
   if (slot == a.m - 1) {
     const int64_t j = (pos + 1) / a.m - 1;
-    const int tpb = (d / kPoolChan) * a.S;
-    pool_block<true>(a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.Bias, d, a.L, a.S, tid, tid,
-               nthr, tid < tpb, true, sh_gate, a.Kc + (b * a.Ncap + j) * d, a.Vc + (b * a.Ncap + j) * d);
+    // the pooling of the prefill compression (same thread layout, same
+    // arithmetic): the staged rows 0..m-2 and the token's own row m-1
+    const int CG = d / kPoolChan, tpb = CG * a.S;
+    const bool in_group = tid < tpb;
+    const int s = tid / CG, c0 = (tid % CG) * kPoolChan;
+    Gate4 st;
+    if (a.L <= kPoolStageRows) {
+      __nv_bfloat16* sm = reinterpret_cast<__nv_bfloat16*>(sh_gate);
+      pool_stage_rows(a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.m - 1, a.m, d, sm, tid,
+                      nthr);
+      if (in_group)
+        pool_slice_staged(st, sm, (size_t)a.m * d, a.Bias, d, a.L, s, c0);
+      else
+        gate_init(st);
+      if (a.S > 1) __syncthreads();  // the merge slots reuse the staged rows
+    } else if (in_group) {
+      pool_slice_direct<true>(st, a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.Bias, d, a.m,
+                              a.L, s, c0);
+    } else {
+      gate_init(st);
+    }
+    if (a.S > 1) gate_tree(st, sh_gate, nthr, tid, s, CG, a.S, in_group);
+    if (in_group && s == 0) gate_store(st, a.Kc + (b * a.Ncap + j) * d + c0, a.Vc + (b * a.Ncap + j) * d + c0);
     if (a.kIc != nullptr) {
       const int cb = a.dI / 2, sb = a.dI / 32;
       if (tid < cb / 4)
@@ -141,10 +161,10 @@ cudaError_t launch_decode_append(const void* Kn, const void* Vn, const void* Zn,
   a.kIs = kIs;
   const int tpb = (d / kPoolChan) * a.S;
   const int threads = tpb > kMinThreads ? tpb : kMinThreads;
-  const size_t smem = (size_t)threads * kGateWords * sizeof(float);
+  const size_t smem = pool_smem_bytes(a.L, a.S, m, d, 1, threads);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kPoolMaxThreads * kGateWords * (int)sizeof(float));
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolMaxSmem);
     if (e != cudaSuccess) return e;
   }
   for (int b0 = 0; b0 < B; b0 += kMaxSeqPerLaunch) {

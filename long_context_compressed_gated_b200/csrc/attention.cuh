@@ -37,6 +37,10 @@ struct AttnArgs {
   // [rows, d/32]; when set, the selected rows are dequantised (exactly) into the
   // bf16 tiles instead of copied from Kc / Vc
   const uint8_t *kc8, *kc8_scales, *vc8, *vc8_scales;
+  // set by launch_attention: work items (prefill token groups) and the number of
+  // item descriptions kept in shared memory (2: the next one is built ahead)
+  int64_t nitems;
+  int slots;
 };
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);

@@ -8,25 +8,37 @@
 //   Kc[c] = sum_p a_p K[p,c],  Vc[c] = sum_p a_p V[p,c].
 //
 // Thread layout of one block: (d/4) * S threads, thread r = s*(d/4) + cg owns
-// channels 4cg..4cg+3 (one 8-byte load per row and array, so a warp reads a
-// whole 256-byte row) of the slice of L consecutive rows s*L .. s*L+L-1.  A
-// slice is pooled in chunks of up to four rows: all of a chunk's loads are
-// issued first, then the chunk's maximum logit per channel (a rescale of the
-// running sums only when it grows), then one exp per element.  The S slices
-// merge pairwise in a fixed tree through shared memory.  Every arithmetic
-// step is an explicit IEEE operation (no contraction left to the compiler),
-// so all callers produce the same bits for a block.
+// channels 4cg..4cg+3 of the slice of L consecutive rows s*L .. s*L+L-1 (a
+// warp covers whole 256-byte rows).  A slice is pooled in chunks of up to four
+// rows: the chunk's base-2 logits g2 = (z + b) * log2(e) and their maximum per
+// channel first (the running sums are rescaled only when it grows), then one
+// exp2 per element, w = exp2(g2 - max) (exp2f: 2 ulp).  The S slices merge
+// pairwise in a fixed tree through shared memory.  Every arithmetic step is an
+// explicit IEEE operation (no contraction left to the compiler), so all
+// callers produce the same bits for a block.
+//
+// Row sources: a CTA whose slices have at most kPoolStageRows rows first copies
+// all of its rows into shared memory with 16-byte cp.async (every load of the
+// CTA in flight at once, no registers held) and pools from there; longer
+// slices load each chunk's rows from global memory into registers.
 #pragma once
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
-constexpr int kPoolChan = 4;          // channels per thread
-constexpr int kPoolChunk = 4;         // rows per chunk of loads
+constexpr int kPoolChan = 4;           // channels per thread
+constexpr int kPoolChunk = 4;          // rows per chunk
 constexpr int kPoolMaxThreads = 512;   // threads of one block's group
 constexpr int kGateWords = 4 * kPoolChan;
+constexpr float kPoolLog2e = 1.44269504088896341f;  // log2(e), rounded to fp32
+constexpr int kPoolStageRows = 8;      // slices of at most this many rows are staged
+// rows of K, V, Z a CTA stages: 512 threads x 8 rows x 4 channels = 16384
+// elements per array, 96 KB
+constexpr int kPoolMaxSmem = 3 * kPoolMaxThreads * kPoolStageRows * kPoolChan * 2;
 
-// Online-softmax state of 4 channels: running max, denominator, two sums.
+// Online-softmax state of 4 channels: running max (of base-2 logits),
+// denominator, two sums.
 struct Gate4 {
   float mx[kPoolChan], den[kPoolChan], k[kPoolChan], v[kPoolChan];
 };
@@ -35,8 +47,9 @@ __device__ __forceinline__ float& gate_word(Gate4& st, int w) {
   return w < 4 ? st.mx[w] : (w < 8 ? st.den[w - 4] : (w < 12 ? st.k[w - 8] : st.v[w - 12]));
 }
 
-__device__ __forceinline__ void bf16x4(const uint2 u, float (&f)[4]) {
-  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+__device__ __forceinline__ void gate_init(Gate4& st) {
+#pragma unroll
+  for (int e = 0; e < kPoolChan; ++e) st.mx[e] = -INFINITY, st.den[e] = st.k[e] = st.v[e] = 0.f;
 }
 
 // Merge b into a (both normalised to their own running max).
@@ -45,7 +58,7 @@ __device__ __forceinline__ void gate_merge(Gate4& a, const Gate4& b) {
   for (int e = 0; e < kPoolChan; ++e) {
     const float m = fmaxf(a.mx[e], b.mx[e]);
     if (m == -INFINITY) continue;
-    const float sa = expf(__fsub_rn(a.mx[e], m)), sb = expf(__fsub_rn(b.mx[e], m));
+    const float sa = exp2f(__fsub_rn(a.mx[e], m)), sb = exp2f(__fsub_rn(b.mx[e], m));
     a.den[e] = __fadd_rn(__fmul_rn(a.den[e], sa), __fmul_rn(b.den[e], sb));
     a.k[e] = __fadd_rn(__fmul_rn(a.k[e], sa), __fmul_rn(b.k[e], sb));
     a.v[e] = __fadd_rn(__fmul_rn(a.v[e], sa), __fmul_rn(b.v[e], sb));
@@ -53,19 +66,85 @@ __device__ __forceinline__ void gate_merge(Gate4& a, const Gate4& b) {
   }
 }
 
-// Pools rows s*L .. s*L+L-1 of a block (rows at K/V/Z + p*d, bias row p at
-// Bias + p*d), channels c0..c0+3.  With kSeparateLast the block's last row
-// (p = m-1) is read from (Klast, Vlast, Zlast): a caller that has not stored it
-// yet passes it separately.
-template <bool kSeparateLast>
-__device__ __forceinline__ void pool_slice(Gate4& st, const __nv_bfloat16* __restrict__ K,
-                                           const __nv_bfloat16* __restrict__ V, const __nv_bfloat16* __restrict__ Z,
-                                           const __nv_bfloat16* __restrict__ Klast,
-                                           const __nv_bfloat16* __restrict__ Vlast,
-                                           const __nv_bfloat16* __restrict__ Zlast, const float* __restrict__ Bias,
-                                           int d, int m, int L, int s, int c0) {
+// The arithmetic of one row, shared by both row sources: base-2 logits and the
+// chunk maximum; the rescale of the running sums when the maximum grows; the
+// weight exp2(g2 - max) accumulated into the denominator and the two sums.
+__device__ __forceinline__ void gate_logits(const uint2 zr, const float4 bb, float (&g2)[kPoolChan],
+                                            float (&cm)[kPoolChan]) {
+  const float z[4] = {bf16_lo(zr.x), bf16_hi(zr.x), bf16_lo(zr.y), bf16_hi(zr.y)};
+  const float b[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-  for (int e = 0; e < kPoolChan; ++e) st.mx[e] = -INFINITY, st.den[e] = st.k[e] = st.v[e] = 0.f;
+  for (int e = 0; e < kPoolChan; ++e) {
+    g2[e] = __fmul_rn(__fadd_rn(z[e], b[e]), kPoolLog2e);
+    cm[e] = fmaxf(cm[e], g2[e]);
+  }
+}
+__device__ __forceinline__ void gate_rescale(Gate4& st, const float (&cm)[kPoolChan]) {
+#pragma unroll
+  for (int e = 0; e < kPoolChan; ++e) {
+    if (cm[e] > st.mx[e]) {
+      const float sc = exp2f(__fsub_rn(st.mx[e], cm[e]));
+      st.den[e] = __fmul_rn(st.den[e], sc);
+      st.k[e] = __fmul_rn(st.k[e], sc);
+      st.v[e] = __fmul_rn(st.v[e], sc);
+      st.mx[e] = cm[e];
+    }
+  }
+}
+__device__ __forceinline__ void gate_accum(Gate4& st, const float (&g2)[kPoolChan], const uint2 kr, const uint2 vr) {
+  const float kf[4] = {bf16_lo(kr.x), bf16_hi(kr.x), bf16_lo(kr.y), bf16_hi(kr.y)};
+  const float vf[4] = {bf16_lo(vr.x), bf16_hi(vr.x), bf16_lo(vr.y), bf16_hi(vr.y)};
+#pragma unroll
+  for (int e = 0; e < kPoolChan; ++e) {
+    const float w = exp2f(__fsub_rn(g2[e], st.mx[e]));
+    st.den[e] = __fadd_rn(st.den[e], w);
+    st.k[e] = __fmaf_rn(w, kf[e], st.k[e]);
+    st.v[e] = __fmaf_rn(w, vf[e], st.v[e]);
+  }
+}
+
+// Copies rows [0, nrows) of Z, K, V (row r at X + r*d, rows contiguous; row
+// `last_row` - or none when negative - from Zlast, Klast, Vlast instead) into
+// shared memory as [Z, K, V][nrows][d] bf16, by all nthr threads of the CTA with
+// 16-byte cp.async (a flat copy of each array), and makes them visible to every
+// thread (CTA barrier: all threads call this).
+__device__ __forceinline__ void pool_stage_rows(const __nv_bfloat16* __restrict__ K,
+                                                const __nv_bfloat16* __restrict__ V,
+                                                const __nv_bfloat16* __restrict__ Z,
+                                                const __nv_bfloat16* __restrict__ Klast,
+                                                const __nv_bfloat16* __restrict__ Vlast,
+                                                const __nv_bfloat16* __restrict__ Zlast, int last_row, int nrows,
+                                                int d, __nv_bfloat16* sm, int tid, int nthr) {
+  const int per = nrows * d / 8;  // 16-byte chunks per array
+  const int last_lo = last_row >= 0 ? last_row * d / 8 : per, last_hi = last_lo + d / 8;
+#pragma unroll
+  for (int arr = 0; arr < 3; ++arr) {
+    const __nv_bfloat16* X = arr == 0 ? Z : (arr == 1 ? K : V);
+    const __nv_bfloat16* Xl = arr == 0 ? Zlast : (arr == 1 ? Klast : Vlast);
+    const uint32_t dst0 = sm100::smem_u32(sm + (size_t)arr * nrows * d);
+#pragma unroll 4
+    for (int c = tid; c < per; c += nthr) {
+      const __nv_bfloat16* src = (c >= last_lo && c < last_hi) ? Xl + (c - last_lo) * 8 : X + (size_t)c * 8;
+      sm100::cp_async16(dst0 + (uint32_t)c * 16u, src, 16u);
+    }
+  }
+  sm100::cp_async_wait_all();
+  __syncthreads();
+}
+
+// Pools rows s*L .. s*L+L-1 of a block, channels c0..c0+3, from global memory:
+// rows at K/V/Z + p*d, the block's last row (p = m-1) from (Klast, Vlast,
+// Zlast) when kSeparateLast.  Bias row p at Bias + p*d (the same rows for
+// every block: cache hits).
+template <bool kSeparateLast>
+__device__ __forceinline__ void pool_slice_direct(Gate4& st, const __nv_bfloat16* __restrict__ K,
+                                                  const __nv_bfloat16* __restrict__ V,
+                                                  const __nv_bfloat16* __restrict__ Z,
+                                                  const __nv_bfloat16* __restrict__ Klast,
+                                                  const __nv_bfloat16* __restrict__ Vlast,
+                                                  const __nv_bfloat16* __restrict__ Zlast,
+                                                  const float* __restrict__ Bias, int d, int m, int L, int s, int c0) {
+  gate_init(st);
   const int p_end = s * L + L;
 #pragma unroll 1
   for (int p0 = s * L; p0 < p_end; p0 += kPoolChunk) {
@@ -81,49 +160,42 @@ __device__ __forceinline__ void pool_slice(Gate4& st, const __nv_bfloat16* __res
         vr[i] = __ldg(reinterpret_cast<const uint2*>(last ? Vlast + c0 : V + off));
       }
     }
-    // the chunk's maximum logit per channel (the bias rows are shared by every
-    // block: cache hits, read where used to keep the registers for the rows)
+    float g2[kPoolChunk][kPoolChan];
     float cm[kPoolChan] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int i = 0; i < kPoolChunk; ++i) {
+    for (int i = 0; i < kPoolChunk; ++i)
+      if (p0 + i < p_end)
+        gate_logits(zr[i], __ldg(reinterpret_cast<const float4*>(Bias + (int64_t)(p0 + i) * d + c0)), g2[i], cm);
+    gate_rescale(st, cm);
+#pragma unroll
+    for (int i = 0; i < kPoolChunk; ++i)
+      if (p0 + i < p_end) gate_accum(st, g2[i], kr[i], vr[i]);
+  }
+}
+
+// The same from rows staged in shared memory: row p of the block's Z at
+// rowz + p*d, its K at + plane, its V at + 2*plane.
+__device__ __forceinline__ void pool_slice_staged(Gate4& st, const __nv_bfloat16* rowz, size_t plane,
+                                                  const float* __restrict__ Bias, int d, int L, int s, int c0) {
+  gate_init(st);
+  const int p_end = s * L + L;
+#pragma unroll 1
+  for (int p0 = s * L; p0 < p_end; p0 += kPoolChunk) {
+    float g2[kPoolChunk][kPoolChan];
+    float cm[kPoolChan] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < kPoolChunk; ++i)
+      if (p0 + i < p_end)
+        gate_logits(*reinterpret_cast<const uint2*>(rowz + (size_t)(p0 + i) * d + c0),
+                    __ldg(reinterpret_cast<const float4*>(Bias + (int64_t)(p0 + i) * d + c0)), g2[i], cm);
+    gate_rescale(st, cm);
+#pragma unroll
+    for (int i = 0; i < kPoolChunk; ++i)
       if (p0 + i < p_end) {
-        const float4 bb = __ldg(reinterpret_cast<const float4*>(Bias + (int64_t)(p0 + i) * d + c0));
-        float z[4];
-        bf16x4(zr[i], z);
-        cm[0] = fmaxf(cm[0], __fadd_rn(z[0], bb.x));
-        cm[1] = fmaxf(cm[1], __fadd_rn(z[1], bb.y));
-        cm[2] = fmaxf(cm[2], __fadd_rn(z[2], bb.z));
-        cm[3] = fmaxf(cm[3], __fadd_rn(z[3], bb.w));
+        const __nv_bfloat16* r = rowz + (size_t)(p0 + i) * d + c0;
+        gate_accum(st, g2[i], *reinterpret_cast<const uint2*>(r + plane),
+                   *reinterpret_cast<const uint2*>(r + 2 * plane));
       }
-    }
-#pragma unroll
-    for (int e = 0; e < kPoolChan; ++e) {
-      if (cm[e] > st.mx[e]) {  // rescale the running sums to the new maximum
-        const float sc = expf(__fsub_rn(st.mx[e], cm[e]));
-        st.den[e] = __fmul_rn(st.den[e], sc);
-        st.k[e] = __fmul_rn(st.k[e], sc);
-        st.v[e] = __fmul_rn(st.v[e], sc);
-        st.mx[e] = cm[e];
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kPoolChunk; ++i) {
-      if (p0 + i < p_end) {
-        const float4 bb = __ldg(reinterpret_cast<const float4*>(Bias + (int64_t)(p0 + i) * d + c0));
-        const float b[4] = {bb.x, bb.y, bb.z, bb.w};
-        float z[4], kf[4], vf[4];
-        bf16x4(zr[i], z);
-        bf16x4(kr[i], kf);
-        bf16x4(vr[i], vf);
-#pragma unroll
-        for (int e = 0; e < kPoolChan; ++e) {
-          const float w = expf(__fsub_rn(__fadd_rn(z[e], b[e]), st.mx[e]));
-          st.den[e] = __fadd_rn(st.den[e], w);
-          st.k[e] = __fmaf_rn(w, kf[e], st.k[e]);
-          st.v[e] = __fmaf_rn(w, vf[e], st.v[e]);
-        }
-      }
-    }
   }
 }
 
@@ -168,40 +240,22 @@ __device__ __forceinline__ void gate_store(const Gate4& st, __nv_bfloat16* __res
   *reinterpret_cast<uint2*>(Vc) = make_uint2(pack_bf16x2(vf[0], vf[1]), pack_bf16x2(vf[2], vf[3]));
 }
 
-// Gated pooling of one block by its group of (d/4)*S threads (r = this
-// thread's index in the group, tid its index in the CTA, nthr the CTA's
-// threads); kSeparateLast as for pool_slice (the same bits either way).  Every thread of the CTA must call this when S > 1; threads
-// outside a group pass in_group = false, inactive groups active = false.
-template <bool kSeparateLast>
-__device__ __forceinline__ void pool_block(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
-                                           const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restrict__ Klast,
-                                           const __nv_bfloat16* __restrict__ Vlast,
-                                           const __nv_bfloat16* __restrict__ Zlast, const float* __restrict__ Bias,
-                                           int d, int L, int S, int r, int tid, int nthr, bool in_group, bool active,
-                                           float* sh, __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Vc) {
-  const int m = L * S;
-  const int CG = d / kPoolChan;
-  const int s = r / CG, c0 = (r % CG) * kPoolChan;
-  active = active && in_group;
-  Gate4 st;
-  if (active) {
-    pool_slice<kSeparateLast>(st, K, V, Z, Klast, Vlast, Zlast, Bias, d, m, L, s, c0);
-  } else {
-#pragma unroll
-    for (int e = 0; e < kPoolChan; ++e) st.mx[e] = -INFINITY, st.den[e] = st.k[e] = st.v[e] = 0.f;
-  }
-  if (S > 1) gate_tree(st, sh, nthr, tid, s, CG, S, in_group);
-  if (active && s == 0) gate_store(st, Kc + c0, Vc + c0);
-}
-
 // Rows per thread L and slices S = m / L of one block: L = m up to 8 rows, else
-// 4 (one chunk of loads per thread), doubled while the group would exceed 512
-// threads.
+// 4, doubled while the group would exceed 512 threads.
 __host__ __device__ inline void pool_shape(int d, int m, int* L, int* S) {
   int l = m <= 8 ? m : 4;
   while ((d / kPoolChan) * (m / l) > kPoolMaxThreads) l *= 2;
   *L = l;
   *S = m / l;
+}
+
+// Shared memory of a CTA of nthr threads pooling `blocks` blocks of m rows with
+// (L, S): the staged rows (L <= kPoolStageRows) - the merge slots reuse them -
+// else the merge slots only.  At most kPoolMaxSmem bytes.
+__host__ __device__ inline size_t pool_smem_bytes(int L, int S, int m, int d, int blocks, int nthr) {
+  const size_t stage = L <= kPoolStageRows ? (size_t)3 * blocks * m * d * 2 : 0;
+  const size_t merge = S > 1 ? (size_t)kGateWords * nthr * 4 : 0;
+  return stage > merge ? stage : merge;
 }
 
 }  // namespace csa

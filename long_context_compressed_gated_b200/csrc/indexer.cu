@@ -523,6 +523,11 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
     // alternate tiles) and after the last one
     const int nrounds = kAlt ? (ntiles + NQ - 1) / NQ : ntiles;
     const int rounds_per_meet = kAlt ? (a.check >= NQ ? a.check / NQ : 1) : a.check;
+    // when every key of the range fits its fixed slot, no buffer is ever cut back:
+    // no meetings at all (the final selection sees every visible key).  Only the
+    // groups of at most two tokens have the room for that (a run-time choice in
+    // the wider groups costs more than it saves: measured on the 8-token groups).
+    const bool meet = G > 2 || (int64_t)ntiles * 128 > cap;
     // insertion of a tile is finished one tile later, so that the latency of the
     // buffer reservation (shared atomic) hides behind the next tile's head sums
     uint64_t pkey[G0];
@@ -634,7 +639,7 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
             if (pbal[t]) pbase[t] = atomicAdd(&s_cnt[g_lo + t], __popc(pbal[t]));
         }
       }
-      if ((rd + 1) % rounds_per_meet != 0 && rd + 1 != nrounds) continue;
+      if (!meet || ((rd + 1) % rounds_per_meet != 0 && rd + 1 != nrounds)) continue;
       // meeting: the warps that insert into a buffer meet; the owner warp cuts it
       // back if the next `check` tiles could overflow it
       finish_insert();
@@ -659,6 +664,10 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
       for (int t = 0; t < G0; ++t) thr[t] = s_thr[g_lo + t];
     }
 
+    if (!meet) {
+      finish_insert();                 // (nothing pending: every key went to its fixed slot)
+      topk::named_sync(gbar, GNT);     // the group's fixed-slot stores, visible to the selection
+    }
     // final exact selection by the group, one buffer at a time: the k best keys of
     // this key range go out unsorted; topk_finalize_kernel merges the ranges and sorts
     for (int t = 0; t < G0; ++t) {
@@ -1030,8 +1039,9 @@ int inject_fault(int code) {
   return 0;
 }
 
-// Candidate capacity per token: whatever shared memory is left (cut-backs are
-// rarer the larger it is), at least k + 128*check and a power of two >= k.
+// Candidate capacity per token: all the shared memory that is left (cut-backs
+// are rarer the larger it is; a range whose keys all fit needs none, and no
+// meetings), at least k + 128*check and a power of two >= k.
 template <int HI, int DI, int G>
 static bool choose_cap(int k, int* cap, int* check) {
   using L = IndexerSmem<HI, DI, G>;
@@ -1042,8 +1052,7 @@ static bool choose_cap(int k, int* cap, int* check) {
   auto fit = [&](int c, int* cp) {
     const int need = k + 128 * c > p ? k + 128 * c : p;
     if (budget < need) return false;
-    int want = 4 * k + 128 * c;  // cut-backs rare: room for several k between them
-    if (want < 4096) want = 4096;
+    int want = budget;
     if (want < need) want = need;
     *cp = (want < budget ? want : budget) & ~127;
     if (*cp < need) *cp = ((need + 127) / 128) * 128;

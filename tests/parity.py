@@ -36,16 +36,19 @@ def fp32_pool_slack(x_bf16, m, Z, B):
     """Worst-case absolute error of the fp32 gated pooling, per (block, channel),
     with u = 2^-24, X = max |x| over the block, G = max |z + b| over the block,
     and the kernel's L rows per slice and S slices:
-      every weight exp(g_i - M) carries a relative error of at most
-        u*G (rounding of z + b) + (L + S) * (2*u*G + 4*u)
-      (each of the at most L-1 in-slice rescales and of the slice merges on its
-      path - ceil(log2 S) <= S-1 in the kernel's pairwise tree - multiplies it by
-      one more exp of a rounded difference: 2uG for the difference, 4u for expf's
-      2-ulp bound); a relative weight error eta moves a weighted mean by at
-      most 2*eta*X; the m-term sums of numerator and denominator plus the L
+      the kernel takes logits in base 2, g2 = RN(RN(z + b) * RN(log2 e)), so every
+      logit carries 3uG (the sum, the rounded constant, the product; an error
+      common to all logits of a block cancels in the normalised mean), and
+      every weight exp2(g2_i - max) a relative error of at most
+        3*u*G + (L + S) * (2*u*G + 4*u)
+      (its own exp2 and each of the at most L-1 in-slice rescales and of the
+      slice merges on its path - ceil(log2 S) <= S-1 in the kernel's pairwise
+      tree - is one exp2 of a rounded difference: 2uG for the difference, 4u for
+      exp2f's 2-ulp bound); a relative weight error eta moves a weighted mean by
+      at most 2*eta*X; the m-term sums of numerator and denominator plus the L
       rescale products add (m + L) * u * X each; the division and the final
       product 2*u*X.  Total:
-        u * X * (2*G*(1 + 2*(L+S)) + 8*(L+S) + 2*(m+L) + 2).
+        u * X * (2*G*(3 + 2*(L+S)) + 8*(L+S) + 2*(m+L) + 2).
     When the weighted sum cancels, this can exceed one bf16 ulp of the (small)
     result; otherwise the bf16 ulp dominates."""
     xf = x_bf16.detach().float().cpu().double().numpy() if hasattr(x_bf16, "detach") else oracle.bf16_words_to_f64(x_bf16)
@@ -58,7 +61,7 @@ def fp32_pool_slack(x_bf16, m, Z, B):
     G = np.abs(g).max(axis=1)
     L, S = _pool_shape(d, m)
     u = 2.0 ** -24
-    return u * X * (2 * G * (1 + 2 * (L + S)) + 8 * (L + S) + 2 * (m + L) + 2)
+    return u * X * (2 * G * (3 + 2 * (L + S)) + 8 * (L + S) + 2 * (m + L) + 2)
 
 
 def assert_within_bf16_ulp(got_bf16, exact_f64, what, slack=None):
