@@ -57,6 +57,9 @@ constexpr int kThreads = (kSchedWarp + 1) * 32;
 constexpr int kRoleWarps = kSchedWarp;    // warps that consume work items (all but the scheduler)
 constexpr float kRescaleSlack = 8.0f;  // raise the running max only when it grows by > 2^8
 constexpr int kSoftmaxBar = 1;         // named barrier of the softmax warps (end of kernel)
+// V ring depth (K has 2): 3 when P lives in tensor memory (V of tile i+3 loads
+// while PV of tile i runs), 2 when P is staged in shared memory
+constexpr int kMaxVStages = 3;
 
 enum TileType : int { kSeg = 0, kHca = 1, kWin = 2 };
 
@@ -156,15 +159,22 @@ struct ItemInfo {
   int ntok, ntiles, valid, split;
 };
 
-template <int D>
+// P (the bf16 weights of a tile) goes either back into tensor memory, into the
+// tile's S columns, and PV reads A from there (TMEM_P: the softmax never waits for
+// PV; the S buffer is released by PV), or into a shared-memory tile (the softmax
+// waits for the previous PV before writing it; the S buffer is released as soon
+// as it has been read).  Measured: the first is faster for dense (HCA) tiles,
+// the second for selected-entry (CSA) tiles.
+template <int D, bool TMEM_P>
 struct AttnSmem {
   static constexpr int kHalf = kRows * 128;                // one 64-column half of a 128-row tile
   static constexpr int kTileBytes = (D / 64) * kHalf;      // 128 rows x D bf16
+  static constexpr int kVS = TMEM_P ? 3 : 2;               // V stages
   static constexpr size_t off_q = 0;
   static constexpr size_t off_k = off_q + kTileBytes;      // 2 stages
-  static constexpr size_t off_v = off_k + 2 * kTileBytes;  // 2 stages
-  static constexpr size_t off_p = off_v + 2 * kTileBytes;  // 128 x 128 bf16
-  static constexpr size_t off_info = off_p + 2 * kHalf;    // [2] ItemInfo
+  static constexpr size_t off_v = off_k + 2 * kTileBytes;  // kVS stages
+  static constexpr size_t off_p = off_v + kVS * kTileBytes;  // 128 x 128 bf16 (shared-memory P)
+  static constexpr size_t off_info = off_p + (TMEM_P ? 0 : 2 * kHalf);  // [2] ItemInfo
   static constexpr size_t off_tiles = off_info + 2 * 128;  // [2][kMaxSegTiles] SEG tiles, packed
   static constexpr size_t off_bar = off_tiles + 2 * kMaxSegTiles * 4;
   static constexpr size_t off_misc = off_bar + 32 * 8;
@@ -174,10 +184,11 @@ struct AttnSmem {
   static size_t bytes(int idx_entries, int slots) { return off_idx + (size_t)slots * idx_entries * 4 + 1024; }
 };
 
-template <int D, bool WANT_LSE>
+template <int D, bool WANT_LSE, bool TMEM_P>
 __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a,
                                                                 const __grid_constant__ AttnMaps maps) {
-  using L = AttnSmem<D>;
+  using L = AttnSmem<D, TMEM_P>;
+  constexpr int kVStages = L::kVS;
   constexpr int KSTEPS_QK = D / 16;
   constexpr int HALVES = D / 64;
   constexpr uint32_t kHalfBytes = kRows * 128;
@@ -193,17 +204,22 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
   uint64_t* q_full = bar + 0;
   uint64_t* k_full = bar + 1;     // [2]
   uint64_t* k_empty = bar + 3;    // [2]
-  uint64_t* v_full = bar + 5;     // [2]
-  uint64_t* v_empty = bar + 7;    // [2]
-  uint64_t* s_full = bar + 9;     // [2]
-  uint64_t* s_free = bar + 11;    // [2]
-  uint64_t* p_full = bar + 13;
-  uint64_t* pv_done = bar + 14;
-  uint64_t* mma_fin = bar + 15;   // every issued MMA complete (before TMEM is freed)
-  uint64_t* q_free = bar + 16;    // the QK products of an item complete: Q may be reloaded
-  uint64_t* o_free = bar + 17;    // an item's output read out of TMEM: the next PV may start
-  uint64_t* list_full = bar + 18;  // [2] an item's description is ready in its slot
-  uint64_t* list_free = bar + 20;  // [2] every role is done with the slot
+  uint64_t* v_full = bar + 5;     // [kVStages] (kMaxVStages reserved)
+  uint64_t* v_empty = bar + 8;    // [kVStages]
+  uint64_t* s_full = bar + 11;    // [2]
+  uint64_t* s_free = bar + 13;    // [2] S buffer (and the P it then holds) consumed by PV
+  // [2] P of a tile written, by tile parity: a softmax warp may finish tile i+1
+  // before another has finished tile i (nothing makes it wait for PV any more)
+  uint64_t* p_full = bar + 15;
+  uint64_t* pv_done = bar + 17;
+  uint64_t* mma_fin = bar + 18;   // every issued MMA complete (before TMEM is freed)
+  uint64_t* q_free = bar + 19;    // the QK products of an item complete: Q may be reloaded
+  // the output of an item with tiles read out of TMEM: the next such item's PV may
+  // start (an item without tiles leaves TMEM alone and takes no part: its epilogue
+  // waits for nothing, so it could otherwise run two phases ahead of the MMA warp)
+  uint64_t* o_free = bar + 20;
+  uint64_t* list_full = bar + 21;  // [2] an item's description is ready in its slot
+  uint64_t* list_free = bar + 23;  // [2] every role is done with the slot
   int* misc = reinterpret_cast<int*>(smem + L::off_misc);  // [1] tmem
   volatile int* s_abort = misc + 48;  // set by the first wait that timed out; every role then stops
   int* s_cnt_all = reinterpret_cast<int*>(smem + L::off_cnt);
@@ -230,14 +246,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], kLoaderThreads + 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], kLoaderThreads + 1);
-      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kSoftmaxWarps);
+      mbar_init(&s_free[i], TMEM_P ? 1 : kSoftmaxWarps);
+      mbar_init(&p_full[i], kSoftmaxWarps);
       mbar_init(&list_full[i], 32);
       mbar_init(&list_free[i], kRoleWarps);
     }
-    mbar_init(p_full, kSoftmaxWarps);
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&v_full[i], kLoaderThreads + 1);
+      mbar_init(&v_empty[i], 1);
+    }
     mbar_init(pv_done, 1);
     mbar_init(mma_fin, 1);
     mbar_init(q_free, 1);
@@ -391,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     const int c = lt % CH, r0 = lt / CH;
     const uint32_t dst_lane = (uint32_t)((c >> 3) * kHalfBytes + r0 * 128 + (((c & 7) ^ (r0 & 7)) << 4));
     // TMA loads this thread has armed and not yet seen consumed: [K/V][stage] parity
-    int armed[2][2] = {{-1, -1}, {-1, -1}};
+    int armed[2][kMaxVStages] = {{-1, -1, -1}, {-1, -1, -1}};
     int q_armed = -1;  // parity of the last Q load issued
     bool live = true;
     int gbase = 0;  // tiles of the earlier items (ring stages and phases run on)
@@ -420,9 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       for (int i = 0; i < inf.ntiles && live; ++i) {
         const Tile tl = tile_at(inf.tl, s_seg, i);
         const int gi = gbase + i;
-        const int st = (int)(gi & 1);
-        const uint32_t ph = (uint32_t)((gi >> 1) & 1);
-        for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
+        for (int which = 0; which < 2; ++which) {  // 0: K (2 stages), 1: V (kVStages)
+          const int st = which ? gi % kVStages : (gi & 1);
+          const uint32_t ph = (uint32_t)((which ? gi / kVStages : gi >> 1) & 1);
           uint64_t* empty = which ? &v_empty[st] : &k_empty[st];
           uint64_t* fullb = which ? &v_full[st] : &k_full[st];
           uint8_t* dst = (which ? s_v : s_k) + (size_t)st * L::kTileBytes;
@@ -496,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     // after an abort, wait (bounded) for the TMA loads still landing in shared memory
     if (lt == 0) {
       for (int w = 0; w < 2; ++w)
-        for (int st = 0; st < 2; ++st)
+        for (int st = 0; st < (w ? kVStages : 2); ++st)
           if (armed[w][st] >= 0) mbar_wait(w ? &v_full[st] : &k_full[st], (uint32_t)armed[w][st]);
       if (q_armed >= 0) mbar_wait(q_full, (uint32_t)q_armed);
     }
@@ -505,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     const uint32_t sq = smem_u32(s_q), sp = smem_u32(s_p);
     bool live = true;
     int gbase = 0;
+    int o_items = 0;  // items with tiles so far (o_free completions to wait for)
     for (int n = 0; live; ++n) {
       const ItemInfo* infp = next_item(n);
       if (infp == nullptr) break;
@@ -545,13 +564,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       if (live && ntiles > 0) live = issue_s(0);
       if (live && ntiles > 1) live = issue_s(1);
       // the previous item's output must be read out of TMEM before this item's first PV
-      if (live && n > 0 && !wait(o_free, (uint32_t)((n - 1) & 1))) live = false;
+      if (live && ntiles > 0) {
+        if (o_items > 0 && !wait(o_free, (uint32_t)((o_items - 1) & 1))) live = false;
+        ++o_items;
+      }
       tc_fence_after();
       bool o_written[2] = {false, false};  // O_A / O_B hold data (else the first PV MMA initialises)
       for (int i = 0; i < ntiles && live; ++i) {
         const int gi = gbase + i;
-        const int st = (int)(gi & 1);
-        if (!wait(p_full, (uint32_t)(gi & 1)) || !wait(&v_full[st], (uint32_t)((gi >> 1) & 1))) {
+        const int st = (int)(gi & 1), vs = gi % kVStages;
+        if (!wait(&p_full[st], (uint32_t)((gi >> 1) & 1)) || !wait(&v_full[vs], (uint32_t)((gi / kVStages) & 1))) {
           live = false;
           break;
         }
@@ -559,17 +581,26 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         tc_fence_after();
         const int width = tile_at(inf.tl, s_seg, i).width;
         if (elect_one()) {
-          const uint32_t sv = smem_u32(s_v + (size_t)st * L::kTileBytes);
+          const uint32_t sv = smem_u32(s_v + (size_t)vs * L::kTileBytes);
+          const uint32_t pcol = tbase + (st ? kTmemS1 : kTmemS0);
           for (int ks = 0; ks < width / 16; ++ks) {
             const int hf = ks >> 2;  // key half: 0 -> O_A, 1 -> O_B
-            const uint32_t aoff = (uint32_t)(hf * kHalfBytes + (ks & 3) * 32);
-            const uint64_t pdesc = make_sdesc(sp + aoff, 16, 1024, kSwizzle128);
             const uint32_t acc = (o_written[hf] || (ks & 3) > 0) ? 1u : 0u;
-            mma_bf16_ss(tbase + (hf ? kTmemOB : kTmemOA), pdesc,
-                        make_sdesc(sv + ks * 2048, kHalfBytes, 1024, kSwizzle128), idesc_bf16(128, D, 0, 1), acc);
+            const uint64_t vdesc = make_sdesc(sv + ks * 2048, kHalfBytes, 1024, kSwizzle128);
+            if constexpr (TMEM_P) {
+              // P (bf16 pairs) in the S buffer's columns: key half hf at columns
+              // 64*hf .. 64*hf+31 of the buffer
+              mma_bf16_ts(tbase + (hf ? kTmemOB : kTmemOA), pcol + (uint32_t)(64 * hf + 8 * (ks & 3)), vdesc,
+                          idesc_bf16(128, D, 0, 1), acc);
+            } else {
+              const uint32_t aoff = (uint32_t)(hf * kHalfBytes + (ks & 3) * 32);
+              mma_bf16_ss(tbase + (hf ? kTmemOB : kTmemOA), make_sdesc(sp + aoff, 16, 1024, kSwizzle128), vdesc,
+                          idesc_bf16(128, D, 0, 1), acc);
+            }
           }
           mma_commit(pv_done);
-          mma_commit(&v_empty[st]);
+          mma_commit(&v_empty[vs]);
+          if constexpr (TMEM_P) mma_commit(&s_free[st]);  // S buffer and its P consumed
         }
         __syncwarp();
         o_written[0] = true;
@@ -599,7 +630,6 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     const float c = a.scale_log2;  // > 0: max of raw logits * c = max of scaled logits
     const int my0 = half * 64;     // first key column of this half
     const uint32_t o_mine = tbase + lane_base + (half ? kTmemOB : kTmemOA);
-    const uint32_t prow = smem_u32(s_p) + (uint32_t)(half * kHalfBytes + row * 128);
     bool live = true;
     int gbase = 0;
     for (int n = 0; live; ++n) {
@@ -612,6 +642,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       int64_t nvis = n_visible(t, a.m);
       if (nvis > a.Nc) nvis = a.Nc;
       float m_run = -INFINITY;
+      // last PV this warp has waited for: a parity wait may be issued only for the
+      // barrier's next phase, never again for one it has already seen complete
+      int pv_waited = gbase - 1;
       float2 l2 = make_float2(0.f, 0.f);  // running row sum of the bf16 weights (two partial sums)
       float2 u2 = make_float2(0.f, 0.f);  // the same of the unrounded weights (for the log-sum-exp)
       for (int i = 0; i < ntiles; ++i) {
@@ -705,19 +738,32 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[st]);
-        // wait until PV of the previous tile finished: P buffer free, O stable
-        if (i > 0) {
-          if (!wait(pv_done, (uint32_t)((gi - 1) & 1))) {
-            live = false;
-            break;
+        if constexpr (!TMEM_P) {
+          // S read: its buffer may take the next QK; then PV of the previous tile
+          // must have finished (the P tile is free, O stable)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[st]);
+          if (i > 0) {
+            if (!wait(pv_done, (uint32_t)((gi - 1) & 1))) {
+              live = false;
+              break;
+            }
+            pv_waited = gi - 1;
+            tc_fence_after();
           }
-          tc_fence_after();
         }
         if (__any_sync(0xffffffffu, raise && i > 0 && alpha != 1.0f)) {
-          // rescale this half's output accumulator (all D columns)
+          // rescale this half's output accumulator (all D columns), once PV of the
+          // previous tile has finished with it
+          if constexpr (TMEM_P) {
+            if (!wait(pv_done, (uint32_t)((gi - 1) & 1))) {
+              live = false;
+              break;
+            }
+            pv_waited = gi - 1;
+            tc_fence_after();
+          }
           const float sc = (raise && i > 0) ? alpha : 1.0f;
 #pragma unroll 1
           for (int b0 = 0; b0 < D; b0 += 32) {
@@ -733,27 +779,44 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
         l2 = make_float2(l2.x * alpha + ps.x, l2.y * alpha + ps.y);
         if (WANT_LSE) u2 = make_float2(u2.x * alpha + pu.x, u2.y * alpha + pu.y);
         m_run = m_new;
-        // store this half's P row (K-major, 128B swizzle)
-        if (my0 < width) {
+        if constexpr (TMEM_P) {
+          // this half's P row (bf16 pairs) into the first 32 columns of its own S
+          // columns, which this warp has read: PV takes A from tensor memory
+          if (my0 < width) {
+            tmem_st32p(scol, pk);
+            tmem_wait_st();
+          }
+        } else {
+          // this half's P row into the shared-memory tile (K-major, 128B swizzle)
+          const uint32_t prow = smem_u32(s_p) + (uint32_t)(half * kHalfBytes + row * 128);
+          if (my0 < width) {
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            if (my0 + cc * 8 < width) {
-              const uint32_t off = (uint32_t)(((cc ^ (row & 7)) << 4));
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + off), "r"(pk[cc * 4]),
-                           "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
-                           : "memory");
+            for (int cc = 0; cc < 8; ++cc) {
+              if (my0 + cc * 8 < width) {
+                const uint32_t off = (uint32_t)(((cc ^ (row & 7)) << 4));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + off), "r"(pk[cc * 4]),
+                             "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
+                             : "memory");
+              }
             }
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[st]);
       }
       // epilogue: the two halves' (max, sum) meet once; O = (O_A f_A + O_B f_B) / l
       float* s_red = s_red_all + (n & 1) * (2 * kRows * 4);
       const int64_t b = inf.b;
-      const bool have_o = ntiles > 0 && live && wait(pv_done, (uint32_t)((gbase + ntiles - 1) & 1));
+      // PV of the last tile.  A parity wait must be for the barrier's next phase:
+      // a warp that has not waited for PV of the tile before (it may be two PVs
+      // behind the last one) waits for that first; one that has already seen it
+      // complete must not wait for it again
+      bool have_o = ntiles > 0 && live;
+      const int last = gbase + ntiles - 1;
+      for (int j = pv_waited + 1 > last - 1 ? pv_waited + 1 : last - 1; have_o && j <= last; ++j)
+        have_o = wait(pv_done, (uint32_t)(j & 1));
       if (have_o) tc_fence_after();
       const float l_mine = have_o ? l2.x + l2.y : 0.f;
       *reinterpret_cast<float4*>(s_red + 4 * (half * kRows + row)) =
@@ -819,7 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       // O of this item is out of TMEM: the next item's PV may overwrite it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
+      if (lane == 0 && ntiles > 0) mbar_arrive(o_free);
       gbase += ntiles;
       release_item(n);
     }
@@ -835,8 +898,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
 
 // ------------------------------------------------------------------ host side
 
-size_t attention_smem_bytes(int d, int idx_entries, int slots) {
-  return d == 128 ? AttnSmem<128>::bytes(idx_entries, slots) : AttnSmem<64>::bytes(idx_entries, slots);
+size_t attention_smem_bytes(int d, bool tmem_p, int idx_entries, int slots) {
+  if (tmem_p)
+    return d == 128 ? AttnSmem<128, true>::bytes(idx_entries, slots) : AttnSmem<64, true>::bytes(idx_entries, slots);
+  return d == 128 ? AttnSmem<128, false>::bytes(idx_entries, slots) : AttnSmem<64, false>::bytes(idx_entries, slots);
 }
 static_assert(sizeof(ItemInfo) <= 128, "item slot");
 
@@ -860,13 +925,21 @@ static bool bf16_map(CUtensorMap* m, const void* base, int64_t rows, int d, int 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool L>
+template <int D, bool L, bool TP>
 static cudaError_t launch_t(const AttnArgs& a, const AttnMaps& maps, unsigned grid, size_t smem,
                             cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(attention_kernel<D, L, TP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attention_kernel<D, L><<<dim3(grid, a.nsplit > 1 ? a.nsplit : 1), kThreads, smem, stream>>>(a, maps);
+  attention_kernel<D, L, TP><<<dim3(grid, a.nsplit > 1 ? a.nsplit : 1), kThreads, smem, stream>>>(a, maps);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_d(const AttnArgs& a, const AttnMaps& maps, unsigned grid, size_t smem, bool lse, bool tp,
+                            cudaStream_t stream) {
+  if (tp) return lse ? launch_t<D, true, true>(a, maps, grid, smem, stream) : launch_t<D, false, true>(a, maps, grid, smem, stream);
+  return lse ? launch_t<D, true, false>(a, maps, grid, smem, stream) : launch_t<D, false, false>(a, maps, grid, smem, stream);
 }
 
 // Merge the split partial outputs: one warp per (sequence, head), lane c owning
@@ -959,8 +1032,9 @@ cudaError_t launch_attention(const AttnArgs& a_in, int d, unsigned grid, cudaStr
   AttnArgs a = a_in;
   const int GQ = kRows / a.H;
   const int idx_entries = a.idx ? GQ * a.k : 0;
-  a.slots = attention_smem_bytes(d, idx_entries, 2) <= 227 * 1024 ? 2 : 1;
-  const size_t smem = attention_smem_bytes(d, idx_entries, a.slots);
+  const bool tp = a.idx == nullptr;  // P in tensor memory for dense (HCA) tiles
+  a.slots = attention_smem_bytes(d, tp, idx_entries, 2) <= 227 * 1024 ? 2 : 1;
+  const size_t smem = attention_smem_bytes(d, tp, idx_entries, a.slots);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   a.nitems = grid;
   if (a.pos == nullptr) {
@@ -974,9 +1048,8 @@ cudaError_t launch_attention(const AttnArgs& a_in, int d, unsigned grid, cudaStr
       !bf16_map(&maps.vr, a.Vr, a.raw_rows, d, 128))
     return cudaErrorInvalidValue;
   const bool lse = a.lse != nullptr || a.nsplit > 1;
-  if (d == 128)
-    return lse ? launch_t<128, true>(a, maps, grid, smem, stream) : launch_t<128, false>(a, maps, grid, smem, stream);
-  return lse ? launch_t<64, true>(a, maps, grid, smem, stream) : launch_t<64, false>(a, maps, grid, smem, stream);
+  if (d == 128) return launch_d<128>(a, maps, grid, smem, lse, tp, stream);
+  return launch_d<64>(a, maps, grid, smem, lse, tp, stream);
 }
 
 }  // namespace csa

@@ -863,59 +863,62 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
       lo = min(lo, s_lo[w]);
       hi = max(hi, s_hi[w]);
     }
-    uint64_t thr;
-    if (hi > lo) {
-      const int bits = 32 - __clz(hi - lo);
-      const int shift = bits > 10 ? bits - 10 : 0;
-      for (int i = tid; i < cnt; i += kFinBlock) atomicAdd(&hist[((uint32_t)(buf[i] >> 32) - lo) >> shift], 1);
-      __syncthreads();
-      if (warp == 0) {
-        int bin, kept;
-        topk::warp_hist_cut(hist, k, lane, &bin, &kept);
-        if (lane == 0) {
-          s_bin = bin;
-          s_kept = kept;
-          s_inbin = hist[bin];
-        }
-      }
-      __syncthreads();
-      const int bin = s_bin, in_bin = s_inbin;
-      const int need = k - (s_kept - in_bin);
-      const uint64_t bin_lo = (uint64_t)(lo + ((uint32_t)bin << shift)) << 32;
-      if (need == in_bin) {
-        thr = bin_lo;
-      } else if (in_bin <= 32) {
-        // the boundary bin's keys (at most 32) into `sel`, sorted in registers
+    // exact threshold: a block-wide radix select on the keys, 10 bits per pass
+    // from the top of their span, until the boundary bin is kept whole or holds at
+    // most 32 keys (then sorted in registers)
+    uint64_t thr = 0;
+    {
+      uint64_t base = (uint64_t)lo << 32;                   // every key lies in [base, base + 2^wl)
+      int wl = (hi > lo ? 32 - __clz(hi - lo) : 0) + 32;
+      int need = k;
+      for (;;) {
+        const int w = wl >= 10 ? 10 : wl;
+        const int sh = wl - w;
+        for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
+        if (tid == 0) s_nsel = 0;
+        __syncthreads();
         for (int i = tid; i < cnt; i += kFinBlock) {
-          const uint64_t v = buf[i];
-          if ((int)(((uint32_t)(v >> 32) - lo) >> shift) == bin) sel[atomicAdd(&s_nsel, 1)] = v;
+          const uint64_t dk = buf[i] - base;
+          if (wl >= 64 || dk < (1ull << wl)) atomicAdd(&hist[(int)(dk >> sh)], 1);
         }
         __syncthreads();
         if (warp == 0) {
-          uint64_t x = lane < in_bin ? sel[lane] : 0;
-          x = topk::warp_sort32_desc(x, lane);
-          const uint64_t t = __shfl_sync(0xffffffffu, x, need - 1);
-          if (lane == 0) s_thr = t;
+          int bin, kept;
+          topk::warp_hist_cut(hist, need, lane, &bin, &kept);
+          if (lane == 0) {
+            s_bin = bin;
+            s_kept = kept;
+            s_inbin = hist[bin];
+          }
         }
         __syncthreads();
-        thr = s_thr;
-      } else {
-        // heavy ties in the boundary bin: exact radix select over all keys
-        if (warp == 0) {
-          const uint64_t t = topk::warp_exact_threshold(buf, cnt, k, hist, lane);
-          if (lane == 0) s_thr = t;
+        const int bin = s_bin, in_bin = s_inbin;
+        need -= s_kept - in_bin;  // keys in the higher bins are all kept
+        base += (uint64_t)bin << sh;
+        wl = sh;
+        if (need == in_bin) {  // the whole boundary bin is kept
+          thr = base;
+          break;
         }
-        __syncthreads();
-        thr = s_thr;
+        if (in_bin <= 32) {
+          // the boundary bin's keys into `sel`, sorted in registers
+          for (int i = tid; i < cnt; i += kFinBlock) {
+            const uint64_t v = buf[i];
+            if (v - base < (1ull << wl)) sel[atomicAdd(&s_nsel, 1)] = v;
+          }
+          __syncthreads();
+          if (warp == 0) {
+            uint64_t x = lane < in_bin ? sel[lane] : 0;
+            x = topk::warp_sort32_desc(x, lane);
+            const uint64_t t = __shfl_sync(0xffffffffu, x, need - 1);
+            if (lane == 0) s_thr = t;
+          }
+          __syncthreads();
+          thr = s_thr;
+          break;
+        }
+        __syncthreads();  // everyone has read s_bin / s_inbin before the next pass
       }
-    } else {
-      // every key has the same score: the order is by index alone
-      if (warp == 0) {
-        const uint64_t t = topk::warp_exact_threshold(buf, cnt, k, hist, lane);
-        if (lane == 0) s_thr = t;
-      }
-      __syncthreads();
-      thr = s_thr;
     }
     // the k keys >= thr, one shared-memory atomic per warp and step
     if (tid == 0) s_nsel = 0;
