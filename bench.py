@@ -37,9 +37,15 @@ NOMINAL_FP4_TFLOPS = 9000.0  # NVIDIA's dense FP4 figure for B200 (context only)
 E2E_CHUNKS = 16  # query chunks of the pipelined end-to-end step
 
 PHASE_TRAFFIC = {
-    # the indexer changed since its full-size DRAM capture: no traffic figure until it is re-taken
-    "indexer_topk": (None, "no full-size capture of the current indexer"),
-    "sparse_attn": (None, "no full-size capture of the current attention kernel"),
+    # DRAM bytes (read + written) of one full-size launch, from the one-pass ncu capture
+    # recorded in profiles/launch_list_bench_default.md; the indexer phase is the
+    # indexer kernel plus the finalize kernel
+    "indexer_topk": (146382336 + 92027904 + 130439936 + 33449728,
+                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of the full-size indexer and finalize "
+                     "launches (profiles/launch_list_bench_default.md)"),
+    "sparse_attn": (625224704 + 487242496,
+                    "ncu dram__bytes_read.sum + dram__bytes_write.sum of a full-size attention launch "
+                    "(profiles/launch_list_bench_default.md)"),
 }
 
 
