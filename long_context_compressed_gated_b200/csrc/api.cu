@@ -111,6 +111,7 @@ struct PosBlock {
 };
 
 __global__ void fill_i64_kernel(int64_t* dst, PosBlock blk, int n) {
+  griddep_launch_dependents();  // the next kernel's setup may overlap this copy
   if ((int)threadIdx.x < n) dst[threadIdx.x] = blk.v[threadIdx.x];
 }
 
@@ -447,6 +448,7 @@ static int decode_impl(const void* q, const uint8_t* qI_codes, const uint8_t* qI
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
+  a.pdl = 1;  // the position upload (and the search) of this call run just before
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Ncap > 0 && !fp8 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
@@ -596,6 +598,7 @@ int csa_decode_attend(const void* q, const void* Kc, const void* Vc, const int32
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
+  a.pdl = 1;  // the position upload (and the search) of this call run just before
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Nloc > 0 ? (int64_t)B * Nloc : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
@@ -709,6 +712,7 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
+  a.pdl = 1;  // the position upload (and the search) of this call run just before
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;

@@ -295,6 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
 
   if (warp == kSchedWarp) {
     // =========================== scheduler: item n's token range, compacted selections, tile list
+    // (the positions and selections may come from the kernel before: read once it completed)
+    griddep_wait();
+    griddep_launch_dependents();
     for (int n = 0;; ++n) {
       const int slot = n % slots;
       const int use = n / slots;
@@ -413,6 +416,21 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
     int q_armed = -1;  // parity of the last Q load issued
     bool live = true;
     int gbase = 0;  // tiles of the earlier items (ring stages and phases run on)
+    // Q of the first item right away: its rows are known from the item number,
+    // so the load overlaps the scheduler's work on the item's tile list
+    auto load_q = [&](int n, int64_t item) {
+      mbar_arrive_expect_tx(q_full, HALVES * kHalfBytes);
+      const int qrow = (int)(decode ? item * H : item * GQ * H);
+      for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(s_q + hf * kHalfBytes, &maps.q, q_full, hf * 64, qrow);
+      q_armed = n & 1;
+    };
+    if (lt == 0) {
+      const int64_t item0 = item_of(0);
+      if (item0 >= 0) {
+        prefetch_tmap(&maps.q);
+        load_q(0, item0);
+      }
+    }
     for (int n = 0; live; ++n) {
       const ItemInfo* infp = next_item(n);
       if (infp == nullptr) break;
@@ -424,16 +442,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       const __nv_bfloat16* Vc = a.Vc + b * a.kc_batch_stride;
       const uint32_t* s_seg = s_seg_all + (n % slots) * kMaxSegTiles;
       const int* s_idx = s_idx_all + (size_t)(n % slots) * idx_entries;
-      if (lt == 0) {
+      if (lt == 0 && n > 0) {
         // Q of this item, once the previous item's QK products are complete
-        if (n > 0 && !wait(q_free, (uint32_t)((n - 1) & 1))) live = false;
-        if (live) {
-          if (n == 0) prefetch_tmap(&maps.q);
-          mbar_arrive_expect_tx(q_full, HALVES * kHalfBytes);
-          const int qrow = (int)(decode ? b * H : inf.row_tok0 * H);
-          for (int hf = 0; hf < HALVES; ++hf) tma_load_2d(s_q + hf * kHalfBytes, &maps.q, q_full, hf * 64, qrow);
-          q_armed = n & 1;
-        }
+        if (!wait(q_free, (uint32_t)((n - 1) & 1))) live = false;
+        if (live) load_q(n, decode ? b : inf.row_tok0 / GQ);
       }
       for (int i = 0; i < inf.ntiles && live; ++i) {
         const Tile tl = tile_at(inf.tl, s_seg, i);
@@ -931,8 +943,8 @@ static cudaError_t launch_t(const AttnArgs& a, const AttnMaps& maps, unsigned gr
   cudaError_t e =
       cudaFuncSetAttribute(attention_kernel<D, L, TP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attention_kernel<D, L, TP><<<dim3(grid, a.nsplit > 1 ? a.nsplit : 1), kThreads, smem, stream>>>(a, maps);
-  return cudaGetLastError();
+  return launch_kernel(attention_kernel<D, L, TP>, dim3(grid, a.nsplit > 1 ? a.nsplit : 1), dim3(kThreads), smem,
+                       stream, a.pdl != 0, a, maps);
 }
 
 template <int D>
@@ -954,6 +966,8 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __r
                                                                 int64_t rows, void* __restrict__ O, int o_f32,
                                                                 int64_t o_batch_stride, float* __restrict__ lse,
                                                                 int64_t sb, int64_t ss) {
+  griddep_wait();  // the partials come from the attention kernel before
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (b, h)
   if (w >= rows) return;
@@ -1003,23 +1017,19 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const float* __r
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int nsplit, int B, int H, int d, void* O,
                            int o_f32, int64_t o_batch_stride, float* lse, int64_t sb, int64_t ss,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool pdl) {
   if (nsplit > kCombineSplits) return cudaErrorInvalidConfiguration;
   const int64_t rows = (int64_t)B * H;
   const unsigned grid = (unsigned)((rows + 7) / 8);
   if (rows == 0) return cudaSuccess;
-  if (d == 128)
-    attention_combine_kernel<128><<<grid, 256, 0, stream>>>(o_part, lse_part, nsplit, H, rows, O, o_f32,
-                                                             o_batch_stride, lse, sb, ss);
-  else
-    attention_combine_kernel<64><<<grid, 256, 0, stream>>>(o_part, lse_part, nsplit, H, rows, O, o_f32,
-                                                            o_batch_stride, lse, sb, ss);
-  return cudaGetLastError();
+  auto kern = d == 128 ? attention_combine_kernel<128> : attention_combine_kernel<64>;
+  return launch_kernel(kern, dim3(grid), dim3(256), 0, stream, pdl, o_part, lse_part, nsplit, H, rows, O, o_f32,
+                       o_batch_stride, lse, sb, ss);
 }
 
 cudaError_t launch_attention_combine(const AttnArgs& a, int B, int d, cudaStream_t stream) {
   return launch_combine(a.o_part, a.lse_part, a.nsplit, B, a.H, d, a.O, a.o_f32, a.o_batch_stride, a.lse, a.nsplit, 1,
-                        stream);
+                        stream, true);
 }
 
 int sm_count();

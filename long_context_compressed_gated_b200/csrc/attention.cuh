@@ -41,6 +41,9 @@ struct AttnArgs {
   // item descriptions kept in shared memory (2: the next one is built ahead)
   int64_t nitems;
   int slots;
+  // 1: a kernel of the same library call runs just before this one (the launch may
+  // overlap it; the scheduler reads positions and selections only once it completed)
+  int pdl;
 };
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);
@@ -51,7 +54,7 @@ int attention_max_seg_tiles();
 // of sequence b at row b*sb + s*ss): O = sum_s exp(lse_s - lse) O_s, lse = log sum exp.
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int nsplit, int B, int H, int d, void* O,
                            int o_f32, int64_t o_batch_stride, float* lse, int64_t sb, int64_t ss,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool pdl = false);
 constexpr int kMaxCombineParts = 16;
 
 }  // namespace csa

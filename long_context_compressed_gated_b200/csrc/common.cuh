@@ -28,6 +28,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Programmatic dependent launch.  A kernel launched with pdl = true may start
+// (and run its setup) while the kernel before it in the stream is still running;
+// griddep_wait() returns once that kernel has completed and its writes are
+// visible, so every read of an earlier kernel's output comes after it, and
+// griddep_launch_dependents() lets the next such kernel start early.  Only the
+// second and later kernels of one library call are launched this way: the first
+// waits for all earlier work of the stream in the ordinary way, so nothing a
+// caller's own kernels write is ever read before its writer has finished.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... P, typename... A>
+cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                          A&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<A&&>(args)...);
+}
+
 // Workspace header: status word + padding to 256 bytes.
 constexpr size_t kWorkspaceHeader = 256;
 

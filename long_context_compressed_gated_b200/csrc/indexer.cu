@@ -64,9 +64,10 @@ constexpr int kHalfBar0 = 1;                  // named barriers 1, 2: the four w
 constexpr int kEpiBar = 3;                    // named barrier 3: all epilogue warps
 constexpr size_t kSmemLimit = 227 * 1024;
 
-// TMEM column map (512 allocated): NB accumulator buffers of N columns from 0
-// (at most 448 columns), scale factors from column 448.
-constexpr uint32_t kTmemSF = 448;
+// TMEM column map (512 allocated): NB accumulator buffers of N columns from 0,
+// then the key scales of each buffer (4 columns each), query scales at column
+// 480, the constant-offset operands' scales at 488 and 492.
+constexpr uint32_t kTmemSFB = 480;
 
 // Tokens per CTA (prefill): 128 accumulator columns (HI >= 16), so that three
 // buffers fit in TMEM; an even count, split between the two epilogue halves.
@@ -77,14 +78,18 @@ struct Geometry {
 
 template <int HI, int G>
 struct TileShape {
-  static constexpr int N = ((G * HI + 15) / 16) * 16;      // MMA N (accumulator columns)
-  static constexpr int NB = G == 1 ? (448 / N >= 8 ? 8 : 4)  // decode: whole barrier groups of 4
-                                   : (448 / N < 8 ? 448 / N : 8);  // accumulator buffers
-  static constexpr uint32_t sfa(int b) { return kTmemSF + 4 * b; }  // key scales, 4 columns each
-  static constexpr uint32_t kSFB = kTmemSF + 32;                    // query scales, 8 columns
-  static constexpr uint32_t kMagicSFA = kTmemSF + 40;              // 4 columns
-  static constexpr uint32_t kMagicSFB = kTmemSF + 44;              // 8 columns
-  static_assert(NB >= 2 && NB * N <= 448, "TMEM budget");
+  static constexpr int N = ((G * HI + 15) / 16) * 16;  // MMA N (accumulator columns)
+  // decode: whole barrier groups of 4 buffers, as many as fit beside their scale
+  // columns (at most 24): the MMA warp runs up to that many tiles ahead of the
+  // epilogue, so that the key stream goes on while the epilogue cuts a buffer back
+  static constexpr int kDecodeNB = (480 / (N + 4)) / 4 * 4 > 24 ? 24 : (480 / (N + 4)) / 4 * 4;
+  static constexpr int NB = G == 1 ? kDecodeNB : (448 / N < 8 ? 448 / N : 8);  // accumulator buffers
+  static constexpr uint32_t kSFA = G == 1 ? (uint32_t)(NB * N) : 448u;
+  static constexpr uint32_t sfa(int b) { return kSFA + 4 * b; }  // key scales, 4 columns each
+  static constexpr uint32_t kSFB = kTmemSFB;                      // query scales, 8 columns
+  static constexpr uint32_t kMagicSFA = kTmemSFB + 8;             // 4 columns
+  static constexpr uint32_t kMagicSFB = kTmemSFB + 12;            // 8 columns
+  static_assert(NB >= 2 && NB * N <= 448 && kSFA + 4 * NB <= kTmemSFB, "TMEM budget");
 };
 
 __device__ __forceinline__ int e2m1_times2(uint32_t code) {
@@ -225,34 +230,15 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cap = a.cap;
   const bool decode = a.pos != nullptr;
-  // A bounded wait of an earlier CTA on this workspace gave up: skip the work
-  // (read now, used after the setup, so the load overlaps it).
-  const int status_at_entry = *reinterpret_cast<volatile int*>(a.status);
-
   // ---- which tokens and which key range
   const int64_t grp = decode ? blockIdx.x : (int64_t)(gridDim.x - 1 - blockIdx.x);  // heavy groups first
   const int64_t row0 = grp * G;
   const int split = blockIdx.y;
-  int64_t tnvis[G];  // entries visible to each token of the group (0 for rows past the end)
-  int64_t nvis_max = 0;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const int64_t r = row0 + g;
-    int64_t t = -1;
-    if (r < a.rows) t = decode ? a.pos[r] : a.t0 + r;
-    int64_t nv = n_visible(t, a.m) - a.j_base;  // entries of this (slice of the) cache visible to t
-    if (nv < 0) nv = 0;
-    if (nv > a.Nc) nv = a.Nc;
-    tnvis[g] = nv;
-    if (nv > nvis_max) nvis_max = nv;
-  }
   const int64_t key_row_base = decode ? row0 * a.Nc : 0;  // per-sequence cache (decode)
   const int64_t j_begin = (int64_t)split * a.split_tiles * 128;
-  int64_t j_end = j_begin + a.split_tiles * 128;
-  if (j_end > nvis_max) j_end = nvis_max;
-  const int ntiles_all = j_end > j_begin ? (int)ceil_div(j_end - j_begin, 128) : 0;
 
-  // ---- setup
+  // ---- setup (barriers, TMEM, constants and the caller's inputs: nothing that an
+  // earlier kernel of the same call writes)
   if (tid == 0) {
     for (int s = 0; s < NSG; ++s) {
       mbar_init(&full[s], 1 + 32);  // TMA transaction arrival + one per producer lane (scales)
@@ -311,6 +297,27 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
       }
     }
   }
+  // the decode positions come from the kernel before (the upload of the positions)
+  griddep_wait();
+  griddep_launch_dependents();
+  // A bounded wait of an earlier CTA on this workspace gave up: skip the work.
+  const int status_at_entry = *reinterpret_cast<volatile int*>(a.status);
+  int64_t tnvis[G];  // entries visible to each token of the group (0 for rows past the end)
+  int64_t nvis_max = 0;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int64_t r = row0 + g;
+    int64_t t = -1;
+    if (r < a.rows) t = decode ? a.pos[r] : a.t0 + r;
+    int64_t nv = n_visible(t, a.m) - a.j_base;  // entries of this (slice of the) cache visible to t
+    if (nv < 0) nv = 0;
+    if (nv > a.Nc) nv = a.Nc;
+    tnvis[g] = nv;
+    if (nv > nvis_max) nvis_max = nv;
+  }
+  int64_t j_end = j_begin + a.split_tiles * 128;
+  if (j_end > nvis_max) j_end = nvis_max;
+  const int ntiles_all = j_end > j_begin ? (int)ceil_div(j_end - j_begin, 128) : 0;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -732,6 +739,8 @@ __global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __re
                                                             float* __restrict__ scores,
                                                             uint64_t* __restrict__ keys_out) {
   extern __shared__ __align__(16) uint8_t fsmem[];
+  griddep_wait();  // the candidate lists come from the kernel before
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   const int64_t r = (int64_t)blockIdx.x * wpb + warp;
@@ -786,6 +795,8 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
                                                                         float* __restrict__ scores,
                                                                         uint64_t* __restrict__ keys_out) {
   extern __shared__ __align__(16) uint8_t bsmem[];
+  griddep_wait();  // the candidate lists come from the kernel before
+  griddep_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t r = blockIdx.x;
   const int cap = topk::next_pow2(nsplit * k);
@@ -961,8 +972,10 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
   }
 }
 
+// pdl: a kernel of the same library call runs just before (the finalize may start
+// during it; it reads the candidates only once that kernel has completed)
 static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, int nsplit, int k, int64_t rows,
-                                   int32_t* idx, float* scores, uint64_t* keys_out, cudaStream_t stream) {
+                                   int32_t* idx, float* scores, uint64_t* keys_out, cudaStream_t stream, bool pdl) {
   if (nsplit > 1) {
     // few rows with many candidates each: a block per row
     const size_t sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
@@ -971,9 +984,8 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
     cudaError_t e =
         cudaFuncSetAttribute(topk_finalize_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_finalize_block_kernel<<<(unsigned)rows, kFinBlock, smem, stream>>>(cand, cand_cnt, nsplit, k, idx, scores,
-                                                                            keys_out);
-    return cudaGetLastError();
+    return launch_kernel(topk_finalize_block_kernel, dim3((unsigned)rows), dim3(kFinBlock), smem, stream, pdl, cand,
+                         cand_cnt, nsplit, k, idx, scores, keys_out);
   }
   const size_t per_warp = (size_t)topk::next_pow2(nsplit * k) * 8 + topk::kWarpBins * 4;
   int wpb = (int)((kSmemLimit - 1024) / per_warp);
@@ -982,9 +994,8 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
   const size_t smem = per_warp * wpb;
   cudaError_t e = cudaFuncSetAttribute(topk_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_finalize_kernel<<<(unsigned)ceil_div(rows, wpb), 32 * wpb, smem, stream>>>(cand, cand_cnt, nsplit, k, rows,
-                                                                                   idx, scores, keys_out);
-  return cudaGetLastError();
+  return launch_kernel(topk_finalize_kernel, dim3((unsigned)ceil_div(rows, wpb)), dim3(32 * wpb), smem, stream, pdl,
+                       cand, cand_cnt, nsplit, k, rows, idx, scores, keys_out);
 }
 
 // Valid keys of each candidate list (nonzero keys first, zero padding after):
@@ -1009,9 +1020,9 @@ cudaError_t launch_topk_merge(const uint64_t* keys, int rows, int lists, int k, 
   }
   if (lists == 1) {
     // one list per row: the warp-per-row pass
-    return launch_finalize(keys, cnt, 1, k, rows, idx, scores, keys_out, stream);
+    return launch_finalize(keys, cnt, 1, k, rows, idx, scores, keys_out, stream, nl > 0);
   }
-  return launch_finalize(keys, cnt, lists, k, rows, idx, scores, keys_out, stream);
+  return launch_finalize(keys, cnt, lists, k, rows, idx, scores, keys_out, stream, nl > 0);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1084,7 +1095,7 @@ static bool choose_cap(int k, int* cap, int* check) {
 
 template <int HI, int DI, int G>
 static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, IndexerArgs a, dim3 grid,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, bool pdl) {
   a.fault = take_injected_fault();
   using L = IndexerSmem<HI, DI, G>;
   CUtensorMap qmap, kmap;
@@ -1096,15 +1107,15 @@ static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, In
   auto kern = indexer_topk_kernel<HI, DI, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, Epi<HI, G>::kBlock, smem, stream>>>(qmap, kmap, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, dim3(Epi<HI, G>::kBlock), smem, stream, pdl, qmap, kmap, a);
 }
 
 template <int HI, int DI>
 static cudaError_t dispatch_g(bool decode, const uint8_t* q_codes, const uint8_t* k_codes, IndexerArgs a,
                               dim3 grid, cudaStream_t stream) {
-  if (decode) return launch_one<HI, DI, 1>(q_codes, k_codes, a, grid, stream);
-  return launch_one<HI, DI, Geometry<HI>::G>(q_codes, k_codes, a, grid, stream);
+  // decode: the positions come from the upload kernel just before
+  if (decode) return launch_one<HI, DI, 1>(q_codes, k_codes, a, grid, stream, true);
+  return launch_one<HI, DI, Geometry<HI>::G>(q_codes, k_codes, a, grid, stream, false);
 }
 
 template <int DI>
@@ -1160,7 +1171,7 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
   if (e != cudaSuccess) return e;
   // a sorting pass per row (one warp each; many rows per SM) is cheaper than
   // sorting inside the indexer CTA, where the sort would sit on the CTA's tail
-  return launch_finalize(cand, cand_cnt, 1, k, T, idx, scores, nullptr, stream);
+  return launch_finalize(cand, cand_cnt, 1, k, T, idx, scores, nullptr, stream, true);
 }
 
 // Decode: rows = B sequences, each with its own cache of Ncap entries and position
@@ -1191,7 +1202,7 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
   cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, true, q_codes, k_codes, a, grid, stream)
                             : dispatch_hi<64>(HI, true, q_codes, k_codes, a, grid, stream);
   if (e != cudaSuccess) return e;
-  return launch_finalize(cand, cand_cnt, nsplit, k, B, idx, scores, keys_out, stream);
+  return launch_finalize(cand, cand_cnt, nsplit, k, B, idx, scores, keys_out, stream, true);
 }
 
 }  // namespace csa
