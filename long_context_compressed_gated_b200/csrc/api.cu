@@ -21,9 +21,9 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
                                    int* cand_cnt, int* status, cudaStream_t stream);
 cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
                                   const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
-                                  int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
-                                  uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
-                                  int* status, cudaStream_t stream, int64_t j_base);
+                                  const int64_t* pos_in, bool pdl, int64_t nvis_max, int64_t Ncap, int HI, int DI,
+                                  int m, int k, int nsplit, uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores,
+                                  uint64_t* keys_out, int* status, cudaStream_t stream, int64_t j_base);
 cudaError_t launch_topk_merge(const uint64_t* keys, int rows, int lists, int k, int* cnt, int32_t* idx,
                               float* scores, uint64_t* keys_out, cudaStream_t stream);
 int inject_fault(int code);
@@ -123,6 +123,20 @@ cudaError_t upload_positions(int64_t* dst, const int64_t* host, int B, cudaStrea
     fill_i64_kernel<<<1, 64, 0, stream>>>(dst + b0, blk, n);
   }
   return cudaGetLastError();
+}
+
+// Decode positions: up to kInlinePos ride in the kernel arguments (nothing is
+// launched); more are copied to the workspace first.  *copied: a copy kernel is
+// the call's first kernel (the ones after it may then start during it).
+cudaError_t stage_positions(int64_t* dst, const int64_t* host, int B, cudaStream_t stream, bool* copied) {
+  *copied = B > kInlinePos;
+  return *copied ? upload_positions(dst, host, B, stream) : cudaSuccess;
+}
+
+void inline_positions(AttnArgs& a, const int64_t* host, int B) {
+  if (B > kInlinePos) return;
+  for (int b = 0; b < B; ++b) a.pos_in[b] = host[b];
+  a.npos_in = B;
 }
 
 
@@ -407,12 +421,14 @@ static int decode_impl(const void* q, const uint8_t* qI_codes, const uint8_t* qI
   float* o_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(cand_cnt) + align256((size_t)B * ns * 4));
   float* lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(o_part) + align256((size_t)B * nsa * H * d * 4));
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  bool copied = false;
+  cudaError_t e = stage_positions(pos_dev, pos, B, s, &copied);
   if (e != cudaSuccess) return cuda_fail(e);
   int32_t* sel = idx ? idx : idx_ws;
   if (Ncap > 0) {
-    e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, nvis_max, Ncap, HI, dI,
-                              m, k, ns, cand, cand_cnt, sel, scores, nullptr, status_word(workspace), s, 0);
+    e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, pos, copied, nvis_max,
+                              Ncap, HI, dI, m, k, ns, cand, cand_cnt, sel, scores, nullptr, status_word(workspace), s,
+                              0);
     if (e != cudaSuccess) return cuda_fail(e);
   } else {
     e = cudaMemsetAsync(sel, 0xFF, (size_t)B * k * 4, s);
@@ -448,7 +464,8 @@ static int decode_impl(const void* q, const uint8_t* qI_codes, const uint8_t* qI
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
-  a.pdl = 1;  // the position upload (and the search) of this call run just before
+  inline_positions(a, pos, B);
+  a.pdl = Ncap > 0 || copied;  // the search (or the position copy) of this call runs just before
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Ncap > 0 && !fp8 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
@@ -523,10 +540,12 @@ int csa_decode_search(const uint8_t* qI_codes, const uint8_t* qI_scales, const u
   uint64_t* cand = reinterpret_cast<uint64_t*>(w + kWorkspaceHeader + align256((size_t)B * 8) +
                                                align256((size_t)B * k * 4));
   int* cand_cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cand) + align256((size_t)B * ns * k * 8));
-  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  bool copied = false;
+  cudaError_t e = stage_positions(pos_dev, pos, B, s, &copied);
   if (e == cudaSuccess)
-    e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, nvis_max, Nloc, HI, dI,
-                              m, k, ns, cand, cand_cnt, nullptr, nullptr, keys, status_word(workspace), s, j_base);
+    e = launch_indexer_decode(qI_codes, qI_scales, w_codes, kI_codes, kI_scales, B, pos_dev, pos, copied, nvis_max,
+                              Nloc, HI, dI, m, k, ns, cand, cand_cnt, nullptr, nullptr, keys, status_word(workspace),
+                              s, j_base);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e);
 }
 
@@ -572,7 +591,8 @@ int csa_decode_attend(const void* q, const void* Kc, const void* Vc, const int32
                        align256((size_t)B * ns * k * 8) + align256((size_t)B * ns * 4);
   const int nsa = decode_attn_splits(B, ceil_div(k, 128) + window_tiles(W, 1));
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  bool copied = false;
+  cudaError_t e = stage_positions(pos_dev, pos, B, s, &copied);
   if (e != cudaSuccess) return cuda_fail(e);
   AttnArgs a{};
   a.Q = static_cast<const __nv_bfloat16*>(q);
@@ -598,7 +618,8 @@ int csa_decode_attend(const void* q, const void* Kc, const void* Vc, const int32
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
-  a.pdl = 1;  // the position upload (and the search) of this call run just before
+  inline_positions(a, pos, B);
+  a.pdl = copied;  // the position copy of this call runs just before
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Nloc > 0 ? (int64_t)B * Nloc : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;
@@ -688,7 +709,8 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
   if ((rc = check_opt(lse))) return rc;
   int64_t* pos_dev = reinterpret_cast<int64_t*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = upload_positions(pos_dev, pos, B, s);
+  bool copied = false;
+  cudaError_t e = stage_positions(pos_dev, pos, B, s, &copied);
   if (e != cudaSuccess) return cuda_fail(e);
   AttnArgs a{};
   a.Q = static_cast<const __nv_bfloat16*>(q);
@@ -712,7 +734,8 @@ int hca_decode(const void* q, const void* Kc, const void* Vc, const void* Kwin, 
   a.raw_batch_stride = (int64_t)W * d;
   a.o_batch_stride = (int64_t)H * d;
   a.pos = pos_dev;
-  a.pdl = 1;  // the position upload (and the search) of this call run just before
+  inline_positions(a, pos, B);
+  a.pdl = copied;  // the position copy of this call runs just before
   a.q_rows = (int64_t)B * H;
   a.kc_rows = Ncap > 0 ? (int64_t)B * Ncap : 1;
   a.raw_rows = W > 0 ? (int64_t)B * W : 1;

@@ -185,7 +185,7 @@ struct AttnSmem {
 };
 
 template <int D, bool WANT_LSE, bool TMEM_P>
-__global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a,
+__global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_constant__ AttnArgs a,
                                                                 const __grid_constant__ AttnMaps maps) {
   using L = AttnSmem<D, TMEM_P>;
   constexpr int kVStages = L::kVS;
@@ -309,31 +309,33 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
       int* s_idx = s_idx_all + (size_t)slot * idx_entries;
       int* s_cnt = s_cnt_all + slot * 32;
       if (item >= 0) {
+        // read now, used at the end: the load overlaps the list's construction
+        const int status_now = *reinterpret_cast<volatile int*>(a.status);
         inf.b = decode ? item : 0;
         inf.split = decode ? (int)blockIdx.y : 0;
         inf.row_tok0 = decode ? 0 : item * GQ;
         const int64_t T = decode ? 1 : a.T;
         inf.ntok = (int)((T - inf.row_tok0) < GQ ? (T - inf.row_tok0) : GQ);
-        const int64_t pos_b = decode ? a.pos[inf.b] : 0;
+        const int64_t pos_b = decode ? a.pos_at(inf.b) : 0;
         inf.raw_lo = decode ? pos_b - a.W + 1 : a.raw_lo;  // absolute position of raw row 0
         inf.t_first = decode ? pos_b : a.t0 + inf.row_tok0;
         inf.t_last = decode ? pos_b : a.t0 + inf.row_tok0 + inf.ntok - 1;
-        // compact each token's selected list (drop -1 / out-of-range); 8 loads per
-        // lane are in flight before any is used
+        // compact each token's selected list (drop -1 / out-of-range); 32 loads per
+        // lane are in flight before any is used (one memory round trip for k <= 1024)
         if (a.idx != nullptr) {
           const int32_t* idx = a.idx + inf.b * (decode ? (int64_t)a.k : 0);
           for (int g = 0; g < inf.ntok; ++g) {
             const int32_t* src = idx + (inf.row_tok0 + g) * a.k;
             int nsel = 0;
-            for (int base = 0; base < a.k; base += 256) {
-              int32_t jv[8];
+            for (int base = 0; base < a.k; base += 1024) {
+              int32_t jv[32];
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
+              for (int u = 0; u < 32; ++u) {
                 const int q = base + 32 * u + lane;
                 jv[u] = q < a.k ? __ldg(src + q) : -1;
               }
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
+              for (int u = 0; u < 32; ++u) {
                 const int64_t jl = (int64_t)jv[u] - a.idx_base;  // row of this (slice of the) cache
                 const bool ok = jv[u] >= 0 && jl >= 0 && jl < a.Nc;
                 const uint32_t bal = __ballot_sync(0xffffffffu, ok);
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const AttnArgs a
           }
           // a bounded wait of an earlier CTA (or kernel on this workspace) gave up:
           // skip the work instead of waiting out every deadline again
-          if (*reinterpret_cast<volatile int*>(a.status) == CSA_ERR_DEVICE_TIMEOUT) nt = 0;
+          if (status_now == CSA_ERR_DEVICE_TIMEOUT) nt = 0;
           tl.count = nt;
           inf.tl = tl;
           inf.ntiles = nt;

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "common.cuh"
+
 namespace csa {
 
 struct AttnArgs {
@@ -25,6 +27,8 @@ struct AttnArgs {
   // decode (pos != null): one sequence per CTA, batch strides in elements
   int64_t q_batch_stride, kc_batch_stride, raw_batch_stride, o_batch_stride;
   const int64_t* pos;       // device, absolute position of each sequence's new token
+  int64_t pos_in[kInlinePos];  // the same positions, when npos_in = B (<= kInlinePos)
+  int npos_in;
   // extents (rows) of the tensors, for the TMA descriptors
   int64_t q_rows, kc_rows, raw_rows;
   // decode with the key tiles of a sequence spread over nsplit CTAs (grid.y):
@@ -44,6 +48,7 @@ struct AttnArgs {
   // 1: a kernel of the same library call runs just before this one (the launch may
   // overlap it; the scheduler reads positions and selections only once it completed)
   int pdl;
+  __device__ __forceinline__ int64_t pos_at(int64_t b) const { return b < npos_in ? pos_in[b] : pos[b]; }
 };
 
 cudaError_t launch_attention(const AttnArgs& a, int d, unsigned grid, cudaStream_t stream);

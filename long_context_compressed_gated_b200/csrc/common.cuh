@@ -57,6 +57,11 @@ cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelEx(&cfg, kern, static_cast<A&&>(args)...);
 }
 
+// Decode positions (absolute position of each sequence's new token) travel
+// inside the kernel arguments for up to kInlinePos sequences; more are first
+// copied into the workspace by a small kernel.
+constexpr int kInlinePos = 64;
+
 // Workspace header: status word + padding to 256 bytes.
 constexpr size_t kWorkspaceHeader = 256;
 

@@ -143,6 +143,8 @@ struct IndexerArgs {
   int64_t rows;             // query rows (prefill T, decode B)
   int64_t t0;               // prefill: absolute position of row 0
   const int64_t* pos;       // decode: absolute position per row (device), else null
+  int64_t pos_in[kInlinePos];  // decode: the same positions, when npos_in = rows (<= kInlinePos)
+  int npos_in;
   int64_t Nc;               // prefill: entries in the cache; decode: Ncap per sequence
   int64_t key_rows;         // rows of the kI tensor (bounds for scale loads)
   int m, k;
@@ -155,6 +157,7 @@ struct IndexerArgs {
   int* cand_cnt;            // [rows, nsplit]    how many of them are valid
   int* status;
   int fault;                // test hook (csa_debug_inject): 1 = the producer skips its first stage group
+  __device__ __forceinline__ int64_t pos_at(int64_t r) const { return r < npos_in ? pos_in[r] : pos[r]; }
 };
 
 template <int HI, int DI, int G>
@@ -175,7 +178,8 @@ struct IndexerSmem {
   static constexpr size_t off_thr = off_cnt + 64 * 4;
   // one score histogram per selection group (a half, or all eight epilogue warps in
   // decode): a group cuts its buffers back one at a time
-  static constexpr size_t off_hist = off_thr + 64 * 8;
+  static constexpr size_t off_nvis = off_thr + 64 * 8;  // entries visible to each token of the group
+  static constexpr size_t off_hist = off_nvis + 64 * 8;
   static constexpr size_t off_grp = off_hist + (size_t)(G == 1 ? 1 : 2) * topk::kWarpBins * 4;  // [2][32] ints
   static constexpr size_t off_bar = off_grp + 256;
   static constexpr size_t off_tslot = off_bar + (2 * kStages + 2 * NB + 2) * 8;
@@ -186,7 +190,7 @@ struct IndexerSmem {
 template <int HI, int DI, int G>
 __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
     indexer_topk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                        const IndexerArgs a) {
+                        const __grid_constant__ IndexerArgs a) {
   using L = IndexerSmem<HI, DI, G>;
   using TS = TileShape<HI, G>;
   constexpr int N = L::N;
@@ -215,6 +219,7 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
   uint8_t* s_mb = smem + L::off_mb;
   int* s_cnt = reinterpret_cast<int*>(smem + L::off_cnt);
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L::off_thr);
+  int64_t* s_nvis = reinterpret_cast<int64_t*>(smem + L::off_nvis);
   int* s_hist = reinterpret_cast<int*>(smem + L::off_hist);
   int* s_grp = reinterpret_cast<int*>(smem + L::off_grp);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
@@ -308,11 +313,12 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
   for (int g = 0; g < G; ++g) {
     const int64_t r = row0 + g;
     int64_t t = -1;
-    if (r < a.rows) t = decode ? a.pos[r] : a.t0 + r;
+    if (r < a.rows) t = decode ? a.pos_at(r) : a.t0 + r;
     int64_t nv = n_visible(t, a.m) - a.j_base;  // entries of this (slice of the) cache visible to t
     if (nv < 0) nv = 0;
     if (nv > a.Nc) nv = a.Nc;
     tnvis[g] = nv;
+    if (tid == 0) s_nvis[g] = nv;
     if (nv > nvis_max) nvis_max = nv;
   }
   int64_t j_end = j_begin + a.split_tiles * 128;
@@ -547,15 +553,9 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
       pbase[t] = 0;
     }
     const uint32_t lt = (1u << lane) - 1u;
-    // entries visible to token gg of the group (recomputed where a loop over the
-    // tokens is not unrolled, so that no register array is indexed at run time)
-    auto token_nvis = [&](int gg) -> int64_t {
-      const int64_t r = row0 + gg;
-      if (r >= a.rows) return 0;
-      int64_t nv = n_visible(decode ? a.pos[r] : a.t0 + r, a.m) - a.j_base;
-      if (nv < 0) nv = 0;
-      return nv > a.Nc ? a.Nc : nv;
-    };
+    // entries visible to token gg of the group (from shared memory where a loop over
+    // the tokens is not unrolled, so that no register array is indexed at run time)
+    auto token_nvis = [&](int gg) -> int64_t { return s_nvis[gg]; };
     // keys held in fixed slots (no cut-back yet): the visible ones among the first n of the range
     auto fixed_count = [&](int64_t nv, int64_t n) -> int {
       int64_t lim = nv < j_end ? nv : j_end;
@@ -780,15 +780,21 @@ __global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __re
 }
 
 // Block-wide finalize for rows with many candidates (a split decode search):
-// 1024 threads per row.  One min/max pass and one 1024-bin histogram over the
-// score range find the bin that holds the k-th key; the keys of that bin are
-// resolved exactly (in-register sort when it holds at most 32, else the warp
-// radix fallback); the k best are compacted, sorted (per-warp register sorts
-// merged through shared memory) and written.  The row's keys are loaded 16 per
-// thread at a time, so the gather costs a few memory round trips.
+// 1024 threads per row, every candidate held in registers (slot u of thread t is
+// candidate u*1024 + t of the row's nsplit*k list slots, 16 slots at most; an
+// empty slot holds key 0, below every valid key).  A block-wide radix select on
+// the registers, 10 bits per pass from the top of the valid keys' span, finds
+// the k-th key (the boundary bin is sorted in registers once it holds at most
+// 32 keys); the k best are compacted into shared memory, sorted (per-warp
+// register sorts merged through shared memory) and written.  All the row's loads
+// are issued before any is used: one memory round trip.
 constexpr int kFinBlock = 1024;
 constexpr int kFinSort = 1024;  // keys sorted by the register/shared hybrid sort
+constexpr int kFinSlots = 16;   // candidate slots per thread: nsplit * k <= kFinSlots * kFinBlock
 
+// U: candidate slots per thread (10 keep the keys in registers for the decode
+// merges, nsplit * k <= 10240; 16 for the widest explicit merges)
+template <int U>
 __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const uint64_t* __restrict__ cand,
                                                                         const int* __restrict__ cand_cnt, int nsplit,
                                                                         int k, int32_t* __restrict__ idx,
@@ -799,158 +805,140 @@ __global__ void __launch_bounds__(kFinBlock) topk_finalize_block_kernel(const ui
   griddep_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t r = blockIdx.x;
-  const int cap = topk::next_pow2(nsplit * k);
-  uint64_t* buf = reinterpret_cast<uint64_t*>(bsmem);    // [cap] gathered candidates
   const int sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
-  uint64_t* sel = buf + cap;                              // [sel_cap] the k best
-  int* hist = reinterpret_cast<int*>(sel + sel_cap);      // [kWarpBins]
-  __shared__ int s_off[kMaxKeyRanges + 1];
+  uint64_t* sel = reinterpret_cast<uint64_t*>(bsmem);  // [sel_cap] the k best
+  int* hist = reinterpret_cast<int*>(sel + sel_cap);   // [kWarpBins]
   __shared__ uint32_t s_lo[kFinBlock / 32], s_hi[kFinBlock / 32];
+  __shared__ int s_n[kFinBlock / 32];
   __shared__ int s_bin, s_kept, s_inbin, s_nsel;
   __shared__ uint64_t s_thr;
-  // gather the per-range lists (offsets by a prefix over the counts).  The loads
-  // of the row are issued kGatherU per thread at a time, so that a row of
-  // nsplit * k keys takes a few memory round trips instead of one per key.
-  constexpr int kGatherU = 16;
   const int total = nsplit * k;
   const uint64_t* src = cand + (size_t)r * total;
-  uint64_t v[kGatherU];
+  const int* cnt_row = cand_cnt + r * nsplit;
+  // slot u holds entry i of list s, q = u * kFinBlock + tid = s * k + i: the list by
+  // a float reciprocal (q < 2^24: the estimate is off by at most one) and an exact
+  // integer correction.  The keys are loaded first; the list counts, read while
+  // they are in flight, then clear the slots past each list's end.
+  const float inv_k = 1.0f / (float)k;
+  __shared__ int s_cnt[kMaxKeyRanges];
+  uint64_t v[U];
 #pragma unroll
-  for (int u = 0; u < kGatherU; ++u) {
-    const int i = u * kFinBlock + tid;
-    v[u] = i < total ? __ldg(src + i) : 0;
+  for (int u = 0; u < U; ++u) {
+    const int q = u * kFinBlock + tid;
+    v[u] = q < total ? __ldg(src + q) : 0;
   }
-  if (tid < nsplit) s_off[tid + 1] = cand_cnt[r * nsplit + tid];
-  if (tid == 0) {
-    s_off[0] = 0;
-    s_nsel = 0;
-  }
-  for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
+  if (tid < nsplit) s_cnt[tid] = __ldg(cnt_row + tid);
   __syncthreads();
-  if (tid == 0)
-    for (int sp = 1; sp <= nsplit; ++sp) s_off[sp] += s_off[sp - 1];
-  __syncthreads();
-  const int cnt = s_off[nsplit];
-  // slot i of the row belongs to range i / k; the valid keys' score range is
-  // taken on the way
   uint32_t lo = 0xFFFFFFFFu, hi = 0;
-  for (int base = 0; base < total; base += kGatherU * kFinBlock) {
-    if (base > 0) {
+  int mine = 0;
 #pragma unroll
-      for (int u = 0; u < kGatherU; ++u) {
-        const int i = base + u * kFinBlock + tid;
-        v[u] = i < total ? __ldg(src + i) : 0;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kGatherU; ++u) {
-      const int i = base + u * kFinBlock + tid;
-      if (i < total) {
-        const int sp = i / k, e = i - sp * k;
-        if (e < s_off[sp + 1] - s_off[sp]) {
-          buf[s_off[sp] + e] = v[u];
-          const uint32_t sc = (uint32_t)(v[u] >> 32);
-          lo = sc < lo ? sc : lo;
-          hi = sc > hi ? sc : hi;
-        }
-      }
+  for (int u = 0; u < U; ++u) {
+    const int q = u * kFinBlock + tid;
+    int sp = (int)((float)q * inv_k);
+    if (sp * k > q) --sp;
+    else if ((sp + 1) * k <= q) ++sp;
+    if (q >= total || q - sp * k >= s_cnt[sp]) v[u] = 0;
+    if (v[u] != 0) {
+      const uint32_t sc = (uint32_t)(v[u] >> 32);
+      lo = sc < lo ? sc : lo;
+      hi = sc > hi ? sc : hi;
+      ++mine;
     }
   }
-  int nout = cnt;
-  if (cnt > k) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    }
-    if (lane == 0) {
-      s_lo[warp] = lo;
-      s_hi[warp] = hi;
-    }
-    __syncthreads();
-    lo = s_lo[0];
-    hi = s_hi[0];
-    for (int w = 1; w < kFinBlock / 32; ++w) {
-      lo = min(lo, s_lo[w]);
-      hi = max(hi, s_hi[w]);
-    }
-    // exact threshold: a block-wide radix select on the keys, 10 bits per pass
-    // from the top of their span, until the boundary bin is kept whole or holds at
-    // most 32 keys (then sorted in registers)
-    uint64_t thr = 0;
-    {
-      uint64_t base = (uint64_t)lo << 32;                   // every key lies in [base, base + 2^wl)
-      int wl = (hi > lo ? 32 - __clz(hi - lo) : 0) + 32;
-      int need = k;
-      for (;;) {
-        const int w = wl >= 10 ? 10 : wl;
-        const int sh = wl - w;
-        for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
-        if (tid == 0) s_nsel = 0;
-        __syncthreads();
-        for (int i = tid; i < cnt; i += kFinBlock) {
-          const uint64_t dk = buf[i] - base;
-          if (wl >= 64 || dk < (1ull << wl)) atomicAdd(&hist[(int)(dk >> sh)], 1);
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  }
+  if (lane == 0) {
+    s_lo[warp] = lo;
+    s_hi[warp] = hi;
+    s_n[warp] = mine;
+  }
+  if (tid == 0) s_nsel = 0;
+  __syncthreads();
+  int cnt = 0;
+  lo = s_lo[0];
+  hi = s_hi[0];
+  for (int w = 0; w < kFinBlock / 32; ++w) {
+    lo = min(lo, s_lo[w]);
+    hi = max(hi, s_hi[w]);
+    cnt += s_n[w];
+  }
+  uint64_t thr = 1;  // every valid key (nonzero)
+  if (cnt > k) {
+    // exact threshold: a block-wide radix select, 10 bits per pass from the top of
+    // the keys' span, until the boundary bin is kept whole or holds at most 32 keys
+    uint64_t base = (uint64_t)lo << 32;  // every valid key lies in [base, base + 2^wl)
+    int wl = (hi > lo ? 32 - __clz(hi - lo) : 0) + 32;
+    int need = k;
+    for (;;) {
+      const int w = wl >= 10 ? 10 : wl;
+      const int sh = wl - w;
+      for (int b = tid; b < topk::kWarpBins; b += kFinBlock) hist[b] = 0;
+      if (tid == 0) s_nsel = 0;
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint64_t dk = v[u] - base;
+        if (v[u] != 0 && (wl >= 64 || dk < (1ull << wl))) atomicAdd(&hist[(int)(dk >> sh)], 1);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int bin, kept;
+        topk::warp_hist_cut(hist, need, lane, &bin, &kept);
+        if (lane == 0) {
+          s_bin = bin;
+          s_kept = kept;
+          s_inbin = hist[bin];
         }
+      }
+      __syncthreads();
+      const int bin = s_bin, in_bin = s_inbin;
+      need -= s_kept - in_bin;  // keys in the higher bins are all kept
+      base += (uint64_t)bin << sh;
+      wl = sh;
+      if (need == in_bin) {  // the whole boundary bin is kept
+        thr = base;
+        break;
+      }
+      if (in_bin <= 32) {
+        // the boundary bin's keys, sorted in registers by one warp
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (v[u] != 0 && v[u] - base < (1ull << wl)) sel[atomicAdd(&s_nsel, 1)] = v[u];
         __syncthreads();
         if (warp == 0) {
-          int bin, kept;
-          topk::warp_hist_cut(hist, need, lane, &bin, &kept);
-          if (lane == 0) {
-            s_bin = bin;
-            s_kept = kept;
-            s_inbin = hist[bin];
-          }
+          uint64_t x = lane < in_bin ? sel[lane] : 0;
+          x = topk::warp_sort32_desc(x, lane);
+          const uint64_t t = __shfl_sync(0xffffffffu, x, need - 1);
+          if (lane == 0) s_thr = t;
         }
         __syncthreads();
-        const int bin = s_bin, in_bin = s_inbin;
-        need -= s_kept - in_bin;  // keys in the higher bins are all kept
-        base += (uint64_t)bin << sh;
-        wl = sh;
-        if (need == in_bin) {  // the whole boundary bin is kept
-          thr = base;
-          break;
-        }
-        if (in_bin <= 32) {
-          // the boundary bin's keys into `sel`, sorted in registers
-          for (int i = tid; i < cnt; i += kFinBlock) {
-            const uint64_t v = buf[i];
-            if (v - base < (1ull << wl)) sel[atomicAdd(&s_nsel, 1)] = v;
-          }
-          __syncthreads();
-          if (warp == 0) {
-            uint64_t x = lane < in_bin ? sel[lane] : 0;
-            x = topk::warp_sort32_desc(x, lane);
-            const uint64_t t = __shfl_sync(0xffffffffu, x, need - 1);
-            if (lane == 0) s_thr = t;
-          }
-          __syncthreads();
-          thr = s_thr;
-          break;
-        }
-        __syncthreads();  // everyone has read s_bin / s_inbin before the next pass
+        thr = s_thr;
+        break;
       }
+      __syncthreads();  // everyone has read s_bin / s_inbin before the next pass
     }
-    // the k keys >= thr, one shared-memory atomic per warp and step
     if (tid == 0) s_nsel = 0;
     __syncthreads();
-    for (int base = 0; base < cnt; base += kFinBlock) {
-      const int i = base + tid;
-      const uint64_t x = i < cnt ? buf[i] : 0;
-      const bool take = i < cnt && x >= thr;
-      const uint32_t mask = __ballot_sync(0xffffffffu, take);
-      if (mask) {
-        int pos = 0;
-        if (lane == 0) pos = atomicAdd(&s_nsel, __popc(mask));
-        pos = __shfl_sync(0xffffffffu, pos, 0);
-        if (take) sel[pos + __popc(mask & ((1u << lane) - 1u))] = x;
-      }
-    }
-    __syncthreads();
-    nout = s_nsel;
-  } else {
-    for (int i = tid; i < cnt; i += kFinBlock) sel[i] = buf[i];
   }
+  // the keys >= thr (at most k of them), one shared-memory atomic per warp and slot
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const bool take = v[u] >= thr;  // thr >= 1: empty slots never
+    const uint32_t mask = __ballot_sync(0xffffffffu, take);
+    if (mask) {
+      int pos = 0;
+      if (lane == 0) pos = atomicAdd(&s_nsel, __popc(mask));
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      if (take) sel[pos + __popc(mask & lt)] = v[u];
+    }
+  }
+  __syncthreads();
+  const int nout = s_nsel;
   const int P = topk::next_pow2(nout > 1 ? nout : 1);
   if (P <= kFinSort) {
     // pad to the register sort's fixed size
@@ -979,13 +967,15 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
   if (nsplit > 1) {
     // few rows with many candidates each: a block per row
     const size_t sel_cap = topk::next_pow2(k) > kFinSort ? topk::next_pow2(k) : kFinSort;
-    const size_t smem = (size_t)topk::next_pow2(nsplit * k) * 8 + sel_cap * 8 + topk::kWarpBins * 4;
-    if (smem > kSmemLimit || nsplit > kMaxKeyRanges) return cudaErrorInvalidConfiguration;
-    cudaError_t e =
-        cudaFuncSetAttribute(topk_finalize_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = sel_cap * 8 + topk::kWarpBins * 4;
+    if ((int64_t)nsplit * k > (int64_t)kFinSlots * kFinBlock || nsplit > kMaxKeyRanges)
+      return cudaErrorInvalidConfiguration;
+    auto kern = (int64_t)nsplit * k <= 10 * kFinBlock ? topk_finalize_block_kernel<10>
+                                                      : topk_finalize_block_kernel<kFinSlots>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(topk_finalize_block_kernel, dim3((unsigned)rows), dim3(kFinBlock), smem, stream, pdl, cand,
-                         cand_cnt, nsplit, k, idx, scores, keys_out);
+    return launch_kernel(kern, dim3((unsigned)rows), dim3(kFinBlock), smem, stream, pdl, cand, cand_cnt, nsplit, k,
+                         idx, scores, keys_out);
   }
   const size_t per_warp = (size_t)topk::next_pow2(nsplit * k) * 8 + topk::kWarpBins * 4;
   int wpb = (int)((kSmemLimit - 1024) / per_warp);
@@ -1094,8 +1084,9 @@ static bool choose_cap(int k, int* cap, int* check) {
 }
 
 template <int HI, int DI, int G>
-static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, IndexerArgs a, dim3 grid,
+static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, const IndexerArgs& a_in, dim3 grid,
                               cudaStream_t stream, bool pdl) {
+  IndexerArgs a = a_in;
   a.fault = take_injected_fault();
   using L = IndexerSmem<HI, DI, G>;
   CUtensorMap qmap, kmap;
@@ -1110,23 +1101,23 @@ static cudaError_t launch_one(const uint8_t* q_codes, const uint8_t* k_codes, In
   return launch_kernel(kern, grid, dim3(Epi<HI, G>::kBlock), smem, stream, pdl, qmap, kmap, a);
 }
 
+// pdl: the decode positions come from a copy kernel of the same call just before
 template <int HI, int DI>
-static cudaError_t dispatch_g(bool decode, const uint8_t* q_codes, const uint8_t* k_codes, IndexerArgs a,
-                              dim3 grid, cudaStream_t stream) {
-  // decode: the positions come from the upload kernel just before
-  if (decode) return launch_one<HI, DI, 1>(q_codes, k_codes, a, grid, stream, true);
+static cudaError_t dispatch_g(bool decode, const uint8_t* q_codes, const uint8_t* k_codes, const IndexerArgs& a,
+                              dim3 grid, cudaStream_t stream, bool pdl) {
+  if (decode) return launch_one<HI, DI, 1>(q_codes, k_codes, a, grid, stream, pdl);
   return launch_one<HI, DI, Geometry<HI>::G>(q_codes, k_codes, a, grid, stream, false);
 }
 
 template <int DI>
-static cudaError_t dispatch_hi(int HI, bool decode, const uint8_t* q_codes, const uint8_t* k_codes, IndexerArgs a,
-                               dim3 grid, cudaStream_t stream) {
+static cudaError_t dispatch_hi(int HI, bool decode, const uint8_t* q_codes, const uint8_t* k_codes,
+                               const IndexerArgs& a, dim3 grid, cudaStream_t stream, bool pdl = false) {
   switch (HI) {
-    case 4: return dispatch_g<4, DI>(decode, q_codes, k_codes, a, grid, stream);
-    case 8: return dispatch_g<8, DI>(decode, q_codes, k_codes, a, grid, stream);
-    case 16: return dispatch_g<16, DI>(decode, q_codes, k_codes, a, grid, stream);
-    case 32: return dispatch_g<32, DI>(decode, q_codes, k_codes, a, grid, stream);
-    case 64: return dispatch_g<64, DI>(decode, q_codes, k_codes, a, grid, stream);
+    case 4: return dispatch_g<4, DI>(decode, q_codes, k_codes, a, grid, stream, pdl);
+    case 8: return dispatch_g<8, DI>(decode, q_codes, k_codes, a, grid, stream, pdl);
+    case 16: return dispatch_g<16, DI>(decode, q_codes, k_codes, a, grid, stream, pdl);
+    case 32: return dispatch_g<32, DI>(decode, q_codes, k_codes, a, grid, stream, pdl);
+    case 64: return dispatch_g<64, DI>(decode, q_codes, k_codes, a, grid, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1175,13 +1166,19 @@ cudaError_t launch_indexer_prefill(const uint8_t* q_codes, const uint8_t* q_scal
 }
 
 // Decode: rows = B sequences, each with its own cache of Ncap entries and position
-// pos[b] (device), key range split `nsplit` ways; candidates merged afterwards.
+// pos[b] (pos_in on the host when B <= kInlinePos, else pos_dev on the device,
+// copied there by the kernel just before: pdl), key range split `nsplit` ways;
+// candidates merged afterwards.
 cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* w_codes,
                                   const uint8_t* k_codes, const uint8_t* k_scales, int B, const int64_t* pos_dev,
-                                  int64_t nvis_max, int64_t Ncap, int HI, int DI, int m, int k, int nsplit,
-                                  uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores, uint64_t* keys_out,
-                                  int* status, cudaStream_t stream, int64_t j_base) {
+                                  const int64_t* pos_in, bool pdl, int64_t nvis_max, int64_t Ncap, int HI, int DI,
+                                  int m, int k, int nsplit, uint64_t* cand, int* cand_cnt, int32_t* idx, float* scores,
+                                  uint64_t* keys_out, int* status, cudaStream_t stream, int64_t j_base) {
   IndexerArgs a{};
+  if (B <= kInlinePos) {
+    for (int b = 0; b < B; ++b) a.pos_in[b] = pos_in[b];
+    a.npos_in = B;
+  }
   a.j_base = j_base;
   a.q_scales = q_scales;
   a.w_codes = w_codes;
@@ -1199,8 +1196,8 @@ cudaError_t launch_indexer_decode(const uint8_t* q_codes, const uint8_t* q_scale
   a.cand_cnt = cand_cnt;
   a.status = status;
   dim3 grid((unsigned)B, (unsigned)nsplit);
-  cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, true, q_codes, k_codes, a, grid, stream)
-                            : dispatch_hi<64>(HI, true, q_codes, k_codes, a, grid, stream);
+  cudaError_t e = DI == 128 ? dispatch_hi<128>(HI, true, q_codes, k_codes, a, grid, stream, pdl)
+                            : dispatch_hi<64>(HI, true, q_codes, k_codes, a, grid, stream, pdl);
   if (e != cudaSuccess) return e;
   return launch_finalize(cand, cand_cnt, nsplit, k, B, idx, scores, keys_out, stream, true);
 }

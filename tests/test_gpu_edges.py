@@ -184,6 +184,33 @@ def test_decode_short_contexts_all_sequences(csa):
         assert_attention_close(O[b:b + 1], o, "decode attention seq %d" % b)
 
 
+def test_decode_positions_beyond_the_inline_limit(csa):
+    """More sequences (70) than the kernel arguments carry positions for: the
+    positions go to the workspace through the copy kernel first, and the search,
+    the merge and the attention read them from there.  Sequences on both sides of
+    the limit (63, 64) are checked, with mixed positions."""
+    B = 70
+    wl = inputs.Workload("dec_b70", H=64, d=128, m=4, k=64, W=32, HI=16, dI=128, batch=B, context=2048, seed=27)
+    g = inputs.decode_batch(wl)
+    pos = [(97 * b + 13) % wl.context for b in range(B)]
+    pos[69] = wl.context - 1
+    scale = 1.0 / math.sqrt(wl.d)
+    gc = {k: v.cuda() for k, v in g.items()}
+    O, lse, idx, scores, ws = csa.csa_decode(gc["q"], gc["qI_codes"], gc["qI_scales"], gc["w_codes"], gc["Kc"],
+                                             gc["Vc"], gc["kI_codes"], gc["kI_scales"], gc["Kwin"], gc["Vwin"], pos,
+                                             wl.m, wl.k, scale)
+    assert csa.csa_check_status(ws) == 0
+    for b in (0, 5, 63, 64, 69):
+        t = pos[b]
+        I = oracle.indexer(g["qI_codes"][b:b + 1], g["qI_scales"][b:b + 1], g["w_codes"][b:b + 1], g["kI_codes"][b],
+                           g["kI_scales"][b], t, wl.m)
+        want_idx, want_top = oracle.topk(I, oracle.n_vis([t], wl.m), wl.k)
+        assert_topk_exact(idx[b:b + 1], scores[b:b + 1], want_idx, want_top, "decode B=70 seq %d" % b)
+        o, l = oracle.attention(g["q"][b:b + 1], g["Kc"][b], g["Vc"][b], g["Kwin"][b], g["Vwin"][b], t, wl.m, wl.W,
+                                scale, sel=want_idx, rows=[0], raw_pos0=t - wl.W + 1)
+        assert_attention_close(O[b:b + 1], o, "decode B=70 attention seq %d" % b)
+
+
 def test_decode_k2048_split_search(csa):
     """Decode with k=2048 over a 64K-token context: the key range is split over
     several CTAs and the merged selection is larger than the block finalize's
