@@ -211,6 +211,29 @@ def test_decode_positions_beyond_the_inline_limit(csa):
         assert_attention_close(O[b:b + 1], o, "decode B=70 attention seq %d" % b)
 
 
+def test_decode_search_long_key_ranges(csa):
+    """Long key ranges (38 sequences of 131072 entries: three ranges of 342 tiles
+    each), so that the search's candidate buffers are cut back several times and
+    meet often.  The k best keys of two sequences are checked against the oracle,
+    bit for bit."""
+    B, N, HI, dI, m, k = 38, 1 << 17, 16, 128, 4, 512
+    qc, qs = inputs.mxfp4((B, HI), dI, 31, "qI")
+    w = inputs.uniform_u8((B, HI), 31, "w", 0, 15)
+    kc, ks = inputs.mxfp4((B, N), dI, 31, "kI")
+    pos = [N * m - 1 - 977 * b for b in range(B)]
+    keys, ws = csa.csa_decode_search(qc.cuda(), qs.cuda(), w.cuda(), kc.cuda(), ks.cuda(), pos, m, k)
+    assert csa.csa_check_status(ws) == 0
+    kk = keys.cpu().numpy().view(np.uint64)
+    units = ((kk >> np.uint64(32)).astype(np.uint32) ^ np.uint32(0x80000000)).view(np.int32)
+    j = (np.uint64(0xFFFFFFFF) - (kk & np.uint64(0xFFFFFFFF))).astype(np.int64)
+    for b in (0, B - 1):
+        t = pos[b]
+        I = oracle.indexer(qc[b:b + 1], qs[b:b + 1], w[b:b + 1], kc[b], ks[b], t, m)
+        want_idx, want_top = oracle.topk(I, oracle.n_vis([t], m), k)
+        assert_topk_exact(torch.from_numpy(j[b:b + 1]), torch.from_numpy(units[b:b + 1].astype(np.float32) / 128.0),
+                          want_idx, want_top, "decode search seq %d" % b)
+
+
 def test_decode_k2048_split_search(csa):
     """Decode with k=2048 over a 64K-token context: the key range is split over
     several CTAs and the merged selection is larger than the block finalize's
