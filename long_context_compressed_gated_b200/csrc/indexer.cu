@@ -546,6 +546,10 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
     uint64_t pkey[G0];
     uint32_t pbal[G0];
     int pbase[G0];
+    // one token per warp (G0 = 1): the range of the scores this thread stores in
+    // fixed slots, so that the final selection skips its range pass
+    constexpr bool kSpan = G0 == 1;
+    uint32_t span_lo = 0xFFFFFFFFu, span_hi = 0u;
 #pragma unroll
     for (int t = 0; t < G0; ++t) {
       pkey[t] = 0;
@@ -635,7 +639,14 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
           if (thr[t] == 0) {
             // no cut-back yet: every visible key is kept, in its fixed slot (the
             // visible keys of a tile are a prefix of it, so the slots stay dense)
-            if (vis) s_cand[(size_t)(g_lo + t) * cap + (size_t)it * 128 + quarter * 32 + lane] = pkey[t];
+            if (vis) {
+              s_cand[(size_t)(g_lo + t) * cap + (size_t)it * 128 + quarter * 32 + lane] = pkey[t];
+              if (kSpan) {
+                const uint32_t su = (uint32_t)(pkey[t] >> 32);
+                span_lo = su < span_lo ? su : span_lo;
+                span_hi = su > span_hi ? su : span_hi;
+              }
+            }
           } else {
             pbal[t] = __ballot_sync(0xffffffffu, vis && pkey[t] >= thr[t]);
           }
@@ -682,14 +693,16 @@ __global__ void __launch_bounds__(Epi<HI, G>::kBlock, 1)
       if (row0 + gg >= a.rows) break;  // uniform over the group
       const int64_t r = row0 + gg;
       uint64_t* buf = s_cand + (size_t)gg * cap;
-      int cnt = s_thr[gg] == 0 ? fixed_count(token_nvis(gg), (int64_t)ntiles * 128) : s_cnt[gg];
-      if (cnt > a.k) {
-        const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, ghist, gscr,
-                                                       gt, gbar);
-        cnt = topk::group_compact_ge<GNT>(buf, cnt, tq, gscr, gt, gbar);
-      }
+      const bool fixed = s_thr[gg] == 0;  // no cut-back: every visible key in its fixed slot
+      int cnt = fixed ? fixed_count(token_nvis(gg), (int64_t)ntiles * 128) : s_cnt[gg];
       uint64_t* out = a.cand + ((size_t)r * a.nsplit + split) * a.k;
-      for (int q = gt; q < cnt; q += GNT) out[q] = buf[q];
+      if (cnt > a.k) {
+        const uint64_t tq = topk::group_threshold<GNT>(buf, cnt, a.k, 0, true, ghist, gscr, gt, gbar,
+                                                       kSpan && fixed, span_lo, span_hi);
+        cnt = topk::group_emit_ge<GNT>(buf, cnt, tq, out, gscr, gt, gbar);
+      } else {
+        for (int q = gt; q < cnt; q += GNT) out[q] = buf[q];
+      }
       if (gt == 0) a.cand_cnt[r * a.nsplit + split] = cnt;
     }
   }

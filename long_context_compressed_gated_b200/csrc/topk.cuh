@@ -349,14 +349,15 @@ __device__ void warp_bitonic_desc(uint64_t* buf, int P, int lane) {
 // boundary histogram bin are kept, unless that keeps more than `room`.
 template <int NT>
 __device__ uint64_t group_threshold(const uint64_t* buf, int cnt, int keep, int room, bool exact, int* hist,
-                                    int* scr, int gt, int bar) {
+                                    int* scr, int gt, int bar, bool span_known = false, uint32_t span_lo = 0,
+                                    uint32_t span_hi = 0) {
   constexpr int NW = NT / 32;
   const int warp = gt >> 5, lane = gt & 31;
   if (cnt <= keep) return 0;
   uint64_t* s_thr64 = reinterpret_cast<uint64_t*>(scr + 2 * NW + 4);  // 8-byte aligned slot
-  // score range
-  uint32_t lo = 0xFFFFFFFFu, hi = 0;
-  for (int i = gt; i < cnt; i += NT) {
+  // score range (span_known: each thread brings the range of the scores it wrote)
+  uint32_t lo = span_known ? span_lo : 0xFFFFFFFFu, hi = span_known ? span_hi : 0;
+  for (int i = gt; i < cnt && !span_known; i += NT) {
     const uint32_t sc = (uint32_t)(buf[i] >> 32);
     lo = sc < lo ? sc : lo;
     hi = sc > hi ? sc : hi;
@@ -473,6 +474,47 @@ __device__ int group_compact_ge(uint64_t* buf, int cnt, uint64_t thr, int* scr, 
     out = total;
   }
   return out;
+}
+
+// The keys of buf[0..cnt) >= thr written to out[0..), in an order fixed by their
+// positions; returns how many.  Rounds of U*NT keys: every thread loads its keys
+// of the round, a per-warp count places them; the counts are double-buffered by
+// round parity, so one barrier per round suffices.  scr: 2*NT/32 ints.
+template <int NT>
+__device__ int group_emit_ge(const uint64_t* buf, int cnt, uint64_t thr, uint64_t* out, int* scr, int gt, int bar) {
+  constexpr int NW = NT / 32, U = 4;
+  const int warp = gt >> 5, lane = gt & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  int done = 0;
+  for (int base = 0, round = 0; base < cnt; base += U * NT, ++round) {
+    int* cnts = scr + (round & 1) * NW;
+    uint64_t v[U];
+    uint32_t bal[U];
+    int mine = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * NT + gt;
+      v[u] = i < cnt ? buf[i] : 0;
+      bal[u] = __ballot_sync(0xffffffffu, i < cnt && v[u] >= thr);
+      mine += __popc(bal[u]);
+    }
+    if (lane == 0) cnts[warp] = mine;
+    named_sync(bar, NT);
+    int woff = done, total = done;
+    for (int w = 0; w < NW; ++w) {
+      const int c = cnts[w];
+      woff += w < warp ? c : 0;
+      total += c;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if ((bal[u] >> lane) & 1u) out[woff + __popc(bal[u] & lt)] = v[u];
+      woff += __popc(bal[u]);
+    }
+    done = total;
+  }
+  named_sync(bar, NT);  // the counts are read before the caller reuses scr
+  return done;
 }
 
 // Lane-major register bitonic sort of 32*R keys, descending: element e = lane*R + r
