@@ -746,6 +746,45 @@ __device__ __forceinline__ void finalize_sorted(const uint64_t* buf, int cnt, in
   }
 }
 
+// One range per row (prefill), at most 32*R candidates: the row's candidates go
+// straight from global memory into registers (all R loads in flight, coalesced:
+// the sort does not care where a key starts), are sorted there and written.
+template <int R>
+__device__ __forceinline__ void finalize_direct(const uint64_t* __restrict__ src, int n, int k, int64_t r,
+                                                int32_t* idx, float* scores, uint64_t* keys_out, int lane) {
+  uint64_t v[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int e = i * 32 + lane;
+    v[i] = e < n ? __ldg(src + e) : 0;
+  }
+  topk::warp_sort_lm_desc<R>(v, lane);
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int q = lane * R + i;
+    if (q < k) {
+      const bool ok = q < n;
+      if (idx) idx[r * k + q] = ok ? (int32_t)topk::key_index(v[i]) : -1;
+      if (scores) scores[r * k + q] = ok ? (float)topk::key_score(v[i]) * (1.0f / 128.0f) : -INFINITY;
+      if (keys_out) keys_out[r * k + q] = ok ? v[i] : 0;
+    }
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(256) topk_finalize_direct_kernel(const uint64_t* __restrict__ cand,
+                                                                   const int* __restrict__ cand_cnt, int k,
+                                                                   int64_t rows, int32_t* __restrict__ idx,
+                                                                   float* __restrict__ scores,
+                                                                   uint64_t* __restrict__ keys_out) {
+  griddep_wait();  // the candidate lists come from the kernel before
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  finalize_direct<R>(cand + (size_t)r * k, cand_cnt[r], k, r, idx, scores, keys_out, lane);
+}
+
 __global__ void __launch_bounds__(256) topk_finalize_kernel(const uint64_t* __restrict__ cand,
                                                             const int* __restrict__ cand_cnt, int nsplit, int k,
                                                             int64_t rows, int32_t* __restrict__ idx,
@@ -988,6 +1027,12 @@ static cudaError_t launch_finalize(const uint64_t* cand, const int* cand_cnt, in
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_kernel(kern, dim3((unsigned)rows), dim3(kFinBlock), smem, stream, pdl, cand, cand_cnt, nsplit, k,
+                         idx, scores, keys_out);
+  }
+  if (nsplit == 1 && k <= 1024) {
+    // one range of at most 1024 keys per row: registers only, no shared memory
+    auto kern = k <= 512 ? topk_finalize_direct_kernel<16> : topk_finalize_direct_kernel<32>;
+    return launch_kernel(kern, dim3((unsigned)ceil_div(rows, 8)), dim3(256), 0, stream, pdl, cand, cand_cnt, k, rows,
                          idx, scores, keys_out);
   }
   const size_t per_warp = (size_t)topk::next_pow2(nsplit * k) * 8 + topk::kWarpBins * 4;
