@@ -38,14 +38,14 @@ E2E_CHUNKS = 16  # query chunks of the pipelined end-to-end step
 
 PHASE_TRAFFIC = {
     # DRAM bytes (read + written) of one full-size launch, from the one-pass ncu capture
-    # recorded in profiles/launch_list_bench_default.md; the indexer phase is the
+    # of the bench's launch list (summary under profiles/); the indexer phase is the
     # indexer kernel plus the finalize kernel
     "indexer_topk": (145393664 + 87410432 + 130292736 + 30677248,
                      "ncu dram__bytes_read.sum + dram__bytes_write.sum of the full-size indexer and finalize "
-                     "launches (profiles/launch_list_bench_default.md)"),
+                     "launches (one-pass capture of the bench's launch list, profiles/)"),
     "sparse_attn": (626069504 + 487205632,
                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of a full-size attention launch "
-                    "(profiles/launch_list_bench_default.md)"),
+                    "(one-pass capture of the bench's launch list, profiles/)"),
 }
 
 
