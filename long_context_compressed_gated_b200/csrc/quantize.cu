@@ -25,6 +25,17 @@ __device__ __forceinline__ uint32_t e2m1_magnitude_code(float y) {
          (uint32_t)(y > 2.5f) + (uint32_t)(y >= 3.5f) + (uint32_t)(y > 5.0f);
 }
 
+// floor(log2 a) of a bf16 magnitude a > 0 given by its bits (sign cleared), from
+// the format's fields: normal 1.m * 2^(E-127); subnormal m * 2^-133.
+__device__ __forceinline__ int floor_log2_bf16(uint32_t bits) {
+  const int E = (int)(bits >> 7);
+  return E > 0 ? E - 127 : (31 - __clz(bits & 0x7Fu)) - 133;
+}
+
+// 2^-X as an fp32 value (X in [-127, 126]: a normal power of two), so that x * 2^-X
+// is the correctly rounded scaling (exact unless the product is subnormal)
+__device__ __forceinline__ float pow2_neg(int X) { return __uint_as_float((uint32_t)(127 - X) << 23); }
+
 __global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const uint4* __restrict__ x, int64_t nblocks, int mode,
                                                              uint4* __restrict__ codes,
                                                              uint8_t* __restrict__ scales) {
@@ -55,18 +66,15 @@ __global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const uint4* __rest
     return;
   }
   int X = -127;
-  if (amax_bits != 0) {
-    int e;
-    frexpf(__uint_as_float(amax_bits << 16), &e);  // amax = f * 2^e, f in [0.5, 1)
-    X = e - 3;                                     // floor(log2 amax) - 2
-  }
-  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  if (amax_bits != 0) X = floor_log2_bf16(amax_bits) - 2;  // at most 125 (finite bf16)
+  X = X < -127 ? -127 : X;
   if (mode == CSA_MX_INDEXER) X = X < -2 ? -2 : (X > 1 ? 1 : X);
+  const float p = pow2_neg(X);
   uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const uint32_t b = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-    const float y = ldexpf(__uint_as_float((b & 0x7FFFu) << 16), -X);  // exact: a power-of-two scaling
+    const float y = __fmul_rn(__uint_as_float((b & 0x7FFFu) << 16), p);
     const uint32_t code = ((b >> 12) & 8u) | e2m1_magnitude_code(y);
     out[i >> 3] |= code << (4 * (i & 7));
   }
@@ -114,18 +122,15 @@ __global__ void __launch_bounds__(256) mxfp8_quantize_kernel(const uint4* __rest
     return;
   }
   int X = -127;
-  if (amax_bits != 0) {
-    int e;
-    frexpf(__uint_as_float(amax_bits << 16), &e);
-    X = e - 9;  // floor(log2 amax) - 8
-  }
-  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  if (amax_bits != 0) X = floor_log2_bf16(amax_bits) - 8;  // at most 119 (finite bf16)
+  X = X < -127 ? -127 : X;
+  const float p = pow2_neg(X);
   uint32_t out[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     // elements 4q .. 4q+3 (words 2q, 2q+1)
-    const float a0 = ldexpf(bf16_lo(w[2 * q]), -X), a1 = ldexpf(bf16_hi(w[2 * q]), -X);
-    const float a2 = ldexpf(bf16_lo(w[2 * q + 1]), -X), a3 = ldexpf(bf16_hi(w[2 * q + 1]), -X);
+    const float a0 = __fmul_rn(bf16_lo(w[2 * q]), p), a1 = __fmul_rn(bf16_hi(w[2 * q]), p);
+    const float a2 = __fmul_rn(bf16_lo(w[2 * q + 1]), p), a3 = __fmul_rn(bf16_hi(w[2 * q + 1]), p);
     out[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
   }
   codes[blk * 2] = make_uint4(out[0], out[1], out[2], out[3]);
