@@ -16,13 +16,14 @@ namespace csa {
 
 namespace {
 
-// E2M1 magnitude code of y >= 0 (y exact in fp32): the number of rounding
-// boundaries y has passed.  The boundaries are the midpoints between the
-// magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; a midpoint itself goes to the even
-// code, hence ">" where the lower neighbour is even and ">=" where it is odd.
-__device__ __forceinline__ uint32_t e2m1_magnitude_code(float y) {
-  return (uint32_t)(y > 0.25f) + (uint32_t)(y >= 0.75f) + (uint32_t)(y > 1.25f) + (uint32_t)(y >= 1.75f) +
-         (uint32_t)(y > 2.5f) + (uint32_t)(y >= 3.5f) + (uint32_t)(y > 5.0f);
+// Two floats -> one byte of two E2M1 codes (round to nearest, ties to the even
+// code, saturating at +-6), a in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float a, float b) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tmov.b16 %0, {t, 0};\n\t}"
+      : "=h"(r)
+      : "f"(b), "f"(a));
+  return r & 0xFFu;
 }
 
 // floor(log2 a) of a bf16 magnitude a > 0 given by its bits (sign cleared), from
@@ -72,11 +73,12 @@ __global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const uint4* __rest
   const float p = pow2_neg(X);
   uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t b = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-    const float y = __fmul_rn(__uint_as_float((b & 0x7FFFu) << 16), p);
-    const uint32_t code = ((b >> 12) & 8u) | e2m1_magnitude_code(y);
-    out[i >> 3] |= code << (4 * (i & 7));
+  for (int i = 0; i < 16; ++i) {
+    // elements 2i (low half of word i) and 2i+1: E2M1 of x / 2^X by the hardware
+    // conversion (nearest, ties to the even code, saturating at +-6, sign kept),
+    // the first element in the low nibble
+    const float y0 = __fmul_rn(bf16_lo(w[i]), p), y1 = __fmul_rn(bf16_hi(w[i]), p);
+    out[i >> 2] |= e2m1x2(y0, y1) << (8 * (i & 3));
   }
   codes[blk] = make_uint4(out[0], out[1], out[2], out[3]);
   scales[blk] = (uint8_t)(X + 127);
