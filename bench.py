@@ -681,19 +681,33 @@ def run_quantize(csa, steps):
 
 def run_compress(csa, wl, steps):
     """The gated compression of the HCA prefill workload alone (m' = 128, 131072
-    tokens: 100 MB of K, V, Z).  The inputs fit in L2, so every step first
-    overwrites a 256 MB buffer; its own time, measured alone, is subtracted."""
-    d = inputs.prefill_layer(wl, device="cuda", with_indexer=False, with_q=False)
+    tokens: 100 MB of K, V, Z).  The inputs fit in L2, so the launches cycle
+    through three copies of them (303 MB, more than twice L2): every launch reads
+    inputs that the two launches before it have evicted, and L2 then holds only
+    clean lines (a flush by writing a large buffer leaves dirty lines whose
+    write-back would land in the timed kernel).  The launches are queued behind a
+    short device-side sleep so that the host's call time stays out of the
+    measurement."""
+    sets = [inputs.prefill_layer(wl, device="cuda", with_indexer=False, with_q=False) for _ in range(3)]
     Kc = torch.empty(wl.T // wl.m_hca, wl.d, dtype=torch.bfloat16, device="cuda")
     Vc = torch.empty_like(Kc)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
-    def step():
-        flush.zero_()
+    def launch(i):
+        d = sets[i % len(sets)]
         csa.csa_compress(d["K"], d["V"], d["Z"], d["B_hca"], wl.m_hca, Kc=Kc, Vc=Vc)
 
-    reps = max(20, steps)
-    ms = _event_ms(step, reps) - _event_ms(lambda: flush.zero_(), reps)
+    reps = 3 * max(10, steps)
+    for i in range(6):
+        launch(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(4_000_000)
+    e0.record()
+    for i in range(reps):
+        launch(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
     by = 3 * wl.T * wl.d * 2 + 2 * (wl.T // wl.m_hca) * wl.d * 2 + wl.m_hca * wl.d * 4
     return {"ms": ms, "bytes": by}
 
@@ -737,7 +751,8 @@ def run_extra(name, csa, peaks, steps, warmup, T=None):
         r = run_compress(csa, w2, steps)
         gbs = r["bytes"] / (r["ms"] * 1e-3) / 1e9
         return {"compress_hca_T%d_m%d" % (w2.T, w2.m_hca): {"ms": r["ms"], "bytes": r["bytes"], "gbs": gbs,
-                                                           "frac_hbm": gbs / peaks["hbm_gbs"], "l2": "flushed"}}
+                                                           "frac_hbm": gbs / peaks["hbm_gbs"],
+                                                           "l2": "three input copies in turn (303 MB)"}}
     if name == "quantize":
         return {"quantize": {k: dict(v, frac_hbm=v["gbs"] / peaks["hbm_gbs"]) for k, v in run_quantize(csa, steps).items()}}
     if name == "stack":

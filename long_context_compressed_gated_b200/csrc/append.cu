@@ -36,7 +36,7 @@ struct AppendArgs {
   const __nv_bfloat16 *Kn, *Vn, *Zn;  // [B, d] the new tokens
   const float* Bias;                  // [m, d]
   const uint8_t *kIc_new, *kIs_new;   // [B, dI/2], [B, dI/32] or null
-  int d, m, W, dI, L, S;
+  int d, m, W, dI, S;
   int64_t Ncap;
   __nv_bfloat16 *Kwin, *Vwin;         // [B, W, d]
   __nv_bfloat16 *Kblk, *Vblk, *Zblk;  // [B, m, d]
@@ -44,8 +44,8 @@ struct AppendArgs {
   uint8_t *kIc, *kIs;                 // [B, Ncap, dI/2], [B, Ncap, dI/32] or null
 };
 
-// blockDim.x = max(256, the pooling group of a block); shared memory:
-// pool_smem_bytes (the staged rows of the pooling, then its merge slots).
+// blockDim.x = max(256, the pooling group of a block); shared memory: the
+// merge scratch of that group (gate_scratch_floats).
 __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const AppendArgs a, const AppendPos P,
                                                                         int b0) {
   extern __shared__ __align__(16) float sh_gate[];
@@ -93,28 +93,42 @@ __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const Ap
   if (slot == a.m - 1) {
     const int64_t j = (pos + 1) / a.m - 1;
     // the pooling of the prefill compression (same thread layout, same
-    // arithmetic): the staged rows 0..m-2 and the token's own row m-1
-    const int CG = d / kPoolChan, tpb = CG * a.S;
-    const bool in_group = tid < tpb;
-    const int s = tid / CG, c0 = (tid % CG) * kPoolChan;
-    Gate4 st;
-    if (a.L <= kPoolStageRows) {
-      __nv_bfloat16* sm = reinterpret_cast<__nv_bfloat16*>(sh_gate);
-      pool_stage_rows(a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.m - 1, a.m, d, sm, tid,
-                      nthr);
-      if (in_group)
-        pool_slice_staged(st, sm, (size_t)a.m * d, a.Bias, d, a.L, s, c0);
-      else
-        gate_init(st);
-      if (a.S > 1) __syncthreads();  // the merge slots reuse the staged rows
-    } else if (in_group) {
-      pool_slice_direct<true>(st, a.Kblk + blk_base, a.Vblk + blk_base, a.Zblk + blk_base, kn, vn, zn, a.Bias, d, a.m,
-                              a.L, s, c0);
-    } else {
+    // arithmetic, same merge order): the staged rows 0..m-2 and the token's
+    // own row m-1, read straight from global memory
+    const int CG = d / kPoolChan, gsize = CG * a.S, R = a.m / a.S;
+    if (tid < gsize) {
+      const int s = tid / CG, cg = tid % CG;
+      const int64_t col = (int64_t)cg * kPoolChan;
+      Gate st;
       gate_init(st);
+      for (int r0 = 0; r0 < R; r0 += kPoolChunk) {
+        const int n = min(kPoolChunk, R - r0);
+        float g2[kPoolChunk][kPoolChan];
+        float cm[kPoolChan];
+#pragma unroll
+        for (int e = 0; e < kPoolChan; ++e) cm[e] = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kPoolChunk; ++q)
+          if (q < n) {
+            const int p = s * R + r0 + q;
+            const __nv_bfloat16* zr = p == a.m - 1 ? zn + col : a.Zblk + blk_base + (int64_t)p * d + col;
+            const float4* br = reinterpret_cast<const float4*>(a.Bias + (int64_t)p * d + col);
+            gate_logits(*reinterpret_cast<const uint4*>(zr), br[0], br[1], g2[q], cm);
+          }
+        gate_rescale(st, cm);
+#pragma unroll
+        for (int q = 0; q < kPoolChunk; ++q)
+          if (q < n) {
+            const int p = s * R + r0 + q;
+            const bool last = p == a.m - 1;
+            const __nv_bfloat16* kr = last ? kn + col : a.Kblk + blk_base + (int64_t)p * d + col;
+            const __nv_bfloat16* vr = last ? vn + col : a.Vblk + blk_base + (int64_t)p * d + col;
+            gate_accum(st, g2[q], *reinterpret_cast<const uint4*>(kr), *reinterpret_cast<const uint4*>(vr));
+          }
+      }
+      gate_group_merge(st, sh_gate, tid, CG, gsize, 1);
+      if (s == 0) gate_store(st, a.Kc + (b * a.Ncap + j) * d + col, a.Vc + (b * a.Ncap + j) * d + col);
     }
-    if (a.S > 1) gate_tree(st, sh_gate, nthr, tid, s, CG, a.S, in_group);
-    if (in_group && s == 0) gate_store(st, a.Kc + (b * a.Ncap + j) * d + c0, a.Vc + (b * a.Ncap + j) * d + c0);
     if (a.kIc != nullptr) {
       const int cb = a.dI / 2, sb = a.dI / 32;
       if (tid < cb / 4)
@@ -148,7 +162,7 @@ cudaError_t launch_decode_append(const void* Kn, const void* Vn, const void* Zn,
   a.m = m;
   a.W = W;
   a.dI = dI;
-  pool_shape(d, m, &a.L, &a.S);
+  a.S = pool_slices(d, m);
   a.Ncap = Ncap;
   a.Kwin = static_cast<__nv_bfloat16*>(Kwin);
   a.Vwin = static_cast<__nv_bfloat16*>(Vwin);
@@ -159,14 +173,9 @@ cudaError_t launch_decode_append(const void* Kn, const void* Vn, const void* Zn,
   a.Vc = static_cast<__nv_bfloat16*>(Vc);
   a.kIc = kIc;
   a.kIs = kIs;
-  const int tpb = (d / kPoolChan) * a.S;
-  const int threads = tpb > kMinThreads ? tpb : kMinThreads;
-  const size_t smem = pool_smem_bytes(a.L, a.S, m, d, 1, threads);
-  if (smem > 48 * 1024) {
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolMaxSmem);
-    if (e != cudaSuccess) return e;
-  }
+  const int gsize = (d / kPoolChan) * a.S;
+  const int threads = gsize > kMinThreads ? gsize : kMinThreads;
+  const size_t smem = (size_t)gate_scratch_floats(gsize, d / kPoolChan) * sizeof(float);
   for (int b0 = 0; b0 < B; b0 += kMaxSeqPerLaunch) {
     AppendPos P{};
     const int n = B - b0 < kMaxSeqPerLaunch ? B - b0 : kMaxSeqPerLaunch;

@@ -6,105 +6,170 @@
 //   Kc[j,c] = sum_i a_i K[i,c],  Vc[j,c] = sum_i a_i V[i,c].
 //
 // HBM-bound: every input byte is read once and every output byte written once.
-// A group of (d/4)*S threads pools one block (compress.cuh): the CTA first
-// copies all rows of its blocks into shared memory with 16-byte cp.async (every
-// load in flight at once, no registers held), each thread then pools 4
-// channels of a slice of L rows, and the slices merge in a fixed pairwise tree,
-// so the result does not depend on scheduling.  A CTA holds 512 threads (one group
-// when the group is larger), capped at 64 registers so that two CTAs - 32
-// warps, ~100 KB of loads in flight - share an SM (measured on the 131072-token
-// HCA compression: 50 us with two CTAs per SM, 63 us with one).
+// One CTA of 512 threads per SM, persistent.  The CTA's threads form groups of
+// d/8 * S threads that each pool one block at a time with the layout of
+// compress.cuh (8 channels of a slice of R = m/S rows per thread); block j goes
+// to CTA j mod grid, so every SM gets the same number of blocks to within one,
+// and a CTA's blocks go to its groups in turn.  Each thread streams its own
+// rows: a two-stage ring of 4-row chunks in shared memory filled by 16-byte
+// cp.async (three row pieces per row: Z, K, V), the next chunk's copies in
+// flight while the current one is pooled, so no barrier of the CTA and no
+// register holds a load in flight.  A group's slices merge when its block's
+// last chunk is pooled (warp shuffles, then the group's first warp).
 #include "common.cuh"
 #include "compress.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
 namespace {
 
-constexpr int kCtaThreads = 512;
+constexpr int kStages = 2;
+constexpr int kBiasSmemMax = 64 * 1024;  // bias tables up to this size are staged in shared memory
+constexpr int kSmemMax = 232448;         // shared memory of one CTA on sm_100
 
-// Thread layout: [block of the CTA][slice s][channel group cg]; blockDim.x =
-// tpb * blocks_per_cta.  Shared memory: pool_smem_bytes (staged rows, then the
-// merge slots).
-template <bool kStaged>
-__global__ void __launch_bounds__(kPoolMaxThreads, 2) compress_kernel(const __nv_bfloat16* __restrict__ K,
-                                                                      const __nv_bfloat16* __restrict__ V,
-                                                                      const __nv_bfloat16* __restrict__ Z,
-                                                                      const float* __restrict__ Bias,
-                                                                      int64_t nblocks, int d, int m, int L, int S,
-                                                                      __nv_bfloat16* __restrict__ Kc,
-                                                                      __nv_bfloat16* __restrict__ Vc) {
+// staged chunk rows: [stage][row][Z, K, V][thread] x 16 bytes
+__host__ __device__ constexpr size_t stage_bytes(int nt) { return (size_t)kStages * kPoolChunk * 3 * nt * 16; }
+
+// Shared memory: the staged rows, then the bias table [m][d] fp32 (kBiasSmem),
+// then the merge scratch of the CTA's groups.
+template <int NT, bool kBiasSmem>
+__global__ void __launch_bounds__(NT, 1) compress_kernel(const __nv_bfloat16* __restrict__ K,
+                                                         const __nv_bfloat16* __restrict__ V,
+                                                         const __nv_bfloat16* __restrict__ Z,
+                                                         const float* __restrict__ Bias, int64_t nblocks, int d, int m,
+                                                         int S, __nv_bfloat16* __restrict__ Kc,
+                                                         __nv_bfloat16* __restrict__ Vc) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
-  const int CG = d / kPoolChan;
-  const int tpb = CG * S;            // threads per compressed block
-  const int bpc = blockDim.x / tpb;  // compressed blocks per CTA
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int local = tid / tpb, r = tid % tpb;
-  const int s = r / CG, c0 = (r % CG) * kPoolChan;
-  const int64_t j0 = (int64_t)blockIdx.x * bpc;
-  const int64_t j = j0 + local;
-  const bool active = j < nblocks;
-  Gate4 st;
-  if (kStaged) {
-    // the CTA's blocks are consecutive rows: one cooperative copy of all of them
-    const int nb = (int)(nblocks - j0 < bpc ? nblocks - j0 : bpc);
-    const int nrows = nb * m;
-    __nv_bfloat16* sm = reinterpret_cast<__nv_bfloat16*>(sm_raw);
-    const int64_t base = j0 * m * d;
-    pool_stage_rows(K + base, V + base, Z + base, nullptr, nullptr, nullptr, -1, nrows, d, sm, tid, nthr);
-    if (active)
-      pool_slice_staged(st, sm + (size_t)local * m * d, (size_t)nrows * d, Bias, d, L, s, c0);
-    else
-      gate_init(st);
-    if (S > 1) {
-      __syncthreads();  // the merge slots reuse the staged rows
-      gate_tree(st, reinterpret_cast<float*>(sm_raw), nthr, tid, s, CG, S, true);
-    }
-  } else {
-    const int64_t base = active ? j * m * d : 0;
-    if (active)
-      pool_slice_direct<false>(st, K + base, V + base, Z + base, nullptr, nullptr, nullptr, Bias, d, m, L, s, c0);
-    else
-      gate_init(st);
-    if (S > 1) gate_tree(st, reinterpret_cast<float*>(sm_raw), nthr, tid, s, CG, S, true);
+  const int tid = threadIdx.x;
+  const int CG = d / kPoolChan, gsize = CG * S, gpc = NT / gsize;
+  const int g = tid / gsize, tg = tid % gsize, s = tg / CG, cg = tg % CG;
+  const int R = m / S, nch = (R + kPoolChunk - 1) / kPoolChunk;
+  float* bias_sm = reinterpret_cast<float*>(sm_raw + stage_bytes(NT));
+  const size_t bias_floats = kBiasSmem ? (size_t)m * d : 0;
+  if (kBiasSmem) {
+    // the bias table, shared by every group of the CTA (all threads, before any leaves)
+    for (int i = tid; i < m * d / 4; i += NT)
+      reinterpret_cast<float4*>(bias_sm)[i] = __ldg(reinterpret_cast<const float4*>(Bias) + i);
+    __syncthreads();
   }
-  if (active && s == 0) gate_store(st, Kc + j * d + c0, Vc + j * d + c0);
+  // blocks of this group: j = blockIdx.x + gridDim.x * (g + gpc * i), i = 0, 1, ...
+  const int64_t j0 = blockIdx.x + (int64_t)gridDim.x * g, jstep = (int64_t)gridDim.x * gpc;
+  if (g >= gpc || j0 >= nblocks) return;  // whole groups leave together
+  const int64_t items = (nblocks - 1 - j0) / jstep + 1;
+  const uint32_t stage0 = sm100::smem_u32(sm_raw) + (uint32_t)tid * 16u;
+  const uint4* stage_ld = reinterpret_cast<const uint4*>(sm_raw) + tid;
+  float* scratch = bias_sm + bias_floats + (size_t)g * gate_scratch_floats(gsize, CG);
+  const float* bias_base = (kBiasSmem ? bias_sm : Bias) + (size_t)s * R * d + cg * kPoolChan;
+  const int64_t col = (int64_t)s * R * d + cg * kPoolChan;  // the thread's piece of its slice's first row
+
+  // the copy stream runs kStages chunks ahead of the pooling
+  int64_t ii = 0;  // item and chunk of the next copy
+  int ic = 0;
+  auto issue = [&](int stg) {
+    if (ii < items) {
+      const int r0 = ic * kPoolChunk, n = min(kPoolChunk, R - r0);
+      const int64_t off = (j0 + jstep * ii) * m * d + col + (int64_t)r0 * d;
+#pragma unroll
+      for (int q = 0; q < kPoolChunk; ++q) {
+        if (q < n) {
+          const uint32_t dst = stage0 + (uint32_t)((stg * kPoolChunk + q) * 3) * (NT * 16u);
+          sm100::cp_async16(dst, Z + off + (int64_t)q * d, 16u);
+          sm100::cp_async16(dst + NT * 16u, K + off + (int64_t)q * d, 16u);
+          sm100::cp_async16(dst + 2u * NT * 16u, V + off + (int64_t)q * d, 16u);
+        }
+      }
+      if (++ic == nch) ic = 0, ++ii;
+    }
+    sm100::cp_async_commit();  // possibly empty: one group per chunk slot keeps the count uniform
+  };
+#pragma unroll
+  for (int stg = 0; stg < kStages; ++stg) issue(stg);
+
+  int stg = 0;
+  for (int64_t i = 0; i < items; ++i) {
+    const int64_t j = j0 + jstep * i;
+    Gate st;
+    gate_init(st);
+    for (int c = 0; c < nch; ++c) {
+      const int r0 = c * kPoolChunk, n = min(kPoolChunk, R - r0);
+      const float* bias = bias_base + (size_t)r0 * d;
+      sm100::cp_async_wait<kStages - 1>();
+      const uint4* sp = stage_ld + (size_t)stg * kPoolChunk * 3 * NT;
+      float g2[kPoolChunk][kPoolChan];
+      float cm[kPoolChan];
+#pragma unroll
+      for (int e = 0; e < kPoolChan; ++e) cm[e] = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < kPoolChunk; ++q)
+        if (q < n) {
+          const float4* br = reinterpret_cast<const float4*>(bias + (size_t)q * d);
+          if (kBiasSmem)
+            gate_logits(sp[(q * 3) * NT], br[0], br[1], g2[q], cm);
+          else
+            gate_logits(sp[(q * 3) * NT], __ldg(br), __ldg(br + 1), g2[q], cm);
+        }
+      gate_rescale(st, cm);
+#pragma unroll
+      for (int q = 0; q < kPoolChunk; ++q)
+        if (q < n) gate_accum(st, g2[q], sp[(q * 3 + 1) * NT], sp[(q * 3 + 2) * NT]);
+      issue(stg);  // this thread's reads of the slot are done: refill it
+      stg = stg + 1 == kStages ? 0 : stg + 1;
+    }
+    gate_group_merge(st, scratch, tg, CG, gsize, 1 + g);
+    if (s == 0) gate_store(st, Kc + j * d + cg * kPoolChan, Vc + j * d + cg * kPoolChan);
+  }
+  sm100::cp_async_wait_all();
+}
+
+template <int NT, bool kBiasSmem>
+size_t smem_bytes(int d, int m, int gsize) {
+  return stage_bytes(NT) + (kBiasSmem ? (size_t)m * d * sizeof(float) : 0) +
+         (size_t)(NT / gsize) * gate_scratch_floats(gsize, d / kPoolChan) * sizeof(float);
+}
+
+template <int NT, bool kBiasSmem>
+cudaError_t launch_t(const void* K, const void* V, const void* Z, const float* B, int64_t nblocks, int d, int m, int S,
+                     void* Kc, void* Vc, int sms, int dev, cudaStream_t stream) {
+  static bool attr_set[64] = {};  // opt in to the largest shared memory once per device
+  if (dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(compress_kernel<NT, kBiasSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemMax);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const int gsize = (d / kPoolChan) * S, gpc = NT / gsize;
+  // enough CTAs that every group has a block, at most one per SM
+  const int64_t need = ceil_div(nblocks, (int64_t)gpc);
+  const int grid = (int)(need < sms ? need : sms);
+  compress_kernel<NT, kBiasSmem><<<grid, NT, smem_bytes<NT, kBiasSmem>(d, m, gsize), stream>>>(
+      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), static_cast<const __nv_bfloat16*>(Z),
+      B, nblocks, d, m, S, static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc));
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-// Host launcher (validated arguments).
+// Host launcher (validated arguments).  512 threads per CTA; when the bias
+// table fits in shared memory it is staged there, with 384 threads if 512
+// threads' rows and the table do not fit together.
 cudaError_t launch_compress(const void* K, const void* V, const void* Z, const float* B, int64_t T, int d, int m,
                             void* Kc, void* Vc, cudaStream_t stream) {
   const int64_t nblocks = T / m;
   if (nblocks == 0) return cudaSuccess;
-  int L, S;
-  pool_shape(d, m, &L, &S);
-  const int tpb = (d / kPoolChan) * S;
-  int bpc = kCtaThreads / tpb;
-  if (bpc < 1) bpc = 1;
-  const int threads = tpb * bpc;
-  const bool staged = L <= kPoolStageRows;
-  const size_t smem = pool_smem_bytes(L, S, m, d, bpc, threads);
-  const int64_t grid = ceil_div(nblocks, bpc);
-  if (smem > 48 * 1024) {
-    static bool attr_set[64] = {};  // opt in to the largest staging area once per device
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_set[dev]) {
-      e = cudaFuncSetAttribute(compress_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolMaxSmem);
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(compress_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolMaxSmem);
-      if (e != cudaSuccess) return e;
-      if (dev < 64) attr_set[dev] = true;
-    }
+  const int S = pool_slices(d, m);
+  const int gsize = (d / kPoolChan) * S;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if ((size_t)m * d * sizeof(float) <= (size_t)kBiasSmemMax) {
+    if (smem_bytes<512, true>(d, m, gsize) <= (size_t)kSmemMax)
+      return launch_t<512, true>(K, V, Z, B, nblocks, d, m, S, Kc, Vc, sms, dev, stream);
+    if (384 % gsize == 0 && smem_bytes<384, true>(d, m, gsize) <= (size_t)kSmemMax)
+      return launch_t<384, true>(K, V, Z, B, nblocks, d, m, S, Kc, Vc, sms, dev, stream);
   }
-  auto kern = staged ? compress_kernel<true> : compress_kernel<false>;
-  kern<<<(unsigned)grid, threads, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), static_cast<const __nv_bfloat16*>(Z),
-      B, nblocks, d, m, L, S, static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc));
-  return cudaGetLastError();
+  return launch_t<512, false>(K, V, Z, B, nblocks, d, m, S, Kc, Vc, sms, dev, stream);
 }
 
 }  // namespace csa

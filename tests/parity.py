@@ -22,33 +22,46 @@ def from_words(w, device):
     return torch.from_numpy(np.ascontiguousarray(w).view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def _pool_shape(d, m):
-    """Rows per thread L and slices S of the GPU pooling of one block (the launch
-    rule of the compression kernel: L = m up to 8, else 4, doubled while
-    (d/4) * (m/L) > 512 threads)."""
-    L = m if m <= 8 else 4
-    while (d // 4) * (m // L) > 512:
-        L *= 2
-    return L, m // L
+def _pool_exp2_depth(d, m):
+    """N, the most exp2 factors on the path of one gate weight in the GPU
+    pooling of a block (its launch rule): S slices of R = m/S rows (S = 1 up to
+    16 rows, else the largest power of two with >= 16 rows per slice and m a
+    multiple of 8S, and d/8 * S <= 512 threads), pooled in chunks of 4 rows; groups of d/8 * S threads
+    merge in-warp pairwise over log2 levels, then the first warp of a group
+    merges the other warps in turn.  A weight meets its own exp2, the rescales
+    after its chunk (at most chunks - 1), one factor per in-warp level and at
+    most nw - 1 factors in the cross-warp merge."""
+    S = 1
+    while 2 * S <= m // 16 and m % (8 * S) == 0 and 2 * S * (d // 8) <= 512:
+        S *= 2
+    chunks = -(-(m // S) // 4)
+    CG = d // 8
+    gsize = CG * S
+    levels, mask = 0, CG
+    while mask < 32 and mask < gsize:
+        levels += 1
+        mask <<= 1
+    nw = gsize // 32 if gsize > 32 else 1
+    return chunks + levels + nw - 1
 
 
 def fp32_pool_slack(x_bf16, m, Z, B):
     """Worst-case absolute error of the fp32 gated pooling, per (block, channel),
     with u = 2^-24, X = max |x| over the block, G = max |z + b| over the block,
-    and the kernel's L rows per slice and S slices:
+    and N = _pool_exp2_depth(d, m):
       the kernel takes logits in base 2, g2 = RN(RN(z + b) * RN(log2 e)), so every
       logit carries 3uG (the sum, the rounded constant, the product; an error
       common to all logits of a block cancels in the normalised mean), and
-      every weight exp2(g2_i - max) a relative error of at most
-        3*u*G + (L + S) * (2*u*G + 4*u)
-      (its own exp2 and each of the at most L-1 in-slice rescales and of the
-      slice merges on its path - ceil(log2 S) <= S-1 in the kernel's pairwise
-      tree - is one exp2 of a rounded difference: 2uG for the difference, 4u for
-      exp2f's 2-ulp bound); a relative weight error eta moves a weighted mean by
-      at most 2*eta*X; the m-term sums of numerator and denominator plus the L
-      rescale products add (m + L) * u * X each; the division and the final
-      product 2*u*X.  Total:
-        u * X * (2*G*(3 + 2*(L+S)) + 8*(L+S) + 2*(m+L) + 2).
+      every weight a relative error of at most
+        3*u*G + N * (2*u*G + 4*u)
+      (each of its N exp2 factors - its own, the in-slice rescales after it and
+      the slice merges on its path - is one exp2 of a rounded difference: 2uG
+      for the difference, 4u for exp2f's 2-ulp bound); a relative weight error
+      eta moves a weighted mean by at most 2*eta*X; the sums of numerator and
+      denominator (m terms, each through at most m - 1 additions in any order,
+      and at most N rescale products) add (m + N) * u * X each; the division and
+      the final product 2*u*X.  Total:
+        u * X * (2*G*(3 + 2*N) + 8*N + 2*(m + N) + 2).
     When the weighted sum cancels, this can exceed one bf16 ulp of the (small)
     result; otherwise the bf16 ulp dominates."""
     xf = x_bf16.detach().float().cpu().double().numpy() if hasattr(x_bf16, "detach") else oracle.bf16_words_to_f64(x_bf16)
@@ -59,9 +72,9 @@ def fp32_pool_slack(x_bf16, m, Z, B):
     X = np.abs(xf[: nb * m]).reshape(nb, m, d).max(axis=1)
     g = zf[: nb * m].reshape(nb, m, d) + bf[None, :, :]
     G = np.abs(g).max(axis=1)
-    L, S = _pool_shape(d, m)
+    N = _pool_exp2_depth(d, m)
     u = 2.0 ** -24
-    return u * X * (2 * G * (3 + 2 * (L + S)) + 8 * (L + S) + 2 * (m + L) + 2)
+    return u * X * (2 * G * (3 + 2 * N) + 8 * N + 2 * (m + N) + 2)
 
 
 def assert_within_bf16_ulp(got_bf16, exact_f64, what, slack=None):

@@ -145,3 +145,30 @@ def test_hca_decode_with_appends(csa):
     Kr, Vr = csa.csa_compress(K[: n * m].cuda(), V[: n * m].cuda(), Z[: n * m].cuda(), Bg, m)
     assert torch.equal(Kc[0, :n], Kr) and torch.equal(Vc[0, :n], Vr)
     assert torch.equal(Kw[0], K[pend - W:pend].cuda())
+
+
+@pytest.mark.parametrize("d,m", [(64, 3), (128, 6), (64, 64), (128, 40), (128, 512), (64, 512)])
+def test_append_pooling_layouts(csa, d, m):
+    """Append 2m + 1 tokens from an empty state: the two completed entries are
+    bit-identical to csa_compress of the same tokens for pooling layouts with
+    sub-warp groups, in-warp levels and cross-warp merges, and within tolerance
+    of the oracle."""
+    from tests.parity import assert_within_bf16_ulp, fp32_pool_slack
+    W, n = 4, 2 * m + 1
+    s = 700 + m + d
+    K, V, Z = (inputs.normal_bf16((n, d), s, x) for x in ("K", "V", "Z"))
+    Bias = inputs.normal_f32((m, d), s, "B", std=0.5)
+    Bg = Bias.cuda()
+    z = lambda *shape: torch.zeros(*shape, dtype=torch.bfloat16, device="cuda")
+    Kw, Vw, Kb, Vb, Zb, Kc, Vc = z(1, W, d), z(1, W, d), z(1, m, d), z(1, m, d), z(1, m, d), z(1, 3, d), z(1, 3, d)
+    Kg, Vg, Zg = K.cuda(), V.cuda(), Z.cuda()
+    for p in range(n):
+        csa.hca_decode_append(Kg[p:p + 1], Vg[p:p + 1], Zg[p:p + 1], Bg, [p], Kw, Vw, Kb, Vb, Zb, Kc, Vc)
+    Kr, Vr = csa.csa_compress(Kg[: 2 * m], Vg[: 2 * m], Zg[: 2 * m], Bg, m)
+    torch.cuda.synchronize()
+    assert torch.equal(Kc[0, :2], Kr) and torch.equal(Vc[0, :2], Vr)
+    assert not Kc[0, 2].any()
+    Kx, Vx = oracle.compress(K[: 2 * m], V[: 2 * m], Z[: 2 * m], Bias, m)
+    assert_within_bf16_ulp(Kr, Kx, "Kc", fp32_pool_slack(K[: 2 * m], m, Z[: 2 * m], Bias))
+    assert_within_bf16_ulp(Vr, Vx, "Vc", fp32_pool_slack(V[: 2 * m], m, Z[: 2 * m], Bias))
+    assert torch.equal(Kw[0], Kg[n - W:n])

@@ -301,7 +301,9 @@ def test_hca_decode(csa):
         np.testing.assert_allclose(lse[b:b + 1].cpu().numpy(), l, atol=2e-3)
 
 
-@pytest.mark.parametrize("T,d,m", [(1000, 128, 4), (1000, 64, 64), (4096, 128, 128), (333, 128, 8), (640, 64, 1)])
+@pytest.mark.parametrize("T,d,m", [(1000, 128, 4), (1000, 64, 64), (4096, 128, 128), (333, 128, 8), (640, 64, 1),
+                                   (1001, 64, 3), (997, 128, 6), (3000, 128, 24), (4000, 64, 40), (2200, 128, 136),
+                                   (5120, 128, 512), (5000, 64, 512), (70000, 128, 4), (300000, 128, 128)])
 def test_compress_edges(csa, T, d, m):
     from tests.parity import assert_within_bf16_ulp, fp32_pool_slack
     g = torch.Generator().manual_seed(T + m)
