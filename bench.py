@@ -696,12 +696,12 @@ def run_compress(csa, wl, steps):
         d = sets[i % len(sets)]
         csa.csa_compress(d["K"], d["V"], d["Z"], d["B_hca"], wl.m_hca, Kc=Kc, Vc=Vc)
 
-    reps = 3 * max(10, steps)
+    reps = 3 * max(50, steps)
     for i in range(6):
         launch(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda._sleep(4_000_000)
+    torch.cuda._sleep(20_000_000)  # ~10 ms at 2 GHz: the host queues all launches meanwhile
     e0.record()
     for i in range(reps):
         launch(i)

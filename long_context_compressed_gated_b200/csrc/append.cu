@@ -103,10 +103,10 @@ __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const Ap
       gate_init(st);
       for (int r0 = 0; r0 < R; r0 += kPoolChunk) {
         const int n = min(kPoolChunk, R - r0);
-        float g2[kPoolChunk][kPoolChan];
-        float cm[kPoolChan];
+        float2 g2[kPoolChunk][4], nm[4];
+        float2 cm[4];
 #pragma unroll
-        for (int e = 0; e < kPoolChan; ++e) cm[e] = -INFINITY;
+        for (int e = 0; e < 4; ++e) cm[e] = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
         for (int q = 0; q < kPoolChunk; ++q)
           if (q < n) {
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const Ap
             const float4* br = reinterpret_cast<const float4*>(a.Bias + (int64_t)p * d + col);
             gate_logits(*reinterpret_cast<const uint4*>(zr), br[0], br[1], g2[q], cm);
           }
-        gate_rescale(st, cm);
+        gate_rescale(st, cm, nm);
 #pragma unroll
         for (int q = 0; q < kPoolChunk; ++q)
           if (q < n) {
@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const Ap
             const bool last = p == a.m - 1;
             const __nv_bfloat16* kr = last ? kn + col : a.Kblk + blk_base + (int64_t)p * d + col;
             const __nv_bfloat16* vr = last ? vn + col : a.Vblk + blk_base + (int64_t)p * d + col;
-            gate_accum(st, g2[q], *reinterpret_cast<const uint4*>(kr), *reinterpret_cast<const uint4*>(vr));
+            gate_accum(st, g2[q], nm, *reinterpret_cast<const uint4*>(kr), *reinterpret_cast<const uint4*>(vr));
           }
       }
       gate_group_merge(st, sh_gate, tid, CG, gsize, 1);

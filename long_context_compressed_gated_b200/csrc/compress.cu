@@ -11,7 +11,7 @@
 // compress.cuh (8 channels of a slice of R = m/S rows per thread); block j goes
 // to CTA j mod grid, so every SM gets the same number of blocks to within one,
 // and a CTA's blocks go to its groups in turn.  Each thread streams its own
-// rows: a two-stage ring of 4-row chunks in shared memory filled by 16-byte
+// rows: a two-stage ring of 2-row chunks in shared memory filled by 16-byte
 // cp.async (three row pieces per row: Z, K, V), the next chunk's copies in
 // flight while the current one is pooled, so no barrier of the CTA and no
 // register holds a load in flight.  A group's slices merge when its block's
@@ -96,10 +96,10 @@ __global__ void __launch_bounds__(NT, 1) compress_kernel(const __nv_bfloat16* __
       const float* bias = bias_base + (size_t)r0 * d;
       sm100::cp_async_wait<kStages - 1>();
       const uint4* sp = stage_ld + (size_t)stg * kPoolChunk * 3 * NT;
-      float g2[kPoolChunk][kPoolChan];
-      float cm[kPoolChan];
+      float2 g2[kPoolChunk][4], nm[4];
+      float2 cm[4];
 #pragma unroll
-      for (int e = 0; e < kPoolChan; ++e) cm[e] = -INFINITY;
+      for (int p = 0; p < 4; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
       for (int q = 0; q < kPoolChunk; ++q)
         if (q < n) {
@@ -109,10 +109,10 @@ __global__ void __launch_bounds__(NT, 1) compress_kernel(const __nv_bfloat16* __
           else
             gate_logits(sp[(q * 3) * NT], __ldg(br), __ldg(br + 1), g2[q], cm);
         }
-      gate_rescale(st, cm);
+      gate_rescale(st, cm, nm);
 #pragma unroll
       for (int q = 0; q < kPoolChunk; ++q)
-        if (q < n) gate_accum(st, g2[q], sp[(q * 3 + 1) * NT], sp[(q * 3 + 2) * NT]);
+        if (q < n) gate_accum(st, g2[q], nm, sp[(q * 3 + 1) * NT], sp[(q * 3 + 2) * NT]);
       issue(stg);  // this thread's reads of the slot are done: refill it
       stg = stg + 1 == kStages ? 0 : stg + 1;
     }

@@ -10,7 +10,7 @@
 // Thread layout of one block (its "group"): S slices of R = m / S consecutive
 // rows times d/8 channel groups; thread t = s*(d/8) + cg owns channels
 // 8cg..8cg+7 (one 16-byte piece of a row) of slice s.  A slice is pooled in
-// chunks of up to four rows: the chunk's base-2 logits g2 = (z + b) * log2(e)
+// chunks of up to two rows: the chunk's base-2 logits g2 = (z + b) * log2(e)
 // and their maximum per channel first, the running sums rescaled when that
 // maximum grows, then one exp2 per element, w = exp2(g2 - max) (the SFU's
 // ex2.approx.ftz: about 2 ulp; results below 2^-126 flush to zero).
@@ -25,7 +25,7 @@
 namespace csa {
 
 constexpr int kPoolChan = 8;           // channels per thread: one 16-byte piece of a row
-constexpr int kPoolChunk = 4;          // rows per chunk
+constexpr int kPoolChunk = 2;          // rows per chunk
 constexpr int kPoolMaxThreads = 512;   // threads of one block's group at most
 constexpr int kGateWords = 4 * kPoolChan;
 constexpr float kPoolLog2e = 1.44269504088896341f;  // log2(e), rounded to fp32
@@ -49,78 +49,93 @@ __device__ __forceinline__ float pool_exp2(float x) {
   return y;
 }
 
-// Online-softmax state of 8 channels: running max (of base-2 logits),
-// denominator, two sums.
+// Online-softmax state of 8 channels as 4 channel pairs: running max (of
+// base-2 logits), denominator, two sums.  The element-wise steps run on pairs
+// (sm_100's packed fp32 add/mul/fma: per component the same IEEE operation,
+// round to nearest even, as the scalar one).
 struct Gate {
-  float mx[kPoolChan], den[kPoolChan], k[kPoolChan], v[kPoolChan];
+  float2 mx[4], den[4], k[4], v[4];
 };
 
+__device__ __forceinline__ float& pair_at(float2* a, int i) { return (i & 1) ? a[i >> 1].y : a[i >> 1].x; }
+
 __device__ __forceinline__ float& gate_word(Gate& st, int w) {
-  return w < 8 ? st.mx[w] : (w < 16 ? st.den[w - 8] : (w < 24 ? st.k[w - 16] : st.v[w - 24]));
+  return w < 8 ? pair_at(st.mx, w) : (w < 16 ? pair_at(st.den, w - 8) : (w < 24 ? pair_at(st.k, w - 16) : pair_at(st.v, w - 24)));
 }
 
 __device__ __forceinline__ void gate_init(Gate& st) {
 #pragma unroll
-  for (int e = 0; e < kPoolChan; ++e) st.mx[e] = -INFINITY, st.den[e] = st.k[e] = st.v[e] = 0.f;
+  for (int p = 0; p < 4; ++p) {
+    st.mx[p] = make_float2(-INFINITY, -INFINITY);
+    st.den[p] = st.k[p] = st.v[p] = make_float2(0.f, 0.f);
+  }
 }
 
 // a <- merge(a, b), both normalised to their own running max.  Every operation
 // is commutative in (a, b), so merge(a, b) and merge(b, a) are the same bits.
-__device__ __forceinline__ void gate_merge(Gate& a, const Gate& b) {
+__device__ __forceinline__ void gate_merge(Gate& a, Gate& b) {
 #pragma unroll
   for (int e = 0; e < kPoolChan; ++e) {
-    const float m = fmaxf(a.mx[e], b.mx[e]);
+    float &amx = pair_at(a.mx, e), &aden = pair_at(a.den, e), &ak = pair_at(a.k, e), &av = pair_at(a.v, e);
+    const float bmx = pair_at(b.mx, e), bden = pair_at(b.den, e), bk = pair_at(b.k, e), bv = pair_at(b.v, e);
+    const float m = fmaxf(amx, bmx);
     if (m == -INFINITY) continue;
-    const float sa = pool_exp2(__fsub_rn(a.mx[e], m)), sb = pool_exp2(__fsub_rn(b.mx[e], m));
-    a.den[e] = __fadd_rn(__fmul_rn(a.den[e], sa), __fmul_rn(b.den[e], sb));
-    a.k[e] = __fadd_rn(__fmul_rn(a.k[e], sa), __fmul_rn(b.k[e], sb));
-    a.v[e] = __fadd_rn(__fmul_rn(a.v[e], sa), __fmul_rn(b.v[e], sb));
-    a.mx[e] = m;
+    const float sa = pool_exp2(__fsub_rn(amx, m)), sb = pool_exp2(__fsub_rn(bmx, m));
+    aden = __fadd_rn(__fmul_rn(aden, sa), __fmul_rn(bden, sb));
+    ak = __fadd_rn(__fmul_rn(ak, sa), __fmul_rn(bk, sb));
+    av = __fadd_rn(__fmul_rn(av, sa), __fmul_rn(bv, sb));
+    amx = m;
   }
 }
 
-__device__ __forceinline__ void unpack8(const uint4 r, float (&f)[8]) {
-  f[0] = bf16_lo(r.x), f[1] = bf16_hi(r.x), f[2] = bf16_lo(r.y), f[3] = bf16_hi(r.y);
-  f[4] = bf16_lo(r.z), f[5] = bf16_hi(r.z), f[6] = bf16_lo(r.w), f[7] = bf16_hi(r.w);
-}
+// bf16 pair (low half first) -> two floats, exactly.
+__device__ __forceinline__ float2 bf16x2_f2(uint32_t w) { return make_float2(bf16_lo(w), bf16_hi(w)); }
 
 // Base-2 logits of one row (8 channels) and the chunk maximum.
-__device__ __forceinline__ void gate_logits(const uint4 zr, const float4 b0, const float4 b1, float (&g2)[kPoolChan],
-                                            float (&cm)[kPoolChan]) {
-  float z[8];
-  unpack8(zr, z);
-  const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+__device__ __forceinline__ void gate_logits(const uint4 zr, const float4 b0, const float4 b1, float2 (&g2)[4],
+                                            float2 (&cm)[4]) {
+  const float2 z[4] = {bf16x2_f2(zr.x), bf16x2_f2(zr.y), bf16x2_f2(zr.z), bf16x2_f2(zr.w)};
+  const float2 b[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                       make_float2(b1.z, b1.w)};
+  const float2 l2e = make_float2(kPoolLog2e, kPoolLog2e);
 #pragma unroll
-  for (int e = 0; e < kPoolChan; ++e) {
-    g2[e] = __fmul_rn(__fadd_rn(z[e], b[e]), kPoolLog2e);
-    cm[e] = fmaxf(cm[e], g2[e]);
+  for (int p = 0; p < 4; ++p) {
+    g2[p] = __fmul2_rn(__fadd2_rn(z[p], b[p]), l2e);
+    cm[p].x = fmaxf(cm[p].x, g2[p].x);
+    cm[p].y = fmaxf(cm[p].y, g2[p].y);
   }
 }
 
 // The running sums follow the chunk maximum when it grows (a multiply by
-// exp2 of the rounded difference; by exactly 1 otherwise).
-__device__ __forceinline__ void gate_rescale(Gate& st, const float (&cm)[kPoolChan]) {
+// exp2 of the rounded difference; by exactly 1 otherwise); nm receives the
+// negated running maxima for gate_accum.
+__device__ __forceinline__ void gate_rescale(Gate& st, const float2 (&cm)[4], float2 (&nm)[4]) {
 #pragma unroll
-  for (int e = 0; e < kPoolChan; ++e) {
-    const bool grow = cm[e] > st.mx[e];
-    const float sc = grow ? pool_exp2(__fsub_rn(st.mx[e], cm[e])) : 1.0f;
-    st.den[e] = __fmul_rn(st.den[e], sc);
-    st.k[e] = __fmul_rn(st.k[e], sc);
-    st.v[e] = __fmul_rn(st.v[e], sc);
-    st.mx[e] = grow ? cm[e] : st.mx[e];
+  for (int p = 0; p < 4; ++p) {
+    const bool gx = cm[p].x > st.mx[p].x, gy = cm[p].y > st.mx[p].y;
+    const float2 sc = make_float2(gx ? pool_exp2(__fsub_rn(st.mx[p].x, cm[p].x)) : 1.0f,
+                                  gy ? pool_exp2(__fsub_rn(st.mx[p].y, cm[p].y)) : 1.0f);
+    st.den[p] = __fmul2_rn(st.den[p], sc);
+    st.k[p] = __fmul2_rn(st.k[p], sc);
+    st.v[p] = __fmul2_rn(st.v[p], sc);
+    st.mx[p] = make_float2(gx ? cm[p].x : st.mx[p].x, gy ? cm[p].y : st.mx[p].y);
+    nm[p] = make_float2(-st.mx[p].x, -st.mx[p].y);
   }
 }
 
-__device__ __forceinline__ void gate_accum(Gate& st, const float (&g2)[kPoolChan], const uint4 kr, const uint4 vr) {
-  float kf[8], vf[8];
-  unpack8(kr, kf);
-  unpack8(vr, vf);
+// One row: w = exp2(g2 - max) (the difference as g2 + (-max): the same
+// rounding), den += w, k += w * K, v += w * V.
+__device__ __forceinline__ void gate_accum(Gate& st, const float2 (&g2)[4], const float2 (&nm)[4], const uint4 kr,
+                                           const uint4 vr) {
+  const float2 kf[4] = {bf16x2_f2(kr.x), bf16x2_f2(kr.y), bf16x2_f2(kr.z), bf16x2_f2(kr.w)};
+  const float2 vf[4] = {bf16x2_f2(vr.x), bf16x2_f2(vr.y), bf16x2_f2(vr.z), bf16x2_f2(vr.w)};
 #pragma unroll
-  for (int e = 0; e < kPoolChan; ++e) {
-    const float w = pool_exp2(__fsub_rn(g2[e], st.mx[e]));
-    st.den[e] = __fadd_rn(st.den[e], w);
-    st.k[e] = __fmaf_rn(w, kf[e], st.k[e]);
-    st.v[e] = __fmaf_rn(w, vf[e], st.v[e]);
+  for (int p = 0; p < 4; ++p) {
+    const float2 dd = __fadd2_rn(g2[p], nm[p]);
+    const float2 w = make_float2(pool_exp2(dd.x), pool_exp2(dd.y));
+    st.den[p] = __fadd2_rn(st.den[p], w);
+    st.k[p] = __ffma2_rn(w, kf[p], st.k[p]);
+    st.v[p] = __ffma2_rn(w, vf[p], st.v[p]);
   }
 }
 
@@ -171,14 +186,13 @@ __host__ __device__ inline int gate_scratch_floats(int gsize, int CG) {
 }
 
 // Normalise and write 8 channels of Kc/Vc (round to nearest even).
-__device__ __forceinline__ void gate_store(const Gate& st, __nv_bfloat16* __restrict__ Kc,
-                                           __nv_bfloat16* __restrict__ Vc) {
+__device__ __forceinline__ void gate_store(Gate& st, __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Vc) {
   float kf[8], vf[8];
 #pragma unroll
   for (int e = 0; e < kPoolChan; ++e) {
-    const float inv = __fdiv_rn(1.0f, st.den[e]);
-    kf[e] = __fmul_rn(st.k[e], inv);
-    vf[e] = __fmul_rn(st.v[e], inv);
+    const float inv = __fdiv_rn(1.0f, pair_at(st.den, e));
+    kf[e] = __fmul_rn(pair_at(st.k, e), inv);
+    vf[e] = __fmul_rn(pair_at(st.v, e), inv);
   }
   *reinterpret_cast<uint4*>(Kc) = make_uint4(pack_bf16x2(kf[0], kf[1]), pack_bf16x2(kf[2], kf[3]),
                                              pack_bf16x2(kf[4], kf[5]), pack_bf16x2(kf[6], kf[7]));

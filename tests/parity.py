@@ -25,16 +25,16 @@ def from_words(w, device):
 def _pool_exp2_depth(d, m):
     """N, the most exp2 factors on the path of one gate weight in the GPU
     pooling of a block (its launch rule): S slices of R = m/S rows (S = 1 up to
-    16 rows, else the largest power of two with >= 16 rows per slice and m a
-    multiple of 8S, and d/8 * S <= 512 threads), pooled in chunks of 4 rows; groups of d/8 * S threads
-    merge in-warp pairwise over log2 levels, then the first warp of a group
-    merges the other warps in turn.  A weight meets its own exp2, the rescales
+    16 rows, else the largest power of two with >= 16 rows per slice, m a
+    multiple of 8S and d/8 * S <= 512 threads), pooled in chunks of 2 rows;
+    groups of d/8 * S threads merge in-warp pairwise over log2 levels, then the
+    first warp of a group merges the other warps in turn.  A weight meets its own exp2, the rescales
     after its chunk (at most chunks - 1), one factor per in-warp level and at
     most nw - 1 factors in the cross-warp merge."""
     S = 1
     while 2 * S <= m // 16 and m % (8 * S) == 0 and 2 * S * (d // 8) <= 512:
         S *= 2
-    chunks = -(-(m // S) // 4)
+    chunks = -(-(m // S) // 2)
     CG = d // 8
     gsize = CG * S
     levels, mask = 0, CG
