@@ -115,7 +115,10 @@ __global__ void __launch_bounds__(kPoolMaxThreads) decode_append_kernel(const Ap
             const float4* br = reinterpret_cast<const float4*>(a.Bias + (int64_t)p * d + col);
             gate_logits(*reinterpret_cast<const uint4*>(zr), br[0], br[1], g2[q], cm);
           }
-        gate_rescale(st, cm, nm);
+        if (r0 == 0)
+          gate_begin(st, cm, nm);
+        else
+          gate_rescale(st, cm, nm);
 #pragma unroll
         for (int q = 0; q < kPoolChunk; ++q)
           if (q < n) {

@@ -61,25 +61,28 @@ __global__ void __launch_bounds__(NT, 1) compress_kernel(const __nv_bfloat16* __
   const uint4* stage_ld = reinterpret_cast<const uint4*>(sm_raw) + tid;
   float* scratch = bias_sm + bias_floats + (size_t)g * gate_scratch_floats(gsize, CG);
   const float* bias_base = (kBiasSmem ? bias_sm : Bias) + (size_t)s * R * d + cg * kPoolChan;
-  const int64_t col = (int64_t)s * R * d + cg * kPoolChan;  // the thread's piece of its slice's first row
-
-  // the copy stream runs kStages chunks ahead of the pooling
-  int64_t ii = 0;  // item and chunk of the next copy
+  // the copy stream runs kStages chunks ahead of the pooling: offset of the
+  // next chunk's first row piece (the thread's slice of its group's first block
+  // to begin with), and the chunk and item it belongs to
+  int64_t ioff = j0 * m * d + (int64_t)s * R * d + cg * kPoolChan;
+  const int64_t item_skip = jstep * m * d - (int64_t)nch * kPoolChunk * d;
+  int64_t ii = 0;
   int ic = 0;
   auto issue = [&](int stg) {
     if (ii < items) {
-      const int r0 = ic * kPoolChunk, n = min(kPoolChunk, R - r0);
-      const int64_t off = (j0 + jstep * ii) * m * d + col + (int64_t)r0 * d;
+      const int n = min(kPoolChunk, R - ic * kPoolChunk);
 #pragma unroll
       for (int q = 0; q < kPoolChunk; ++q) {
         if (q < n) {
           const uint32_t dst = stage0 + (uint32_t)((stg * kPoolChunk + q) * 3) * (NT * 16u);
-          sm100::cp_async16(dst, Z + off + (int64_t)q * d, 16u);
-          sm100::cp_async16(dst + NT * 16u, K + off + (int64_t)q * d, 16u);
-          sm100::cp_async16(dst + 2u * NT * 16u, V + off + (int64_t)q * d, 16u);
+          const int64_t off = ioff + (int64_t)q * d;
+          sm100::cp_async16(dst, Z + off, 16u);
+          sm100::cp_async16(dst + NT * 16u, K + off, 16u);
+          sm100::cp_async16(dst + 2u * NT * 16u, V + off, 16u);
         }
       }
-      if (++ic == nch) ic = 0, ++ii;
+      ioff += (int64_t)kPoolChunk * d;
+      if (++ic == nch) ic = 0, ++ii, ioff += item_skip;
     }
     sm100::cp_async_commit();  // possibly empty: one group per chunk slot keeps the count uniform
   };
@@ -109,7 +112,10 @@ __global__ void __launch_bounds__(NT, 1) compress_kernel(const __nv_bfloat16* __
           else
             gate_logits(sp[(q * 3) * NT], __ldg(br), __ldg(br + 1), g2[q], cm);
         }
-      gate_rescale(st, cm, nm);
+      if (c == 0)
+        gate_begin(st, cm, nm);
+      else
+        gate_rescale(st, cm, nm);
 #pragma unroll
       for (int q = 0; q < kPoolChunk; ++q)
         if (q < n) gate_accum(st, g2[q], nm, sp[(q * 3 + 1) * NT], sp[(q * 3 + 2) * NT]);

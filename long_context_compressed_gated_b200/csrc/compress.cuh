@@ -123,6 +123,16 @@ __device__ __forceinline__ void gate_rescale(Gate& st, const float2 (&cm)[4], fl
   }
 }
 
+// gate_rescale on a state fresh from gate_init (the slice's first chunk): the
+// sums are +0 and stay +0 (+0 * exp2(-inf) = +0), so only the maximum moves.
+__device__ __forceinline__ void gate_begin(Gate& st, const float2 (&cm)[4], float2 (&nm)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    st.mx[p] = cm[p];
+    nm[p] = make_float2(-cm[p].x, -cm[p].y);
+  }
+}
+
 // One row: w = exp2(g2 - max) (the difference as g2 + (-max): the same
 // rounding), den += w, k += w * K, v += w * V.
 __device__ __forceinline__ void gate_accum(Gate& st, const float2 (&g2)[4], const float2 (&nm)[4], const uint4 kr,
