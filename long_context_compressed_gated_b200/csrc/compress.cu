@@ -6,7 +6,8 @@
 //   Kc[j,c] = sum_i a_i K[i,c],  Vc[j,c] = sum_i a_i V[i,c].
 //
 // HBM-bound: every input byte is read once and every output byte written once.
-// One CTA of 512 threads per SM, persistent.  The CTA's threads form groups of
+// One CTA of 512 threads per SM (384 where 512 threads' staging and the bias
+// table do not fit together), persistent.  The CTA's threads form groups of
 // d/8 * S threads that each pool one block at a time with the layout of
 // compress.cuh (8 channels of a slice of R = m/S rows per thread); block j goes
 // to CTA j mod grid, so every SM gets the same number of blocks to within one,
@@ -14,8 +15,11 @@
 // rows: a two-stage ring of 2-row chunks in shared memory filled by 16-byte
 // cp.async (three row pieces per row: Z, K, V), the next chunk's copies in
 // flight while the current one is pooled, so no barrier of the CTA and no
-// register holds a load in flight.  A group's slices merge when its block's
-// last chunk is pooled (warp shuffles, then the group's first warp).
+// register holds a load in flight.  The bias table B [m, d] is copied into
+// shared memory once per CTA when it is at most 64 KB (every chunk would
+// otherwise wait on an L2 round trip for its rows of B).  A group's slices
+// merge when its block's last chunk is pooled (warp shuffles, then the group's
+// first warp).
 #include "common.cuh"
 #include "compress.cuh"
 #include "sm100.cuh"
